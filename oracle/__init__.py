@@ -1,0 +1,170 @@
+"""fp64 CPU oracle for flex attention -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's
+``cpu_baseline`` / reference leg may import this package.  It shares no code
+with the CUDA library: ``flex_oracle.c`` restates the method from its
+definition (see the header of that file for the formulas and their sources).
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, library special cases, exact identities, hand-worked golden
+values); nothing is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "flex_oracle.c")
+_LIB = os.path.join(_HERE, "_flex_oracle.so")
+
+SCORE_MODS = {"none": 0, "alibi": 1}
+MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset": 3,
+             # causal=True is the same keep rule as causal_via_mask
+             "causal_fast": 1}
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile flex_oracle.c into a shared library next to it (gcc -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm", "-lpthread"]
+        subprocess.check_call(cmd)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.oracle_fwd.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, I64, P, P, P, I]
+        lib.oracle_fwd.restype = I
+        lib.oracle_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P, I]
+        lib.oracle_decode.restype = I
+        lib.oracle_mask_matrix.argtypes = [I, I, I, I, I, P]
+        lib.oracle_mask_matrix.restype = I
+        lib.oracle_tile_map.argtypes = [I, I, I, I, I, I, I, P]
+        lib.oracle_tile_map.restype = I
+        lib.oracle_alibi_slope.argtypes = [I, I]
+        lib.oracle_alibi_slope.restype = D
+        _lib = lib
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return 0
+    if t.dtype == torch.float16:
+        return 1
+    raise TypeError(f"oracle takes bf16/f16 tensors, got {t.dtype}")
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """The raw 16-bit patterns of a CPU bf16/f16 tensor (contiguous copy)."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
+        rows=None, want_probs=False, threads=None):
+    """Oracle forward.  q [B,H,Sq,D], k/v [B,Hkv,Skv,D] (CPU bf16/f16 tensors).
+
+    rows: optional int64 array of flattened (b*H + h)*Sq + i row indices.
+    Returns (O, LSE[, P]) as float64 numpy arrays; O is [B,H,Sq,D] / LSE
+    [B,H,Sq] for all rows, or [n,D] / [n] for a row subset.
+    """
+    lib = _load()
+    B, H, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k.shape
+    assert Bk == B and Dk == D and tuple(v.shape) == tuple(k.shape)
+    assert q.dtype == k.dtype == v.dtype
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    if rows is None:
+        n = B * H * Sq
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n = int(rows_arr.size)
+    o = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    probs = np.zeros((n, Skv), dtype=np.float64) if want_probs else None
+    rc = lib.oracle_fwd(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, _dtype_code(q),
+                        B, H, Hkv, Sq, Skv, D, float(scale),
+                        SCORE_MODS[score_mod], MASK_MODS[mask_mod], int(window), int(offset),
+                        None if rows_arr is None else rows_arr.ctypes.data, n,
+                        o.ctypes.data, lse.ctypes.data,
+                        None if probs is None else probs.ctypes.data,
+                        int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_fwd rejected its arguments (rc={rc})")
+    if rows is None:
+        o = o.reshape(B, H, Sq, D)
+        lse = lse.reshape(B, H, Sq)
+        if probs is not None:
+            probs = probs.reshape(B, H, Sq, Skv)
+    return (o, lse, probs) if want_probs else (o, lse)
+
+
+def decode(q, k_cache, v_cache, kv_len, scale, mask=None, threads=None):
+    """Oracle decode.  q [B,H,1,D]; caches [B,Hkv,cap,D]; kv_len [B] int32;
+    mask optional [B,H,1,cap] (f16/bf16).  Returns (O [B,H,1,D], LSE [B,H,1])."""
+    lib = _load()
+    B, H, one, D = q.shape
+    assert one == 1
+    _, Hkv, cap, _ = k_cache.shape
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    lens = np.ascontiguousarray(kv_len.detach().cpu().numpy().astype(np.int32))
+    mb = _bits(mask) if mask is not None else None
+    mdt = _dtype_code(mask) if mask is not None else 0
+    o = np.zeros((B * H, D), dtype=np.float64)
+    lse = np.zeros((B * H,), dtype=np.float64)
+    rc = lib.oracle_decode(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, lens.ctypes.data,
+                           None if mb is None else mb.ctypes.data, mdt, _dtype_code(q),
+                           B, H, Hkv, cap, D, float(scale), o.ctypes.data, lse.ctypes.data,
+                           int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_decode rejected its arguments (rc={rc})")
+    return o.reshape(B, H, 1, D), lse.reshape(B, H, 1)
+
+
+def mask_matrix(mask_mod, Sq, Skv, window=0, offset=0) -> np.ndarray:
+    """uint8 [Sq, Skv]: 1 where mask_mod keeps (i, j)."""
+    lib = _load()
+    out = np.zeros((Sq, Skv), dtype=np.uint8)
+    lib.oracle_mask_matrix(MASK_MODS[mask_mod], Sq, Skv, int(window), int(offset), out.ctypes.data)
+    return out
+
+
+def tile_map(mask_mod, Sq, Skv, window=0, offset=0, bm=128, bn=128) -> np.ndarray:
+    """uint8 [ceil(Sq/bm), ceil(Skv/bn)]: 0 EMPTY, 1 FULL, 2 PARTIAL."""
+    lib = _load()
+    nq, nk = -(-Sq // bm), -(-Skv // bn)
+    out = np.zeros((nq, nk), dtype=np.uint8)
+    rc = lib.oracle_tile_map(MASK_MODS[mask_mod], Sq, Skv, int(window), int(offset), bm, bn, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("bad tile size")
+    return out
+
+
+def alibi_slope(h: int, H: int) -> float:
+    return float(_load().oracle_alibi_slope(h, H))
+
+
+def fwd_flops(B, H, Sq, Skv, D) -> float:
+    """Dense forward work 4*B*H*Sq*Skv*D (two matmuls of 2*Sq*Skv*D each)."""
+    return 4.0 * B * H * Sq * Skv * D

@@ -1,0 +1,343 @@
+/*
+ * flex_oracle.c -- plain fp64 CPU oracle for flex attention (forward + decode).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or constant with the CUDA library; every rule below is
+ * written again from the method's definition.
+ *
+ * What it computes (one query row i of batch b, query head h):
+ *
+ *   hk     = h / (H / Hkv)                       GQA: contiguous head groups
+ *                                                 (torch-mlir PR 4366 "[TORCH] Added
+ *                                                 flex_attention hop function",
+ *                                                 Description: enable_gqa operand)
+ *   x_j    = scale * sum_d Q[b,h,i,d] K[b,hk,j,d]  score, scaled first
+ *   x_j   += score_mod(...)                      alibi: slope_h * (j - i),
+ *                                                 slope_h = 2^(-8 (h+1) / H)
+ *                                                 (FlyDSL PR 931 "Add flex_attention
+ *                                                 (score_mod / mask_mod) ...",
+ *                                                 Summary: score_mod runs after the
+ *                                                 scale and before the mask)
+ *   keep_j = mask_mod(b,h,i,j)                   causal: j <= i;
+ *                                                 sliding window W: j <= i && i-j < W;
+ *                                                 offset o: j <= i + o
+ *   M      = max over kept j of x_j
+ *   l      = sum over kept j of exp(x_j - M)
+ *   O[i]   = sum over kept j of exp(x_j - M) / l * V[b,hk,j,:]
+ *   LSE[i] = M + ln l        (natural log)
+ *   no kept j  ->  O[i] = 0, LSE[i] = -inf       (FlyDSL PR 931, Summary:
+ *                                                 fully-masked rows give 0/-inf)
+ *
+ * Decode (IREE issue 19015 "[ROCM] Support dynamic key-value cache sequence
+ * length", example IR: one query row against a KV cache of dynamic length and an
+ * f16 additive mask operand): x_j = scale * q.k_j + mask[b,h,j] for j < kv_len[b];
+ * keep_j = (x_j != -inf); then the same softmax as above.
+ *
+ * Tile map: for a BM x BN grid over (query, key) positions, a tile is
+ *   EMPTY(0)   if no element with i < Sq has keep && j < Skv,
+ *   FULL(1)    if every element with i < Sq has keep && j < Skv,
+ *   PARTIAL(2) otherwise.
+ *
+ * Everything is a direct loop in double precision; rows are split across
+ * POSIX threads and nothing else is reordered.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Oracle-local identifiers; the Python wrapper maps names onto these. */
+#define OR_SCORE_NONE 0
+#define OR_SCORE_ALIBI 1
+
+#define OR_MASK_NONE 0
+#define OR_MASK_CAUSAL 1
+#define OR_MASK_SLIDING 2
+#define OR_MASK_OFFSET 3
+
+#define OR_DT_BF16 0
+#define OR_DT_F16 1
+
+/* ---- exact conversion of stored 16-bit values to double ---------------- */
+
+static double bf16_bits_to_double(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+static double f16_bits_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -24);               /* subnormal: m * 2^-24 */
+  } else if (e == 31) {
+    v = (m == 0) ? INFINITY : NAN;
+  } else {
+    v = ldexp((double)(m + 1024), e - 25);   /* (1 + m/1024) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+static double elem(const uint16_t* p, int64_t idx, int dtype) {
+  return dtype == OR_DT_BF16 ? bf16_bits_to_double(p[idx]) : f16_bits_to_double(p[idx]);
+}
+
+/* ---- the hooks, written from their definitions -------------------------- */
+
+double oracle_alibi_slope(int h, int H) { return pow(2.0, -8.0 * (double)(h + 1) / (double)H); }
+
+int oracle_mask_keep(int mask_mod, int64_t i, int64_t j, int window, int offset) {
+  switch (mask_mod) {
+    case OR_MASK_NONE: return 1;
+    case OR_MASK_CAUSAL: return j <= i;
+    case OR_MASK_SLIDING: return (j <= i) && (i - j < (int64_t)window);
+    case OR_MASK_OFFSET: return j <= i + (int64_t)offset;
+    default: return 0;
+  }
+}
+
+/* ---- forward -------------------------------------------------------------- */
+
+typedef struct {
+  const uint16_t *q, *k, *v;
+  int dtype, B, H, Hkv, Sq, Skv, D;
+  double scale;
+  int score_mod, mask_mod, window, offset;
+  const int64_t* rows;   /* flattened (b*H + h)*Sq + i; NULL = all rows */
+  int64_t n_rows;
+  double* o;             /* [n_rows, D] */
+  double* lse;           /* [n_rows] */
+  double* probs;         /* optional [n_rows, Skv] normalised weights */
+  int64_t r0, r1;
+} fwd_job;
+
+static void fwd_row(const fwd_job* J, int64_t r, double* x, unsigned char* keep) {
+  int64_t flat = J->rows ? J->rows[r] : r;
+  int64_t i = flat % J->Sq;
+  int64_t bh = flat / J->Sq;
+  int h = (int)(bh % J->H);
+  int b = (int)(bh / J->H);
+  int G = J->H / J->Hkv;
+  int hk = h / G;
+  int D = J->D;
+  const int64_t qbase = flat * D;
+  const int64_t kvbase = ((int64_t)b * J->Hkv + hk) * (int64_t)J->Skv * D;
+  double slope = (J->score_mod == OR_SCORE_ALIBI) ? oracle_alibi_slope(h, J->H) : 0.0;
+
+  double M = -INFINITY;
+  int any = 0;
+  for (int64_t j = 0; j < J->Skv; ++j) {
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d)
+      dot += elem(J->q, qbase + d, J->dtype) * elem(J->k, kvbase + j * D + d, J->dtype);
+    double s = J->scale * dot;
+    if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);
+    x[j] = s;
+    keep[j] = (unsigned char)oracle_mask_keep(J->mask_mod, i, j, J->window, J->offset);
+    if (keep[j]) {
+      any = 1;
+      if (s > M) M = s;
+    }
+  }
+  double* o = J->o + r * D;
+  for (int d = 0; d < D; ++d) o[d] = 0.0;
+  if (!any) {
+    J->lse[r] = -INFINITY;
+    if (J->probs)
+      for (int64_t j = 0; j < J->Skv; ++j) J->probs[r * J->Skv + j] = 0.0;
+    return;
+  }
+  double l = 0.0;
+  for (int64_t j = 0; j < J->Skv; ++j)
+    if (keep[j]) l += exp(x[j] - M);
+  for (int64_t j = 0; j < J->Skv; ++j) {
+    double p = keep[j] ? exp(x[j] - M) / l : 0.0;
+    if (J->probs) J->probs[r * J->Skv + j] = p;
+    if (p != 0.0)
+      for (int d = 0; d < D; ++d) o[d] += p * elem(J->v, kvbase + j * D + d, J->dtype);
+  }
+  J->lse[r] = M + log(l);
+}
+
+static void* fwd_worker(void* arg) {
+  fwd_job* J = (fwd_job*)arg;
+  double* x = (double*)malloc(sizeof(double) * (size_t)J->Skv);
+  unsigned char* keep = (unsigned char*)malloc((size_t)J->Skv);
+  if (x && keep)
+    for (int64_t r = J->r0; r < J->r1; ++r) fwd_row(J, r, x, keep);
+  free(x);
+  free(keep);
+  return NULL;
+}
+
+static int run_jobs(fwd_job* base, int64_t n_rows, int nthreads, void* (*fn)(void*), size_t job_size) {
+  if (nthreads < 1) nthreads = 1;
+  if ((int64_t)nthreads > n_rows) nthreads = (int)(n_rows > 0 ? n_rows : 1);
+  char* jobs = (char*)malloc(job_size * (size_t)nthreads);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  if (!jobs || !th) { free(jobs); free(th); return -1; }
+  for (int t = 0; t < nthreads; ++t) {
+    fwd_job* J = (fwd_job*)(jobs + job_size * (size_t)t);
+    memcpy(J, base, job_size);
+    J->r0 = n_rows * t / nthreads;
+    J->r1 = n_rows * (t + 1) / nthreads;
+  }
+  int started = 0;
+  for (int t = 1; t < nthreads; ++t) {
+    if (pthread_create(&th[t], NULL, fn, jobs + job_size * (size_t)t) != 0) break;
+    started = t;
+  }
+  fn(jobs);
+  for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
+  /* any worker that failed to start: run it here */
+  for (int t = started + 1; t < nthreads; ++t) fn(jobs + job_size * (size_t)t);
+  free(jobs);
+  free(th);
+  return 0;
+}
+
+/* Forward over selected rows (rows == NULL: all B*H*Sq rows). */
+int oracle_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dtype,
+               int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
+               int score_mod, int mask_mod, int window, int offset,
+               const int64_t* rows, int64_t n_rows,
+               double* o, double* lse, double* probs, int nthreads) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv != 0 || Sq <= 0 || Skv <= 0 || D <= 0) return -1;
+  fwd_job J;
+  memset(&J, 0, sizeof J);
+  J.q = q; J.k = k; J.v = v; J.dtype = dtype;
+  J.B = B; J.H = H; J.Hkv = Hkv; J.Sq = Sq; J.Skv = Skv; J.D = D;
+  J.scale = scale; J.score_mod = score_mod; J.mask_mod = mask_mod;
+  J.window = window; J.offset = offset;
+  J.rows = rows;
+  J.n_rows = rows ? n_rows : (int64_t)B * H * Sq;
+  J.o = o; J.lse = lse; J.probs = probs;
+  return run_jobs(&J, J.n_rows, nthreads, fwd_worker, sizeof J);
+}
+
+/* ---- decode ---------------------------------------------------------------- */
+
+typedef struct {
+  const uint16_t *q, *kc, *vc, *mask;
+  const int32_t* kv_len;
+  int dtype, mask_dtype, B, H, Hkv, cap, D;
+  double scale;
+  double* o;    /* [B*H, D] */
+  double* lse;  /* [B*H]    */
+  int64_t r0, r1;
+} dec_job;
+
+static void dec_row(const dec_job* J, int64_t r, double* x) {
+  int h = (int)(r % J->H);
+  int b = (int)(r / J->H);
+  int hk = h / (J->H / J->Hkv);
+  int D = J->D;
+  int64_t L = J->kv_len[b];
+  const int64_t kvbase = ((int64_t)b * J->Hkv + hk) * (int64_t)J->cap * D;
+  double M = -INFINITY;
+  for (int64_t j = 0; j < L; ++j) {
+    double dot = 0.0;
+    for (int d = 0; d < D; ++d)
+      dot += elem(J->q, r * D + d, J->dtype) * elem(J->kc, kvbase + j * D + d, J->dtype);
+    double s = J->scale * dot;
+    if (J->mask) s += elem(J->mask, r * (int64_t)J->cap + j, J->mask_dtype);
+    x[j] = s;
+    if (s > M) M = s;
+  }
+  double* o = J->o + r * D;
+  for (int d = 0; d < D; ++d) o[d] = 0.0;
+  if (M == -INFINITY) {   /* kv_len == 0 or every position masked */
+    J->lse[r] = -INFINITY;
+    return;
+  }
+  double l = 0.0;
+  for (int64_t j = 0; j < L; ++j)
+    if (x[j] != -INFINITY) l += exp(x[j] - M);
+  for (int64_t j = 0; j < L; ++j) {
+    if (x[j] == -INFINITY) continue;
+    double p = exp(x[j] - M) / l;
+    for (int d = 0; d < D; ++d) o[d] += p * elem(J->vc, kvbase + j * D + d, J->dtype);
+  }
+  J->lse[r] = M + log(l);
+}
+
+static void* dec_worker(void* arg) {
+  dec_job* J = (dec_job*)arg;
+  double* x = (double*)malloc(sizeof(double) * (size_t)(J->cap > 0 ? J->cap : 1));
+  if (x)
+    for (int64_t r = J->r0; r < J->r1; ++r) dec_row(J, r, x);
+  free(x);
+  return NULL;
+}
+
+int oracle_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                  const int32_t* kv_len, const uint16_t* mask, int mask_dtype, int dtype,
+                  int B, int H, int Hkv, int cap, int D, double scale,
+                  double* o, double* lse, int nthreads) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv != 0 || cap <= 0 || D <= 0) return -1;
+  for (int b = 0; b < B; ++b)
+    if (kv_len[b] < 0 || kv_len[b] > cap) return -2;
+  dec_job J;
+  memset(&J, 0, sizeof J);
+  J.q = q; J.kc = kc; J.vc = vc; J.mask = mask; J.kv_len = kv_len;
+  J.dtype = dtype; J.mask_dtype = mask_dtype;
+  J.B = B; J.H = H; J.Hkv = Hkv; J.cap = cap; J.D = D; J.scale = scale;
+  J.o = o; J.lse = lse;
+  int64_t n = (int64_t)B * H;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > n) nthreads = (int)(n > 0 ? n : 1);
+  dec_job* jobs = (dec_job*)malloc(sizeof(dec_job) * (size_t)nthreads);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  if (!jobs || !th) { free(jobs); free(th); return -3; }
+  for (int t = 0; t < nthreads; ++t) {
+    jobs[t] = J;
+    jobs[t].r0 = n * t / nthreads;
+    jobs[t].r1 = n * (t + 1) / nthreads;
+  }
+  int started = 0;
+  for (int t = 1; t < nthreads; ++t) {
+    if (pthread_create(&th[t], NULL, dec_worker, &jobs[t]) != 0) break;
+    started = t;
+  }
+  dec_worker(&jobs[0]);
+  for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
+  for (int t = started + 1; t < nthreads; ++t) dec_worker(&jobs[t]);
+  free(jobs);
+  free(th);
+  return 0;
+}
+
+/* ---- element mask and tile map (brute force) ------------------------------- */
+
+/* keep[i*Skv + j] = mask_mod(i, j) for every i < Sq, j < Skv. */
+int oracle_mask_matrix(int mask_mod, int Sq, int Skv, int window, int offset, uint8_t* keep) {
+  for (int64_t i = 0; i < Sq; ++i)
+    for (int64_t j = 0; j < Skv; ++j)
+      keep[i * Skv + j] = (uint8_t)oracle_mask_keep(mask_mod, i, j, window, offset);
+  return 0;
+}
+
+/* map[t*nkv + u] in {0 EMPTY, 1 FULL, 2 PARTIAL}; nq = ceil(Sq/BM), nkv = ceil(Skv/BN). */
+int oracle_tile_map(int mask_mod, int Sq, int Skv, int window, int offset, int BM, int BN, uint8_t* map) {
+  if (BM <= 0 || BN <= 0) return -1;
+  int nq = (Sq + BM - 1) / BM, nkv = (Skv + BN - 1) / BN;
+  for (int t = 0; t < nq; ++t) {
+    for (int u = 0; u < nkv; ++u) {
+      int64_t kept = 0, total = 0;
+      for (int64_t i = (int64_t)t * BM; i < (int64_t)(t + 1) * BM && i < Sq; ++i) {
+        for (int64_t j = (int64_t)u * BN; j < (int64_t)(u + 1) * BN; ++j) {
+          ++total;
+          if (j < Skv && oracle_mask_keep(mask_mod, i, j, window, offset)) ++kept;
+        }
+      }
+      map[(int64_t)t * nkv + u] = (uint8_t)(kept == 0 ? 0 : (kept == total ? 1 : 2));
+    }
+  }
+  return 0;
+}
