@@ -1,0 +1,174 @@
+"""Python binding for the sm_100a flex-attention library (libflexattn.so).
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels
+behind the C ABI of ``include/flex_attn.h``.  Tensors are torch CUDA tensors; the
+binding passes their device pointers and the current CUDA stream.  There is no
+fallback: if the shared library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libflexattn.so")
+
+# enum values of include/flex_attn.h
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "misaligned", 4: "workspace",
+          5: "CUDA error", 6: "device timeout"}
+DTYPES = {torch.bfloat16: 0, torch.float16: 1}
+SCORE_MODS = {"none": 0, "alibi": 1}
+MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset": 3, "causal_fast": 4}
+FLAG_TILE_MAP = 1
+
+# The symbols include/flex_attn.h declares.
+EXPORTED = ["flex_attn_fwd", "flex_attn_decode_workspace_size", "flex_attn_decode",
+            "flex_attn_mask_eval", "flex_attn_tile_sizes", "flex_attn_device_status",
+            "flex_status_string"]
+
+
+class FlexAttnError(RuntimeError):
+    pass
+
+
+class ModParams(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_int32), ("offset", ctypes.c_int32),
+                ("flags", ctypes.c_uint32), ("tile_map_out", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libflexattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FlexAttnError(f"{path} is missing: run `python -m attention_flex_attn_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.flex_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams), I, P]
+    lib.flex_attn_fwd.restype = I
+    lib.flex_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
+    lib.flex_attn_decode_workspace_size.restype = SZ
+    lib.flex_attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, P]
+    lib.flex_attn_decode.restype = I
+    lib.flex_attn_mask_eval.argtypes = [I, ctypes.POINTER(ModParams), I, I, P, P]
+    lib.flex_attn_mask_eval.restype = I
+    lib.flex_attn_tile_sizes.argtypes = [I, ctypes.POINTER(I), ctypes.POINTER(I)]
+    lib.flex_attn_tile_sizes.restype = None
+    lib.flex_attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I]
+    lib.flex_attn_device_status.restype = I
+    lib.flex_status_string.argtypes = [I]
+    lib.flex_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise FlexAttnError(f"{what}: {STATUS.get(rc, rc)} (status {rc})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _cuda_tensor(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise FlexAttnError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise FlexAttnError(f"{name} must be contiguous")
+
+
+def tile_sizes(D: int = 128):
+    lib = load_library()
+    bm, bn = ctypes.c_int(), ctypes.c_int()
+    lib.flex_attn_tile_sizes(D, ctypes.byref(bm), ctypes.byref(bn))
+    return bm.value, bn.value
+
+
+def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
+        return_lse=True, out=None, lse_out=None, tile_map=None):
+    """Flex-attention forward.  q [B,H,Sq,D], k/v [B,Hkv,Skv,D] (bf16 or f16, CUDA).
+
+    Returns (O, LSE) (LSE is None when return_lse is False).  ``tile_map``: optional
+    uint8 CUDA tensor of ceil(Sq/BM)*ceil(Skv/BN) bytes that receives the tile classes
+    of batch 0 / head 0.
+    """
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda_tensor(t, n)
+    B, H, Sq, D = q.shape
+    Bk, Hkv, Skv, Dk = k.shape
+    if Bk != B or Dk != D or tuple(v.shape) != tuple(k.shape) or not (q.dtype == k.dtype == v.dtype):
+        raise FlexAttnError("shape/dtype mismatch between q, k, v")
+    if q.dtype not in DTYPES:
+        raise FlexAttnError(f"unsupported dtype {q.dtype}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = out if out is not None else torch.empty_like(q)
+    lse = None
+    if return_lse:
+        lse = lse_out if lse_out is not None else torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    mp = ModParams(int(window), int(offset), FLAG_TILE_MAP if tile_map is not None else 0,
+                   tile_map.data_ptr() if tile_map is not None else None)
+    rc = lib.flex_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
+                           float(scale), SCORE_MODS[score_mod], MASK_MODS[mask_mod], ctypes.byref(mp),
+                           DTYPES[q.dtype], _stream(q.device))
+    _check(rc, "flex_attn_fwd")
+    return o, lse
+
+
+def decode_workspace_size(B, H, Hkv, cap, D) -> int:
+    return int(load_library().flex_attn_decode_workspace_size(B, H, Hkv, cap, D))
+
+
+def decode(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None, workspace=None):
+    """Decode attention.  q [B,H,1,D]; caches [B,Hkv,cap,D]; kv_len [B] int32 (CUDA);
+    mask optional [B,H,1,cap] of q's dtype.  Returns (O [B,H,1,D], LSE [B,H,1])."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (kv_len, "kv_len")):
+        _cuda_tensor(t, n)
+    if mask is not None:
+        _cuda_tensor(mask, "mask")
+    B, H, one, D = q.shape
+    _, Hkv, cap, _ = k_cache.shape
+    if one != 1 or kv_len.dtype != torch.int32:
+        raise FlexAttnError("decode takes q [B,H,1,D] and int32 kv_len")
+    o = out if out is not None else torch.empty_like(q)
+    lse = lse_out if lse_out is not None else torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, H, Hkv, cap, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = lib.flex_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_len), _ptr(mask), _ptr(o), _ptr(lse),
+                              B, H, Hkv, cap, D, float(scale), DTYPES[q.dtype], _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(rc, "flex_attn_decode")
+    return o, lse
+
+
+def mask_eval(mask_mod, Sq, Skv, window=0, offset=0, device="cuda"):
+    """uint8 [Sq, Skv] CUDA tensor of the forward kernel's keep decisions."""
+    lib = load_library()
+    keep = torch.empty((Sq, Skv), dtype=torch.uint8, device=device)
+    mp = ModParams(int(window), int(offset), 0, None)
+    rc = lib.flex_attn_mask_eval(MASK_MODS[mask_mod], ctypes.byref(mp), Sq, Skv, _ptr(keep), _stream(keep.device))
+    _check(rc, "flex_attn_mask_eval")
+    return keep
+
+
+def device_status(reset: bool = True) -> int:
+    """Reads (and clears) the device status word; synchronises the device."""
+    lib = load_library()
+    v = ctypes.c_uint32(0)
+    _check(lib.flex_attn_device_status(ctypes.byref(v), 1 if reset else 0), "flex_attn_device_status")
+    return int(v.value)

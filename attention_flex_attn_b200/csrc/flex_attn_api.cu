@@ -1,0 +1,337 @@
+// flex_attn_api.cu -- the C ABI declared in include/flex_attn.h: host-side argument
+// checks, TMA tensor-map encoding, compile-time dispatch over (head dim, dtype,
+// score_mod, mask_mod), and kernel launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "flex_attn.h"
+#include "flex_decode.cuh"
+#include "flex_fwd_sm100.cuh"
+#include "mask_rules.cuh"
+
+namespace flexattn {
+
+// Device status word (bits documented with flex_attn_device_status).
+__device__ unsigned int g_status;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [rows3 x rows x D] 16-bit tensor, box = 64 elements x 128 rows x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, flex_dtype_t dt, int D, int rows, int64_t outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const CUtensorMapDataType t = dt == FLEX_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(D) * 2 * rows};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Per-device "attribute already set" bits, one set per kernel instantiation (the tag
+// parameters make every forward instantiation own its static).
+template <int D, typename T, int SCORE, int MASK, typename K>
+bool ensure_smem_attr(K kernel, int bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
+unsigned* status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+  return static_cast<unsigned*>(p);
+}
+
+// ---------------------------------------------------------------- forward dispatch
+
+template <int D, typename T, int SCORE, int MASK>
+flex_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
+                         int n_units, cudaStream_t stream) {
+  auto kern = flex_fwd_kernel<D, T, SCORE, MASK>;
+  if (!ensure_smem_attr<D, T, SCORE, MASK>(kern, FwdSmem<D>::kAlloc)) return FLEX_ERR_CUDA;
+  kern<<<n_units, kFwdThreads, FwdSmem<D>::kAlloc, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
+}
+
+template <int D, typename T, int SCORE>
+flex_status_t dispatch_mask(int mask, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const FwdParams& p, int n_units, cudaStream_t s) {
+  switch (mask) {
+    case kMaskNone: return launch_fwd<D, T, SCORE, kMaskNone>(mq, mk, mv, p, n_units, s);
+    case kMaskCausal: return launch_fwd<D, T, SCORE, kMaskCausal>(mq, mk, mv, p, n_units, s);
+    case kMaskSliding: return launch_fwd<D, T, SCORE, kMaskSliding>(mq, mk, mv, p, n_units, s);
+    case kMaskOffset: return launch_fwd<D, T, SCORE, kMaskOffset>(mq, mk, mv, p, n_units, s);
+  }
+  return FLEX_ERR_INVALID_ARG;
+}
+
+template <int D, typename T>
+flex_status_t dispatch_score(int score, int mask, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, const FwdParams& p, int n_units, cudaStream_t s) {
+  if (score == kScoreNone) return dispatch_mask<D, T, kScoreNone>(mask, mq, mk, mv, p, n_units, s);
+  return dispatch_mask<D, T, kScoreAlibi>(mask, mq, mk, mv, p, n_units, s);
+}
+
+// ---------------------------------------------------------------- mask evaluation (debug)
+
+// Composes exactly the decisions the forward kernel takes for element (i, j): is the key
+// tile of j visited by the query tile of i, and if so FULL or inside the row interval.
+template <int MASK>
+__global__ void mask_eval_kernel(MaskArgs m, int Sq, int Skv, uint8_t* keep) {
+  const int64_t total = static_cast<int64_t>(Sq) * Skv;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(idx / Skv), j = static_cast<int>(idx % Skv);
+    const int q0 = (i / kBM) * kBM, q1 = min(q0 + kBM, Sq);
+    int t_lo, t_hi;
+    tile_range<MASK>(q0, q1, kBN, m, t_lo, t_hi);
+    const int u = j / kBN, k0 = u * kBN;
+    uint8_t kv = 0;
+    if (u >= t_lo && u < t_hi) {
+      if (tile_class<MASK>(q0, q1, k0, kBN, m) == kTileFull) {
+        kv = 1;
+      } else {
+        int lo, hi;
+        col_interval<MASK>(i, k0, m, lo, hi);
+        kv = (j - k0 >= lo && j - k0 <= hi) ? 1 : 0;
+      }
+    }
+    keep[idx] = kv;
+  }
+}
+
+// ---------------------------------------------------------------- decode dispatch
+
+template <int D, typename T, int GT>
+flex_status_t launch_decode(const DecodeParams& p, cudaStream_t s) {
+  dim3 grid(p.n_splits, p.B * p.Hkv * (p.G / GT));
+  decode_split_kernel<D, T, GT><<<grid, kDecThreads, 0, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FLEX_ERR_CUDA;
+  const int rows = p.B * p.H;
+  decode_combine_kernel<D, T><<<(rows + kDecWarps - 1) / kDecWarps, kDecThreads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
+}
+
+template <int D, typename T>
+flex_status_t decode_by_group(const DecodeParams& p, cudaStream_t s) {
+  if (p.G % 8 == 0) return launch_decode<D, T, 8>(p, s);
+  if (p.G % 4 == 0) return launch_decode<D, T, 4>(p, s);
+  if (p.G % 2 == 0) return launch_decode<D, T, 2>(p, s);
+  return launch_decode<D, T, 1>(p, s);
+}
+
+int decode_splits(int cap) { return (cap + kChunk - 1) / kChunk; }
+
+}  // namespace
+}  // namespace flexattn
+
+using namespace flexattn;
+
+extern "C" {
+
+flex_status_t flex_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                            int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
+                            const flex_mod_params_t* mod_params, flex_dtype_t dtype, flex_stream_t stream) {
+  if (!q || !k || !v || !o) return FLEX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
+  if (dtype != FLEX_DTYPE_BF16 && dtype != FLEX_DTYPE_F16) return FLEX_ERR_UNSUPPORTED;
+  if (score_mod_id != FLEX_SCORE_NONE && score_mod_id != FLEX_SCORE_ALIBI) return FLEX_ERR_INVALID_ARG;
+  int mask = -1;
+  switch (mask_mod_id) {
+    case FLEX_MASK_NONE: mask = kMaskNone; break;
+    case FLEX_MASK_CAUSAL:
+    case FLEX_MASK_CAUSAL_FAST: mask = kMaskCausal; break;
+    case FLEX_MASK_SLIDING_WINDOW: mask = kMaskSliding; break;
+    case FLEX_MASK_KV_LE_Q_PLUS_OFFSET: mask = kMaskOffset; break;
+    default: return FLEX_ERR_INVALID_ARG;
+  }
+  const flex_mod_params_t zero{};
+  const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
+  if (mask == kMaskSliding && mp.window < 1) return FLEX_ERR_INVALID_ARG;
+  const bool want_map = (mp.flags & FLEX_FLAG_TILE_MAP) != 0;
+  if (want_map && !mp.tile_map_out) return FLEX_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return FLEX_ERR_MISALIGNED;
+  const int64_t bh = static_cast<int64_t>(B) * H;
+  const int n_qtiles = (Sq + kBM - 1) / kBM;
+  const int n_pairs = (n_qtiles + 1) / 2;
+  const int64_t n_units = bh * n_pairs;
+  if (n_units > 0x7fffffff || static_cast<int64_t>(B) * Hkv > 0x7fffffff) return FLEX_ERR_UNSUPPORTED;
+
+  unsigned* st = status_ptr();
+  if (!st) return FLEX_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, dtype, D, Sq, bh) || !make_map(&mk, k, dtype, D, Skv, static_cast<int64_t>(B) * Hkv) ||
+      !make_map(&mv, v, dtype, D, Skv, static_cast<int64_t>(B) * Hkv))
+    return FLEX_ERR_CUDA;
+
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.tile_map = want_map ? mp.tile_map_out : nullptr;
+  p.status = st;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.n_qtiles = n_qtiles;
+  p.n_ktiles = (Skv + kBN - 1) / kBN;
+  p.n_pairs = n_pairs;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = MaskArgs{Skv, mp.window, mp.offset};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int units = static_cast<int>(n_units);
+  if (D == 128) {
+    return dtype == FLEX_DTYPE_BF16 ? dispatch_score<128, __nv_bfloat16>(score_mod_id, mask, mq, mk, mv, p, units, s)
+                                    : dispatch_score<128, __half>(score_mod_id, mask, mq, mk, mv, p, units, s);
+  }
+  return dtype == FLEX_DTYPE_BF16 ? dispatch_score<64, __nv_bfloat16>(score_mod_id, mask, mq, mk, mv, p, units, s)
+                                  : dispatch_score<64, __half>(score_mod_id, mask, mq, mk, mv, p, units, s);
+}
+
+size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D) {
+  if (B < 1 || H < 1 || Hkv < 1 || cap < 1 || D < 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * H;
+  const size_t ns = static_cast<size_t>(decode_splits(cap));
+  const size_t o_bytes = rows * ns * D * sizeof(float);
+  const size_t o_round = (o_bytes + 255) & ~static_cast<size_t>(255);
+  return o_round + rows * ns * sizeof(float);
+}
+
+flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_len,
+                               const void* additive_mask, void* o, float* lse, int B, int H, int Hkv, int cap, int D,
+                               float scale, flex_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                               flex_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !kv_len || !o) return FLEX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || cap < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
+  if (dtype != FLEX_DTYPE_BF16 && dtype != FLEX_DTYPE_F16) return FLEX_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * Hkv * (H / Hkv) > 65535LL * 8) return FLEX_ERR_UNSUPPORTED;
+  const size_t need = flex_attn_decode_workspace_size(B, H, Hkv, cap, D);
+  if (!workspace || workspace_bytes < need) return FLEX_ERR_WORKSPACE;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(workspace) ||
+      (lse && !aligned16(lse)) || (additive_mask && !aligned16(additive_mask)) || !aligned16(kv_len))
+    return FLEX_ERR_MISALIGNED;
+  unsigned* st = status_ptr();
+  if (!st) return FLEX_ERR_CUDA;
+  DecodeParams p{};
+  p.q = q;
+  p.k = k_cache;
+  p.v = v_cache;
+  p.kv_len = kv_len;
+  p.mask = additive_mask;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.cap = cap;
+  p.n_splits = decode_splits(cap);
+  const size_t rows = static_cast<size_t>(B) * H;
+  const size_t o_bytes = rows * p.n_splits * D * sizeof(float);
+  p.part_o = static_cast<float*>(workspace);
+  p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((o_bytes + 255) & ~static_cast<size_t>(255)));
+  p.status = st;
+  p.scale_log2 = scale * kLog2e;
+  const int grid_y = B * Hkv * (p.G / (p.G % 8 == 0 ? 8 : p.G % 4 == 0 ? 4 : p.G % 2 == 0 ? 2 : 1));
+  if (grid_y > 65535) return FLEX_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (D == 128)
+    return dtype == FLEX_DTYPE_BF16 ? decode_by_group<128, __nv_bfloat16>(p, s) : decode_by_group<128, __half>(p, s);
+  return dtype == FLEX_DTYPE_BF16 ? decode_by_group<64, __nv_bfloat16>(p, s) : decode_by_group<64, __half>(p, s);
+}
+
+flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_params, int Sq, int Skv,
+                                  uint8_t* keep, flex_stream_t stream) {
+  if (!keep || Sq < 1 || Skv < 1) return FLEX_ERR_INVALID_ARG;
+  const flex_mod_params_t zero{};
+  const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
+  MaskArgs m{Skv, mp.window, mp.offset};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t total = static_cast<int64_t>(Sq) * Skv;
+  const int grid = static_cast<int>(total / 256 + 1 > 4096 ? 4096 : total / 256 + 1);
+  switch (mask_mod_id) {
+    case FLEX_MASK_NONE: mask_eval_kernel<kMaskNone><<<grid, 256, 0, s>>>(m, Sq, Skv, keep); break;
+    case FLEX_MASK_CAUSAL:
+    case FLEX_MASK_CAUSAL_FAST: mask_eval_kernel<kMaskCausal><<<grid, 256, 0, s>>>(m, Sq, Skv, keep); break;
+    case FLEX_MASK_SLIDING_WINDOW:
+      if (mp.window < 1) return FLEX_ERR_INVALID_ARG;
+      mask_eval_kernel<kMaskSliding><<<grid, 256, 0, s>>>(m, Sq, Skv, keep);
+      break;
+    case FLEX_MASK_KV_LE_Q_PLUS_OFFSET: mask_eval_kernel<kMaskOffset><<<grid, 256, 0, s>>>(m, Sq, Skv, keep); break;
+    default: return FLEX_ERR_INVALID_ARG;
+  }
+  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
+}
+
+void flex_attn_tile_sizes(int D, int* bm, int* bn) {
+  (void)D;
+  if (bm) *bm = kBM;
+  if (bn) *bn = kBN;
+}
+
+flex_status_t flex_attn_device_status(uint32_t* status_out, int reset) {
+  if (!status_out) return FLEX_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FLEX_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return FLEX_ERR_CUDA;
+  *status_out = v;
+  if (reset) {
+    const unsigned z = 0;
+    if (cudaMemcpyToSymbol(g_status, &z, sizeof z) != cudaSuccess) return FLEX_ERR_CUDA;
+  }
+  return FLEX_OK;
+}
+
+const char* flex_status_string(flex_status_t s) {
+  switch (s) {
+    case FLEX_OK: return "ok";
+    case FLEX_ERR_INVALID_ARG: return "invalid argument";
+    case FLEX_ERR_UNSUPPORTED: return "unsupported head dim, dtype or size";
+    case FLEX_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case FLEX_ERR_WORKSPACE: return "decode workspace missing or too small";
+    case FLEX_ERR_CUDA: return "CUDA call failed";
+    case FLEX_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

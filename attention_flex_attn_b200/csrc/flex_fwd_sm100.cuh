@@ -1,0 +1,454 @@
+// flex_fwd_sm100.cuh -- flex-attention forward kernel for sm_100a.
+//
+// Computes, per query row i of (batch b, head h),
+//   O = softmax(mask_mod(score_mod(scale * Q K^T))) V  and  LSE = log-sum-exp (natural log),
+// following FlyDSL PR 931 "Add flex_attention (score_mod / mask_mod) on the generic
+// flash-attention kernel", Summary (score_mod sees the scaled score and runs before the
+// mask; fully masked rows give O = 0 / LSE = -inf) with the hooks chosen at compile time,
+// so the no-mod instantiation carries no hook code at all.
+//
+// One CTA owns two 128-row query tiles of one (b, h) and walks the key/value tiles both
+// of them need:
+//   warp 9      TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory slots
+//   warp 8      MMA issuer (one thread): S_k = Q_k K_j^T and O_k += P_k V_j with tcgen05,
+//               accumulators in tensor memory
+//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: each thread owns one
+//               query row (= one TMEM lane), reads its S row from TMEM, applies score_mod,
+//               mask (PARTIAL tiles only) and the online base-2 softmax, writes P (16-bit)
+//               back into TMEM over S, rescales its O row when the running max grows by
+//               more than 2^8, and finally normalises O and writes O and LSE.
+// The MMA order S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ... lets one softmax
+// warpgroup work while the tensor core runs the other tile's matmuls.
+//
+// Tensor memory (512 columns x 128 lanes): S0 [0,128) S1 [128,256) O0 [256,256+D)
+// O1 [384,384+D); P_k aliases the first 64 columns of S_k (two 16-bit values per column).
+// Shared memory: Q0, Q1 and NS key/value slots, each a 128-row tile stored as D/64 chunks
+// of [128 rows x 128 bytes] in the 128-byte swizzled layout TMA writes and the tensor
+// core reads.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "mask_rules.cuh"
+#include "ptx_sm100.cuh"
+
+namespace flexattn {
+
+constexpr int kBM = 128;        // query rows per tile (tcgen05 M)
+constexpr int kBN = 128;        // keys per tile
+constexpr int kFwdThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+constexpr unsigned kStatusFwdTimeout = 2u;
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  uint8_t* tile_map;   // debug tile map or nullptr
+  unsigned* status;    // device status word
+  int H, Hkv, G, Sq, Skv;
+  int n_qtiles, n_ktiles, n_pairs;
+  float scale_log2;    // scale * log2(e)
+  MaskArgs mask;
+};
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kTileBytes = kBM * D * 2;          // one 128-row tile
+  static constexpr int kChunkBytes = kBM * 128;           // one 64-element-wide chunk
+  static constexpr int kSlots = D == 128 ? 4 : 8;         // key/value ring depth
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
+  // barriers: q, full[NS], empty[NS], s_full[2], p_full[2], o_full[2], drain; then tmem addr
+  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kTmemPtrOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
+};
+
+template <typename T>
+struct DtypeBits;
+template <>
+struct DtypeBits<__nv_bfloat16> {
+  static constexpr uint32_t kFmt = 1;
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+template <>
+struct DtypeBits<__half> {
+  static constexpr uint32_t kFmt = 0;
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+
+template <int D, typename T, int SCORE, int MASK>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    flex_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdSmem<D>;
+  constexpr int NS = L::kSlots;
+  constexpr int kChunks = D / 64;
+  constexpr uint32_t kTmemCols = 512;
+  constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);
+  constexpr uint32_t kIdescPV = idesc_f16(DtypeBits<T>::kFmt, kBM, D, 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw_addr);
+
+  const uint32_t bar_q = sbase + L::kBarOff;
+  auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
+  auto bar_s = [&](int k) { return sbase + L::kBarOff + 8u * (1 + 2 * NS + k); };
+  auto bar_p = [&](int k) { return sbase + L::kBarOff + 8u * (3 + 2 * NS + k); };
+  auto bar_o = [&](int k) { return sbase + L::kBarOff + 8u * (5 + 2 * NS + k); };
+  const uint32_t bar_drain = sbase + L::kBarOff + 8u * (7 + 2 * NS);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---------------------------------------------------------------- work unit
+  const int bh = blockIdx.x / p.n_pairs;
+  const int pair = p.n_pairs - 1 - (blockIdx.x % p.n_pairs);  // heavier (later) rows first
+  const int h = bh % p.H;
+  const int b = bh / p.H;
+  const int bkv = b * p.Hkv + h / p.G;
+
+  int q0[2], q1[2], lo[2], hi[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int qt = 2 * pair + k;
+    q0[k] = qt * kBM;
+    q1[k] = min(q0[k] + kBM, p.Sq);
+    lo[k] = hi[k] = 0;
+    if (qt < p.n_qtiles) tile_range<MASK>(q0[k], q1[k], kBN, p.mask, lo[k], hi[k]);
+  }
+  const bool act0 = lo[0] < hi[0], act1 = lo[1] < hi[1];
+  const int ulo = act0 ? (act1 ? min(lo[0], lo[1]) : lo[0]) : lo[1];
+  const int uhi = act0 ? (act1 ? max(hi[0], hi[1]) : hi[0]) : hi[1];
+  const bool any_work = act0 || act1;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(bar_s(k), 1);
+      mbar_init(bar_p(k), kBM);
+      mbar_init(bar_o(k), 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+
+  auto tile_smem = [&](int off_tiles) { return sbase + static_cast<uint32_t>(off_tiles); };
+  const uint32_t q_smem0 = tile_smem(L::kQOff);
+  auto q_smem = [&](int k) { return q_smem0 + static_cast<uint32_t>(k * L::kTileBytes); };
+  auto kv_smem = [&](int s) { return sbase + static_cast<uint32_t>(L::kKVOff + s * L::kTileBytes); };
+
+  if (warp == 9) {
+    // ============================================================ TMA producer
+    if (lane == 0 && any_work) {
+      const int bytes_q = (act0 ? 1 : 0) * L::kTileBytes + (act1 ? 1 : 0) * L::kTileBytes;
+      mbar_arrive_expect_tx(bar_q, bytes_q);
+      for (int k = 0; k < 2; ++k) {
+        if (!(k == 0 ? act0 : act1)) continue;
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(q_smem(k) + c * L::kChunkBytes, &tmQ, bar_q, c * 64, q0[k], bh);
+      }
+      int r = 0;
+      bool ok = true;
+      for (int j = ulo; j < uhi && ok; ++j) {
+        for (int which = 0; which < 2 && ok; ++which, ++r) {
+          const int s = r % NS;
+          const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
+          if (!mbar_wait(bar_empty(s), ph ^ 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs) ||
+              *abort_flag) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
+          const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(kv_smem(s) + c * L::kChunkBytes, map, bar_full(s), c * 64, j * kBN, bkv);
+        }
+      }
+      // Every load issued must land before the CTA can exit.
+      const int issued = r;
+      for (int e = issued - NS < 0 ? 0 : issued - NS; e < issued; ++e)
+        mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusFwdTimeout,
+                  kWaitTimeoutNs);
+      mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+    }
+  } else if (warp == 8) {
+    // ============================================================ MMA issuer
+    if (lane == 0 && any_work) {
+      bool ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+      tc_fence_after();
+      int np[2] = {0, 0};
+      auto issue_s = [&](int k, int slot) {
+        const uint32_t d = tmem + 128u * k;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * L::kChunkBytes + (kk % 4) * 32;
+          const uint64_t ad = smem_desc(q_smem(k) + off, 16, 1024, kSwizzle128B);
+          const uint64_t bd = smem_desc(kv_smem(slot) + off, 16, 1024, kSwizzle128B);
+          mma_ss(d, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int k, int slot, bool acc) {
+        const uint32_t d = tmem + 256u + 128u * k;
+        const uint32_t a = tmem + 128u * k;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd = smem_desc(kv_smem(slot) + kk * 2048, L::kChunkBytes, 1024, kSwizzle128B);
+          mma_ts(d, a + 8u * kk, bd, kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int j = ulo; j < uhi && ok; ++j) {
+        const int rK = 2 * (j - ulo), rV = rK + 1;
+        const int sK = rK % NS, sV = rV % NS;
+        if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+                       kStatusFwdTimeout, kWaitTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int k = 0; k < 2; ++k) {
+          if (j == lo[k] && lo[k] < hi[k]) {
+            issue_s(k, sK);
+            mma_commit(bar_s(k));
+          }
+        }
+        mma_commit(bar_empty(sK));
+        if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
+                       kStatusFwdTimeout, kWaitTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        for (int k = 0; k < 2 && ok; ++k) {
+          if (j < lo[k] || j >= hi[k]) continue;
+          if (!mbar_wait(bar_p(k), static_cast<uint32_t>(np[k]) & 1u, p.status, kStatusFwdTimeout,
+                         kWaitTimeoutNs) ||
+              *abort_flag) {
+            ok = false;
+            break;
+          }
+          ++np[k];
+          tc_fence_after();
+          issue_pv(k, sV, j > lo[k]);
+          if (j + 1 < hi[k]) {
+            const int rK2 = rK + 2;
+            if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status,
+                           kStatusFwdTimeout, kWaitTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(k, rK2 % NS);
+            mma_commit(bar_s(k));
+          } else {
+            mma_commit(bar_o(k));
+          }
+        }
+        mma_commit(bar_empty(sV));
+      }
+      if (!ok) *abort_flag = 1;
+      // Drain: all MMAs this thread issued have completed before TMEM is released.
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+    }
+  } else {
+    // ============================================================ softmax warpgroups
+    const int k = warp >> 2;          // query tile of this warpgroup
+    const int wq = warp & 3;          // TMEM lane quarter
+    const int row = wq * 32 + lane;   // row inside the tile == TMEM lane
+    const int qi = q0[k] + row;       // absolute query index
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 128u * k;
+    const uint32_t tO = tmem + lane_off + 256u + 128u * k;
+    const bool tile_valid = (2 * pair + k) < p.n_qtiles;
+    const bool write_map = p.tile_map != nullptr && bh == 0 && tile_valid && threadIdx.x % 128 == 0;
+    const int qt = 2 * pair + k;
+
+    if (write_map) {
+      for (int u = 0; u < p.n_ktiles; ++u)
+        if (u < lo[k] || u >= hi[k]) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + u] = kTileEmpty;
+    }
+
+    float m_used = -INFINITY;  // running max in log2 units (the reference of P and O)
+    float l_sum = 0.f;
+    const float sc = SCORE == kScoreAlibi ? 1.0f : p.scale_log2;
+    float slope2 = 0.f;
+    if (SCORE == kScoreAlibi) slope2 = exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H)) * kLog2e;
+
+    bool ok = true;
+    int n = 0;
+    for (int j = lo[k]; j < hi[k]; ++j, ++n) {
+      // Warp-uniform decision: the TMEM loads below are warp-collective.
+      const bool got = mbar_wait(bar_s(k), static_cast<uint32_t>(n) & 1u, p.status, kStatusFwdTimeout,
+                                 kWaitTimeoutNs) &&
+                       !*abort_flag;
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int k0 = j * kBN;
+      const int cls = tile_class<MASK>(q0[k], q1[k], k0, kBN, p.mask);
+      if (write_map) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] = static_cast<uint8_t>(cls);
+
+      float s[kBN];
+      {
+        uint32_t r[64];
+        tmem_ld64(tS, r);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
+        tmem_ld64(tS + 64u, r);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[64 + c] = __uint_as_float(r[c]);
+      }
+      if (SCORE == kScoreAlibi) {
+        const float base = slope2 * static_cast<float>(k0 - qi);
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) s[c] = fmaf(s[c], p.scale_log2, fmaf(slope2, static_cast<float>(c), base));
+      }
+      if (cls == kTilePartial) {
+        int c_lo, c_hi;
+        col_interval<MASK>(qi, k0, p.mask, c_lo, c_hi);
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if (c < c_lo || c > c_hi) s[c] = -INFINITY;
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < kBN; c += 4) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]);
+        mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
+      const bool need = mx > m_used + kRescaleThreshold;  // false while both are -inf
+      if (__any_sync(0xffffffffu, need)) {
+        float alpha = 1.0f;
+        if (need) {
+          alpha = ex2_approx(m_used - mx);  // 0 when m_used == -inf
+          m_used = mx;
+          l_sum *= alpha;
+        }
+        if (n > 0) {
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(tO + c, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tO + c, r);
+          }
+        }
+      }
+      const float m_safe = m_used == -INFINITY ? 0.f : m_used;
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float e0 = ex2_approx(fmaf(s[64 * half + c], sc, -m_safe));
+          const float e1 = ex2_approx(fmaf(s[64 * half + c + 1], sc, -m_safe));
+          ls0 += e0;
+          ls1 += e1;
+          pk[c / 2] = DtypeBits<T>::pack(e0, e1);
+        }
+        tmem_st32(tS + 32u * half, pk);
+      }
+      l_sum += ls0 + ls1;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p(k));
+    }
+    if (!ok) *abort_flag = 1;
+
+    // ---------------------------------------------------------------- epilogue
+    if (tile_valid) {
+      bool ran = ok && lo[k] < hi[k];
+      if (ran) {
+        const bool got = mbar_wait(bar_o(k), 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          *abort_flag = 1;
+          ran = false;
+        }
+        tc_fence_after();
+      }
+      const bool row_ok = qi < p.Sq;
+      const bool has_mass = ran && l_sum > 0.f;
+      const float inv = has_mass ? 1.0f / l_sum : 0.f;
+      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<int64_t>(bh) * p.Sq + qi) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        if (ran) {
+          tmem_ld32(tO + c, r);
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a = has_mass ? __uint_as_float(r[2 * e]) * inv : 0.f;
+          const float bb = has_mass ? __uint_as_float(r[2 * e + 1]) * inv : 0.f;
+          w[e] = DtypeBits<T>::pack(a, bb);
+        }
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+      if (row_ok && p.lse != nullptr) {
+        p.lse[static_cast<int64_t>(bh) * p.Sq + qi] =
+            has_mass ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace flexattn

@@ -1,0 +1,100 @@
+// mask_rules.cuh -- the mask_mod keep rules of the forward kernel, in the two forms it
+// uses: per tile (which key tiles a query tile must visit, and whether a visited tile
+// needs per-element masking) and per row (the contiguous interval of kept key columns
+// inside one key tile).
+//
+// Keep rules (FlyDSL PR 931 "Add flex_attention (score_mod / mask_mod) on the generic
+// flash-attention kernel", Summary: built-in causal / sliding_window mask_mods, plus an
+// offset rule for cross-attention), indices absolute (top-left aligned):
+//   NONE:            keep
+//   CAUSAL:          j <= i
+//   SLIDING_WINDOW:  j <= i  &&  i - j < W
+//   KV_LE_Q_PLUS_OFF j <= i + off
+// and every rule also requires j < Skv (the pad rule for a ragged last key tile).
+//
+// For each rule the kept keys of row i form one interval [a(i), b(i)] with a and b
+// non-decreasing in i, so the kept keys of a query tile (rows q0..q1-1) form the
+// interval [a(q0), b(q1-1)], and a key tile [k0, k1) is FULL exactly when
+// a(q1-1) <= k0 and k1 - 1 <= b(q0) and k1 <= Skv.
+#pragma once
+
+#include <cstdint>
+
+namespace flexattn {
+
+enum MaskKind : int { kMaskNone = 0, kMaskCausal = 1, kMaskSliding = 2, kMaskOffset = 3 };
+enum ScoreKind : int { kScoreNone = 0, kScoreAlibi = 1 };
+enum TileClass : int { kTileEmpty = 0, kTileFull = 1, kTilePartial = 2 };
+
+struct MaskArgs {
+  int Skv;
+  int window;
+  int offset;
+};
+
+// Kept key interval [lo, hi] (inclusive, may be empty: lo > hi) of query row i.
+template <int MASK>
+__host__ __device__ __forceinline__ void row_interval(int64_t i, const MaskArgs& m, int64_t& lo,
+                                                      int64_t& hi) {
+  lo = 0;
+  hi = static_cast<int64_t>(m.Skv) - 1;
+  if (MASK == kMaskCausal) {
+    hi = i < hi ? i : hi;
+  } else if (MASK == kMaskSliding) {
+    hi = i < hi ? i : hi;
+    const int64_t a = i - m.window + 1;
+    lo = a > 0 ? a : 0;
+  } else if (MASK == kMaskOffset) {
+    const int64_t b = i + m.offset;
+    hi = b < hi ? b : hi;
+  }
+}
+
+// Key-tile range [t_lo, t_hi) that rows [q0, q1) (q1 exclusive, already clipped to Sq)
+// must visit; empty (t_lo == t_hi == 0) when no key of these rows is kept.
+template <int MASK>
+__host__ __device__ __forceinline__ void tile_range(int q0, int q1, int BN, const MaskArgs& m,
+                                                    int& t_lo, int& t_hi) {
+  int64_t lo_first, hi_first, lo_last, hi_last;
+  row_interval<MASK>(q0, m, lo_first, hi_first);
+  row_interval<MASK>(q1 - 1, m, lo_last, hi_last);
+  const int64_t jlo = lo_first;  // a() is non-decreasing
+  const int64_t jhi = hi_last;   // b() is non-decreasing
+  if (q1 <= q0 || jhi < jlo || jhi < 0) {
+    t_lo = t_hi = 0;
+    return;
+  }
+  t_lo = static_cast<int>(jlo / BN);
+  t_hi = static_cast<int>(jhi / BN) + 1;
+}
+
+// FULL or PARTIAL for a key tile [k0, k0 + BN) inside the visited range.
+template <int MASK>
+__host__ __device__ __forceinline__ int tile_class(int q0, int q1, int k0, int BN, const MaskArgs& m) {
+  const int64_t k1 = static_cast<int64_t>(k0) + BN;
+  if (k1 > m.Skv) return kTilePartial;
+  if (MASK == kMaskNone) return kTileFull;
+  int64_t lo_first, hi_first, lo_last, hi_last;
+  row_interval<MASK>(q0, m, lo_first, hi_first);
+  row_interval<MASK>(q1 - 1, m, lo_last, hi_last);
+  return (lo_last <= k0 && k1 - 1 <= hi_first) ? kTileFull : kTilePartial;
+}
+
+// Column interval [c_lo, c_hi] (relative to k0) kept in row i of a key tile at k0.
+template <int MASK>
+__host__ __device__ __forceinline__ void col_interval(int64_t i, int k0, const MaskArgs& m, int& c_lo,
+                                                      int& c_hi) {
+  int64_t lo, hi;
+  row_interval<MASK>(i, m, lo, hi);
+  lo -= k0;
+  hi -= k0;
+  // clamp to a range that fits in int and keeps "lo > hi" meaning empty
+  c_lo = static_cast<int>(lo < -1 ? -1 : (lo > 1 << 20 ? 1 << 20 : lo));
+  c_hi = static_cast<int>(hi < -1 ? -1 : (hi > 1 << 20 ? 1 << 20 : hi));
+  if (lo > hi) {
+    c_lo = 1;
+    c_hi = 0;
+  }
+}
+
+}  // namespace flexattn

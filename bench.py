@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark of the flex-attention hot path on B200.
+
+One step = one flex forward over the long-context workload (B=2, H=Hkv=32,
+S=8192, D=128, bf16, no_mod) followed by one decode over the dynamic KV cache
+workload (B=16, H=Hkv=32, cap=8192, D=128, f16, kv_len ~ U[1, 8192], 10% -inf
+additive mask).  Inputs are seeded synthetic tensors made on the device; every
+input is larger than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs the same workload
+on its own GPU (independent replicas, weak scaling; no collective in the data
+path) and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "flex-attn fwd TFLOPS (B2 H32 D128 S8192 bf16); decode KV-read HBM GB/s"
+FWD = dict(B=2, H=32, Hkv=32, S=8192, D=128, sigma=0.5, seed=4000)
+DEC = dict(B=16, H=32, Hkv=32, cap=8192, D=128, scale=0.08837890625, seed=3032, mask_p=0.1)
+# FlyDSL flex_attention on MI300X, no_mod, B=2 H=32 D=128 S=8192 (context, other hardware)
+PAGES_NO_MOD_8192_TFLOPS = 470.1
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# dram read+write bytes per launch from ncu, keyed by the hash of the kernel sources
+# they were measured on (a changed kernel reports null until it is captured again)
+MEASURED_TRAFFIC = {}
+KERNEL_SOURCES = ["attention_flex_attn_b200/csrc/flex_fwd_sm100.cuh",
+                  "attention_flex_attn_b200/csrc/ptx_sm100.cuh",
+                  "attention_flex_attn_b200/csrc/mask_rules.cuh",
+                  "attention_flex_attn_b200/csrc/flex_decode.cuh"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def fwd_flops(B, H, Sq, Skv, D):
+    return 4.0 * B * H * Sq * Skv * D
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"]))}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def make_inputs(dev):
+    import torch
+    import synth
+    f = FWD
+    q, k, v = synth.qkv(f["B"], f["H"], f["Hkv"], f["S"], f["S"], f["D"], seed=f["seed"], sigma=f["sigma"],
+                        device=dev)
+    d = DEC
+    qd = synth.normal_tensor((d["B"], d["H"], 1, d["D"]), d["seed"] * 8 + 1, dtype="f16", device=dev)
+    kc = synth.normal_tensor((d["B"], d["Hkv"], d["cap"], d["D"]), d["seed"] * 8 + 2, dtype="f16", device=dev)
+    vc = synth.normal_tensor((d["B"], d["Hkv"], d["cap"], d["D"]), d["seed"] * 8 + 3, dtype="f16", device=dev)
+    lens = synth.kv_lengths(d["B"], d["cap"], d["seed"] * 8 + 4).to(dev)
+    mask = synth.bernoulli_neg_inf_mask((d["B"], d["H"], 1, d["cap"]), d["mask_p"], d["seed"] * 8 + 5,
+                                        dtype="f16").to(dev)
+    return (q, k, v), (qd, kc, vc, lens, mask)
+
+
+def decode_bytes(lens, H, Hkv, D, with_mask):
+    """Algorithmic bytes of one decode: K and V rows read for every valid position,
+    mask entries for valid positions, Q read, O (f16) and LSE (fp32) written."""
+    tot = int(sum(int(x) for x in lens))
+    b = tot * Hkv * D * 2 * 2
+    if with_mask:
+        b += tot * H * 2
+    B = len(lens)
+    b += B * H * D * 2 * 2 + B * H * 4
+    return b
+
+
+def cpu_oracle_sample(q, k, v, target_s=15.0):
+    """Times the fp64 oracle on a bounded row sample of the forward workload."""
+    import numpy as np
+    import oracle
+    B, H, S, D = q.shape
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(0)
+    n = max(threads, 8)
+    rows = np.sort(rng.choice(B * H * S, size=n, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.fwd(qc, kc, vc, scale=1 / math.sqrt(D), rows=rows, threads=threads)
+    dt = time.perf_counter() - t0
+    n2 = int(min(B * H * S, max(n, n * target_s / max(dt, 1e-3))))
+    rows = np.sort(rng.choice(B * H * S, size=n2, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.fwd(qc, kc, vc, scale=1 / math.sqrt(D), rows=rows, threads=threads)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * n2 * S * D
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{n2} random query rows of the B2 H32 S8192 D128 no_mod forward (8192 keys each), "
+                      f"fp64, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: bounded row samples on the host cores."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    if rank != 0:
+        return 0
+    f = FWD
+    q, k, v = synth.qkv(f["B"], f["H"], f["Hkv"], f["S"], f["S"], f["D"], seed=f["seed"], sigma=f["sigma"])
+    B, H, S, D = q.shape
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(1)
+    probe = np.sort(rng.choice(B * H * S, size=max(threads, 8), replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.fwd(q, k, v, scale=1 / math.sqrt(D), rows=probe, threads=threads)
+    per_row = (time.perf_counter() - t0) / probe.size
+    budget = 120.0 / (args.steps + args.warmup)
+    n = int(max(threads, min(B * H * S, budget / max(per_row, 1e-6))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(B * H * S, size=n, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.fwd(q, k, v, scale=1 / math.sqrt(D), rows=rows, threads=threads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    dt = sum(times)
+    flops = 4.0 * n * S * D * len(times)
+    val = flops / dt / 1e12
+    line = {"metric": METRIC, "value": val, "unit": "TFLOPS", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "flex fwd B2 H32 Hkv32 S8192 D128 no_mod, oracle row sample per step",
+                       "rows_per_step": n},
+            "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} random query rows per step (8192 keys each), fp64"},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the per-case and e2e measurements")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import attention_flex_attn_b200 as fa
+
+    fa.load_library()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    (q, k, v), (qd, kc, vc, lens, mask) = make_inputs(dev)
+    f, d = FWD, DEC
+    scale = 1.0 / math.sqrt(f["D"])
+    o = torch.empty_like(q)
+    lse = torch.empty((f["B"], f["H"], f["S"]), dtype=torch.float32, device=dev)
+    od = torch.empty_like(qd)
+    lsed = torch.empty((d["B"], d["H"], 1), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.decode_workspace_size(d["B"], d["H"], d["Hkv"], d["cap"], d["D"]), dtype=torch.uint8,
+                     device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        fa.fwd(q, k, v, scale=scale, out=o, lse_out=lse)
+        if ev is not None:
+            ev[1].record()
+        fa.decode(qd, kc, vc, lens, d["scale"], mask=mask, out=od, lse_out=lsed, workspace=ws)
+        if ev is not None:
+            ev[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.15)
+    start.record()
+    for i in range(args.steps):
+        step(evs[i])
+    end.record()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    t = torch.tensor([total_ms, sum(fwd_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_sum, dec_sum = (float(x) for x in t.tolist())
+    if fa.device_status() != 0:
+        raise RuntimeError("device status set during the timed steps")
+
+    flops = fwd_flops(f["B"], f["H"], f["S"], f["S"], f["D"])
+    fwd_avg_s = fwd_sum / args.steps / 1e3
+    dec_avg_s = dec_sum / args.steps / 1e3
+    dbytes = decode_bytes(lens.tolist(), d["H"], d["Hkv"], d["D"], True)
+    value = world * flops / fwd_avg_s / 1e12  # whole-job forward TFLOPS (max-over-ranks time)
+    peaks, peak_kind = load_peaks()
+    achieved = flops / fwd_avg_s / 1e12
+    traffic = MEASURED_TRAFFIC.get(kernel_hash())
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": value / world / PAGES_NO_MOD_8192_TFLOPS,
+        "vs_baseline_ref": "FlyDSL flex_attention no_mod on MI300X, 470.1 TFLOPS (other hardware, context)",
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "flex fwd B2 H32 Hkv32 S8192 D128 bf16 no_mod + decode B16 H32 Hkv32 cap8192 "
+                               "D128 f16 kv_len~U[1,8192] mask10%",
+                   "global_batch": f["B"] * world, "seq_len": f["S"], "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (forward Q/K/V 384 MiB, decode caches 2 GiB); no flush"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 burst", "kernel": "flex_fwd_kernel<128,bf16,none,none>"},
+        "decode": {"gbs": dbytes / dec_avg_s / 1e9, "ms": dec_avg_s * 1e3, "bytes": dbytes,
+                   "roofline": {"bound": "hbm", "achieved": dbytes / dec_avg_s / 1e9, "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": dbytes / dec_avg_s / 1e9 / peaks["hbm_gbs"],
+                                "peak_source": peak_kind}},
+        "fwd_ms": fwd_avg_s * 1e3,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "kernel_hash": kernel_hash(),
+    }
+
+    if not args.no_extras:
+        line["cases"] = per_case(fa, q, k, v, scale, o, lse, args)
+        line["decode_cases"] = decode_cases(fa, dev, args)
+        line["e2e"] = e2e(fa, q, k, v, scale, args, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(q, k, v)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def _time_fn(fn, iters, warm):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters / 1e3
+
+
+def per_case(fa, q, k, v, scale, o, lse, args):
+    """TFLOPS of the other hook cases on the same inputs (BASELINE convention: causal halved)."""
+    B, H, S, D = q.shape
+    dense = fwd_flops(B, H, S, S, D)
+    W = 1024
+    useful_window = 4.0 * D * B * H * (W * (W + 1) // 2 + (S - W) * W)
+    cases = {"no_mod": dict(), "alibi": dict(score_mod="alibi"),
+             "sliding_window_1024": dict(mask_mod="sliding_window", window=W),
+             "causal_via_mask": dict(mask_mod="causal"), "causal_fast": dict(mask_mod="causal_fast")}
+    out = {}
+    for name, mods in cases.items():
+        t = _time_fn(lambda: fa.fwd(q, k, v, scale=scale, out=o, lse_out=lse, **mods), 20, 3)
+        causal = "causal" in name
+        out[name] = {"us": t * 1e6, "tflops": (dense * (0.5 if causal else 1.0)) / t / 1e12,
+                     "tflops_dense_equiv": dense / t / 1e12}
+        if name.startswith("sliding"):
+            out[name]["tflops_useful"] = useful_window / t / 1e12
+    return out
+
+
+def decode_cases(fa, dev, args):
+    """Decode GB/s for the other rows of the decode configuration."""
+    import torch
+    import synth
+    d = DEC
+    res = {}
+    for Hkv in (32, 8):
+        for long_kv in (False, True):
+            seed = 3300 + Hkv
+            qd = synth.normal_tensor((d["B"], d["H"], 1, d["D"]), seed * 8 + 1, dtype="f16", device=dev)
+            kc = synth.normal_tensor((d["B"], Hkv, d["cap"], d["D"]), seed * 8 + 2, dtype="f16", device=dev)
+            vc = synth.normal_tensor((d["B"], Hkv, d["cap"], d["D"]), seed * 8 + 3, dtype="f16", device=dev)
+            lens = (torch.full((d["B"],), d["cap"], dtype=torch.int32) if long_kv
+                    else synth.kv_lengths(d["B"], d["cap"], seed * 8 + 4))
+            mask = synth.bernoulli_neg_inf_mask((d["B"], d["H"], 1, d["cap"]), 0.1, seed * 8 + 5, dtype="f16").to(dev)
+            lens_d = lens.to(dev)
+            ws = torch.empty(fa.decode_workspace_size(d["B"], d["H"], Hkv, d["cap"], d["D"]), dtype=torch.uint8,
+                             device=dev)
+            for with_mask in (False, True):
+                t = _time_fn(lambda: fa.decode(qd, kc, vc, lens_d, d["scale"], mask=mask if with_mask else None,
+                                               workspace=ws), 20, 3)
+                by = decode_bytes(lens.tolist(), d["H"], Hkv, d["D"], with_mask)
+                key = f"Hkv{Hkv}_{'long' if long_kv else 'random'}_{'mask' if with_mask else 'nomask'}"
+                res[key] = {"us": t * 1e6, "gbs": by / t / 1e9}
+            del qd, kc, vc, mask, ws
+    return res
+
+
+def e2e(fa, q, k, v, scale, args, dev, world):
+    """Forward through the public API with host buffers: H2D of Q/K/V from pinned memory,
+    the kernel, D2H of O and LSE, all inside the timed region."""
+    import torch
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    hl = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
+    B, H, S, D = q.shape
+    flops = fwd_flops(B, H, S, S, D)
+
+    def once():
+        dq, dk, dv = (t.to(dev, non_blocking=True) for t in (hq, hk, hv))
+        o, lse = fa.fwd(dq, dk, dv, scale=scale)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    iters = max(3, min(args.steps, 10))
+    t = _time_fn(once, iters, 2)
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = q.numel() * q.element_size() + hl.numel() * 4
+    return {"value": world * flops / t / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "what": "forward with host Q/K/V in pinned memory, copies included"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

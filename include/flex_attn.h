@@ -1,0 +1,165 @@
+/*
+ * flex_attn.h -- C ABI of the B200 (sm_100a) flex-attention library.
+ *
+ * The library computes the fused attention forward pass
+ *
+ *     O = softmax( mask_mod( score_mod( scale * Q K^T ) ) ) V,   LSE = log-sum-exp per row
+ *
+ * with PyTorch flex_attention's per-element hooks, and a decode variant for one
+ * query row against a KV cache of dynamic length.
+ *
+ * Sources for the operation (page title, section):
+ *  - FlyDSL PR 931 "Add flex_attention (score_mod / mask_mod) on the generic
+ *    flash-attention kernel", Summary: score_mod(score, b, h, q_idx, kv_idx) gets the
+ *    already scaled score and runs before the mask; mask_mod(b, h, q_idx, kv_idx)
+ *    keeps or drops an element; built-in alibi / sliding_window / causal mods;
+ *    fully masked rows give O = 0 and LSE = -inf.
+ *  - torch-mlir PR 4366 "[TORCH] Added flex_attention hop function", Description:
+ *    the operands query, key, value, scale, enable_gqa, return_lse.
+ *  - IREE issue 19015 "[ROCM] Support dynamic key-value cache sequence length",
+ *    example IR: decode with q [B,H,1,D], K/V cache [B,H,?,D], an f16 additive mask
+ *    [B,H,1,?] and an f32 accumulation region.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named q/k/v/o/lse/kv_len/mask/workspace are DEVICE pointers on the
+ *    current CUDA device, owned by the caller.  The library keeps no per-call state
+ *    and allocates no device memory.
+ *  - Layouts are dense row-major: Q/O [B, H, Sq, D]; K/V [B, Hkv, Skv, D];
+ *    LSE [B, H, Sq] fp32 (natural log); KV cache [B, Hkv, cap, D].
+ *  - Every pointer must be 16-byte aligned.
+ *  - GQA: query head h reads key/value head h / (H / Hkv); H % Hkv must be 0.
+ *  - Argument checks run on the host before any launch; a failed check returns an
+ *    error code and launches nothing.  Work is enqueued on `stream` and the call
+ *    returns without synchronising.
+ *  - Problems that only the device can see (a kv_len outside [0, cap], a wait that
+ *    ran out of time) set bits in a device status word instead of trapping; read it
+ *    with flex_attn_device_status().
+ */
+#ifndef FLEX_ATTN_H_
+#define FLEX_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* flex_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  FLEX_OK = 0,
+  FLEX_ERR_INVALID_ARG = 1,   /* null pointer, bad size, H % Hkv != 0, bad mod parameter */
+  FLEX_ERR_UNSUPPORTED = 2,   /* head dim or dtype the kernels do not cover */
+  FLEX_ERR_MISALIGNED = 3,    /* a pointer that is not 16-byte aligned */
+  FLEX_ERR_WORKSPACE = 4,     /* decode workspace missing or too small */
+  FLEX_ERR_CUDA = 5,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+  FLEX_ERR_DEVICE_TIMEOUT = 6 /* reported through flex_attn_device_status() only */
+} flex_status_t;
+
+typedef enum { FLEX_DTYPE_BF16 = 0, FLEX_DTYPE_F16 = 1 } flex_dtype_t;
+
+/* score_mod: applied to s = scale * q.k before any mask (FlyDSL PR 931, Summary). */
+typedef enum {
+  FLEX_SCORE_NONE = 0,
+  FLEX_SCORE_ALIBI = 1 /* s += slope_h * (kv_idx - q_idx), slope_h = 2^(-8 (h+1) / H) */
+} flex_score_mod_t;
+
+/* mask_mod: keep (q_idx, kv_idx) iff the rule holds; indices are absolute (top-left). */
+typedef enum {
+  FLEX_MASK_NONE = 0,
+  FLEX_MASK_CAUSAL = 1,                /* causal_via_mask: kv_idx <= q_idx                  */
+  FLEX_MASK_SLIDING_WINDOW = 2,        /* kv_idx <= q_idx && q_idx - kv_idx < window        */
+  FLEX_MASK_KV_LE_Q_PLUS_OFFSET = 3,   /* kv_idx <= q_idx + offset (offset may be negative) */
+  FLEX_MASK_CAUSAL_FAST = 4            /* causal=True: the same keep rule as CAUSAL          */
+} flex_mask_mod_t;
+
+/* Tile classification written by the debug tile map (one byte per tile). */
+enum { FLEX_TILE_EMPTY = 0, FLEX_TILE_FULL = 1, FLEX_TILE_PARTIAL = 2 };
+
+#define FLEX_FLAG_TILE_MAP 1u /* write tile_map_out (see flex_mod_params_t) */
+
+typedef struct {
+  int32_t window;  /* FLEX_MASK_SLIDING_WINDOW: number of keys kept, >= 1 */
+  int32_t offset;  /* FLEX_MASK_KV_LE_Q_PLUS_OFFSET */
+  uint32_t flags;  /* FLEX_FLAG_* */
+  /* Debug: device buffer of ceil(Sq/BM) * ceil(Skv/BN) bytes.  With FLEX_FLAG_TILE_MAP
+   * set, the work units of batch 0 / head 0 write the class of every (q-tile, kv-tile)
+   * they process (FULL or PARTIAL) and EMPTY for every tile they skip. */
+  uint8_t* tile_map_out;
+} flex_mod_params_t;
+
+/*
+ * flex_attn_fwd -- fused forward pass (FlyDSL PR 931, Summary; torch-mlir PR 4366,
+ * Description).
+ *
+ *   q   [B, H,   Sq,  D]  dtype         k, v [B, Hkv, Skv, D]  dtype
+ *   o   [B, H,   Sq,  D]  dtype (out)   lse  [B, H, Sq] fp32 (out; NULL = return_lse false)
+ *   scale: multiplies q.k before score_mod; finite and > 0.
+ *   score_mod_id: flex_score_mod_t; mask_mod_id: flex_mask_mod_t.
+ *   mod_params: may be NULL when no mask parameter is needed.
+ *   D in {64, 128}; dtype in {BF16, F16}; B, H, Hkv, Sq, Skv >= 1.
+ * Accumulation is fp32; P and O are rounded to dtype with round-to-nearest-even.
+ * Rows whose every key is masked get O = +0 and LSE = -inf.
+ * Returns FLEX_OK or an error code (nothing is launched on error).
+ */
+flex_status_t flex_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int H, int Hkv, int Sq, int Skv, int D, float scale,
+                            int score_mod_id, int mask_mod_id, const flex_mod_params_t* mod_params,
+                            flex_dtype_t dtype, flex_stream_t stream);
+
+/*
+ * flex_attn_decode_workspace_size -- bytes of device workspace flex_attn_decode needs
+ * for these sizes (the split-KV partial outputs and their log-sum-exps).
+ */
+size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D);
+
+/*
+ * flex_attn_decode -- one query row per (batch, head) against a KV cache of
+ * per-sequence dynamic length (IREE issue 19015, example IR).
+ *
+ *   q        [B, H, 1, D]     dtype          k_cache, v_cache [B, Hkv, cap, D] dtype
+ *   kv_len   [B] int32 (device): valid length of each sequence, 0 <= kv_len[b] <= cap;
+ *            positions >= kv_len[b] are never read.  kv_len[b] == 0 gives O = 0, LSE = -inf.
+ *            A value outside [0, cap] sets a device status bit and that sequence's
+ *            rows are written as O = 0, LSE = -inf.
+ *   additive_mask [B, H, 1, cap] dtype, or NULL: added to scale * q.k (after scaling);
+ *            -inf drops a position.
+ *   o        [B, H, 1, D] dtype (out);  lse [B, H, 1] fp32 (out, NULL allowed).
+ *   workspace: device buffer of at least flex_attn_decode_workspace_size() bytes,
+ *            16-byte aligned; its contents on entry do not matter.
+ *   scale: finite and > 0.  D in {64, 128}; dtype in {BF16, F16}.
+ */
+flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* kv_len, const void* additive_mask, void* o,
+                               float* lse, int B, int H, int Hkv, int cap, int D, float scale,
+                               flex_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                               flex_stream_t stream);
+
+/*
+ * flex_attn_mask_eval -- debug: evaluates the device mask rule the forward kernel uses
+ * into keep[Sq * Skv] (uint8, device, 1 = kept) for element-exact comparison.
+ * Covers mask_mod and the j < Skv pad rule.
+ */
+flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_params,
+                                  int Sq, int Skv, uint8_t* keep, flex_stream_t stream);
+
+/* flex_attn_tile_sizes -- the (BM, BN) tile geometry the forward kernel uses for D. */
+void flex_attn_tile_sizes(int D, int* bm, int* bn);
+
+/*
+ * flex_attn_device_status -- reads (and, if reset != 0, clears) the device status
+ * word on the current device.  Synchronises the device.  Bits:
+ *   1 = a decode kv_len outside [0, cap];  2 = a forward-kernel wait ran out of time;
+ *   4 = a decode-kernel wait ran out of time.
+ */
+flex_status_t flex_attn_device_status(uint32_t* status_out, int reset);
+
+/* flex_status_string -- a static description of a status code. */
+const char* flex_status_string(flex_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLEX_ATTN_H_ */

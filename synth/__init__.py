@@ -80,11 +80,60 @@ def torch_dtype(name) -> torch.dtype:
     return _DTYPES[name]
 
 
-def normal_tensor(shape, seed: int, sigma: float = 1.0, dtype="bf16") -> torch.Tensor:
-    """CPU tensor of iid N(0, sigma^2) values rounded (RN-even) to ``dtype``."""
+def _as_i64(c: int) -> int:
+    c &= 0xFFFFFFFFFFFFFFFF
+    return c - (1 << 64) if c >= (1 << 63) else c
+
+
+_T_GOLDEN, _T_M1, _T_M2 = _as_i64(0x9E3779B97F4A7C15), _as_i64(0xBF58476D1CE4E5B9), _as_i64(0x94D049BB133111EB)
+
+
+def _shr(x: torch.Tensor, s: int) -> torch.Tensor:
+    """Logical right shift of int64 bit patterns."""
+    return (x >> s) & ((1 << (64 - s)) - 1)
+
+
+def _splitmix64_t(x: torch.Tensor) -> torch.Tensor:
+    z = x + _T_GOLDEN
+    z = (z ^ _shr(z, 30)) * _T_M1
+    z = (z ^ _shr(z, 27)) * _T_M2
+    return z ^ _shr(z, 31)
+
+
+def normal_fp64_torch(seed: int, n: int, device) -> torch.Tensor:
+    """Same stream as normal_fp64 (identical uniforms), computed with torch on ``device``."""
+    key = _as_i64(int(_stream_key(seed)))
+    out = torch.empty(n, dtype=torch.float64, device=device)
+    npairs = (n + 1) // 2
+    step = 1 << 24
+    for p0 in range(0, npairs, step):
+        p1 = min(npairs, p0 + step)
+        ctr = torch.arange(2 * p0, 2 * p1, dtype=torch.int64, device=device)
+        bits = _splitmix64_t(ctr * _T_GOLDEN + key)
+        u = (_shr(bits, 11).to(torch.float64) + 1.0) * (1.0 / 9007199254740992.0)
+        u1, u2 = u[0::2], u[1::2]
+        r = torch.sqrt(-2.0 * torch.log(u1))
+        t = (2.0 * np.pi) * u2
+        pair = torch.stack((r * torch.cos(t), r * torch.sin(t)), dim=1).reshape(-1)
+        lo, hi = 2 * p0, min(n, 2 * p1)
+        out[lo:hi] = pair[: hi - lo]
+    return out
+
+
+def normal_tensor(shape, seed: int, sigma: float = 1.0, dtype="bf16", device=None) -> torch.Tensor:
+    """Tensor of iid N(0, sigma^2) values rounded (RN-even) to ``dtype``.
+
+    device None: computed with numpy on the CPU.  Otherwise the torch implementation of
+    the same counter stream runs on ``device`` (used for large inputs); uniforms are
+    bit-identical, the fp64 Box-Muller may differ in the last ulp.
+    """
     n = int(np.prod(shape)) if len(shape) else 1
-    z = normal_fp64(seed, n) * sigma
-    return torch.from_numpy(z).reshape(tuple(shape)).to(torch_dtype(dtype))
+    if device is None:
+        z = normal_fp64(seed, n) * sigma
+        return torch.from_numpy(z).reshape(tuple(shape)).to(torch_dtype(dtype))
+    z = normal_fp64_torch(seed, n, device)
+    z.mul_(sigma)
+    return z.to(torch_dtype(dtype)).reshape(tuple(shape))
 
 
 def kv_lengths(batch: int, cap: int, seed: int, lo: int = 1) -> torch.Tensor:
@@ -109,9 +158,9 @@ def case_seed(config: int, case: int, rep: int = 0) -> int:
     return 1000 * config + 10 * case + rep
 
 
-def qkv(B, H, Hkv, Sq, Skv, D, seed, sigma=1.0, dtype="bf16"):
-    """Q [B,H,Sq,D], K/V [B,Hkv,Skv,D] with independent streams seed+{1,2,3}."""
-    q = normal_tensor((B, H, Sq, D), seed * 8 + 1, sigma, dtype)
-    k = normal_tensor((B, Hkv, Skv, D), seed * 8 + 2, sigma, dtype)
-    v = normal_tensor((B, Hkv, Skv, D), seed * 8 + 3, sigma, dtype)
+def qkv(B, H, Hkv, Sq, Skv, D, seed, sigma=1.0, dtype="bf16", device=None):
+    """Q [B,H,Sq,D], K/V [B,Hkv,Skv,D] with independent streams seed*8+{1,2,3}."""
+    q = normal_tensor((B, H, Sq, D), seed * 8 + 1, sigma, dtype, device)
+    k = normal_tensor((B, Hkv, Skv, D), seed * 8 + 2, sigma, dtype, device)
+    v = normal_tensor((B, Hkv, Skv, D), seed * 8 + 3, sigma, dtype, device)
     return q, k, v

@@ -1,0 +1,104 @@
+"""CPU checks of the C ABI: the library loads, exports what the header declares, and
+rejects bad arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_flex_attn_b200 as fa
+from attention_flex_attn_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.load_library()
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "flex_attn.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(flex_\w+)\s*\(", txt)))
+
+
+def test_header_symbols_exported(lib):
+    names = _declared()
+    assert names, "no declarations found"
+    assert sorted(fa.EXPORTED) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.flex_status_string(code)
+    assert lib.flex_status_string(99) == b"unknown status"
+
+
+def test_tile_sizes(lib):
+    assert fa.tile_sizes(128) == (128, 128)
+    assert fa.tile_sizes(64) == (128, 128)
+
+
+def test_workspace_size(lib):
+    # ceil(8192/256) = 32 splits; o part [16*32, 32, 128] fp32 + lse part
+    n = fa.decode_workspace_size(16, 32, 8, 8192, 128)
+    assert n == 16 * 32 * 32 * 128 * 4 + 16 * 32 * 32 * 4
+    assert fa.decode_workspace_size(0, 32, 8, 8192, 128) == 0
+
+
+P = ctypes.c_void_p
+
+
+def _fwd(lib, q=16, k=16, v=16, o=16, lse=None, B=1, H=2, Hkv=1, Sq=8, Skv=8, D=128, scale=0.1,
+         score=0, mask=0, mp=None, dtype=0):
+    return lib.flex_attn_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, Hkv, Sq, Skv, D, scale, score, mask,
+                             ctypes.byref(mp) if mp is not None else None, dtype, None)
+
+
+def test_fwd_rejects_bad_args_on_host(lib):
+    assert _fwd(lib, q=0) == 1
+    assert _fwd(lib, B=0) == 1
+    assert _fwd(lib, H=3, Hkv=2) == 1
+    assert _fwd(lib, Sq=0) == 1
+    assert _fwd(lib, scale=0.0) == 1
+    assert _fwd(lib, scale=float("nan")) == 1
+    assert _fwd(lib, D=96) == 2
+    assert _fwd(lib, dtype=7) == 2
+    assert _fwd(lib, score=5) == 1
+    assert _fwd(lib, mask=9) == 1
+    assert _fwd(lib, mask=2, mp=fa.ModParams(0, 0, 0, None)) == 1      # window < 1
+    assert _fwd(lib, mp=fa.ModParams(1, 0, 1, None)) == 1              # tile map without buffer
+    assert _fwd(lib, q=17) == 3
+    assert _fwd(lib, lse=20) == 3
+
+
+def test_decode_rejects_bad_args_on_host(lib):
+    def dec(q=16, k=16, v=16, kl=16, m=None, o=16, lse=None, B=2, H=4, Hkv=2, cap=64, D=128, scale=0.1,
+            dtype=1, ws=16, wsb=1 << 20):
+        return lib.flex_attn_decode(P(q), P(k), P(v), P(kl), P(m), P(o), P(lse), B, H, Hkv, cap, D, scale,
+                                    dtype, P(ws), wsb, None)
+    assert dec(kl=0) == 1
+    assert dec(H=3) == 1
+    assert dec(cap=0) == 1
+    assert dec(D=80) == 2
+    assert dec(ws=0) == 4
+    assert dec(wsb=16) == 4
+    assert dec(m=18) == 3
+    assert dec(kl=4) == 3
+
+
+def test_mask_eval_rejects_bad_args(lib):
+    assert lib.flex_attn_mask_eval(0, None, 0, 4, P(16), None) == 1
+    assert lib.flex_attn_mask_eval(7, None, 4, 4, P(16), None) == 1
+    assert lib.flex_attn_mask_eval(0, None, 4, 4, P(0), None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(fa.FlexAttnError):
+        fa.fwd(q, q, q)
