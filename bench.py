@@ -215,6 +215,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-case and e2e measurements")
+    ap.add_argument("--profile", choices=["fwd", "fwd8192", "decode"], default=None,
+                    help="run only a few launches of one kernel (for ncu captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -225,6 +227,8 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.profile:
+        return profile_case(args.profile)
 
     import torch
     import torch.distributed as dist
@@ -419,6 +423,34 @@ def e2e(fa, q, k, v, scale, args, dev, world):
     d2h = q.numel() * q.element_size() + hl.numel() * 4
     return {"value": world * flops / t / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "what": "forward with host Q/K/V in pinned memory, copies included"}
+
+
+def profile_case(which):
+    """A few launches of one kernel on a case larger than L2 but a few GB at most:
+    fwd = B2 H32 S4096 D128 bf16 no_mod (192 MiB of Q/K/V); fwd8192 = the full forward
+    workload; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
+    import torch
+    import synth
+    import attention_flex_attn_b200 as fa
+    fa.load_library()
+    dev = torch.device("cuda", 0)
+    if which.startswith("fwd"):
+        S = 8192 if which == "fwd8192" else 4096
+        q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
+        for _ in range(4):
+            fa.fwd(q, k, v)
+    else:
+        qd = synth.normal_tensor((16, 32, 1, 128), 11, dtype="f16", device=dev)
+        kc = synth.normal_tensor((16, 8, 8192, 128), 12, dtype="f16", device=dev)
+        vc = synth.normal_tensor((16, 8, 8192, 128), 13, dtype="f16", device=dev)
+        lens = torch.full((16,), 8192, dtype=torch.int32, device=dev)
+        mask = synth.bernoulli_neg_inf_mask((16, 32, 1, 8192), 0.1, 14, dtype="f16").to(dev)
+        for _ in range(4):
+            fa.decode(qd, kc, vc, lens, 0.08837890625, mask=mask)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    print(f"profile {which} ok")
+    return 0
 
 
 if __name__ == "__main__":
