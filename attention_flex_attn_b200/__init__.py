@@ -26,7 +26,7 @@ FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
 EXPORTED = ["flex_attn_fwd", "flex_attn_decode_workspace_size", "flex_attn_decode",
-            "flex_attn_mask_eval", "flex_attn_tile_sizes", "flex_attn_device_status",
+            "flex_attn_decode_noalloc", "flex_attn_mask_eval", "flex_attn_tile_sizes", "flex_attn_device_status",
             "flex_status_string"]
 
 
@@ -57,6 +57,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_decode_workspace_size.restype = SZ
     lib.flex_attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, P]
     lib.flex_attn_decode.restype = I
+    lib.flex_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P]
+    lib.flex_attn_decode_noalloc.restype = I
     lib.flex_attn_mask_eval.argtypes = [I, ctypes.POINTER(ModParams), I, I, P, P]
     lib.flex_attn_mask_eval.restype = I
     lib.flex_attn_tile_sizes.argtypes = [I, ctypes.POINTER(I), ctypes.POINTER(I)]
@@ -153,6 +155,33 @@ def decode(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None
                               B, H, Hkv, cap, D, float(scale), DTYPES[q.dtype], _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(q.device))
     _check(rc, "flex_attn_decode")
+    return o, lse
+
+
+# Bytes of the scratch array compiled into the library for decode_noalloc.
+DECODE_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def decode_noalloc(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None):
+    """Decode through flex_attn_decode_noalloc: no workspace argument and no device
+    allocation inside the library; it uses the scratch array compiled into the library
+    (shared by all calls on a device, so calls must not overlap on the GPU).  Outputs
+    are allocated here only when ``out`` / ``lse_out`` are not given."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (kv_len, "kv_len")):
+        _cuda_tensor(t, n)
+    if mask is not None:
+        _cuda_tensor(mask, "mask")
+    B, H, one, D = q.shape
+    _, Hkv, cap, _ = k_cache.shape
+    if one != 1 or kv_len.dtype != torch.int32:
+        raise FlexAttnError("decode takes q [B,H,1,D] and int32 kv_len")
+    o = out if out is not None else torch.empty_like(q)
+    lse = lse_out if lse_out is not None else torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    rc = lib.flex_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_len), _ptr(mask), _ptr(o),
+                                      _ptr(lse), B, H, Hkv, cap, D, float(scale), DTYPES[q.dtype],
+                                      _stream(q.device))
+    _check(rc, "flex_attn_decode_noalloc")
     return o, lse
 
 

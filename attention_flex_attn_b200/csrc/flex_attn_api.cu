@@ -69,6 +69,25 @@ bool ensure_smem_attr(K kernel, int bytes) {
   return true;
 }
 
+// Scratch for flex_attn_decode_noalloc: compiled into the library so that callers who
+// cannot allocate device memory still get a workspace.  One copy per device, shared by
+// every call on that device.
+__device__ __align__(256) unsigned char g_decode_scratch[FLEX_DECODE_STATIC_SCRATCH_BYTES];
+
+// Device address of g_decode_scratch on the current device, looked up once per device
+// (host code only sees a host-side stand-in under that name, never usable on the GPU).
+void* decode_scratch_ptr() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<void*> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
+  cache[dev].store(p, std::memory_order_release);
+  return p;
+}
+
 unsigned* status_ptr() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
@@ -277,6 +296,19 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
   if (D == 128)
     return dtype == FLEX_DTYPE_BF16 ? decode_by_group<128, __nv_bfloat16>(p, s) : decode_by_group<128, __half>(p, s);
   return dtype == FLEX_DTYPE_BF16 ? decode_by_group<64, __nv_bfloat16>(p, s) : decode_by_group<64, __half>(p, s);
+}
+
+flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* kv_len, const void* additive_mask, void* o, float* lse,
+                                       int B, int H, int Hkv, int cap, int D, float scale, flex_dtype_t dtype,
+                                       flex_stream_t stream) {
+  const size_t need = flex_attn_decode_workspace_size(B, H, Hkv, cap, D);
+  if (need == 0) return FLEX_ERR_INVALID_ARG;
+  if (need > FLEX_DECODE_STATIC_SCRATCH_BYTES) return FLEX_ERR_WORKSPACE;
+  void* scratch = decode_scratch_ptr();
+  if (!scratch) return FLEX_ERR_CUDA;
+  return flex_attn_decode(q, k_cache, v_cache, kv_len, additive_mask, o, lse, B, H, Hkv, cap, D, scale, dtype,
+                          scratch, FLEX_DECODE_STATIC_SCRATCH_BYTES, stream);
 }
 
 flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_params, int Sq, int Skv,

@@ -137,6 +137,33 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
                                flex_stream_t stream);
 
 /*
+ * flex_attn_decode_noalloc -- flex_attn_decode without a caller-supplied workspace.
+ * (No counterpart on the source pages: this entry point exists for callers of this
+ * library.)  Some callers cannot allocate device memory at call time: hosts that load
+ * operators through a fixed interface which passes only inputs and outputs, processes
+ * that reserved their whole memory budget up front, and latency-bound decode loops that
+ * must not pay for cudaMalloc/cudaFree (both synchronise the device).  This variant
+ * needs no workspace: it uses a scratch array of FLEX_DECODE_STATIC_SCRATCH_BYTES
+ * compiled into the library, which every GPU that loads the library keeps until the
+ * process exits.  It calls no allocator of any kind.
+ *   Arguments, layouts and errors are those of flex_attn_decode.  Sizes whose workspace
+ *   (flex_attn_decode_workspace_size) exceeds FLEX_DECODE_STATIC_SCRATCH_BYTES return
+ *   FLEX_ERR_WORKSPACE and launch nothing.
+ *   The first call on a device looks up the device address of the scratch array
+ *   (cudaGetSymbolAddress, with that device current); make that first call before any
+ *   stream capture on the device.
+ *   All calls on a device share the one array and it keeps the last call's contents;
+ *   the kernels write every scratch entry they read, so nothing needs clearing, but
+ *   calls that overlap on the GPU (e.g. on two streams at once) race on it and must be
+ *   serialised by the caller.
+ */
+#define FLEX_DECODE_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* kv_len, const void* additive_mask, void* o,
+                                       float* lse, int B, int H, int Hkv, int cap, int D, float scale,
+                                       flex_dtype_t dtype, flex_stream_t stream);
+
+/*
  * flex_attn_mask_eval -- debug: evaluates the device mask rule the forward kernel uses
  * into keep[Sq * Skv] (uint8, device, 1 = kept) for element-exact comparison.
  * Covers mask_mod and the j < Skv pad rule.

@@ -102,3 +102,10 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(fa.FlexAttnError):
         fa.fwd(q, q, q)
+
+
+def test_static_scratch_limit_matches_header():
+    txt = open(os.path.join(ROOT, "include", "flex_attn.h")).read()
+    m = re.search(r"#define FLEX_DECODE_STATIC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", txt)
+    assert m, "FLEX_DECODE_STATIC_SCRATCH_BYTES not found"
+    assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == fa.DECODE_STATIC_SCRATCH_BYTES
