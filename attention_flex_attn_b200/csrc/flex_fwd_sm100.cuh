@@ -8,15 +8,20 @@
 // so the no-mod instantiation carries no hook code at all.
 //
 // One CTA owns two 128-row query tiles of one (b, h) and walks the key/value tiles both
-// of them need:
-//   warp 9      TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory slots
-//   warp 8      MMA issuer (one thread): S_k = Q_k K_j^T and O_k += P_k V_j with tcgen05,
-//               accumulators in tensor memory
-//   warps 0-3   softmax for query tile 0, warps 4-7 for query tile 1: each thread owns one
+// of them need.  Three warpgroups:
+//   warp 0      MMA issuer (one thread): S_k = Q_k K_j^T and O_k += P_k V_j with tcgen05,
+//               accumulators in tensor memory.  It is warp 0 so that the warp scheduler of
+//               its sub-partition, shared with two busy softmax warps, serves it first.
+//   warp 1      TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory slots
+//   warps 2-3   idle (they only give their registers to the softmax warpgroups)
+//   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1: each thread owns one
 //               query row (= one TMEM lane), reads its S row from TMEM, applies score_mod,
 //               mask (PARTIAL tiles only) and the online base-2 softmax, writes P (16-bit)
-//               back into TMEM over S, rescales its O row when the running max grows by
-//               more than 2^8, and finally normalises O and writes O and LSE.
+//               back into TMEM over S in two 64-column halves (each signalled on its own
+//               barrier so the P.V matmul can start on the first half), rescales its O row
+//               when the running max grows by more than 2^8, and finally normalises O and
+//               writes O and LSE.  kEmuPairsPerHalf of each 32 column pairs can evaluate
+//               2^x as a polynomial on the FMA pipe instead of the MUFU unit.
 // The MMA order S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ... lets one softmax
 // warpgroup work while the tensor core runs the other tile's matmuls.
 //
@@ -39,7 +44,18 @@ namespace flexattn {
 
 constexpr int kBM = 128;        // query rows per tile (tcgen05 M)
 constexpr int kBN = 128;        // keys per tile
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 384;
+constexpr int kMmaWarp = 0;
+constexpr int kTmaWarp = 1;
+constexpr int kSoftmaxWarp0 = 4;        // warps 4-7: query tile 0, warps 8-11: query tile 1
+constexpr uint32_t kSoftmaxRegs = 200;  // per thread, softmax warpgroups after setmaxnreg
+constexpr uint32_t kAuxRegs = 96;       // per thread, producer/MMA warpgroup after setmaxnreg
+// 256 * 200 + 128 * 96 = 63488 <= 384 * 168 (the launch allotment at 384 threads); per
+// SM sub-partition (one warp of each warpgroup) 200 + 200 + 96 <= 512
+static_assert(256 * kSoftmaxRegs + 128 * kAuxRegs <= (65536 / kFwdThreads) / 8 * 8 * kFwdThreads,
+              "setmaxnreg split exceeds the registers the block is launched with");
+static_assert(2 * kSoftmaxRegs + kAuxRegs <= 512, "per sub-partition register file exceeded");
+constexpr int kEmuPairsPerHalf = 0;     // of 32 column pairs per 64-column half run on the FMA pipe
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
@@ -61,15 +77,19 @@ template <int D>
 struct FwdSmem {
   static constexpr int kTileBytes = kBM * D * 2;          // one 128-row tile
   static constexpr int kChunkBytes = kBM * 128;           // one 64-element-wide chunk
-  static constexpr int kSlots = D == 128 ? 4 : 8;         // key/value ring depth
+  // Key/value ring depth.  K_j and V_j take consecutive entries; K_j is released as soon
+  // as both S_k(j) are issued, V_j only after both P_k V_j, so with 5 slots V_{j+2} waits
+  // on K_j rather than on V_j and gets about two tile steps of load lead time.
+  static constexpr int kSlots = D == 128 ? 5 : 12;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  // barriers: q, full[NS], empty[NS], s_full[2], p_full[2], o_full[2], drain; then tmem addr
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1;
+  // barriers: q, full[NS], empty[NS], s_full[2], p_half[2][2], o_full[2], drain; then tmem addr
+  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 4 + 2 + 1;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemPtrOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
+  static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
 };
 
 template <typename T>
@@ -111,9 +131,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
   auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
   auto bar_s = [&](int k) { return sbase + L::kBarOff + 8u * (1 + 2 * NS + k); };
-  auto bar_p = [&](int k) { return sbase + L::kBarOff + 8u * (3 + 2 * NS + k); };
-  auto bar_o = [&](int k) { return sbase + L::kBarOff + 8u * (5 + 2 * NS + k); };
-  const uint32_t bar_drain = sbase + L::kBarOff + 8u * (7 + 2 * NS);
+  auto bar_p = [&](int k, int half) { return sbase + L::kBarOff + 8u * (3 + 2 * NS + 2 * k + half); };
+  auto bar_o = [&](int k) { return sbase + L::kBarOff + 8u * (7 + 2 * NS + k); };
+  const uint32_t bar_drain = sbase + L::kBarOff + 8u * (9 + 2 * NS);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
 
@@ -150,19 +170,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar_s(k), 1);
-      mbar_init(bar_p(k), kBM);
+      mbar_init(bar_p(k, 0), kBM);
+      mbar_init(bar_p(k, 1), kBM);
       mbar_init(bar_o(k), 1);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == kTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
     tmem_relinquish();
   }
@@ -171,14 +192,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
 
-  auto tile_smem = [&](int off_tiles) { return sbase + static_cast<uint32_t>(off_tiles); };
-  const uint32_t q_smem0 = tile_smem(L::kQOff);
+  const uint32_t q_smem0 = sbase + static_cast<uint32_t>(L::kQOff);
   auto q_smem = [&](int k) { return q_smem0 + static_cast<uint32_t>(k * L::kTileBytes); };
   auto kv_smem = [&](int s) { return sbase + static_cast<uint32_t>(L::kKVOff + s * L::kTileBytes); };
 
-  if (warp == 9) {
-    // ============================================================ TMA producer
-    if (lane == 0 && any_work) {
+  if (warp < kSoftmaxWarp0) {
+    regs_dec<kAuxRegs>();
+    if (warp == kTmaWarp && lane == 0 && any_work) {
+      // ============================================================ TMA producer
       const int bytes_q = (act0 ? 1 : 0) * L::kTileBytes + (act1 ? 1 : 0) * L::kTileBytes;
       mbar_arrive_expect_tx(bar_q, bytes_q);
       for (int k = 0; k < 2; ++k) {
@@ -210,45 +231,51 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusFwdTimeout,
                   kWaitTimeoutNs);
       mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
-    }
-  } else if (warp == 8) {
-    // ============================================================ MMA issuer
-    if (lane == 0 && any_work) {
+    } else if (warp == kMmaWarp && lane == 0 && any_work) {
+      // ============================================================ MMA issuer
       bool ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
       tc_fence_after();
       int np[2] = {0, 0};
+      // descriptor of chunk 0 / k-step 0; k-step kk adds ((kk/4)*chunk + (kk%4)*32) >> 4
+      const uint64_t dq0 = smem_desc(q_smem(0), 16, 1024, kSwizzle128B);
       auto issue_s = [&](int k, int slot) {
         const uint32_t d = tmem + 128u * k;
+        const uint64_t aq = dq0 + static_cast<uint64_t>((k * L::kTileBytes) >> 4);
+        const uint64_t bk = smem_desc(kv_smem(slot), 16, 1024, kSwizzle128B);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * L::kChunkBytes + (kk % 4) * 32;
-          const uint64_t ad = smem_desc(q_smem(k) + off, 16, 1024, kSwizzle128B);
-          const uint64_t bd = smem_desc(kv_smem(slot) + off, 16, 1024, kSwizzle128B);
-          mma_ss(d, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
+          mma_ss(d, aq + off, bk + off, kIdescS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int k, int slot, bool acc) {
+      auto issue_pv = [&](int k, int slot, bool acc, int kk0, int kk1) {
         const uint32_t d = tmem + 256u + 128u * k;
         const uint32_t a = tmem + 128u * k;
+        const uint64_t bv = smem_desc(kv_smem(slot), L::kChunkBytes, 1024, kSwizzle128B);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc(kv_smem(slot) + kk * 2048, L::kChunkBytes, 1024, kSwizzle128B);
-          mma_ts(d, a + 8u * kk, bd, kIdescPV, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = kk0; kk < kk1; ++kk)
+          mma_ts(d, a + 8u * kk, bv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                 (acc || kk > 0) ? 1u : 0u);
       };
       for (int j = ulo; j < uhi && ok; ++j) {
         const int rK = 2 * (j - ulo), rV = rK + 1;
         const int sK = rK % NS, sV = rV % NS;
-        if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
-                       kStatusFwdTimeout, kWaitTimeoutNs)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int k = 0; k < 2; ++k) {
-          if (j == lo[k] && lo[k] < hi[k]) {
-            issue_s(k, sK);
-            mma_commit(bar_s(k));
+        const bool first0 = act0 && j == lo[0], first1 = act1 && j == lo[1];
+        if (first0 || first1) {
+          // K_j was not needed before: wait for it here (otherwise the previous step did)
+          if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+                         kStatusFwdTimeout, kWaitTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (first0) {
+            issue_s(0, sK);
+            mma_commit(bar_s(0));
+          }
+          if (first1) {
+            issue_s(1, sK);
+            mma_commit(bar_s(1));
           }
         }
         mma_commit(bar_empty(sK));
@@ -257,25 +284,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ok = false;
           break;
         }
+        bool next_k_ready = false;
         for (int k = 0; k < 2 && ok; ++k) {
           if (j < lo[k] || j >= hi[k]) continue;
-          if (!mbar_wait(bar_p(k), static_cast<uint32_t>(np[k]) & 1u, p.status, kStatusFwdTimeout,
-                         kWaitTimeoutNs) ||
-              *abort_flag) {
-            ok = false;
-            break;
-          }
-          ++np[k];
-          tc_fence_after();
-          issue_pv(k, sV, j > lo[k]);
-          if (j + 1 < hi[k]) {
-            const int rK2 = rK + 2;
-            if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status,
-                           kStatusFwdTimeout, kWaitTimeoutNs)) {
+          const uint32_t par = static_cast<uint32_t>(np[k]) & 1u;
+          for (int half = 0; half < 2; ++half) {
+            if (!mbar_wait(bar_p(k, half), par, p.status, kStatusFwdTimeout, kWaitTimeoutNs) || *abort_flag) {
               ok = false;
               break;
             }
             tc_fence_after();
+            issue_pv(k, sV, j > lo[k], 4 * half, 4 * half + 4);
+          }
+          if (!ok) break;
+          ++np[k];
+          if (j + 1 < hi[k]) {
+            const int rK2 = rK + 2;
+            if (!next_k_ready) {
+              if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status,
+                             kStatusFwdTimeout, kWaitTimeoutNs)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              next_k_ready = true;
+            }
             issue_s(k, rK2 % NS);
             mma_commit(bar_s(k));
           } else {
@@ -290,8 +323,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_wait(bar_drain, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
     }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // ============================================================ softmax warpgroups
-    const int k = warp >> 2;          // query tile of this warpgroup
+    const int k = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
     const int wq = warp & 3;          // TMEM lane quarter
     const int row = wq * 32 + lane;   // row inside the tile == TMEM lane
     const int qi = q0[k] + row;       // absolute query index
@@ -329,16 +363,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int cls = tile_class<MASK>(q0[k], q1[k], k0, kBN, p.mask);
       if (write_map) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] = static_cast<uint8_t>(cls);
 
-      float s[kBN];
-      {
-        uint32_t r[64];
-        tmem_ld64(tS, r);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(r[c]);
-        tmem_ld64(tS + 64u, r);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[64 + c] = __uint_as_float(r[c]);
-      }
+      uint32_t sr[kBN];
+      tmem_ld128(tS, sr);
+      float* s = reinterpret_cast<float*>(sr);
       if (SCORE == kScoreAlibi) {
         const float base = slope2 * static_cast<float>(k0 - qi);
 #pragma unroll
@@ -351,15 +378,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int c = 0; c < kBN; ++c)
           if (c < c_lo || c > c_hi) s[c] = -INFINITY;
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      float mx0 = max3f(s[0], s[1], s[2]), mx1 = max3f(s[3], s[4], s[5]);
+      float mx2 = max3f(s[6], s[7], s[8]), mx3 = max3f(s[9], s[10], s[11]);
 #pragma unroll
-      for (int c = 4; c < kBN; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
+      for (int c = 12; c + 8 <= kBN - 4; c += 8) {
+        mx0 = max3f(mx0, s[c], s[c + 1]);
+        mx1 = max3f(mx1, s[c + 2], s[c + 3]);
+        mx2 = max3f(mx2, s[c + 4], s[c + 5]);
+        mx3 = max3f(mx3, s[c + 6], s[c + 7]);
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
+      mx0 = max3f(mx0, s[kBN - 4], s[kBN - 3]);
+      mx1 = max3f(mx1, s[kBN - 2], s[kBN - 1]);
+      const float mx = max3f(mx0, mx1, fmaxf(mx2, mx3)) * sc;
       const bool need = mx > m_used + kRescaleThreshold;  // false while both are -inf
       if (__any_sync(0xffffffffu, need)) {
         float alpha = 1.0f;
@@ -369,35 +399,53 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           l_sum *= alpha;
         }
         if (n > 0) {
+          const uint64_t a2 = pack2(alpha, alpha);
 #pragma unroll 1
           for (int c = 0; c < D; c += 32) {
             uint32_t r[32];
             tmem_ld32(tO + c, r);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              const uint64_t v = mul2(pack2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), a2);
+              r[e] = static_cast<uint32_t>(v);
+              r[e + 1] = static_cast<uint32_t>(v >> 32);
+            }
             tmem_st32(tO + c, r);
           }
         }
       }
       const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-      float ls0 = 0.f, ls1 = 0.f;
+      const uint64_t sc2 = pack2(sc, sc);
+      const uint64_t nm2 = pack2(-m_safe, -m_safe);
+      uint64_t acc2 = 0;  // two running partial sums (0.0f, 0.0f)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float e0 = ex2_approx(fmaf(s[64 * half + c], sc, -m_safe));
-          const float e1 = ex2_approx(fmaf(s[64 * half + c + 1], sc, -m_safe));
-          ls0 += e0;
-          ls1 += e1;
-          pk[c / 2] = DtypeBits<T>::pack(e0, e1);
+        for (int i = 0; i < 32; ++i) {
+          const int c = 64 * half + 2 * i;
+          const uint64_t x2 = fma2(pack2(s[c], s[c + 1]), sc2, nm2);
+          uint64_t e2;
+          if (i >= 32 - kEmuPairsPerHalf) {
+            e2 = exp2_poly2(x2);
+          } else {
+            float x0, x1;
+            unpack2(x2, x0, x1);
+            e2 = pack2(ex2_approx(x0), ex2_approx(x1));
+          }
+          acc2 = add2(acc2, e2);
+          float e0, e1;
+          unpack2(e2, e0, e1);
+          pk[i] = DtypeBits<T>::pack(e0, e1);
         }
         tmem_st32(tS + 32u * half, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p(k, half));
       }
-      l_sum += ls0 + ls1;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar_p(k));
+      float a0, a1;
+      unpack2(acc2, a0, a1);
+      l_sum += a0 + a1;
     }
     if (!ok) *abort_flag = 1;
 
@@ -413,7 +461,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
       }
       const bool row_ok = qi < p.Sq;
-      const bool has_mass = ran && l_sum > 0.f;
+      // A row has mass iff it ever saw a kept (finite) score.  The polynomial 2^x returns
+      // ~2^-125 rather than 0 for masked scores, so l_sum alone cannot tell.
+      const bool has_mass = ran && m_used != -INFINITY && l_sum > 0.f;
       const float inv = has_mass ? 1.0f / l_sum : 0.f;
       T* orow = reinterpret_cast<T*>(p.o) + (static_cast<int64_t>(bh) * p.Sq + qi) * D;
 #pragma unroll 1
@@ -445,7 +495,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
