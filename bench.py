@@ -60,6 +60,23 @@ def fwd_flops(B, H, Sq, Skv, D):
     return 4.0 * B * H * Sq * Skv * D
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings (every rank gets the result).  Ranks run
+    independent replicas, so the job takes as long as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(world, flops_per_rank, seconds):
+    """Whole-job throughput of `world` replicas that each did flops_per_rank in `seconds`
+    (the max over ranks)."""
+    return world * flops_per_rank / seconds / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -290,10 +307,7 @@ def main():
     total_ms = start.elapsed_time(end)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    t = torch.tensor([total_ms, sum(fwd_ms), sum(dec_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_sum, dec_sum = (float(x) for x in t.tolist())
+    total_ms, fwd_sum, dec_sum = max_over_ranks([total_ms, sum(fwd_ms), sum(dec_ms)], device=dev)
     if fa.device_status() != 0:
         raise RuntimeError("device status set during the timed steps")
 
@@ -301,7 +315,7 @@ def main():
     fwd_avg_s = fwd_sum / args.steps / 1e3
     dec_avg_s = dec_sum / args.steps / 1e3
     dbytes = decode_bytes(lens.tolist(), d["H"], d["Hkv"], d["D"], True)
-    value = world * flops / fwd_avg_s / 1e12  # whole-job forward TFLOPS (max-over-ranks time)
+    value = whole_job_tflops(world, flops, fwd_avg_s)  # max-over-ranks time
     peaks, peak_kind = load_peaks()
     achieved = flops / fwd_avg_s / 1e12
     traffic = MEASURED_TRAFFIC.get(kernel_hash())
