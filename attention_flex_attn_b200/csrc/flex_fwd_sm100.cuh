@@ -22,8 +22,9 @@
 //               when the running max grows by more than 2^8, and finally normalises O and
 //               writes O and LSE.  kEmuPairsPerHalf of each 32 column pairs can evaluate
 //               2^x as a polynomial on the FMA pipe instead of the MUFU unit.
-// The MMA order S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ... lets one softmax
-// warpgroup work while the tensor core runs the other tile's matmuls.
+// Key tiles are visited from the last to the first.  With t counting steps, the MMA order
+// S0(t0) S1(t0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ... lets one softmax warpgroup work
+// while the tensor core runs the other tile's matmuls.
 //
 // Tensor memory (512 columns x 128 lanes): S0 [0,128) S1 [128,256) O0 [256,256+D)
 // O1 [384,384+D); P_k aliases the first 64 columns of S_k (two 16-bit values per column).
@@ -209,7 +210,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       int r = 0;
       bool ok = true;
-      for (int j = ulo; j < uhi && ok; ++j) {
+      for (int t = 0; t < uhi - ulo && ok; ++t) {
+        const int j = uhi - 1 - t;  // key tiles from last to first
         for (int which = 0; which < 2 && ok; ++which, ++r) {
           const int s = r % NS;
           const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
@@ -257,10 +259,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_ts(d, a + 8u * kk, bv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
                  (acc || kk > 0) ? 1u : 0u);
       };
-      for (int j = ulo; j < uhi && ok; ++j) {
-        const int rK = 2 * (j - ulo), rV = rK + 1;
+      for (int t = 0; t < uhi - ulo && ok; ++t) {
+        const int j = uhi - 1 - t;  // key tiles from last to first
+        const int rK = 2 * t, rV = rK + 1;
         const int sK = rK % NS, sV = rV % NS;
-        const bool first0 = act0 && j == lo[0], first1 = act1 && j == lo[1];
+        const bool first0 = act0 && j == hi[0] - 1, first1 = act1 && j == hi[1] - 1;
         if (first0 || first1) {
           // K_j was not needed before: wait for it here (otherwise the previous step did)
           if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
@@ -289,17 +292,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (j < lo[k] || j >= hi[k]) continue;
           const uint32_t par = static_cast<uint32_t>(np[k]) & 1u;
           for (int half = 0; half < 2; ++half) {
-            if (!mbar_wait(bar_p(k, half), par, p.status, kStatusFwdTimeout, kWaitTimeoutNs) || *abort_flag) {
+            if (!mbar_wait(bar_p(k, half), par, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_pv(k, sV, j > lo[k], 4 * half, 4 * half + 4);
+            issue_pv(k, sV, j < hi[k] - 1, 4 * half, 4 * half + 4);
           }
           if (!ok) break;
           ++np[k];
-          if (j + 1 < hi[k]) {
-            const int rK2 = rK + 2;
+          if (j - 1 >= lo[k]) {
+            const int rK2 = rK + 2;  // K_{j-1}
             if (!next_k_ready) {
               if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status,
                              kStatusFwdTimeout, kWaitTimeoutNs)) {
@@ -349,7 +352,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     bool ok = true;
     int n = 0;
-    for (int j = lo[k]; j < hi[k]; ++j, ++n) {
+    // Key tiles from last to first: with alibi the bias grows with the key index, so the
+    // row maximum is met on the first tile and the lazy rescale of O almost never runs.
+    for (int j = hi[k] - 1; j >= lo[k]; --j, ++n) {
       // Warp-uniform decision: the TMEM loads below are warp-collective.
       const bool got = mbar_wait(bar_s(k), static_cast<uint32_t>(n) & 1u, p.status, kStatusFwdTimeout,
                                  kWaitTimeoutNs) &&
