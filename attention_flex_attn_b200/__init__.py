@@ -26,8 +26,8 @@ FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
 EXPORTED = ["flex_attn_fwd", "flex_attn_decode_workspace_size", "flex_attn_decode",
-            "flex_attn_decode_noalloc", "flex_attn_mask_eval", "flex_attn_tile_sizes", "flex_attn_device_status",
-            "flex_status_string"]
+            "flex_attn_decode_noalloc", "flex_attn_mask_eval", "flex_attn_selftest_wait_timeout",
+            "flex_attn_tile_sizes", "flex_attn_device_status", "flex_status_string"]
 
 
 class FlexAttnError(RuntimeError):
@@ -61,6 +61,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_decode_noalloc.restype = I
     lib.flex_attn_mask_eval.argtypes = [I, ctypes.POINTER(ModParams), I, I, P, P]
     lib.flex_attn_mask_eval.restype = I
+    lib.flex_attn_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
+    lib.flex_attn_selftest_wait_timeout.restype = I
     lib.flex_attn_tile_sizes.argtypes = [I, ctypes.POINTER(I), ctypes.POINTER(I)]
     lib.flex_attn_tile_sizes.restype = None
     lib.flex_attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I]
@@ -193,6 +195,14 @@ def mask_eval(mask_mod, Sq, Skv, window=0, offset=0, device="cuda"):
     rc = lib.flex_attn_mask_eval(MASK_MODS[mask_mod], ctypes.byref(mp), Sq, Skv, _ptr(keep), _stream(keep.device))
     _check(rc, "flex_attn_mask_eval")
     return keep
+
+
+def selftest_wait_timeout(timeout_us: int, device="cuda"):
+    """Runs the failure-detection self-test (a bounded wait on a barrier nothing arrives
+    on); afterwards device_status() has bit 8 set."""
+    lib = load_library()
+    dev = torch.device(device)
+    _check(lib.flex_attn_selftest_wait_timeout(int(timeout_us), _stream(dev)), "flex_attn_selftest_wait_timeout")
 
 
 def device_status(reset: bool = True) -> int:

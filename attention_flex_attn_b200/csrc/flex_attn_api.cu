@@ -165,14 +165,36 @@ flex_status_t launch_decode(const DecodeParams& p, cudaStream_t s) {
 }
 
 template <int D, typename T>
+flex_status_t launch_decode_gqa(const DecodeParams& p, cudaStream_t s) {
+  dim3 grid(p.n_splits, p.B * p.Hkv * ((p.G + kGqaRows - 1) / kGqaRows));
+  decode_gqa_kernel<D, T><<<grid, kDecThreads, 0, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FLEX_ERR_CUDA;
+  const int rows = p.B * p.H;
+  decode_combine_kernel<D, T><<<(rows + kDecWarps - 1) / kDecWarps, kDecThreads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
+}
+
+// One query head per kv head streams on CUDA cores; grouped heads go to the tensor-core
+// kernel, whose work per byte does not grow with the group size.
+template <int D, typename T>
 flex_status_t decode_by_group(const DecodeParams& p, cudaStream_t s) {
-  if (p.G % 8 == 0) return launch_decode<D, T, 8>(p, s);
-  if (p.G % 4 == 0) return launch_decode<D, T, 4>(p, s);
-  if (p.G % 2 == 0) return launch_decode<D, T, 2>(p, s);
+  if (p.G >= 2) return launch_decode_gqa<D, T>(p, s);
   return launch_decode<D, T, 1>(p, s);
 }
 
 int decode_splits(int cap) { return (cap + kChunk - 1) / kChunk; }
+
+constexpr unsigned kStatusSelftestTimeout = 8u;
+
+// One thread waits on a barrier that nothing arrives on, with the bounded wait the
+// kernels use; the wait must give up, set the status bit and let the kernel end.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned* status) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  fence_barrier_init();
+  mbar_wait(b, 0, status, kStatusSelftestTimeout, timeout_ns);
+}
 
 }  // namespace
 }  // namespace flexattn
@@ -290,7 +312,7 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
   p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((o_bytes + 255) & ~static_cast<size_t>(255)));
   p.status = st;
   p.scale_log2 = scale * kLog2e;
-  const int grid_y = B * Hkv * (p.G / (p.G % 8 == 0 ? 8 : p.G % 4 == 0 ? 4 : p.G % 2 == 0 ? 2 : 1));
+  const int64_t grid_y = static_cast<int64_t>(B) * Hkv * (p.G >= 2 ? (p.G + kGqaRows - 1) / kGqaRows : 1);
   if (grid_y > 65535) return FLEX_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (D == 128)
@@ -331,6 +353,15 @@ flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_
     case FLEX_MASK_KV_LE_Q_PLUS_OFFSET: mask_eval_kernel<kMaskOffset><<<grid, 256, 0, s>>>(m, Sq, Skv, keep); break;
     default: return FLEX_ERR_INVALID_ARG;
   }
+  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
+}
+
+flex_status_t flex_attn_selftest_wait_timeout(uint32_t timeout_us, flex_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 2000000u) return FLEX_ERR_INVALID_ARG;
+  unsigned* st = status_ptr();
+  if (!st) return FLEX_ERR_CUDA;
+  selftest_wait_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull, st);
   return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
 }
 

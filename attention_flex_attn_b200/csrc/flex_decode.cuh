@@ -18,6 +18,7 @@
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx_sm100.cuh"
 
@@ -239,6 +240,242 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
     const int64_t row = static_cast<int64_t>(b) * p.H + h0 + g;
     p.part_o[(row * p.n_splits + split) * D + d] = l > 0.f ? x / l : 0.f;
     if (d == 0) p.part_lse[row * p.n_splits + split] = l > 0.f ? s_m[g] + lg2_approx(l) : -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Grouped-query decode (G = H / Hkv >= 2): the G query heads of one kv head share every
+// K/V byte, so the per-byte arithmetic grows with G.  This kernel puts up to 16 heads in
+// the 16 rows of warp-level tensor-core MMAs (mma.sync m16n8k16, fp32 accumulate), which
+// makes the arithmetic per byte independent of G and leaves the kernel bound by HBM.
+// Each warp owns 64 keys of the 256-key chunk:
+//  * S = Q K^T: K rows are loaded straight into B fragments, 16 bytes per lane.  Within
+//    each 32-wide slice of the head dimension the contraction index is permuted the same
+//    way in the Q (A) and K (B) fragments, so each lane reads 8 consecutive elements.
+//  * the warp-local softmax works on the accumulator fragments; P is repacked in
+//    registers as the A fragment of P V (the accumulator layout of S over two 8-key
+//    tiles is the A layout of one 16-key step).
+//  * V rows are loaded 16 bytes per lane and transposed in registers with movmatrix into
+//    B fragments; this permutes the head dimension of O, which is undone on the store.
+// The four warps' partial results are merged through shared memory into one (O, LSE)
+// partial per chunk, in the same workspace format as decode_split_kernel.
+constexpr int kGqaRows = 16;
+constexpr int kGqaKeysPerWarp = kChunk / kDecWarps;  // 64
+
+template <typename T>
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack_pair(float lo, float hi) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+__device__ __forceinline__ uint32_t u4_at(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const DecodeParams p) {
+  constexpr int KC = D / 32;  // 32-wide slices of the head dimension
+  __shared__ float s_m[kDecWarps][kGqaRows], s_l[kDecWarps][kGqaRows];
+  __shared__ __align__(16) float s_o[kDecWarps][kGqaRows][D];
+
+  const int split = blockIdx.x;
+  const int ngrp = (p.G + kGqaRows - 1) / kGqaRows;
+  const int grp = blockIdx.y % ngrp;
+  const int bk = blockIdx.y / ngrp;
+  const int hkv = bk % p.Hkv;
+  const int b = bk / p.Hkv;
+  const int h0 = hkv * p.G + grp * kGqaRows;
+  const int gt = min(kGqaRows, p.G - grp * kGqaRows);  // valid MMA rows (query heads)
+
+  const int L = checked_len(p, b);
+  const int j0 = split * kChunk;
+  if (L <= 0 || j0 >= L) return;
+  const int n = min(kChunk, L - j0);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int kw0 = warp * kGqaKeysPerWarp;
+  const T* kbase = reinterpret_cast<const T*>(p.k) + ((static_cast<int64_t>(b) * p.Hkv + hkv) * p.cap + j0) * D;
+  const T* vbase = reinterpret_cast<const T*>(p.v) + ((static_cast<int64_t>(b) * p.Hkv + hkv) * p.cap + j0) * D;
+
+  // Q fragments: rows g and g + 8, head-dimension elements 32c + 8q .. 32c + 8q + 7.
+  uint4 qa[KC][2];
+#pragma unroll
+  for (int c = 0; c < KC; ++c)
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = g + 8 * hr;
+      qa[c][hr] = row < gt ? *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
+                                                             (static_cast<int64_t>(b) * p.H + h0 + row) * D + 32 * c + 8 * q)
+                           : make_uint4(0, 0, 0, 0);
+    }
+
+  // ---- S = Q K^T over this warp's 64 keys (8 tiles of 8 keys)
+  float sc[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; nt += 2) {
+    uint4 kr[2][KC];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int key = kw0 + (nt + t) * 8 + g;
+#pragma unroll
+      for (int c = 0; c < KC; ++c)
+        kr[t][c] = key < n ? ldg_nc_v4(kbase + static_cast<int64_t>(key) * D + 32 * c + 8 * q) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < KC; ++c)
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+          const uint32_t a[4] = {u4_at(qa[c][0], 2 * sub), u4_at(qa[c][1], 2 * sub), u4_at(qa[c][0], 2 * sub + 1),
+                                 u4_at(qa[c][1], 2 * sub + 1)};
+          mma16816<T>(acc, a, u4_at(kr[t][c], 2 * sub), u4_at(kr[t][c], 2 * sub + 1));
+        }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt + t][e] = acc[e];
+    }
+  }
+
+  // ---- scale (base 2), padding, additive mask; warp-local softmax per row
+  const T* mrow0 = nullptr;
+  const T* mrow1 = nullptr;
+  if (p.mask != nullptr) {
+    if (g < gt) mrow0 = reinterpret_cast<const T*>(p.mask) + (static_cast<int64_t>(b) * p.H + h0 + g) * p.cap + j0;
+    if (g + 8 < gt) mrow1 = reinterpret_cast<const T*>(p.mask) + (static_cast<int64_t>(b) * p.H + h0 + g + 8) * p.cap + j0;
+  }
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = kw0 + nt * 8 + 2 * q + (e & 1);
+      const bool upper = e >= 2;
+      const int row = g + 8 * (upper ? 1 : 0);
+      float x = -INFINITY;
+      if (key < n && row < gt) {
+        x = sc[nt][e] * p.scale_log2;
+        const T* mr = upper ? mrow1 : mrow0;
+        if (mr) x += to_float(mr[key]) * kDecLog2e;
+      }
+      sc[nt][e] = x;
+      if (upper) m1 = fmaxf(m1, x);
+      else m0 = fmaxf(m0, x);
+    }
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+  }
+  const float ms0 = m0 == -INFINITY ? 0.f : m0, ms1 = m1 == -INFINITY ? 0.f : m1;
+  float l0 = 0.f, l1 = 0.f;
+  uint32_t pa[4][4];  // A fragments of P for the four 16-key steps
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+    const float p0 = ex2_approx(sc[nt][0] - ms0), p1 = ex2_approx(sc[nt][1] - ms0);
+    const float p2 = ex2_approx(sc[nt][2] - ms1), p3 = ex2_approx(sc[nt][3] - ms1);
+    l0 += p0 + p1;
+    l1 += p2 + p3;
+    pa[nt >> 1][(nt & 1) * 2 + 0] = pack_pair<T>(p0, p1);
+    pa[nt >> 1][(nt & 1) * 2 + 1] = pack_pair<T>(p2, p3);
+  }
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+
+  // ---- O = P V: per 16-key step and 32-wide slice, two 16-byte loads and 8 transposes
+  float o[KC][4][4];
+#pragma unroll
+  for (int c = 0; c < KC; ++c)
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[c][r][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    const int keyA = kw0 + 16 * ks + g, keyB = keyA + 8;
+    uint4 va[KC], vb[KC];
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      va[c] = keyA < n ? ldg_nc_v4(vbase + static_cast<int64_t>(keyA) * D + 32 * c + 8 * q) : make_uint4(0, 0, 0, 0);
+      vb[c] = keyB < n ? ldg_nc_v4(vbase + static_cast<int64_t>(keyB) * D + 32 * c + 8 * q) : make_uint4(0, 0, 0, 0);
+    }
+    // A fragment rows g / g+8, k = 2q, 2q+1 (keys 16ks + 2q..) and 2q+8, 2q+9 (keys 16ks + 8 + 2q..)
+    const uint32_t a[4] = {pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3]};
+#pragma unroll
+    for (int c = 0; c < KC; ++c)
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        mma16816<T>(o[c][r], a, transpose8x8(u4_at(va[c], r)), transpose8x8(u4_at(vb[c], r)));
+  }
+
+  // ---- merge the four warps (each relative to its own row max) into one chunk partial
+  if (q == 0) {
+    s_m[warp][g] = m0;
+    s_m[warp][g + 8] = m1;
+    s_l[warp][g] = l0;
+    s_l[warp][g + 8] = l1;
+  }
+  // o[c][r][0..1] hold rows g, o[c][r][2..3] row g + 8, head-dim 32c + 8q + 2r + {0, 1}
+#pragma unroll
+  for (int c = 0; c < KC; ++c)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int d = 32 * c + 8 * q + 2 * r;
+      *reinterpret_cast<float2*>(&s_o[warp][g][d]) = make_float2(o[c][r][0], o[c][r][1]);
+      *reinterpret_cast<float2*>(&s_o[warp][g + 8][d]) = make_float2(o[c][r][2], o[c][r][3]);
+    }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < gt * D; idx += kDecThreads) {
+    const int row = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, s_m[w][row]);
+    float acc = 0.f, wsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float mw = s_m[w][row];
+        if (mw == -INFINITY) continue;
+        const float f = ex2_approx(mw - M);
+        wsum = fmaf(f, s_l[w][row], wsum);
+        acc = fmaf(f, s_o[w][row][d], acc);
+      }
+    }
+    const int64_t grow = static_cast<int64_t>(b) * p.H + h0 + row;
+    p.part_o[(grow * p.n_splits + split) * D + d] = wsum > 0.f ? acc / wsum : 0.f;
+    if (d == 0) p.part_lse[grow * p.n_splits + split] = wsum > 0.f ? M + lg2_approx(wsum) : -INFINITY;
   }
 }
 

@@ -171,6 +171,16 @@ flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const
 flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_params,
                                   int Sq, int Skv, uint8_t* keep, flex_stream_t stream);
 
+/*
+ * flex_attn_selftest_wait_timeout -- failure-detection self-test (no counterpart on the
+ * source pages).  Launches one thread that waits, with the same bounded mbarrier wait the
+ * forward kernel uses, on a barrier nothing ever arrives on; after timeout_us
+ * microseconds (1 .. 2,000,000) the wait gives up and sets status bit 8.  Shows that an
+ * expired wait ends the kernel normally, reports through the status word, and leaves the
+ * context usable.  Asynchronous on `stream`.
+ */
+flex_status_t flex_attn_selftest_wait_timeout(uint32_t timeout_us, flex_stream_t stream);
+
 /* flex_attn_tile_sizes -- the (BM, BN) tile geometry the forward kernel uses for D. */
 void flex_attn_tile_sizes(int D, int* bm, int* bn);
 
@@ -178,7 +188,7 @@ void flex_attn_tile_sizes(int D, int* bm, int* bn);
  * flex_attn_device_status -- reads (and, if reset != 0, clears) the device status
  * word on the current device.  Synchronises the device.  Bits:
  *   1 = a decode kv_len outside [0, cap];  2 = a forward-kernel wait ran out of time;
- *   4 = a decode-kernel wait ran out of time.
+ *   4 = a decode-kernel wait ran out of time;  8 = the self-test wait ran out (expected).
  */
 flex_status_t flex_attn_device_status(uint32_t* status_out, int reset);
 

@@ -38,23 +38,34 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def _bind(lib):
+    P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    lib.oracle_fwd.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, I64, P, P, P, I]
+    lib.oracle_fwd.restype = I
+    lib.oracle_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P, I]
+    lib.oracle_decode.restype = I
+    lib.oracle_mask_matrix.argtypes = [I, I, I, I, I, P]
+    lib.oracle_mask_matrix.restype = I
+    lib.oracle_tile_map.argtypes = [I, I, I, I, I, I, I, P]
+    lib.oracle_tile_map.restype = I
+    lib.oracle_alibi_slope.argtypes = [I, I]
+    lib.oracle_alibi_slope.restype = D
+    return lib
+
+
+def use_library(path=None):
+    """Test hook: route the wrappers through another build of flex_oracle.c (for the
+    mutation test of the pins); path None goes back to the normal build."""
+    global _lib
+    _lib = None if path is None else _bind(ctypes.CDLL(path))
+
+
 def _load():
     global _lib
     if _lib is None:
         build()
         lib = ctypes.CDLL(_LIB)
-        P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
-        lib.oracle_fwd.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, I64, P, P, P, I]
-        lib.oracle_fwd.restype = I
-        lib.oracle_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P, I]
-        lib.oracle_decode.restype = I
-        lib.oracle_mask_matrix.argtypes = [I, I, I, I, I, P]
-        lib.oracle_mask_matrix.restype = I
-        lib.oracle_tile_map.argtypes = [I, I, I, I, I, I, I, P]
-        lib.oracle_tile_map.restype = I
-        lib.oracle_alibi_slope.argtypes = [I, I]
-        lib.oracle_alibi_slope.restype = D
-        _lib = lib
+        _lib = _bind(lib)
     return _lib
 
 

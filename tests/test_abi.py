@@ -109,3 +109,8 @@ def test_static_scratch_limit_matches_header():
     m = re.search(r"#define FLEX_DECODE_STATIC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", txt)
     assert m, "FLEX_DECODE_STATIC_SCRATCH_BYTES not found"
     assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == fa.DECODE_STATIC_SCRATCH_BYTES
+
+
+def test_selftest_rejects_bad_timeouts(lib):
+    assert lib.flex_attn_selftest_wait_timeout(0, None) == 1
+    assert lib.flex_attn_selftest_wait_timeout(2000001, None) == 1

@@ -59,7 +59,7 @@ def test_decode_split_boundaries(lens, D, dtype):
     _check(*args)
 
 
-@pytest.mark.parametrize("H,Hkv", [(6, 2), (12, 4), (5, 5), (16, 2)])
+@pytest.mark.parametrize("H,Hkv", [(6, 2), (12, 4), (5, 5), (16, 2), (32, 2), (40, 2), (64, 4)])
 def test_decode_group_sizes(H, Hkv):
     args = _inputs(3, H, Hkv, 700, 128, seed=3300 + H, mask_p=0.3)
     _check(*args)
