@@ -40,12 +40,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 MEASURED_TRAFFIC = {
     # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 403,697,408 B read +
     # 114,692,864 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
-    "627e09257dec1da2": 518390272,
+    "1d7a0e1b91413d40": 518390272,
 }
+# the forward kernel's sources: the roofline traffic below belongs to that kernel
 KERNEL_SOURCES = ["attention_flex_attn_b200/csrc/flex_fwd_sm100.cuh",
                   "attention_flex_attn_b200/csrc/ptx_sm100.cuh",
-                  "attention_flex_attn_b200/csrc/mask_rules.cuh",
-                  "attention_flex_attn_b200/csrc/flex_decode.cuh"]
+                  "attention_flex_attn_b200/csrc/mask_rules.cuh"]
 
 
 def kernel_hash() -> str:
