@@ -479,7 +479,10 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const Decode
   }
 }
 
-// One warp per (b, h) row: merge the chunks written by decode_split_kernel.
+// One warp per (b, h) row: merge the chunks written by the split kernels.  Lane s holds the
+// log-sum-exp of chunk s (chunks beyond 32 are folded in a second round), the weights
+// 2^(lse_s - lse) are broadcast by shuffle, and the partial outputs of eight chunks are
+// loaded at a time so their latencies overlap.
 template <int D, typename T>
 __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const DecodeParams p) {
   constexpr int PER = D / 32;
@@ -503,14 +506,30 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const Decod
   for (int e = 0; e < PER; ++e) o[e] = 0.f;
   float W = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < ns; ++s) {
-      const float ls = plse[s];
-      if (ls == -INFINITY) continue;
-      const float w = ex2_approx(ls - M);
-      W += w;
-      const float* po = p.part_o + (static_cast<int64_t>(row) * p.n_splits + s) * D + lane * PER;
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+      // weight of chunk s0 + lane (0 for empty or missing chunks)
+      const int sl = s0 + lane;
+      const float ls = sl < ns ? plse[sl] : -INFINITY;
+      const float wl = ls == -INFINITY ? 0.f : ex2_approx(ls - M);
+      float wsum = wl;
 #pragma unroll
-      for (int e = 0; e < PER; ++e) o[e] = fmaf(w, po[e], o[e]);
+      for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+      W += wsum;
+      const int cnt = min(32, ns - s0);
+      const float* po = p.part_o + (static_cast<int64_t>(row) * p.n_splits + s0) * D + lane * PER;
+      for (int t0 = 0; t0 < cnt; t0 += 8) {
+        float v[8][PER];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+#pragma unroll
+          for (int e = 0; e < PER; ++e) v[t][e] = t0 + t < cnt ? po[(t0 + t) * D + e] : 0.f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float w = __shfl_sync(0xffffffffu, wl, (t0 + t) & 31);
+#pragma unroll
+          for (int e = 0; e < PER; ++e) o[e] = fmaf(w, v[t][e], o[e]);
+        }
+      }
     }
   }
   T* out = reinterpret_cast<T*>(p.o) + static_cast<int64_t>(row) * D + lane * PER;
