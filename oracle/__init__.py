@@ -6,8 +6,8 @@ with the CUDA library: ``flex_oracle.c`` restates the method from its
 definition (see the header of that file for the formulas and their sources).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-(closed forms, library special cases, exact identities, hand-worked golden
-values); nothing is "parity unpinned".
+and ``tests/test_oracle_block_pins.py`` (closed forms, library special cases,
+exact identities, hand-worked golden values); nothing is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -50,6 +50,9 @@ def _bind(lib):
     lib.oracle_tile_map.restype = I
     lib.oracle_alibi_slope.argtypes = [I, I]
     lib.oracle_alibi_slope.restype = D
+    lib.oracle_fwd_block_sparse.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, P, I, I, I,
+                                            P, I64, P, P, I]
+    lib.oracle_fwd_block_sparse.restype = I
     return lib
 
 
@@ -129,6 +132,83 @@ def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset
         if probs is not None:
             probs = probs.reshape(B, H, Sq, Skv)
     return (o, lse, probs) if want_probs else (o, lse)
+
+
+def _i32(a):
+    if a is None:
+        return None
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def fwd_block_sparse(q, k, v, kv_num, kv_idx, full_num=None, full_idx=None, scale=None,
+                     score_mod="none", mask_mod="none", window=0, offset=0, bm=128, bn=128,
+                     rows=None, threads=None):
+    """Oracle forward with a block mask (BlockMask: FlyDSL PR 931 "Add flex_attention
+    (score_mod / mask_mod) ...", Out of scope, names block sparsity as the next phase;
+    the list convention is PyTorch's).
+
+    kv_num / full_num: [Bm, Hm, ceil(Sq/bm)] int32 block counts; kv_idx / full_idx:
+    [Bm, Hm, ceil(Sq/bm), max_blocks] int32 key-block indices; Bm in {1, B} and Hm in
+    {1, H} broadcast like numpy.  Either pair may be None (no blocks of that kind).
+    Key j of query row i is kept iff j < Skv and its block j // bn is listed as full
+    for the tile i // bm, or listed as partial and mask_mod(i, j) holds.  A count is
+    clamped to [0, max_blocks]; an index outside [0, ceil(Skv/bn)) names no block.
+    Returns (O, LSE) like fwd()."""
+    lib = _load()
+    B, H, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    nq = -(-Sq // bm)
+    kn, ki, fn, fi = _i32(kv_num), _i32(kv_idx), _i32(full_num), _i32(full_idx)
+    if kn is None and fn is None:
+        raise ValueError("a block mask needs at least one of the partial / full lists")
+    max_blocks = (ki if ki is not None else fi).shape[-1]
+
+    def expand(a, tail):
+        return None if a is None else np.ascontiguousarray(np.broadcast_to(a, (B, H, nq) + tail))
+    kn, fn = expand(kn, ()), expand(fn, ())
+    ki, fi = expand(ki, (max_blocks,)), expand(fi, (max_blocks,))
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    if rows is None:
+        n, rows_arr = B * H * Sq, None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n = int(rows_arr.size)
+    o = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    ptr = lambda a: None if a is None else a.ctypes.data
+    rc = lib.oracle_fwd_block_sparse(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, _dtype_code(q),
+                                     B, H, Hkv, Sq, Skv, D, float(scale), SCORE_MODS[score_mod],
+                                     MASK_MODS[mask_mod], int(window), int(offset),
+                                     ptr(kn), ptr(ki), ptr(fn), ptr(fi), int(max_blocks), int(bm), int(bn),
+                                     None if rows_arr is None else rows_arr.ctypes.data, n,
+                                     o.ctypes.data, lse.ctypes.data, int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_fwd_block_sparse rejected its arguments (rc={rc})")
+    if rows is None:
+        return o.reshape(B, H, Sq, D), lse.reshape(B, H, Sq)
+    return o, lse
+
+
+def block_mask_from_tile_map(tmap, B, H, max_blocks=None):
+    """Partial/full block lists that reproduce a tile map (2 -> partial, 1 -> full)."""
+    nq, nk = tmap.shape
+    mb = max_blocks or nk
+    kv_num = np.zeros((B, H, nq), np.int32)
+    kv_idx = np.zeros((B, H, nq, mb), np.int32)
+    full_num = np.zeros((B, H, nq), np.int32)
+    full_idx = np.zeros((B, H, nq, mb), np.int32)
+    for t in range(nq):
+        part = [u for u in range(nk) if tmap[t, u] == 2]
+        full = [u for u in range(nk) if tmap[t, u] == 1]
+        kv_num[:, :, t] = len(part)
+        kv_idx[:, :, t, :len(part)] = part
+        full_num[:, :, t] = len(full)
+        full_idx[:, :, t, :len(full)] = full
+    return kv_num, kv_idx, full_num, full_idx
 
 
 def decode(q, k_cache, v_cache, kv_len, scale, mask=None, threads=None):

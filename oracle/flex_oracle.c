@@ -34,6 +34,13 @@
  * f16 additive mask operand): x_j = scale * q.k_j + mask[b,h,j] for j < kv_len[b];
  * keep_j = (x_j != -inf); then the same softmax as above.
  *
+ * Block-sparse forward (BlockMask; FlyDSL PR 931, "Out of scope (future phases)":
+ * block sparsity named as the next phase, with no definition given).  Reading: the
+ * PyTorch BlockMask convention.  For query tile t = i / BM of (b, h), a key j with
+ * block u = j / BN is kept iff j < Skv and (u is in the full list of t, or u is in
+ * the partial list of t and mask_mod(i, j) holds).  Unlisted blocks are dropped.
+ * Everything else (scale, score_mod, softmax, 0/-inf rows) is the forward above.
+ *
  * Tile map: for a BM x BN grid over (query, key) positions, a tile is
  *   EMPTY(0)   if no element with i < Sq has keep && j < Skv,
  *   FULL(1)    if every element with i < Sq has keep && j < Skv,
@@ -102,6 +109,36 @@ int oracle_mask_keep(int mask_mod, int64_t i, int64_t j, int window, int offset)
   }
 }
 
+/* Block mask (BlockMask).  Reading: PyTorch's convention.  For query tile t of one
+ * (b, h) (tile_row = (b*H + h) * n_qtiles + t), the key blocks u listed in
+ * full_idx[tile_row, 0 .. full_num) are kept wholesale (only j < Skv applies), those in
+ * kv_idx[tile_row, 0 .. kv_num) keep (i, j) iff mask_mod(i, j) && j < Skv, and every
+ * other block is dropped.  A block on both lists counts as full.  Counts are clamped
+ * to [0, max_blocks]; an index outside [0, ceil(Skv/BN)) matches no key. */
+typedef struct {
+  const int32_t *kv_num, *kv_idx, *full_num, *full_idx;
+  int max_blocks, BM, BN, n_qtiles;
+} block_lists;
+
+static int block_listed(const int32_t* num, const int32_t* idx, int64_t row, int max_blocks, int64_t u) {
+  if (!num || !idx) return 0;
+  int32_t cnt = num[row];
+  if (cnt > max_blocks) cnt = max_blocks;
+  for (int32_t c = 0; c < cnt; ++c)
+    if ((int64_t)idx[row * max_blocks + c] == u) return 1;
+  return 0;
+}
+
+static int block_keep(const block_lists* L, int64_t bh, int mask_mod, int64_t i, int64_t j, int Skv,
+                      int window, int offset) {
+  if (j >= Skv) return 0;
+  int64_t tile_row = bh * L->n_qtiles + i / L->BM;
+  int64_t u = j / L->BN;
+  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;
+  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return oracle_mask_keep(mask_mod, i, j, window, offset);
+  return 0;
+}
+
 /* ---- forward -------------------------------------------------------------- */
 
 typedef struct {
@@ -114,6 +151,7 @@ typedef struct {
   double* o;             /* [n_rows, D] */
   double* lse;           /* [n_rows] */
   double* probs;         /* optional [n_rows, Skv] normalised weights */
+  const block_lists* blk; /* block mask, or NULL for mask_mod alone */
   int64_t r0, r1;
 } fwd_job;
 
@@ -139,7 +177,8 @@ static void fwd_row(const fwd_job* J, int64_t r, double* x, unsigned char* keep)
     double s = J->scale * dot;
     if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);
     x[j] = s;
-    keep[j] = (unsigned char)oracle_mask_keep(J->mask_mod, i, j, J->window, J->offset);
+    keep[j] = (unsigned char)(J->blk ? block_keep(J->blk, bh, J->mask_mod, i, j, J->Skv, J->window, J->offset)
+                                     : oracle_mask_keep(J->mask_mod, i, j, J->window, J->offset));
     if (keep[j]) {
       any = 1;
       if (s > M) M = s;
@@ -311,6 +350,32 @@ int oracle_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
   free(jobs);
   free(th);
   return 0;
+}
+
+/* Block-sparse forward over selected rows: the forward above with the keep rule of the
+ * block lists.  kv_num/full_num are [B*H*n_qtiles] and kv_idx/full_idx
+ * [B*H*n_qtiles*max_blocks] int32, n_qtiles = ceil(Sq/BM); either pair may be NULL. */
+int oracle_fwd_block_sparse(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dtype,
+                            int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
+                            int score_mod, int mask_mod, int window, int offset,
+                            const int32_t* kv_num, const int32_t* kv_idx, const int32_t* full_num,
+                            const int32_t* full_idx, int max_blocks, int BM, int BN,
+                            const int64_t* rows, int64_t n_rows, double* o, double* lse, int nthreads) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv != 0 || Sq <= 0 || Skv <= 0 || D <= 0) return -1;
+  if (BM <= 0 || BN <= 0 || max_blocks < 0) return -1;
+  block_lists L;
+  L.kv_num = kv_num; L.kv_idx = kv_idx; L.full_num = full_num; L.full_idx = full_idx;
+  L.max_blocks = max_blocks; L.BM = BM; L.BN = BN; L.n_qtiles = (Sq + BM - 1) / BM;
+  fwd_job J;
+  memset(&J, 0, sizeof J);
+  J.q = q; J.k = k; J.v = v; J.dtype = dtype;
+  J.B = B; J.H = H; J.Hkv = Hkv; J.Sq = Sq; J.Skv = Skv; J.D = D;
+  J.scale = scale; J.score_mod = score_mod; J.mask_mod = mask_mod;
+  J.window = window; J.offset = offset;
+  J.rows = rows;
+  J.n_rows = rows ? n_rows : (int64_t)B * H * Sq;
+  J.o = o; J.lse = lse; J.blk = &L;
+  return run_jobs(&J, J.n_rows, nthreads, fwd_worker, sizeof J);
 }
 
 /* ---- element mask and tile map (brute force) ------------------------------- */

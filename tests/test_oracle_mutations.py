@@ -1,5 +1,5 @@
 """Plants plausible mistakes in copies of the C oracle and checks that the pins in
-test_oracle_pins.py catch every one (each mutant must fail at least one pin).
+test_oracle_pins.py and test_oracle_block_pins.py catch every one (each mutant must fail at least one pin).
 Everything runs on the CPU against a temporary build; the real oracle is untouched.
 Mutants that leave the mathematics unchanged (e.g. dropping the fully-masked guard,
 which still yields p = 0 and log 0 = -inf) are not listed: no test could tell them apart."""
@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import oracle
+import tests.test_oracle_block_pins as bpins
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "flex_oracle.c")
@@ -40,6 +41,12 @@ MUTANTS = [
      "  if (M == -INFINITY) {   /* kv_len == 0 or every position masked */\n    J->lse[r] = 0.0;"),
     ("tile classes swapped", "(kept == total ? 1 : 2)", "(kept == total ? 2 : 1)"),
     ("tile ignores pad", "if (j < Skv && oracle_mask_keep(", "if (oracle_mask_keep("),
+    ("block: full list ignored", "  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;\n", ""),
+    ("block: partial skips mask_mod", "u)) return oracle_mask_keep(mask_mod, i, j, window, offset);", "u)) return 1;"),
+    ("block: partial beats full",
+     "  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;\n  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return oracle_mask_keep(mask_mod, i, j, window, offset);",
+     "  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return oracle_mask_keep(mask_mod, i, j, window, offset);\n  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;"),
+    ("block: query tile from BN", "int64_t tile_row = bh * L->n_qtiles + i / L->BM;", "int64_t tile_row = bh * L->n_qtiles + i / L->BN;"),
     ("bf16 decoded as truncated", "  uint32_t u = ((uint32_t)b) << 16;", "  uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
 ]
 
@@ -64,6 +71,12 @@ CHECKS = [
     (pins.test_decode_finite_mask_added_after_scale, {"L": 7}),
     (pins.test_tile_map_closed_forms, {}),
     (pins.test_mask_matrix_counts, {}),
+    (bpins.test_block_sparse_equals_dense_masked_softmax, {"mask": "causal", "window": 0, "offset": 0, "score": "none"}),
+    (bpins.test_block_sparse_equals_dense_masked_softmax, {"mask": "sliding_window", "window": 6, "offset": 0,
+                                                            "score": "alibi"}),
+    (bpins.test_full_block_beats_partial_and_ignores_mask_mod, {}),
+    (bpins.test_every_block_full_equals_no_mask, {}),
+    (bpins.test_empty_block_mask_gives_zero_rows, {}),
 ]
 
 
