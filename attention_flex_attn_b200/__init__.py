@@ -25,7 +25,7 @@ MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset":
 FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
-EXPORTED = ["flex_attn_fwd", "flex_attn_decode_workspace_size", "flex_attn_decode",
+EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_decode_workspace_size", "flex_attn_decode",
             "flex_attn_decode_noalloc", "flex_attn_mask_eval", "flex_attn_selftest_wait_timeout",
             "flex_attn_tile_sizes", "flex_attn_device_status", "flex_status_string"]
 
@@ -37,6 +37,14 @@ class FlexAttnError(RuntimeError):
 class ModParams(ctypes.Structure):
     _fields_ = [("window", ctypes.c_int32), ("offset", ctypes.c_int32),
                 ("flags", ctypes.c_uint32), ("tile_map_out", ctypes.c_void_p)]
+
+
+class BlockMaskC(ctypes.Structure):
+    """flex_block_mask_t of include/flex_attn.h."""
+    _fields_ = [("kv_num_blocks", ctypes.c_void_p), ("kv_indices", ctypes.c_void_p),
+                ("full_kv_num_blocks", ctypes.c_void_p), ("full_kv_indices", ctypes.c_void_p),
+                ("max_blocks", ctypes.c_int32), ("batch", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("q_block_size", ctypes.c_int32), ("kv_block_size", ctypes.c_int32)]
 
 
 _lib = None
@@ -53,6 +61,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.flex_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams), I, P]
     lib.flex_attn_fwd.restype = I
+    lib.flex_attn_fwd_block_sparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams),
+                                               ctypes.POINTER(BlockMaskC), I, P]
+    lib.flex_attn_fwd_block_sparse.restype = I
     lib.flex_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.flex_attn_decode_workspace_size.restype = SZ
     lib.flex_attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, P]
@@ -100,15 +111,7 @@ def tile_sizes(D: int = 128):
     return bm.value, bn.value
 
 
-def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
-        return_lse=True, out=None, lse_out=None, tile_map=None):
-    """Flex-attention forward.  q [B,H,Sq,D], k/v [B,Hkv,Skv,D] (bf16 or f16, CUDA).
-
-    Returns (O, LSE) (LSE is None when return_lse is False).  ``tile_map``: optional
-    uint8 CUDA tensor of ceil(Sq/BM)*ceil(Skv/BN) bytes that receives the tile classes
-    of batch 0 / head 0.
-    """
-    lib = load_library()
+def _fwd_args(q, k, v, scale, return_lse, out, lse_out):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _cuda_tensor(t, n)
     B, H, Sq, D = q.shape
@@ -123,12 +126,65 @@ def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset
     lse = None
     if return_lse:
         lse = lse_out if lse_out is not None else torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    return B, H, Hkv, Sq, Skv, D, float(scale), o, lse
+
+
+def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
+        return_lse=True, out=None, lse_out=None, tile_map=None):
+    """Flex-attention forward.  q [B,H,Sq,D], k/v [B,Hkv,Skv,D] (bf16 or f16, CUDA).
+
+    Returns (O, LSE) (LSE is None when return_lse is False).  ``tile_map``: optional
+    uint8 CUDA tensor of ceil(Sq/BM)*ceil(Skv/BN) bytes that receives the tile classes
+    of batch 0 / head 0.
+    """
+    lib = load_library()
+    B, H, Hkv, Sq, Skv, D, scale, o, lse = _fwd_args(q, k, v, scale, return_lse, out, lse_out)
     mp = ModParams(int(window), int(offset), FLAG_TILE_MAP if tile_map is not None else 0,
                    tile_map.data_ptr() if tile_map is not None else None)
     rc = lib.flex_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
-                           float(scale), SCORE_MODS[score_mod], MASK_MODS[mask_mod], ctypes.byref(mp),
+                           scale, SCORE_MODS[score_mod], MASK_MODS[mask_mod], ctypes.byref(mp),
                            DTYPES[q.dtype], _stream(q.device))
     _check(rc, "flex_attn_fwd")
+    return o, lse
+
+
+def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None, full_kv_indices=None,
+                     scale=None, score_mod="none", mask_mod="none", window=0, offset=0, return_lse=True,
+                     out=None, lse_out=None, tile_map=None, block_size=128):
+    """Forward with a block mask (flex_attn_fwd_block_sparse).  The block lists are int32
+    CUDA tensors: counts [Bm, Hm, ceil(Sq/128)], indices [Bm, Hm, ceil(Sq/128), max_blocks],
+    Bm in {1, B}, Hm in {1, H}; either (counts, indices) pair may be None, not both.
+    Partial blocks apply mask_mod, full blocks only the key-length rule."""
+    lib = load_library()
+    B, H, Hkv, Sq, Skv, D, scale, o, lse = _fwd_args(q, k, v, scale, return_lse, out, lse_out)
+    pairs = [(kv_num_blocks, kv_indices, "kv"), (full_kv_num_blocks, full_kv_indices, "full_kv")]
+    shape = None
+    for num, idx, name in pairs:
+        if (num is None) != (idx is None):
+            raise FlexAttnError(f"{name}_num_blocks and {name}_indices go together")
+        if num is None:
+            continue
+        _cuda_tensor(num, f"{name}_num_blocks")
+        _cuda_tensor(idx, f"{name}_indices")
+        if num.dtype != torch.int32 or idx.dtype != torch.int32:
+            raise FlexAttnError("block mask tensors must be int32")
+        if num.dim() != 3 or idx.dim() != 4 or tuple(idx.shape[:3]) != tuple(num.shape):
+            raise FlexAttnError("block mask shapes: counts [Bm, Hm, nq], indices [Bm, Hm, nq, max_blocks]")
+        if shape is not None and tuple(idx.shape) != shape:
+            raise FlexAttnError("partial and full block lists differ in shape")
+        shape = tuple(idx.shape)
+    if shape is None:
+        raise FlexAttnError("a block mask needs the partial or the full lists")
+    bm = BlockMaskC(_ptr(kv_num_blocks), _ptr(kv_indices), _ptr(full_kv_num_blocks), _ptr(full_kv_indices),
+                    shape[3], shape[0], shape[1], int(block_size), int(block_size))
+    if shape[2] != -(-Sq // 128):
+        raise FlexAttnError(f"block mask has {shape[2]} query tiles, Sq={Sq} needs {-(-Sq // 128)}")
+    mp = ModParams(int(window), int(offset), FLAG_TILE_MAP if tile_map is not None else 0,
+                   tile_map.data_ptr() if tile_map is not None else None)
+    rc = lib.flex_attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
+                                        scale, SCORE_MODS[score_mod], MASK_MODS[mask_mod], ctypes.byref(mp),
+                                        ctypes.byref(bm), DTYPES[q.dtype], _stream(q.device))
+    _check(rc, "flex_attn_fwd_block_sparse")
     return o, lse
 
 

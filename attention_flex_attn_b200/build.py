@@ -16,17 +16,18 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libflexattn.so")
-SOURCES = [os.path.join(CSRC, "flex_attn_api.cu")]
+OBJ_DIR = os.path.join(PKG, "_build")
+# Translation units: the forward kernels per (head dim, block mask), decode, and the C ABI.
+# They compile in parallel and link into one shared library.
+SOURCES = [os.path.join(CSRC, f) for f in (
+    "flex_fwd_d128.cu", "flex_fwd_d128_blocks.cu", "flex_fwd_d64.cu", "flex_fwd_d64_blocks.cu",
+    "flex_decode_launch.cu", "flex_attn_api.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, "flex_attn.h")]
 
-NVCC_FLAGS = [
-    "-gencode", "arch=compute_100a,code=sm_100a",
-    "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared",
-    "--expt-relaxed-constexpr",
-    "-cudart", "static",
-]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+COMPILE_FLAGS = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
+LINK_FLAGS = [*ARCH, "-shared", "-cudart", "static"]
 
 
 def nvcc() -> str:
@@ -38,16 +39,24 @@ def stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS)
+    return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS + [os.path.abspath(__file__)])
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if not force and not stale():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp", *SOURCES]
-    if verbose_ptxas:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    subprocess.check_call(cmd)
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(OBJ_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
+        objs.append(obj)
+        cmd = [nvcc(), *COMPILE_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+        procs.append((src, subprocess.Popen(cmd)))
+    failed = [src for src, pr in procs if pr.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, "nvcc " + " ".join(os.path.basename(f) for f in failed))
+    subprocess.check_call([nvcc(), *LINK_FLAGS, "-o", LIB + ".tmp", *objs])
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

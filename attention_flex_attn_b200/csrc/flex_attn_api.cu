@@ -1,6 +1,7 @@
 // flex_attn_api.cu -- the C ABI declared in include/flex_attn.h: host-side argument
-// checks, TMA tensor-map encoding, compile-time dispatch over (head dim, dtype,
-// score_mod, mask_mod), and kernel launches on the caller's stream.
+// checks, TMA tensor-map encoding and the choice of launcher (head dim, block mask);
+// the launchers in flex_fwd_d*.cu and flex_decode_launch.cu dispatch over (dtype,
+// score_mod, mask_mod) and launch on the caller's stream.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -12,8 +13,7 @@
 #include <mutex>
 
 #include "flex_attn.h"
-#include "flex_decode.cuh"
-#include "flex_fwd_sm100.cuh"
+#include "launch.cuh"
 #include "mask_rules.cuh"
 
 namespace flexattn {
@@ -24,6 +24,7 @@ __device__ unsigned int g_status;
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // ---------------------------------------------------------------- tensor maps
 
@@ -55,20 +56,6 @@ bool make_map(CUtensorMap* map, const void* base, flex_dtype_t dt, int D, int ro
   return r == CUDA_SUCCESS;
 }
 
-// Per-device "attribute already set" bits, one set per kernel instantiation (the tag
-// parameters make every forward instantiation own its static).
-template <int D, typename T, int SCORE, int MASK, typename K>
-bool ensure_smem_attr(K kernel, int bytes) {
-  static std::atomic<uint64_t> done{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  const uint64_t bit = 1ull << (dev & 63);
-  if (done.load(std::memory_order_acquire) & bit) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
-  done.fetch_or(bit, std::memory_order_acq_rel);
-  return true;
-}
-
 // Scratch for flex_attn_decode_noalloc: compiled into the library so that callers who
 // cannot allocate device memory still get a workspace.  One copy per device, shared by
 // every call on that device.
@@ -92,36 +79,6 @@ unsigned* status_ptr() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
   return static_cast<unsigned*>(p);
-}
-
-// ---------------------------------------------------------------- forward dispatch
-
-template <int D, typename T, int SCORE, int MASK>
-flex_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
-                         int n_units, cudaStream_t stream) {
-  auto kern = flex_fwd_kernel<D, T, SCORE, MASK>;
-  if (!ensure_smem_attr<D, T, SCORE, MASK>(kern, FwdSmem<D>::kAlloc)) return FLEX_ERR_CUDA;
-  kern<<<n_units, kFwdThreads, FwdSmem<D>::kAlloc, stream>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
-}
-
-template <int D, typename T, int SCORE>
-flex_status_t dispatch_mask(int mask, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const FwdParams& p, int n_units, cudaStream_t s) {
-  switch (mask) {
-    case kMaskNone: return launch_fwd<D, T, SCORE, kMaskNone>(mq, mk, mv, p, n_units, s);
-    case kMaskCausal: return launch_fwd<D, T, SCORE, kMaskCausal>(mq, mk, mv, p, n_units, s);
-    case kMaskSliding: return launch_fwd<D, T, SCORE, kMaskSliding>(mq, mk, mv, p, n_units, s);
-    case kMaskOffset: return launch_fwd<D, T, SCORE, kMaskOffset>(mq, mk, mv, p, n_units, s);
-  }
-  return FLEX_ERR_INVALID_ARG;
-}
-
-template <int D, typename T>
-flex_status_t dispatch_score(int score, int mask, const CUtensorMap& mq, const CUtensorMap& mk,
-                             const CUtensorMap& mv, const FwdParams& p, int n_units, cudaStream_t s) {
-  if (score == kScoreNone) return dispatch_mask<D, T, kScoreNone>(mask, mq, mk, mv, p, n_units, s);
-  return dispatch_mask<D, T, kScoreAlibi>(mask, mq, mk, mv, p, n_units, s);
 }
 
 // ---------------------------------------------------------------- mask evaluation (debug)
@@ -152,36 +109,6 @@ __global__ void mask_eval_kernel(MaskArgs m, int Sq, int Skv, uint8_t* keep) {
   }
 }
 
-// ---------------------------------------------------------------- decode dispatch
-
-template <int D, typename T, int GT>
-flex_status_t launch_decode(const DecodeParams& p, cudaStream_t s) {
-  dim3 grid(p.n_splits, p.B * p.Hkv * (p.G / GT));
-  decode_split_kernel<D, T, GT><<<grid, kDecThreads, 0, s>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return FLEX_ERR_CUDA;
-  const int rows = p.B * p.H;
-  decode_combine_kernel<D, T><<<(rows + kDecWarps - 1) / kDecWarps, kDecThreads, 0, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
-}
-
-template <int D, typename T>
-flex_status_t launch_decode_gqa(const DecodeParams& p, cudaStream_t s) {
-  dim3 grid(p.n_splits, p.B * p.Hkv * ((p.G + kGqaRows - 1) / kGqaRows));
-  decode_gqa_kernel<D, T><<<grid, kDecThreads, 0, s>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return FLEX_ERR_CUDA;
-  const int rows = p.B * p.H;
-  decode_combine_kernel<D, T><<<(rows + kDecWarps - 1) / kDecWarps, kDecThreads, 0, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
-}
-
-// One query head per kv head streams on CUDA cores; grouped heads go to the tensor-core
-// kernel, whose work per byte does not grow with the group size.
-template <int D, typename T>
-flex_status_t decode_by_group(const DecodeParams& p, cudaStream_t s) {
-  if (p.G >= 2) return launch_decode_gqa<D, T>(p, s);
-  return launch_decode<D, T, 1>(p, s);
-}
-
 int decode_splits(int cap) { return (cap + kChunk - 1) / kChunk; }
 
 constexpr unsigned kStatusSelftestTimeout = 8u;
@@ -196,16 +123,11 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned* status) {
   mbar_wait(b, 0, status, kStatusSelftestTimeout, timeout_ns);
 }
 
-}  // namespace
-}  // namespace flexattn
-
-using namespace flexattn;
-
-extern "C" {
-
-flex_status_t flex_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
-                            int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
-                            const flex_mod_params_t* mod_params, flex_dtype_t dtype, flex_stream_t stream) {
+// Shared body of flex_attn_fwd (bm == nullptr) and flex_attn_fwd_block_sparse.
+flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                         int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
+                         const flex_mod_params_t* mod_params, const flex_block_mask_t* bm, flex_dtype_t dtype,
+                         flex_stream_t stream) {
   if (!q || !k || !v || !o) return FLEX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
@@ -228,6 +150,21 @@ flex_status_t flex_attn_fwd(const void* q, const void* k, const void* v, void* o
   if (want_map && !mp.tile_map_out) return FLEX_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
     return FLEX_ERR_MISALIGNED;
+  if (bm) {
+    const bool has_part = bm->kv_num_blocks != nullptr, has_full = bm->full_kv_num_blocks != nullptr;
+    if (has_part != (bm->kv_indices != nullptr) || has_full != (bm->full_kv_indices != nullptr))
+      return FLEX_ERR_INVALID_ARG;
+    if (!has_part && !has_full) return FLEX_ERR_INVALID_ARG;
+    if (bm->max_blocks < 1 || (bm->batch != 1 && bm->batch != B) || (bm->heads != 1 && bm->heads != H))
+      return FLEX_ERR_INVALID_ARG;
+    if (bm->q_block_size != kBM || bm->kv_block_size != kBN) return FLEX_ERR_UNSUPPORTED;
+    if ((Skv + kBN - 1) / kBN > kMaxBlockKeyTiles) return FLEX_ERR_UNSUPPORTED;
+    const int64_t idx_elems = static_cast<int64_t>(bm->batch) * bm->heads * ((Sq + kBM - 1) / kBM) * bm->max_blocks;
+    if (idx_elems > 0x7fffffffLL) return FLEX_ERR_UNSUPPORTED;
+    if (!aligned4(bm->kv_num_blocks) || !aligned4(bm->kv_indices) || !aligned4(bm->full_kv_num_blocks) ||
+        !aligned4(bm->full_kv_indices))
+      return FLEX_ERR_MISALIGNED;
+  }
   const int64_t bh = static_cast<int64_t>(B) * H;
   const int n_qtiles = (Sq + kBM - 1) / kBM;
   const int n_pairs = (n_qtiles + 1) / 2;
@@ -258,12 +195,43 @@ flex_status_t flex_attn_fwd(const void* q, const void* k, const void* v, void* o
   p.mask = MaskArgs{Skv, mp.window, mp.offset};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int units = static_cast<int>(n_units);
-  if (D == 128) {
-    return dtype == FLEX_DTYPE_BF16 ? dispatch_score<128, __nv_bfloat16>(score_mod_id, mask, mq, mk, mv, p, units, s)
-                                    : dispatch_score<128, __half>(score_mod_id, mask, mq, mk, mv, p, units, s);
+  if (bm) {
+    p.blk_num[0] = bm->kv_num_blocks;
+    p.blk_idx[0] = bm->kv_indices;
+    p.blk_num[1] = bm->full_kv_num_blocks;
+    p.blk_idx[1] = bm->full_kv_indices;
+    p.blk_max = bm->max_blocks;
+    p.blk_b_stride = bm->batch == 1 ? 0 : bm->heads;
+    p.blk_h_stride = bm->heads == 1 ? 0 : 1;
+    return D == 128 ? fwd_dispatch<128, true>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s)
+                    : fwd_dispatch<64, true>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s);
   }
-  return dtype == FLEX_DTYPE_BF16 ? dispatch_score<64, __nv_bfloat16>(score_mod_id, mask, mq, mk, mv, p, units, s)
-                                  : dispatch_score<64, __half>(score_mod_id, mask, mq, mk, mv, p, units, s);
+  return D == 128 ? fwd_dispatch<128, false>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s)
+                  : fwd_dispatch<64, false>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s);
+}
+
+}  // namespace
+}  // namespace flexattn
+
+using namespace flexattn;
+
+extern "C" {
+
+flex_status_t flex_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                            int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
+                            const flex_mod_params_t* mod_params, flex_dtype_t dtype, flex_stream_t stream) {
+  return fwd_common(q, k, v, o, lse, B, H, Hkv, Sq, Skv, D, scale, score_mod_id, mask_mod_id, mod_params, nullptr,
+                    dtype, stream);
+}
+
+flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                         int H, int Hkv, int Sq, int Skv, int D, float scale, int score_mod_id,
+                                         int mask_mod_id, const flex_mod_params_t* mod_params,
+                                         const flex_block_mask_t* block_mask, flex_dtype_t dtype,
+                                         flex_stream_t stream) {
+  if (!block_mask) return FLEX_ERR_INVALID_ARG;
+  return fwd_common(q, k, v, o, lse, B, H, Hkv, Sq, Skv, D, scale, score_mod_id, mask_mod_id, mod_params,
+                    block_mask, dtype, stream);
 }
 
 size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D) {
@@ -314,10 +282,7 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
   p.scale_log2 = scale * kLog2e;
   const int64_t grid_y = static_cast<int64_t>(B) * Hkv * (p.G >= 2 ? (p.G + kGqaRows - 1) / kGqaRows : 1);
   if (grid_y > 65535) return FLEX_ERR_UNSUPPORTED;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (D == 128)
-    return dtype == FLEX_DTYPE_BF16 ? decode_by_group<128, __nv_bfloat16>(p, s) : decode_by_group<128, __half>(p, s);
-  return dtype == FLEX_DTYPE_BF16 ? decode_by_group<64, __nv_bfloat16>(p, s) : decode_by_group<64, __half>(p, s);
+  return decode_dispatch(D, dtype, p, reinterpret_cast<cudaStream_t>(stream));
 }
 
 flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -22,6 +22,10 @@
 //               when the running max grows by more than 2^8, and finally normalises O and
 //               writes O and LSE.  kEmuPairsPerHalf of each 32 column pairs can evaluate
 //               2^x as a polynomial on the FMA pipe instead of the MUFU unit.
+// With a block mask (the BLOCKS instantiations) each query tile visits the key tiles its
+// partial and full lists name instead of the range its mask_mod implies; the CTA walks the
+// union of its two tiles' sets, and a tile absent from one set is simply not issued for
+// that query tile.  The sets live in shared memory as bitmaps built at the start.
 // Key tiles are visited from the last to the first.  With t counting steps, the MMA order
 // S0(t0) S1(t0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ... lets one softmax warpgroup work
 // while the tensor core runs the other tile's matmuls.
@@ -62,6 +66,11 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr unsigned kStatusFwdTimeout = 2u;
+// Block mask: key tiles a bitmap can name (Skv <= 2048 * 128), and its size in words.
+constexpr int kMaxBlockKeyTiles = 2048;
+constexpr int kBlkWords = kMaxBlockKeyTiles / 32;
+// A FULL-listed key tile that runs past Skv: only the key-length rule masks it.
+constexpr int kTileFullRagged = 3;
 
 struct FwdParams {
   void* o;
@@ -72,9 +81,16 @@ struct FwdParams {
   int n_qtiles, n_ktiles, n_pairs;
   float scale_log2;    // scale * log2(e)
   MaskArgs mask;
+  // Block mask (BLOCKS instantiations): [0] partial lists, [1] full lists; counts are
+  // [rows x n_qtiles], indices [rows x n_qtiles x blk_max]; row of (b, h) =
+  // b * blk_b_stride + h * blk_h_stride (a stride of 0 shares one row).
+  const int32_t* blk_num[2];
+  const int32_t* blk_idx[2];
+  int blk_max;
+  int blk_b_stride, blk_h_stride;
 };
 
-template <int D>
+template <int D, bool BLOCKS = false>
 struct FwdSmem {
   static constexpr int kTileBytes = kBM * D * 2;          // one 128-row tile
   static constexpr int kChunkBytes = kBM * 128;           // one 64-element-wide chunk
@@ -88,7 +104,9 @@ struct FwdSmem {
   // barriers: q, full[NS], empty[NS], s_full[2], p_half[2][2], o_full[2], drain; then tmem addr
   static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 4 + 2 + 1;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kTmemPtrOff + 16;
+  // block-mask bitmaps: full0, full1, act0, act1, union (kBlkWords words each)
+  static constexpr int kBlkOff = kTmemPtrOff + 16;
+  static constexpr int kBytes = kBlkOff + (BLOCKS ? 5 * kBlkWords * 4 : 0);
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
   static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
 };
@@ -112,11 +130,24 @@ struct DtypeBits<__half> {
   }
 };
 
-template <int D, typename T, int SCORE, int MASK>
+// Highest set bit below j in a kBlkWords-word bitmap, or -1 (j <= kMaxBlockKeyTiles).
+__device__ __forceinline__ int bits_prev(const uint32_t* w, int j) {
+  if (j <= 0) return -1;
+  int wi = (j - 1) >> 5;
+  uint32_t m = w[wi] & (0xffffffffu >> (31 - ((j - 1) & 31)));
+  while (true) {
+    if (m) return (wi << 5) + 31 - __clz(m);
+    if (--wi < 0) return -1;
+    m = w[wi];
+  }
+}
+__device__ __forceinline__ bool bits_has(const uint32_t* w, int j) { return (w[j >> 5] >> (j & 31)) & 1u; }
+
+template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     flex_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using L = FwdSmem<D>;
+  using L = FwdSmem<D, BLOCKS>;
   constexpr int NS = L::kSlots;
   constexpr int kChunks = D / 64;
   constexpr uint32_t kTmemCols = 512;
@@ -157,10 +188,80 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     lo[k] = hi[k] = 0;
     if (qt < p.n_qtiles) tile_range<MASK>(q0[k], q1[k], kBN, p.mask, lo[k], hi[k]);
   }
-  const bool act0 = lo[0] < hi[0], act1 = lo[1] < hi[1];
-  const int ulo = act0 ? (act1 ? min(lo[0], lo[1]) : lo[0]) : lo[1];
-  const int uhi = act0 ? (act1 ? max(hi[0], hi[1]) : hi[0]) : hi[1];
-  const bool any_work = act0 || act1;
+
+  // ---------------------------------------------------------------- block-mask bitmaps
+  // full_k: tiles listed full; act_k: every tile query tile k visits; uni: act_0 | act_1.
+  uint32_t* blk = reinterpret_cast<uint32_t*>(sgen + L::kBlkOff);
+  auto full_bits = [&](int k) { return blk + k * kBlkWords; };
+  auto act_bits = [&](int k) { return blk + (2 + k) * kBlkWords; };
+  const uint32_t* uni_bits = blk + 4 * kBlkWords;
+  if constexpr (BLOCKS) {
+    for (int w = threadIdx.x; w < 5 * kBlkWords; w += kFwdThreads) blk[w] = 0u;
+    __syncthreads();
+    const int64_t row0 = static_cast<int64_t>(b) * p.blk_b_stride + static_cast<int64_t>(h) * p.blk_h_stride;
+    // list l = 2 * k + f: query tile 2 * pair + k, f = 0 partial / 1 full (selects, not
+    // indexing, so that nothing here is forced into local memory)
+    auto count = [&](int k, int f) {
+      const int qt = 2 * pair + k;
+      const int32_t* num = f ? p.blk_num[1] : p.blk_num[0];
+      const int c = (qt < p.n_qtiles && num != nullptr) ? num[row0 * p.n_qtiles + qt] : 0;
+      return c < 0 ? 0 : (c > p.blk_max ? p.blk_max : c);
+    };
+    const int c00 = count(0, 0), c01 = count(0, 1), c10 = count(1, 0), c11 = count(1, 1);
+    for (int e = threadIdx.x; e < 4 * p.blk_max; e += kFwdThreads) {
+      const int l = e / p.blk_max, c = e - l * p.blk_max;
+      const int k = l >> 1, f = l & 1;
+      const int cl = k ? (f ? c11 : c10) : (f ? c01 : c00);
+      if (c >= cl) continue;
+      const int32_t* idx = f ? p.blk_idx[1] : p.blk_idx[0];
+      const int u = idx[(row0 * p.n_qtiles + 2 * pair + k) * p.blk_max + c];
+      if (u < 0 || u >= p.n_ktiles) continue;
+      bool full = f == 1;
+      if (!full) {
+        // a partial tile outside the mask_mod range keeps nothing; one the mask keeps
+        // whole needs no per-element mask
+        if (u < (k ? lo[1] : lo[0]) || u >= (k ? hi[1] : hi[0])) continue;
+        full = tile_class<MASK>(k ? q0[1] : q0[0], k ? q1[1] : q1[0], u * kBN, kBN, p.mask) == kTileFull;
+      }
+      const uint32_t bit = 1u << (u & 31);
+      if (full) atomicOr(full_bits(k) + (u >> 5), bit);
+      atomicOr(act_bits(k) + (u >> 5), bit);
+    }
+    __syncthreads();
+    for (int w = threadIdx.x; w < kBlkWords; w += kFwdThreads) blk[4 * kBlkWords + w] = act_bits(0)[w] | act_bits(1)[w];
+  }
+  // Visit order of query tile k and of the union: first tile, then the next one below j.
+  auto first_of = [&](int k) -> int {
+    if constexpr (BLOCKS) return bits_prev(act_bits(k), p.n_ktiles);
+    else return lo[k] < hi[k] ? hi[k] - 1 : -1;
+  };
+  auto next_of = [&](int k, int j) -> int {
+    if constexpr (BLOCKS) return bits_prev(act_bits(k), j);
+    else return j - 1 >= lo[k] ? j - 1 : -1;
+  };
+  auto has = [&](int k, int j) -> bool {
+    if constexpr (BLOCKS) return bits_has(act_bits(k), j);
+    else return j >= lo[k] && j < hi[k];
+  };
+  bool act0, act1;
+  int ulo = 0, uhi = 0;
+  if constexpr (BLOCKS) {
+    // act_k is read after the setup barrier below
+    act0 = act1 = false;
+  } else {
+    act0 = lo[0] < hi[0];
+    act1 = lo[1] < hi[1];
+    ulo = act0 ? (act1 ? min(lo[0], lo[1]) : lo[0]) : lo[1];
+    uhi = act0 ? (act1 ? max(hi[0], hi[1]) : hi[0]) : hi[1];
+  }
+  auto union_first = [&]() -> int {
+    if constexpr (BLOCKS) return bits_prev(uni_bits, p.n_ktiles);
+    else return (act0 || act1) ? uhi - 1 : -1;
+  };
+  auto union_next = [&](int j) -> int {
+    if constexpr (BLOCKS) return bits_prev(uni_bits, j);
+    else return j - 1 >= ulo ? j - 1 : -1;
+  };
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -192,6 +293,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
+  if constexpr (BLOCKS) {
+    act0 = first_of(0) >= 0;
+    act1 = first_of(1) >= 0;
+  }
+  const bool any_work = act0 || act1;
 
   const uint32_t q_smem0 = sbase + static_cast<uint32_t>(L::kQOff);
   auto q_smem = [&](int k) { return q_smem0 + static_cast<uint32_t>(k * L::kTileBytes); };
@@ -210,8 +316,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       int r = 0;
       bool ok = true;
-      for (int t = 0; t < uhi - ulo && ok; ++t) {
-        const int j = uhi - 1 - t;  // key tiles from last to first
+      for (int j = union_first(); j >= 0 && ok; j = union_next(j)) {  // key tiles from last to first
         for (int which = 0; which < 2 && ok; ++which, ++r) {
           const int s = r % NS;
           const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
@@ -259,12 +364,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_ts(d, a + 8u * kk, bv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
                  (acc || kk > 0) ? 1u : 0u);
       };
-      for (int t = 0; t < uhi - ulo && ok; ++t) {
-        const int j = uhi - 1 - t;  // key tiles from last to first
+      // s_ready[k]: S_k of the current key tile was issued during the previous step.
+      bool s_ready[2] = {false, false}, started[2] = {false, false};
+      int t = 0;
+      for (int j = union_first(); j >= 0 && ok; j = union_next(j), ++t) {  // last to first
         const int rK = 2 * t, rV = rK + 1;
         const int sK = rK % NS, sV = rV % NS;
-        const bool first0 = act0 && j == hi[0] - 1, first1 = act1 && j == hi[1] - 1;
-        if (first0 || first1) {
+        const bool in0 = act0 && has(0, j), in1 = act1 && has(1, j);
+        const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
+        if (need0 || need1) {
           // K_j was not needed before: wait for it here (otherwise the previous step did)
           if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
                          kStatusFwdTimeout, kWaitTimeoutNs)) {
@@ -272,11 +380,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             break;
           }
           tc_fence_after();
-          if (first0) {
+          if (need0) {
             issue_s(0, sK);
             mma_commit(bar_s(0));
           }
-          if (first1) {
+          if (need1) {
             issue_s(1, sK);
             mma_commit(bar_s(1));
           }
@@ -287,9 +395,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ok = false;
           break;
         }
+        const int jn = union_next(j);
         bool next_k_ready = false;
         for (int k = 0; k < 2 && ok; ++k) {
-          if (j < lo[k] || j >= hi[k]) continue;
+          s_ready[k] = false;
+          if (!(k == 0 ? in0 : in1)) continue;
           const uint32_t par = static_cast<uint32_t>(np[k]) & 1u;
           for (int half = 0; half < 2; ++half) {
             if (!mbar_wait(bar_p(k, half), par, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
@@ -297,12 +407,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               break;
             }
             tc_fence_after();
-            issue_pv(k, sV, j < hi[k] - 1, 4 * half, 4 * half + 4);
+            issue_pv(k, sV, started[k], 4 * half, 4 * half + 4);
           }
           if (!ok) break;
+          started[k] = true;
           ++np[k];
-          if (j - 1 >= lo[k]) {
-            const int rK2 = rK + 2;  // K_{j-1}
+          const int nk = next_of(k, j);
+          if (nk >= 0 && nk == jn) {
+            const int rK2 = rK + 2;  // K of the next step
             if (!next_k_ready) {
               if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status,
                              kStatusFwdTimeout, kWaitTimeoutNs)) {
@@ -314,9 +426,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             issue_s(k, rK2 % NS);
             mma_commit(bar_s(k));
-          } else {
+            s_ready[k] = true;
+          } else if (nk < 0) {
             mma_commit(bar_o(k));
           }
+          // otherwise S_k(nk) is issued at the step of key tile nk
         }
         mma_commit(bar_empty(sV));
       }
@@ -339,9 +453,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const bool write_map = p.tile_map != nullptr && bh == 0 && tile_valid && threadIdx.x % 128 == 0;
     const int qt = 2 * pair + k;
 
+    const bool act_k = k == 0 ? act0 : act1;
     if (write_map) {
       for (int u = 0; u < p.n_ktiles; ++u)
-        if (u < lo[k] || u >= hi[k]) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + u] = kTileEmpty;
+        if (!act_k || !has(k, u)) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + u] = kTileEmpty;
     }
 
     float m_used = -INFINITY;  // running max in log2 units (the reference of P and O)
@@ -354,7 +469,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int n = 0;
     // Key tiles from last to first: with alibi the bias grows with the key index, so the
     // row maximum is met on the first tile and the lazy rescale of O almost never runs.
-    for (int j = hi[k] - 1; j >= lo[k]; --j, ++n) {
+    for (int j = act_k ? first_of(k) : -1; j >= 0; j = next_of(k, j), ++n) {
       // Warp-uniform decision: the TMEM loads below are warp-collective.
       const bool got = mbar_wait(bar_s(k), static_cast<uint32_t>(n) & 1u, p.status, kStatusFwdTimeout,
                                  kWaitTimeoutNs) &&
@@ -365,8 +480,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tc_fence_after();
       const int k0 = j * kBN;
-      const int cls = tile_class<MASK>(q0[k], q1[k], k0, kBN, p.mask);
-      if (write_map) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] = static_cast<uint8_t>(cls);
+      int cls;
+      if constexpr (BLOCKS)
+        cls = bits_has(full_bits(k), j) ? (k0 + kBN > p.Skv ? kTileFullRagged : kTileFull) : kTilePartial;
+      else
+        cls = tile_class<MASK>(q0[k], q1[k], k0, kBN, p.mask);
+      if (write_map)
+        p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] =
+            static_cast<uint8_t>(cls == kTileFullRagged ? kTilePartial : cls);
 
       uint32_t sr[kBN];
       tmem_ld128(tS, sr);
@@ -376,9 +497,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN; ++c) s[c] = fmaf(s[c], p.scale_log2, fmaf(slope2, static_cast<float>(c), base));
       }
-      if (cls == kTilePartial) {
+      if (cls != kTileFull) {
         int c_lo, c_hi;
-        col_interval<MASK>(qi, k0, p.mask, c_lo, c_hi);
+        if (BLOCKS && cls == kTileFullRagged)
+          col_interval<kMaskNone>(qi, k0, p.mask, c_lo, c_hi);
+        else
+          col_interval<MASK>(qi, k0, p.mask, c_lo, c_hi);
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
           if (c < c_lo || c > c_hi) s[c] = -INFINITY;
@@ -456,7 +580,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     // ---------------------------------------------------------------- epilogue
     if (tile_valid) {
-      bool ran = ok && lo[k] < hi[k];
+      bool ran = ok && act_k;
       if (ran) {
         const bool got = mbar_wait(bar_o(k), 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
         if (!__all_sync(0xffffffffu, got)) {

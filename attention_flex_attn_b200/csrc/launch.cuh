@@ -1,0 +1,37 @@
+// launch.cuh -- host-side launchers shared between the translation units of the
+// library: each forward (head dim, block mask) combination and the decode path is
+// instantiated in a .cu file of its own so that they compile in parallel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "flex_attn.h"
+#include "flex_decode.cuh"
+#include "flex_fwd_sm100.cuh"
+
+namespace flexattn {
+
+// Forward over every (dtype, score_mod, mask_mod) instantiation of one head dim and
+// block-mask mode.  Instantiated in flex_fwd_d{64,128}{,_blocks}.cu.
+template <int D, bool BLOCKS>
+flex_status_t fwd_dispatch(flex_dtype_t dtype, int score, int mask, const CUtensorMap& mq, const CUtensorMap& mk,
+                           const CUtensorMap& mv, const FwdParams& p, int n_units, cudaStream_t s);
+
+extern template flex_status_t fwd_dispatch<64, false>(flex_dtype_t, int, int, const CUtensorMap&,
+                                                      const CUtensorMap&, const CUtensorMap&, const FwdParams&,
+                                                      int, cudaStream_t);
+extern template flex_status_t fwd_dispatch<128, false>(flex_dtype_t, int, int, const CUtensorMap&,
+                                                       const CUtensorMap&, const CUtensorMap&, const FwdParams&,
+                                                       int, cudaStream_t);
+extern template flex_status_t fwd_dispatch<64, true>(flex_dtype_t, int, int, const CUtensorMap&,
+                                                     const CUtensorMap&, const CUtensorMap&, const FwdParams&,
+                                                     int, cudaStream_t);
+extern template flex_status_t fwd_dispatch<128, true>(flex_dtype_t, int, int, const CUtensorMap&,
+                                                      const CUtensorMap&, const CUtensorMap&, const FwdParams&,
+                                                      int, cudaStream_t);
+
+// Split-KV decode + combine (flex_decode_launch.cu).
+flex_status_t decode_dispatch(int D, flex_dtype_t dtype, const DecodeParams& p, cudaStream_t s);
+
+}  // namespace flexattn

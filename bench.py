@@ -388,7 +388,45 @@ def per_case(fa, q, k, v, scale, o, lse, args):
                      "tflops_dense_equiv": dense / t / 1e12}
         if name.startswith("sliding"):
             out[name]["tflops_useful"] = useful_window / t / 1e12
+    out.update(block_cases(fa, q, k, v, scale, o, lse))
     return out
+
+
+def block_lists(sel):
+    """[B, H, nq, nk] boolean block selection -> (counts, indices) int32, selected first."""
+    import numpy as np
+    num = sel.sum(-1).astype(np.int32)
+    idx = np.argsort(~sel, axis=-1, kind="stable").astype(np.int32)
+    return num, idx
+
+
+def block_cases(fa, q, k, v, scale, o, lse):
+    """Block-mask forward (flex_attn_fwd_block_sparse) on the forward inputs: causal given
+    as lists (diagonal blocks partial, the rest full), and random per-head lists with half
+    of the key blocks of every query tile full.  TFLOPS count the listed blocks whole
+    (4 * D * 128 * 128 per block), the causal case halves the dense count as above."""
+    import numpy as np
+    import torch
+    B, H, S, D = q.shape
+    nq = nk = S // 128
+    dev = q.device
+    res = {}
+    diag = np.eye(nq, nk, dtype=bool)
+    below = np.tril(np.ones((nq, nk), dtype=bool), -1)
+    kn, ki = block_lists(np.broadcast_to(diag, (1, 1, nq, nk)))
+    fn, fi = block_lists(np.broadcast_to(below, (1, 1, nq, nk)))
+    lists = [torch.from_numpy(a).to(dev) for a in (kn, ki, fn, fi)]
+    t = _time_fn(lambda: fa.fwd_block_sparse(q, k, v, *lists, scale=scale, mask_mod="causal", out=o,
+                                             lse_out=lse), 20, 3)
+    res["block_causal_lists"] = {"us": t * 1e6, "tflops": 0.5 * fwd_flops(B, H, S, S, D) / t / 1e12}
+    rng = np.random.default_rng(4100)
+    sel = rng.random((B, H, nq, nk)) < 0.5
+    fn, fi = block_lists(sel)
+    lists = [torch.from_numpy(a).to(dev) for a in (fn, fi)]
+    t = _time_fn(lambda: fa.fwd_block_sparse(q, k, v, None, None, *lists, scale=scale, out=o, lse_out=lse), 20, 3)
+    flops = 4.0 * D * 128 * 128 * float(sel.sum())
+    res["block_random_half_full"] = {"us": t * 1e6, "tflops": flops / t / 1e12, "density": float(sel.mean())}
+    return res
 
 
 def decode_cases(fa, dev, args):

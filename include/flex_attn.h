@@ -109,6 +109,51 @@ flex_status_t flex_attn_fwd(const void* q, const void* k, const void* v, void* o
                             flex_dtype_t dtype, flex_stream_t stream);
 
 /*
+ * flex_block_mask_t -- a block mask (BlockMask): per query tile of 128 rows, lists of key
+ * blocks of 128 keys.  FlyDSL PR 931 (Out of scope) names block sparsity as the next
+ * phase without defining it; the lists follow PyTorch's BlockMask convention:
+ *   - a key block on the query tile's full list is kept whole (only kv_idx < Skv applies);
+ *   - a key block on its partial list keeps the elements mask_mod keeps;
+ *   - every other key block is dropped; a block on both lists counts as full.
+ * Arrays are DEVICE int32, dense row-major, owned by the caller, 4-byte aligned:
+ *   kv_num_blocks, full_kv_num_blocks  [batch, heads, ceil(Sq/128)]
+ *   kv_indices, full_kv_indices        [batch, heads, ceil(Sq/128), max_blocks]
+ * Either (num, indices) pair may be NULL (no blocks of that kind), not both.  batch is 1
+ * (one mask for every batch) or B; heads is 1 or H.  Only the first num entries of an
+ * index row are read; num is clamped to [0, max_blocks] on the device, an index outside
+ * [0, ceil(Skv/128)) names no block, and a repeated index counts once, so no value in
+ * these arrays can make the kernel read out of bounds.  The order of the entries does
+ * not matter.
+ */
+typedef struct {
+  const int32_t* kv_num_blocks;
+  const int32_t* kv_indices;
+  const int32_t* full_kv_num_blocks;
+  const int32_t* full_kv_indices;
+  int32_t max_blocks;     /* >= 1 */
+  int32_t batch;          /* 1 or B */
+  int32_t heads;          /* 1 or H */
+  int32_t q_block_size;   /* must be 128 (FLEX_ERR_UNSUPPORTED otherwise) */
+  int32_t kv_block_size;  /* must be 128 (FLEX_ERR_UNSUPPORTED otherwise) */
+} flex_block_mask_t;
+
+/*
+ * flex_attn_fwd_block_sparse -- flex_attn_fwd with a block mask: the key tiles each query
+ * tile visits come from block_mask instead of from the range mask_mod implies; partial
+ * blocks still apply mask_mod element by element (and blocks that mask_mod drops whole are
+ * skipped), full blocks apply only kv_idx < Skv.  Arguments, layouts and errors are those
+ * of flex_attn_fwd, plus: block_mask non-NULL and valid as described above; Skv at most
+ * 2048 * 128 = 262144 (FLEX_ERR_UNSUPPORTED beyond); mod_params->tile_map_out, if asked
+ * for, records what the kernel visited (FULL, or PARTIAL for tiles it masks).
+ */
+flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                                         int B, int H, int Hkv, int Sq, int Skv, int D, float scale,
+                                         int score_mod_id, int mask_mod_id,
+                                         const flex_mod_params_t* mod_params,
+                                         const flex_block_mask_t* block_mask, flex_dtype_t dtype,
+                                         flex_stream_t stream);
+
+/*
  * flex_attn_decode_workspace_size -- bytes of device workspace flex_attn_decode needs
  * for these sizes (the split-KV partial outputs and their log-sum-exps).
  */

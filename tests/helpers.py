@@ -50,3 +50,31 @@ def gather_rows(t, rows):
     """t [B,H,S,...] -> rows of the flattened [B*H*S, ...] view."""
     flat = t.reshape(-1, *t.shape[3:]) if t.dim() > 3 else t.reshape(-1)
     return flat[torch.as_tensor(rows, device=t.device)]
+
+
+def random_block_lists(rng, B, H, nq, nk, max_blocks, p_full=0.3, p_part=0.3):
+    """Random block-mask lists (numpy int32): counts [B,H,nq], indices [B,H,nq,max_blocks]
+    for partial and full blocks, with the irregularities a caller may pass -- a repeated
+    index, an index naming no block (-1, nk, nk+5), garbage after the count, counts above
+    max_blocks or below 0."""
+    kn = np.zeros((B, H, nq), np.int32)
+    ki = np.zeros((B, H, nq, max_blocks), np.int32)
+    fn = np.zeros((B, H, nq), np.int32)
+    fi = np.zeros((B, H, nq, max_blocks), np.int32)
+    for b in range(B):
+        for h in range(H):
+            for t in range(nq):
+                for num, idx, pr in ((kn, ki, p_part), (fn, fi, p_full)):
+                    chosen = [u for u in range(nk) if rng.random() < pr]
+                    if chosen and rng.random() < 0.3:
+                        chosen.append(chosen[0])            # a duplicate
+                    if rng.random() < 0.2:
+                        chosen.append(int(rng.choice([-1, nk, nk + 5])))  # names no block
+                    rng.shuffle(chosen)
+                    chosen = chosen[:max_blocks]
+                    idx[b, h, t, :len(chosen)] = chosen
+                    idx[b, h, t, len(chosen):] = rng.integers(-3, nk + 3, max_blocks - len(chosen))
+                    c = len(chosen)
+                    r = rng.random()
+                    num[b, h, t] = c if r < 0.8 else (max_blocks + 3 if r < 0.9 else -2)
+    return kn, ki, fn, fi

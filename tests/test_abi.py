@@ -114,3 +114,24 @@ def test_static_scratch_limit_matches_header():
 def test_selftest_rejects_bad_timeouts(lib):
     assert lib.flex_attn_selftest_wait_timeout(0, None) == 1
     assert lib.flex_attn_selftest_wait_timeout(2000001, None) == 1
+
+
+def test_block_sparse_rejects_bad_args_on_host(lib):
+    def bs(bm, Sq=8, Skv=8, **kw):
+        return lib.flex_attn_fwd_block_sparse(P(16), P(16), P(16), P(16), None, 1, 2, 1, Sq, Skv, 128, 0.1, 0, 0,
+                                              None, ctypes.byref(bm) if bm is not None else None, 0, None)
+
+    def mask(num=32, idx=64, fnum=None, fidx=None, maxb=1, batch=1, heads=1, qb=128, kb=128):
+        return fa.BlockMaskC(num, idx, fnum, fidx, maxb, batch, heads, qb, kb)
+    assert bs(None) == 1
+    assert bs(mask(num=None, idx=None)) == 1              # neither list
+    assert bs(mask(idx=None)) == 1                        # counts without indices
+    assert bs(mask(fnum=32)) == 1                         # full counts without indices
+    assert bs(mask(maxb=0)) == 1
+    assert bs(mask(batch=3)) == 1                         # batch must be 1 or B
+    assert bs(mask(heads=3)) == 1                         # heads must be 1 or H
+    assert bs(mask(qb=64)) == 2
+    assert bs(mask(kb=256)) == 2
+    assert bs(mask(), Skv=2048 * 128 + 1) == 2            # beyond what the bitmaps name
+    assert bs(mask(num=34)) == 3                          # not 4-byte aligned
+    assert bs(mask(fnum=32, fidx=66)) == 3

@@ -18,6 +18,7 @@ import pytest
 import torch
 
 import synth
+from tests.helpers import random_block_lists as _random_lists
 
 TOL = 1e-12
 
@@ -69,30 +70,6 @@ def _torch_masked(q, k, v, keep, scale, alibi=False):
     o = p @ vv
     lse = torch.logsumexp(s, -1)
     return o.numpy(), lse.numpy()
-
-
-def _random_lists(rng, B, H, nq, nk, max_blocks, p_full=0.3, p_part=0.3):
-    kn = np.zeros((B, H, nq), np.int32)
-    ki = np.zeros((B, H, nq, max_blocks), np.int32)
-    fn = np.zeros((B, H, nq), np.int32)
-    fi = np.zeros((B, H, nq, max_blocks), np.int32)
-    for b in range(B):
-        for h in range(H):
-            for t in range(nq):
-                for num, idx, pr in ((kn, ki, p_part), (fn, fi, p_full)):
-                    chosen = [u for u in range(nk) if rng.random() < pr]
-                    if chosen and rng.random() < 0.3:
-                        chosen.append(chosen[0])            # a duplicate
-                    if rng.random() < 0.2:
-                        chosen.append(int(rng.choice([-1, nk, nk + 5])))  # names no block
-                    rng.shuffle(chosen)
-                    chosen = chosen[:max_blocks]
-                    idx[b, h, t, :len(chosen)] = chosen
-                    idx[b, h, t, len(chosen):] = rng.integers(-3, nk + 3, max_blocks - len(chosen))
-                    c = len(chosen)
-                    r = rng.random()
-                    num[b, h, t] = c if r < 0.8 else (max_blocks + 3 if r < 0.9 else -2)
-    return kn, ki, fn, fi
 
 
 @pytest.mark.parametrize("mask,window,offset,score", [
