@@ -41,6 +41,7 @@
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "mask_rules.cuh"
 #include "ptx_sm100.cuh"
@@ -71,6 +72,17 @@ constexpr int kMaxBlockKeyTiles = 2048;
 constexpr int kBlkWords = kMaxBlockKeyTiles / 32;
 // A FULL-listed key tile that runs past Skv: only the key-length rule masks it.
 constexpr int kTileFullRagged = 3;
+
+// Step record: what the MMA issuer does at one step of the CTA's walk over key tiles.
+// The TMA producer, which walks the same tiles ahead of time, writes the record of step
+// t + 1 before it signals V of step t, so the issuer never walks the sets itself.
+constexpr uint32_t kRecIn0 = 1u << 0;    // query tile 0 visits this key tile
+constexpr uint32_t kRecIn1 = 1u << 1;
+constexpr uint32_t kRecPre0 = 1u << 2;   // ... and its next key tile is the next step's
+constexpr uint32_t kRecPre1 = 1u << 3;
+constexpr uint32_t kRecLast0 = 1u << 4;  // ... and this is its last key tile
+constexpr uint32_t kRecLast1 = 1u << 5;
+constexpr uint32_t kRecEnd = 1u << 6;    // no step: the walk is over
 
 struct FwdParams {
   void* o;
@@ -104,9 +116,12 @@ struct FwdSmem {
   // barriers: q, full[NS], empty[NS], s_full[2], p_half[2][2], o_full[2], drain; then tmem addr
   static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 4 + 2 + 1;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
-  // block-mask bitmaps: full0, full1, act0, act1, union (kBlkWords words each)
-  static constexpr int kBlkOff = kTmemPtrOff + 16;
-  static constexpr int kBytes = kBlkOff + (BLOCKS ? 5 * kBlkWords * 4 : 0);
+  // step records (kRec*): one per key/value slot, plus the first step's
+  static constexpr int kRecOff = kTmemPtrOff + 16;
+  static constexpr int kRecBytes = ((kSlots + 1) * 4 + 15) / 16 * 16;
+  // block-mask bitmaps: full0, full1, act0, act1 (kBlkWords words each)
+  static constexpr int kBlkOff = kRecOff + kRecBytes;
+  static constexpr int kBytes = kBlkOff + (BLOCKS ? 4 * kBlkWords * 4 : 0);
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
   static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
 };
@@ -130,17 +145,48 @@ struct DtypeBits<__half> {
   }
 };
 
-// Highest set bit below j in a kBlkWords-word bitmap, or -1 (j <= kMaxBlockKeyTiles).
-__device__ __forceinline__ int bits_prev(const uint32_t* w, int j) {
-  if (j <= 0) return -1;
-  int wi = (j - 1) >> 5;
-  uint32_t m = w[wi] & (0xffffffffu >> (31 - ((j - 1) & 31)));
-  while (true) {
-    if (m) return (wi << 5) + 31 - __clz(m);
-    if (--wi < 0) return -1;
-    m = w[wi];
+// Walk of the key tiles one query tile visits, from the last to the first.  cur is the
+// current tile (-1 once the walk is over), advance() moves to the next one.
+//
+// BitCursor walks the set bits of a shared-memory bitmap with the current 32-bit word in
+// a register, so a step costs a few ALU operations and one shared-memory load per 32
+// tiles; the companion bitmap (the FULL tiles) is read alongside into cur_full.
+struct BitCursor {
+  const uint32_t* set;
+  const uint32_t* comp;
+  int wi;
+  uint32_t bits, cword;
+  int cur;
+  bool cur_full;
+  __device__ __forceinline__ void advance() {
+    while (bits == 0) {
+      if (--wi < 0) {
+        cur = -1;
+        return;
+      }
+      bits = set[wi];
+      cword = comp[wi];
+    }
+    const int bit = 31 - __clz(bits);
+    bits &= ~(1u << bit);
+    cur = (wi << 5) + bit;
+    cur_full = (cword >> bit) & 1u;
   }
-}
+  // n_tiles <= kMaxBlockKeyTiles; bits at or above n_tiles are clear.
+  __device__ __forceinline__ BitCursor(const uint32_t* s, const uint32_t* c, int n_tiles)
+      : set(s), comp(c), wi((n_tiles + 31) >> 5), bits(0), cword(0), cur(-1), cur_full(false) {
+    advance();
+  }
+};
+
+// RangeCursor walks the contiguous range [lo, hi) that a mask_mod implies.
+struct RangeCursor {
+  int lo, cur;
+  bool cur_full = false;
+  __device__ __forceinline__ RangeCursor(int l, int h) : lo(l), cur(h - 1 >= l ? h - 1 : -1) {}
+  __device__ __forceinline__ void advance() { cur = cur - 1 >= lo ? cur - 1 : -1; }
+};
+
 __device__ __forceinline__ bool bits_has(const uint32_t* w, int j) { return (w[j >> 5] >> (j & 31)) & 1u; }
 
 template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
@@ -168,6 +214,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t bar_drain = sbase + L::kBarOff + 8u * (9 + 2 * NS);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
+  uint32_t* rec_smem = reinterpret_cast<uint32_t*>(sgen + L::kRecOff);  // [NS] per V slot, [NS] first
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -179,7 +226,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int b = bh / p.H;
   const int bkv = b * p.Hkv + h / p.G;
 
+  // Per query tile k of the pair.  Read through sel() wherever k is not a compile-time
+  // constant, so that no array is indexed at run time (that would put it in local memory).
   int q0[2], q1[2], lo[2], hi[2];
+  auto sel = [](const int (&a)[2], int k) { return k ? a[1] : a[0]; };
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int qt = 2 * pair + k;
@@ -190,13 +240,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 
   // ---------------------------------------------------------------- block-mask bitmaps
-  // full_k: tiles listed full; act_k: every tile query tile k visits; uni: act_0 | act_1.
+  // full_k: tiles listed full; act_k: every tile query tile k visits.  Complete at the
+  // setup barrier below.
   uint32_t* blk = reinterpret_cast<uint32_t*>(sgen + L::kBlkOff);
   auto full_bits = [&](int k) { return blk + k * kBlkWords; };
   auto act_bits = [&](int k) { return blk + (2 + k) * kBlkWords; };
-  const uint32_t* uni_bits = blk + 4 * kBlkWords;
   if constexpr (BLOCKS) {
-    for (int w = threadIdx.x; w < 5 * kBlkWords; w += kFwdThreads) blk[w] = 0u;
+    for (int w = threadIdx.x; w < 4 * kBlkWords; w += kFwdThreads) blk[w] = 0u;
     __syncthreads();
     const int64_t row0 = static_cast<int64_t>(b) * p.blk_b_stride + static_cast<int64_t>(h) * p.blk_h_stride;
     // list l = 2 * k + f: query tile 2 * pair + k, f = 0 partial / 1 full (selects, not
@@ -220,47 +270,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (!full) {
         // a partial tile outside the mask_mod range keeps nothing; one the mask keeps
         // whole needs no per-element mask
-        if (u < (k ? lo[1] : lo[0]) || u >= (k ? hi[1] : hi[0])) continue;
-        full = tile_class<MASK>(k ? q0[1] : q0[0], k ? q1[1] : q1[0], u * kBN, kBN, p.mask) == kTileFull;
+        if (u < sel(lo, k) || u >= sel(hi, k)) continue;
+        full = tile_class<MASK>(sel(q0, k), sel(q1, k), u * kBN, kBN, p.mask) == kTileFull;
       }
       const uint32_t bit = 1u << (u & 31);
       if (full) atomicOr(full_bits(k) + (u >> 5), bit);
       atomicOr(act_bits(k) + (u >> 5), bit);
     }
-    __syncthreads();
-    for (int w = threadIdx.x; w < kBlkWords; w += kFwdThreads) blk[4 * kBlkWords + w] = act_bits(0)[w] | act_bits(1)[w];
   }
-  // Visit order of query tile k and of the union: first tile, then the next one below j.
-  auto first_of = [&](int k) -> int {
-    if constexpr (BLOCKS) return bits_prev(act_bits(k), p.n_ktiles);
-    else return lo[k] < hi[k] ? hi[k] - 1 : -1;
+  // The walk over query tile k's key tiles (valid after the setup barrier); the CTA's
+  // steps are the union of both walks: j = max of the two cursors.
+  auto cursor = [&](int k) {
+    if constexpr (BLOCKS) return BitCursor(act_bits(k), full_bits(k), p.n_ktiles);
+    else return RangeCursor(sel(lo, k), sel(hi, k));
   };
-  auto next_of = [&](int k, int j) -> int {
-    if constexpr (BLOCKS) return bits_prev(act_bits(k), j);
-    else return j - 1 >= lo[k] ? j - 1 : -1;
-  };
-  auto has = [&](int k, int j) -> bool {
+  auto has = [&](int k, int j) -> bool {  // debug tile map only
     if constexpr (BLOCKS) return bits_has(act_bits(k), j);
-    else return j >= lo[k] && j < hi[k];
-  };
-  bool act0, act1;
-  int ulo = 0, uhi = 0;
-  if constexpr (BLOCKS) {
-    // act_k is read after the setup barrier below
-    act0 = act1 = false;
-  } else {
-    act0 = lo[0] < hi[0];
-    act1 = lo[1] < hi[1];
-    ulo = act0 ? (act1 ? min(lo[0], lo[1]) : lo[0]) : lo[1];
-    uhi = act0 ? (act1 ? max(hi[0], hi[1]) : hi[0]) : hi[1];
-  }
-  auto union_first = [&]() -> int {
-    if constexpr (BLOCKS) return bits_prev(uni_bits, p.n_ktiles);
-    else return (act0 || act1) ? uhi - 1 : -1;
-  };
-  auto union_next = [&](int j) -> int {
-    if constexpr (BLOCKS) return bits_prev(uni_bits, j);
-    else return j - 1 >= ulo ? j - 1 : -1;
+    else return j >= sel(lo, k) && j < sel(hi, k);
   };
 
   // ---------------------------------------------------------------- setup
@@ -293,10 +319,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  if constexpr (BLOCKS) {
-    act0 = first_of(0) >= 0;
-    act1 = first_of(1) >= 0;
-  }
+  const bool act0 = cursor(0).cur >= 0, act1 = cursor(1).cur >= 0;
   const bool any_work = act0 || act1;
 
   const uint32_t q_smem0 = sbase + static_cast<uint32_t>(L::kQOff);
@@ -307,16 +330,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     regs_dec<kAuxRegs>();
     if (warp == kTmaWarp && lane == 0 && any_work) {
       // ============================================================ TMA producer
+      int r = 0;
+      bool ok = true;
+      auto c0 = cursor(0), c1 = cursor(1);
+      // record of the step at max(a0.cur, a1.cur) (copies: the caller's cursors stay put)
+      auto make_rec = [](auto a0, auto a1) -> uint32_t {
+        const int j = max(a0.cur, a1.cur);
+        if (j < 0) return kRecEnd;
+        const bool i0 = a0.cur == j, i1 = a1.cur == j;
+        if (i0) a0.advance();
+        if (i1) a1.advance();
+        const int jn = max(a0.cur, a1.cur);
+        uint32_t rec = (i0 ? kRecIn0 : 0u) | (i1 ? kRecIn1 : 0u);
+        if (i0) rec |= a0.cur < 0 ? kRecLast0 : (a0.cur == jn ? kRecPre0 : 0u);
+        if (i1) rec |= a1.cur < 0 ? kRecLast1 : (a1.cur == jn ? kRecPre1 : 0u);
+        return rec;
+      };
+      // The first record is published with the Q barrier, which the issuer waits on first.
+      rec_smem[NS] = make_rec(c0, c1);
       const int bytes_q = (act0 ? 1 : 0) * L::kTileBytes + (act1 ? 1 : 0) * L::kTileBytes;
       mbar_arrive_expect_tx(bar_q, bytes_q);
       for (int k = 0; k < 2; ++k) {
         if (!(k == 0 ? act0 : act1)) continue;
         for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(q_smem(k) + c * L::kChunkBytes, &tmQ, bar_q, c * 64, q0[k], bh);
+          tma_load_3d(q_smem(k) + c * L::kChunkBytes, &tmQ, bar_q, c * 64, sel(q0, k), bh);
       }
-      int r = 0;
-      bool ok = true;
-      for (int j = union_first(); j >= 0 && ok; j = union_next(j)) {  // key tiles from last to first
+      for (int j = max(c0.cur, c1.cur); j >= 0 && ok; j = max(c0.cur, c1.cur)) {  // last to first
+        if (c0.cur == j) c0.advance();
+        if (c1.cur == j) c1.advance();
+        const uint32_t next_rec = make_rec(c0, c1);
         for (int which = 0; which < 2 && ok; ++which, ++r) {
           const int s = r % NS;
           const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
@@ -326,6 +368,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             ok = false;
             break;
           }
+          if (which == 1) rec_smem[s] = next_rec;  // released by the arrive below
           mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
           const CUtensorMap* map = which == 0 ? &tmK : &tmV;
           for (int c = 0; c < kChunks; ++c)
@@ -366,11 +409,43 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       // s_ready[k]: S_k of the current key tile was issued during the previous step.
       bool s_ready[2] = {false, false}, started[2] = {false, false};
-      int t = 0;
-      for (int j = union_first(); j >= 0 && ok; j = union_next(j), ++t) {  // last to first
+      // P_k V_j for query tile k (a compile-time constant, so the per-tile state stays in
+      // registers), then S_k of its next key tile if that is the next step's tile (pre), or
+      // the O_k completion signal after its last key tile (last); otherwise S_k waits for the
+      // step of its next key tile.
+      auto tile_step = [&](auto kc, bool pre, bool last, int rK, int sV, bool& next_k_ready) -> bool {
+        constexpr int k = decltype(kc)::value;
+        s_ready[k] = false;
+        const uint32_t par = static_cast<uint32_t>(np[k]) & 1u;
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(bar_p(k, half), par, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) return false;
+          tc_fence_after();
+          issue_pv(k, sV, started[k], 4 * half, 4 * half + 4);
+        }
+        started[k] = true;
+        ++np[k];
+        if (pre) {
+          const int rK2 = rK + 2;  // K of the next step
+          if (!next_k_ready) {
+            if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status,
+                           kStatusFwdTimeout, kWaitTimeoutNs))
+              return false;
+            tc_fence_after();
+            next_k_ready = true;
+          }
+          issue_s(k, rK2 % NS);
+          mma_commit(bar_s(k));
+          s_ready[k] = true;
+        } else if (last) {
+          mma_commit(bar_o(k));
+        }
+        return true;
+      };
+      uint32_t rec = rec_smem[NS];  // published with the Q barrier
+      for (int t = 0; !(rec & kRecEnd) && ok; ++t) {
         const int rK = 2 * t, rV = rK + 1;
         const int sK = rK % NS, sV = rV % NS;
-        const bool in0 = act0 && has(0, j), in1 = act1 && has(1, j);
+        const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
         const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
         if (need0 || need1) {
           // K_j was not needed before: wait for it here (otherwise the previous step did)
@@ -395,44 +470,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ok = false;
           break;
         }
-        const int jn = union_next(j);
+        const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
         bool next_k_ready = false;
-        for (int k = 0; k < 2 && ok; ++k) {
-          s_ready[k] = false;
-          if (!(k == 0 ? in0 : in1)) continue;
-          const uint32_t par = static_cast<uint32_t>(np[k]) & 1u;
-          for (int half = 0; half < 2; ++half) {
-            if (!mbar_wait(bar_p(k, half), par, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_pv(k, sV, started[k], 4 * half, 4 * half + 4);
-          }
-          if (!ok) break;
-          started[k] = true;
-          ++np[k];
-          const int nk = next_of(k, j);
-          if (nk >= 0 && nk == jn) {
-            const int rK2 = rK + 2;  // K of the next step
-            if (!next_k_ready) {
-              if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status,
-                             kStatusFwdTimeout, kWaitTimeoutNs)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              next_k_ready = true;
-            }
-            issue_s(k, rK2 % NS);
-            mma_commit(bar_s(k));
-            s_ready[k] = true;
-          } else if (nk < 0) {
-            mma_commit(bar_o(k));
-          }
-          // otherwise S_k(nk) is issued at the step of key tile nk
-        }
+        if (in0)
+          ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
+        if (ok && in1)
+          ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
+        if (!ok) break;
         mma_commit(bar_empty(sV));
+        rec = next_rec;
       }
       if (!ok) *abort_flag = 1;
       // Drain: all MMAs this thread issued have completed before TMEM is released.
@@ -445,7 +491,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int k = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
     const int wq = warp & 3;          // TMEM lane quarter
     const int row = wq * 32 + lane;   // row inside the tile == TMEM lane
-    const int qi = q0[k] + row;       // absolute query index
+    const int q0k = sel(q0, k), q1k = sel(q1, k);
+    const int qi = q0k + row;         // absolute query index
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + 128u * k;
     const uint32_t tO = tmem + lane_off + 256u + 128u * k;
@@ -469,7 +516,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int n = 0;
     // Key tiles from last to first: with alibi the bias grows with the key index, so the
     // row maximum is met on the first tile and the lazy rescale of O almost never runs.
-    for (int j = act_k ? first_of(k) : -1; j >= 0; j = next_of(k, j), ++n) {
+    auto cur = cursor(k);
+    for (int j = cur.cur; j >= 0; j = cur.cur, ++n) {
+      // With a block mask the class comes from the walk (FULL listed or not).
+      const int cls_blk =
+          cur.cur_full ? (j * kBN + kBN > p.Skv ? kTileFullRagged : kTileFull) : kTilePartial;
+      cur.advance();
       // Warp-uniform decision: the TMEM loads below are warp-collective.
       const bool got = mbar_wait(bar_s(k), static_cast<uint32_t>(n) & 1u, p.status, kStatusFwdTimeout,
                                  kWaitTimeoutNs) &&
@@ -480,11 +532,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tc_fence_after();
       const int k0 = j * kBN;
-      int cls;
-      if constexpr (BLOCKS)
-        cls = bits_has(full_bits(k), j) ? (k0 + kBN > p.Skv ? kTileFullRagged : kTileFull) : kTilePartial;
-      else
-        cls = tile_class<MASK>(q0[k], q1[k], k0, kBN, p.mask);
+      const int cls = BLOCKS ? cls_blk : tile_class<MASK>(q0k, q1k, k0, kBN, p.mask);
       if (write_map)
         p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] =
             static_cast<uint8_t>(cls == kTileFullRagged ? kTilePartial : cls);
