@@ -38,9 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram read+write bytes per launch from ncu, keyed by the hash of the kernel sources
 # they were measured on (a changed kernel reports null until it is captured again)
 MEASURED_TRAFFIC = {
-    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 403,697,408 B read +
-    # 114,692,864 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
-    "1d7a0e1b91413d40": 518390272,
+    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 402,740,480 B read +
+    # 116,575,744 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
+    "60a6582866216d8d": 519316224,
 }
 # the forward kernel's sources: the roofline traffic below belongs to that kernel
 KERNEL_SOURCES = ["attention_flex_attn_b200/csrc/flex_fwd_sm100.cuh",
@@ -236,7 +236,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-case and e2e measurements")
-    ap.add_argument("--profile", choices=["fwd", "fwd8192", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "decode"], default=None,
                     help="run only a few launches of one kernel (for ncu captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -402,9 +402,10 @@ def block_lists(sel):
 
 def block_cases(fa, q, k, v, scale, o, lse):
     """Block-mask forward (flex_attn_fwd_block_sparse) on the forward inputs: causal given
-    as lists (diagonal blocks partial, the rest full), and random per-head lists with half
-    of the key blocks of every query tile full.  TFLOPS count the listed blocks whole
-    (4 * D * 128 * 128 per block), the causal case halves the dense count as above."""
+    as lists (diagonal blocks partial, the rest full); causal attention inside documents
+    of 4..24 whole tiles (useful TFLOPS = 4 * D * kept pairs); random per-head lists with
+    half of the key blocks of every query tile full (TFLOPS count the listed blocks whole,
+    4 * D * 128 * 128 per block).  The causal case halves the dense count as above."""
     import numpy as np
     import torch
     B, H, S, D = q.shape
@@ -419,6 +420,33 @@ def block_cases(fa, q, k, v, scale, o, lse):
     t = _time_fn(lambda: fa.fwd_block_sparse(q, k, v, *lists, scale=scale, mask_mod="causal", out=o,
                                              lse_out=lse), 20, 3)
     res["block_causal_lists"] = {"us": t * 1e6, "tflops": 0.5 * fwd_flops(B, H, S, S, D) / t / 1e12}
+    # documents of 4..24 whole tiles (512..3072 tokens), causal inside each document:
+    # the diagonal block partial, earlier blocks of the same document full
+    rng = np.random.default_rng(4101)
+    starts, t = [], 0
+    while t < nq:
+        starts.append(t)
+        t += int(rng.integers(4, 25))
+    doc_start = np.zeros(nq, np.int64)
+    for s0 in starts:
+        doc_start[s0:] = s0
+    part = np.zeros((1, 1, nq, nk), bool)
+    full = np.zeros((1, 1, nq, nk), bool)
+    for qt in range(nq):
+        part[0, 0, qt, qt] = True
+        full[0, 0, qt, doc_start[qt]:qt] = True
+    kn, ki = block_lists(part)
+    fn, fi = block_lists(full)
+    lists = [torch.from_numpy(a).to(dev) for a in (kn, ki, fn, fi)]
+    t = _time_fn(lambda: fa.fwd_block_sparse(q, k, v, *lists, scale=scale, mask_mod="causal", out=o,
+                                             lse_out=lse), 20, 3)
+    pairs = 0.0  # kept (query, key) pairs per (b, h)
+    ends = starts[1:] + [nq]
+    for s0, e0 in zip(starts, ends):
+        n = (e0 - s0) * 128
+        pairs += n * (n + 1) / 2
+    res["block_document_causal"] = {"us": t * 1e6, "tflops_useful": 4.0 * D * B * H * pairs / t / 1e12,
+                                    "documents": len(starts)}
     rng = np.random.default_rng(4100)
     sel = rng.random((B, H, nq, nk)) < 0.5
     fn, fi = block_lists(sel)
@@ -484,13 +512,22 @@ def e2e(fa, q, k, v, scale, args, dev, world):
 def profile_case(which):
     """A few launches of one kernel on a case larger than L2 but a few GB at most:
     fwd = B2 H32 S4096 D128 bf16 no_mod (192 MiB of Q/K/V); fwd8192 = the full forward
-    workload; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
+    workload; fwd_blocks = the S4096 inputs with random per-head block lists, half of the
+    key blocks of every query tile full; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
     import torch
     import synth
     import attention_flex_attn_b200 as fa
     fa.load_library()
     dev = torch.device("cuda", 0)
-    if which.startswith("fwd"):
+    if which == "fwd_blocks":
+        import numpy as np
+        S, nq = 4096, 32
+        q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
+        sel = np.random.default_rng(4100).random((2, 32, nq, nq)) < 0.5
+        fn, fi = (torch.from_numpy(a).to(dev) for a in block_lists(sel))
+        for _ in range(4):
+            fa.fwd_block_sparse(q, k, v, None, None, fn, fi)
+    elif which.startswith("fwd"):
         S = 8192 if which == "fwd8192" else 4096
         q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
         for _ in range(4):
