@@ -25,7 +25,9 @@ _LIB = os.path.join(_HERE, "_flex_oracle.so")
 SCORE_MODS = {"none": 0, "alibi": 1}
 MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset": 3,
              # causal=True is the same keep rule as causal_via_mask
-             "causal_fast": 1}
+             "causal_fast": 1,
+             # tensor-capturing: same document under per-batch boundary offsets (+ causal)
+             "document": 5, "document_causal": 6}
 
 _lib = None
 
@@ -40,18 +42,18 @@ def build(force: bool = False) -> str:
 
 def _bind(lib):
     P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
-    lib.oracle_fwd.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, I64, P, P, P, I]
+    lib.oracle_fwd.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, I, P, I64, P, P, P, I]
     lib.oracle_fwd.restype = I
     lib.oracle_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, D, P, P, I]
     lib.oracle_decode.restype = I
-    lib.oracle_mask_matrix.argtypes = [I, I, I, I, I, P]
+    lib.oracle_mask_matrix.argtypes = [I, I, I, I, I, P, P, I, P]
     lib.oracle_mask_matrix.restype = I
-    lib.oracle_tile_map.argtypes = [I, I, I, I, I, I, I, P]
+    lib.oracle_tile_map.argtypes = [I, I, I, I, I, P, P, I, I, I, P]
     lib.oracle_tile_map.restype = I
     lib.oracle_alibi_slope.argtypes = [I, I]
     lib.oracle_alibi_slope.restype = D
-    lib.oracle_fwd_block_sparse.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, P, I, I, I,
-                                            P, I64, P, P, I]
+    lib.oracle_fwd_block_sparse.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, I,
+                                            P, P, P, P, I, I, I, P, I64, P, P, I]
     lib.oracle_fwd_block_sparse.restype = I
     return lib
 
@@ -92,16 +94,46 @@ def default_threads() -> int:
         return os.cpu_count() or 1
 
 
+def _captured(B, H, mask_mod, alibi_slopes, doc_offsets, doc_offsets_kv):
+    """float64 [H] slopes and int32 [B, n_docs + 1] boundary arrays (or None), and n_docs."""
+    slopes = None
+    if alibi_slopes is not None:
+        if isinstance(alibi_slopes, torch.Tensor):
+            alibi_slopes = alibi_slopes.detach().cpu().double().numpy()
+        slopes = np.ascontiguousarray(np.asarray(alibi_slopes, dtype=np.float64).reshape(H))
+    oq = okv = None
+    n_docs = 0
+    if mask_mod in ("document", "document_causal"):
+        if doc_offsets is None:
+            raise ValueError("document masks need doc_offsets")
+        oq = _i32(doc_offsets).reshape(B, -1)
+        okv = oq if doc_offsets_kv is None else _i32(doc_offsets_kv).reshape(B, -1)
+        if okv.shape != oq.shape:
+            raise ValueError("doc_offsets and doc_offsets_kv differ in shape")
+        oq, okv = np.ascontiguousarray(oq), np.ascontiguousarray(okv)
+        n_docs = oq.shape[1] - 1
+    return slopes, oq, okv, n_docs
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
 def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
-        rows=None, want_probs=False, threads=None):
+        rows=None, want_probs=False, threads=None, alibi_slopes=None, doc_offsets=None,
+        doc_offsets_kv=None):
     """Oracle forward.  q [B,H,Sq,D], k/v [B,Hkv,Skv,D] (CPU bf16/f16 tensors).
 
     rows: optional int64 array of flattened (b*H + h)*Sq + i row indices.
+    alibi_slopes: [H] slopes for score_mod="alibi" (default: 2^(-8(h+1)/H)).
+    doc_offsets / doc_offsets_kv: [B, n_docs + 1] document boundaries of the query / key
+    positions for mask_mod "document" / "document_causal" (kv defaults to the query's).
     Returns (O, LSE[, P]) as float64 numpy arrays; O is [B,H,Sq,D] / LSE
     [B,H,Sq] for all rows, or [n,D] / [n] for a row subset.
     """
     lib = _load()
     B, H, Sq, D = q.shape
+    slopes, oq, okv, n_docs = _captured(B, H, mask_mod, alibi_slopes, doc_offsets, doc_offsets_kv)
     Bk, Hkv, Skv, Dk = k.shape
     assert Bk == B and Dk == D and tuple(v.shape) == tuple(k.shape)
     assert q.dtype == k.dtype == v.dtype
@@ -120,6 +152,7 @@ def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset
     rc = lib.oracle_fwd(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, _dtype_code(q),
                         B, H, Hkv, Sq, Skv, D, float(scale),
                         SCORE_MODS[score_mod], MASK_MODS[mask_mod], int(window), int(offset),
+                        _p(slopes), _p(oq), _p(okv), n_docs,
                         None if rows_arr is None else rows_arr.ctypes.data, n,
                         o.ctypes.data, lse.ctypes.data,
                         None if probs is None else probs.ctypes.data,
@@ -144,7 +177,7 @@ def _i32(a):
 
 def fwd_block_sparse(q, k, v, kv_num, kv_idx, full_num=None, full_idx=None, scale=None,
                      score_mod="none", mask_mod="none", window=0, offset=0, bm=128, bn=128,
-                     rows=None, threads=None):
+                     rows=None, threads=None, alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None):
     """Oracle forward with a block mask (BlockMask: FlyDSL PR 931 "Add flex_attention
     (score_mod / mask_mod) ...", Out of scope, names block sparsity as the next phase;
     the list convention is PyTorch's).
@@ -159,6 +192,7 @@ def fwd_block_sparse(q, k, v, kv_num, kv_idx, full_num=None, full_idx=None, scal
     lib = _load()
     B, H, Sq, D = q.shape
     _, Hkv, Skv, _ = k.shape
+    slopes, oq, okv, n_docs = _captured(B, H, mask_mod, alibi_slopes, doc_offsets, doc_offsets_kv)
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     nq = -(-Sq // bm)
@@ -183,6 +217,7 @@ def fwd_block_sparse(q, k, v, kv_num, kv_idx, full_num=None, full_idx=None, scal
     rc = lib.oracle_fwd_block_sparse(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, _dtype_code(q),
                                      B, H, Hkv, Sq, Skv, D, float(scale), SCORE_MODS[score_mod],
                                      MASK_MODS[mask_mod], int(window), int(offset),
+                                     _p(slopes), _p(oq), _p(okv), n_docs,
                                      ptr(kn), ptr(ki), ptr(fn), ptr(fi), int(max_blocks), int(bm), int(bn),
                                      None if rows_arr is None else rows_arr.ctypes.data, n,
                                      o.ctypes.data, lse.ctypes.data, int(threads or default_threads()))
@@ -233,22 +268,30 @@ def decode(q, k_cache, v_cache, kv_len, scale, mask=None, threads=None):
     return o.reshape(B, H, 1, D), lse.reshape(B, H, 1)
 
 
-def mask_matrix(mask_mod, Sq, Skv, window=0, offset=0) -> np.ndarray:
-    """uint8 [Sq, Skv]: 1 where mask_mod keeps (i, j)."""
+def mask_matrix(mask_mod, Sq, Skv, window=0, offset=0, doc_offsets=None, doc_offsets_kv=None) -> np.ndarray:
+    """uint8 [Sq, Skv]: 1 where mask_mod keeps (i, j) (document masks: one batch's
+    boundaries, [n_docs + 1])."""
     lib = _load()
+    _, oq, okv, n_docs = _captured(1, 1, mask_mod, None, doc_offsets, doc_offsets_kv)
     out = np.zeros((Sq, Skv), dtype=np.uint8)
-    lib.oracle_mask_matrix(MASK_MODS[mask_mod], Sq, Skv, int(window), int(offset), out.ctypes.data)
+    rc = lib.oracle_mask_matrix(MASK_MODS[mask_mod], Sq, Skv, int(window), int(offset), _p(oq), _p(okv), n_docs,
+                                out.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_mask_matrix rejected its arguments (rc={rc})")
     return out
 
 
-def tile_map(mask_mod, Sq, Skv, window=0, offset=0, bm=128, bn=128) -> np.ndarray:
+def tile_map(mask_mod, Sq, Skv, window=0, offset=0, bm=128, bn=128, doc_offsets=None,
+             doc_offsets_kv=None) -> np.ndarray:
     """uint8 [ceil(Sq/bm), ceil(Skv/bn)]: 0 EMPTY, 1 FULL, 2 PARTIAL."""
     lib = _load()
+    _, oq, okv, n_docs = _captured(1, 1, mask_mod, None, doc_offsets, doc_offsets_kv)
     nq, nk = -(-Sq // bm), -(-Skv // bn)
     out = np.zeros((nq, nk), dtype=np.uint8)
-    rc = lib.oracle_tile_map(MASK_MODS[mask_mod], Sq, Skv, int(window), int(offset), bm, bn, out.ctypes.data)
+    rc = lib.oracle_tile_map(MASK_MODS[mask_mod], Sq, Skv, int(window), int(offset), _p(oq), _p(okv), n_docs,
+                             bm, bn, out.ctypes.data)
     if rc != 0:
-        raise ValueError("bad tile size")
+        raise ValueError(f"oracle_tile_map rejected its arguments (rc={rc})")
     return out
 
 

@@ -34,6 +34,10 @@
  * f16 additive mask operand): x_j = scale * q.k_j + mask[b,h,j] for j < kv_len[b];
  * keep_j = (x_j != -inf); then the same softmax as above.
  *
+ * Tensor-capturing mods (FlyDSL PR 931, Out of scope: a later phase, undefined; the
+ * readings are stated at keep_rule below): alibi with a captured per-head slope table,
+ * and a document mask (optionally causal) over per-batch document boundaries.
+ *
  * Block-sparse forward (BlockMask; FlyDSL PR 931, "Out of scope (future phases)":
  * block sparsity named as the next phase, with no definition given).  Reading: the
  * PyTorch BlockMask convention.  For query tile t = i / BM of (b, h), a key j with
@@ -63,6 +67,8 @@
 #define OR_MASK_CAUSAL 1
 #define OR_MASK_SLIDING 2
 #define OR_MASK_OFFSET 3
+#define OR_MASK_DOC 5
+#define OR_MASK_DOC_CAUSAL 6
 
 #define OR_DT_BF16 0
 #define OR_DT_F16 1
@@ -109,6 +115,40 @@ int oracle_mask_keep(int mask_mod, int64_t i, int64_t j, int window, int offset)
   }
 }
 
+/* Tensor-capturing mods (FlyDSL PR 931, Out of scope: "tensor-capturing mods" named as a
+ * later phase, undefined).  Readings:
+ *  - alibi with a captured per-head slope table: s += slopes[h] * (j - i);
+ *  - document mask over packed sequences: the captured tensors give, per batch b, the
+ *    document boundaries off_q[b][0..n_docs] of the query positions and off_kv[b][..]
+ *    of the key positions; position p is in document d iff off[d] <= p < off[d+1], and
+ *    in none if no such d.  Keep (i, j) iff i and j are in the same document d (and,
+ *    for the causal form, j <= i in absolute positions). */
+typedef struct {
+  const double* slopes;          /* [H], or NULL for the built-in slopes */
+  const int32_t *off_q, *off_kv; /* [B][n_docs + 1] */
+  int n_docs;
+} captured_mods;
+
+/* Document d with off[d] <= pos < off[d+1], or -1 (a plain scan of the boundaries). */
+static int64_t doc_of(const int32_t* off, int n_docs, int64_t pos) {
+  for (int d = 0; d < n_docs; ++d)
+    if ((int64_t)off[d] <= pos && pos < (int64_t)off[d + 1]) return d;
+  return -1;
+}
+
+/* The keep rule of element (i, j) of batch b, mask_mod with its parameters. */
+static int keep_rule(int mask_mod, int window, int offset, const captured_mods* C, int b, int64_t i,
+                     int64_t j) {
+  if (mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) {
+    const int32_t* oq = C->off_q + (int64_t)b * (C->n_docs + 1);
+    const int32_t* okv = C->off_kv + (int64_t)b * (C->n_docs + 1);
+    int64_t dq = doc_of(oq, C->n_docs, i);
+    if (dq < 0 || dq != doc_of(okv, C->n_docs, j)) return 0;
+    return mask_mod == OR_MASK_DOC || j <= i;
+  }
+  return oracle_mask_keep(mask_mod, i, j, window, offset);
+}
+
 /* Block mask (BlockMask).  Reading: PyTorch's convention.  For query tile t of one
  * (b, h) (tile_row = (b*H + h) * n_qtiles + t), the key blocks u listed in
  * full_idx[tile_row, 0 .. full_num) are kept wholesale (only j < Skv applies), those in
@@ -130,12 +170,12 @@ static int block_listed(const int32_t* num, const int32_t* idx, int64_t row, int
 }
 
 static int block_keep(const block_lists* L, int64_t bh, int mask_mod, int64_t i, int64_t j, int Skv,
-                      int window, int offset) {
+                      int window, int offset, const captured_mods* C, int b) {
   if (j >= Skv) return 0;
   int64_t tile_row = bh * L->n_qtiles + i / L->BM;
   int64_t u = j / L->BN;
   if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;
-  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return oracle_mask_keep(mask_mod, i, j, window, offset);
+  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return keep_rule(mask_mod, window, offset, C, b, i, j);
   return 0;
 }
 
@@ -152,6 +192,7 @@ typedef struct {
   double* lse;           /* [n_rows] */
   double* probs;         /* optional [n_rows, Skv] normalised weights */
   const block_lists* blk; /* block mask, or NULL for mask_mod alone */
+  captured_mods cap;      /* captured tensors of the mods */
   int64_t r0, r1;
 } fwd_job;
 
@@ -166,7 +207,8 @@ static void fwd_row(const fwd_job* J, int64_t r, double* x, unsigned char* keep)
   int D = J->D;
   const int64_t qbase = flat * D;
   const int64_t kvbase = ((int64_t)b * J->Hkv + hk) * (int64_t)J->Skv * D;
-  double slope = (J->score_mod == OR_SCORE_ALIBI) ? oracle_alibi_slope(h, J->H) : 0.0;
+  double slope = 0.0;
+  if (J->score_mod == OR_SCORE_ALIBI) slope = J->cap.slopes ? J->cap.slopes[h] : oracle_alibi_slope(h, J->H);
 
   double M = -INFINITY;
   int any = 0;
@@ -177,8 +219,9 @@ static void fwd_row(const fwd_job* J, int64_t r, double* x, unsigned char* keep)
     double s = J->scale * dot;
     if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);
     x[j] = s;
-    keep[j] = (unsigned char)(J->blk ? block_keep(J->blk, bh, J->mask_mod, i, j, J->Skv, J->window, J->offset)
-                                     : oracle_mask_keep(J->mask_mod, i, j, J->window, J->offset));
+    keep[j] = (unsigned char)(J->blk ? block_keep(J->blk, bh, J->mask_mod, i, j, J->Skv, J->window, J->offset,
+                                                  &J->cap, b)
+                                     : keep_rule(J->mask_mod, J->window, J->offset, &J->cap, b, i, j));
     if (keep[j]) {
       any = 1;
       if (s > M) M = s;
@@ -242,9 +285,11 @@ static int run_jobs(fwd_job* base, int64_t n_rows, int nthreads, void* (*fn)(voi
 }
 
 /* Forward over selected rows (rows == NULL: all B*H*Sq rows). */
+/* slopes, off_q, off_kv: the captured tensors (NULL when the mods take none). */
 int oracle_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dtype,
                int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
                int score_mod, int mask_mod, int window, int offset,
+               const double* slopes, const int32_t* off_q, const int32_t* off_kv, int n_docs,
                const int64_t* rows, int64_t n_rows,
                double* o, double* lse, double* probs, int nthreads) {
   if (H <= 0 || Hkv <= 0 || H % Hkv != 0 || Sq <= 0 || Skv <= 0 || D <= 0) return -1;
@@ -257,6 +302,8 @@ int oracle_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dtyp
   J.rows = rows;
   J.n_rows = rows ? n_rows : (int64_t)B * H * Sq;
   J.o = o; J.lse = lse; J.probs = probs;
+  J.cap.slopes = slopes; J.cap.off_q = off_q; J.cap.off_kv = off_kv; J.cap.n_docs = n_docs;
+  if ((mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) && (!off_q || !off_kv || n_docs < 0)) return -2;
   return run_jobs(&J, J.n_rows, nthreads, fwd_worker, sizeof J);
 }
 
@@ -358,6 +405,7 @@ int oracle_decode(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
 int oracle_fwd_block_sparse(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dtype,
                             int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
                             int score_mod, int mask_mod, int window, int offset,
+                            const double* slopes, const int32_t* off_q, const int32_t* off_kv, int n_docs,
                             const int32_t* kv_num, const int32_t* kv_idx, const int32_t* full_num,
                             const int32_t* full_idx, int max_blocks, int BM, int BN,
                             const int64_t* rows, int64_t n_rows, double* o, double* lse, int nthreads) {
@@ -375,22 +423,31 @@ int oracle_fwd_block_sparse(const uint16_t* q, const uint16_t* k, const uint16_t
   J.rows = rows;
   J.n_rows = rows ? n_rows : (int64_t)B * H * Sq;
   J.o = o; J.lse = lse; J.blk = &L;
+  J.cap.slopes = slopes; J.cap.off_q = off_q; J.cap.off_kv = off_kv; J.cap.n_docs = n_docs;
+  if ((mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) && (!off_q || !off_kv || n_docs < 0)) return -2;
   return run_jobs(&J, J.n_rows, nthreads, fwd_worker, sizeof J);
 }
 
 /* ---- element mask and tile map (brute force) ------------------------------- */
 
-/* keep[i*Skv + j] = mask_mod(i, j) for every i < Sq, j < Skv. */
-int oracle_mask_matrix(int mask_mod, int Sq, int Skv, int window, int offset, uint8_t* keep) {
+/* keep[i*Skv + j] = mask_mod(i, j) for every i < Sq, j < Skv (document masks: the
+ * boundaries off_q / off_kv of one batch, n_docs + 1 entries each). */
+int oracle_mask_matrix(int mask_mod, int Sq, int Skv, int window, int offset, const int32_t* off_q,
+                       const int32_t* off_kv, int n_docs, uint8_t* keep) {
+  captured_mods C = {NULL, off_q, off_kv, n_docs};
+  if ((mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) && (!off_q || !off_kv)) return -2;
   for (int64_t i = 0; i < Sq; ++i)
     for (int64_t j = 0; j < Skv; ++j)
-      keep[i * Skv + j] = (uint8_t)oracle_mask_keep(mask_mod, i, j, window, offset);
+      keep[i * Skv + j] = (uint8_t)keep_rule(mask_mod, window, offset, &C, 0, i, j);
   return 0;
 }
 
 /* map[t*nkv + u] in {0 EMPTY, 1 FULL, 2 PARTIAL}; nq = ceil(Sq/BM), nkv = ceil(Skv/BN). */
-int oracle_tile_map(int mask_mod, int Sq, int Skv, int window, int offset, int BM, int BN, uint8_t* map) {
+int oracle_tile_map(int mask_mod, int Sq, int Skv, int window, int offset, const int32_t* off_q,
+                    const int32_t* off_kv, int n_docs, int BM, int BN, uint8_t* map) {
+  captured_mods C = {NULL, off_q, off_kv, n_docs};
   if (BM <= 0 || BN <= 0) return -1;
+  if ((mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) && (!off_q || !off_kv)) return -2;
   int nq = (Sq + BM - 1) / BM, nkv = (Skv + BN - 1) / BN;
   for (int t = 0; t < nq; ++t) {
     for (int u = 0; u < nkv; ++u) {
@@ -398,7 +455,7 @@ int oracle_tile_map(int mask_mod, int Sq, int Skv, int window, int offset, int B
       for (int64_t i = (int64_t)t * BM; i < (int64_t)(t + 1) * BM && i < Sq; ++i) {
         for (int64_t j = (int64_t)u * BN; j < (int64_t)(u + 1) * BN; ++j) {
           ++total;
-          if (j < Skv && oracle_mask_keep(mask_mod, i, j, window, offset)) ++kept;
+          if (j < Skv && keep_rule(mask_mod, window, offset, &C, 0, i, j)) ++kept;
         }
       }
       map[(int64_t)t * nkv + u] = (uint8_t)(kept == 0 ? 0 : (kept == total ? 1 : 2));

@@ -1,5 +1,5 @@
 """Plants plausible mistakes in copies of the C oracle and checks that the pins in
-test_oracle_pins.py and test_oracle_block_pins.py catch every one (each mutant must fail at least one pin).
+test_oracle_pins.py, test_oracle_block_pins.py and test_oracle_mods_pins.py catch every one (each mutant must fail at least one pin).
 Everything runs on the CPU against a temporary build; the real oracle is untouched.
 Mutants that leave the mathematics unchanged (e.g. dropping the fully-masked guard,
 which still yields p = 0 and log 0 = -inf) are not listed: no test could tell them apart."""
@@ -12,6 +12,7 @@ import torch
 
 import oracle
 import tests.test_oracle_block_pins as bpins
+import tests.test_oracle_mods_pins as mpins
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "flex_oracle.c")
@@ -40,13 +41,20 @@ MUTANTS = [
     ("decode empty row LSE 0", "  if (M == -INFINITY) {   /* kv_len == 0 or every position masked */\n    J->lse[r] = -INFINITY;",
      "  if (M == -INFINITY) {   /* kv_len == 0 or every position masked */\n    J->lse[r] = 0.0;"),
     ("tile classes swapped", "(kept == total ? 1 : 2)", "(kept == total ? 2 : 1)"),
-    ("tile ignores pad", "if (j < Skv && oracle_mask_keep(", "if (oracle_mask_keep("),
+    ("tile ignores pad", "if (j < Skv && keep_rule(", "if (keep_rule("),
     ("block: full list ignored", "  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;\n", ""),
-    ("block: partial skips mask_mod", "u)) return oracle_mask_keep(mask_mod, i, j, window, offset);", "u)) return 1;"),
+    ("block: partial skips mask_mod", "u)) return keep_rule(mask_mod, window, offset, C, b, i, j);", "u)) return 1;"),
     ("block: partial beats full",
-     "  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;\n  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return oracle_mask_keep(mask_mod, i, j, window, offset);",
-     "  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return oracle_mask_keep(mask_mod, i, j, window, offset);\n  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;"),
+     "  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;\n  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return keep_rule(mask_mod, window, offset, C, b, i, j);",
+     "  if (block_listed(L->kv_num, L->kv_idx, tile_row, L->max_blocks, u)) return keep_rule(mask_mod, window, offset, C, b, i, j);\n  if (block_listed(L->full_num, L->full_idx, tile_row, L->max_blocks, u)) return 1;"),
     ("block: query tile from BN", "int64_t tile_row = bh * L->n_qtiles + i / L->BM;", "int64_t tile_row = bh * L->n_qtiles + i / L->BN;"),
+    ("document end inclusive", "pos < (int64_t)off[d + 1]) return d;", "pos <= (int64_t)off[d + 1]) return d;"),
+    ("document causal ignored", "return mask_mod == OR_MASK_DOC || j <= i;", "return 1;"),
+    ("document keys use query boundaries", "const int32_t* okv = C->off_kv + (int64_t)b", "const int32_t* okv = C->off_q + (int64_t)b"),
+    ("document of batch 0 for every batch", "const int32_t* oq = C->off_q + (int64_t)b * (C->n_docs + 1);",
+     "const int32_t* oq = C->off_q;"),
+    ("slope table ignored", "slope = J->cap.slopes ? J->cap.slopes[h] : oracle_alibi_slope(h, J->H);",
+     "slope = oracle_alibi_slope(h, J->H);"),
     ("bf16 decoded as truncated", "  uint32_t u = ((uint32_t)b) << 16;", "  uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
 ]
 
@@ -77,6 +85,11 @@ CHECKS = [
     (bpins.test_full_block_beats_partial_and_ignores_mask_mod, {}),
     (bpins.test_every_block_full_equals_no_mask, {}),
     (bpins.test_empty_block_mask_gives_zero_rows, {}),
+    (mpins.test_random_slope_table_equals_torch, {}),
+    (mpins.test_document_masks_equal_torch, {"case": "packed", "causal": True}),
+    (mpins.test_document_masks_equal_torch, {"case": "tail_unassigned", "causal": False}),
+    (mpins.test_document_masks_equal_torch, {"case": "cross", "causal": False}),
+    (mpins.test_document_mask_matrix_and_tile_map, {"causal": True}),
 ]
 
 
