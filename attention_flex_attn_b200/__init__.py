@@ -21,7 +21,9 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "misaligned", 4: 
           5: "CUDA error", 6: "device timeout"}
 DTYPES = {torch.bfloat16: 0, torch.float16: 1}
 SCORE_MODS = {"none": 0, "alibi": 1}
-MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset": 3, "causal_fast": 4}
+SCORE_ALIBI_SLOPES = 2  # alibi with a captured slope tensor
+MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset": 3, "causal_fast": 4,
+             "document": 5, "document_causal": 6}
 FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
@@ -36,7 +38,9 @@ class FlexAttnError(RuntimeError):
 
 class ModParams(ctypes.Structure):
     _fields_ = [("window", ctypes.c_int32), ("offset", ctypes.c_int32),
-                ("flags", ctypes.c_uint32), ("tile_map_out", ctypes.c_void_p)]
+                ("flags", ctypes.c_uint32), ("tile_map_out", ctypes.c_void_p),
+                ("alibi_slopes", ctypes.c_void_p), ("doc_offsets_q", ctypes.c_void_p),
+                ("doc_offsets_kv", ctypes.c_void_p), ("n_docs", ctypes.c_int32)]
 
 
 class BlockMaskC(ctypes.Structure):
@@ -129,20 +133,56 @@ def _fwd_args(q, k, v, scale, return_lse, out, lse_out):
     return B, H, Hkv, Sq, Skv, D, float(scale), o, lse
 
 
+def _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
+                doc_offsets_kv):
+    """ModParams and the score_mod id; the captured tensors are checked, not copied."""
+    score = SCORE_MODS[score_mod]
+    slopes_ptr = None
+    if alibi_slopes is not None:
+        if score_mod != "alibi":
+            raise FlexAttnError("alibi_slopes go with score_mod='alibi'")
+        _cuda_tensor(alibi_slopes, "alibi_slopes")
+        if alibi_slopes.dtype != torch.float32 or alibi_slopes.numel() != H:
+            raise FlexAttnError("alibi_slopes must be float32 with H entries")
+        score, slopes_ptr = SCORE_ALIBI_SLOPES, alibi_slopes.data_ptr()
+    oq = okv = None
+    n_docs = 0
+    if mask_mod in ("document", "document_causal"):
+        if doc_offsets is None:
+            raise FlexAttnError("document masks need doc_offsets [B, n_docs + 1] (int32, CUDA)")
+        for t, n in ((doc_offsets, "doc_offsets"), (doc_offsets_kv, "doc_offsets_kv")):
+            if t is None:
+                continue
+            _cuda_tensor(t, n)
+            if t.dtype != torch.int32 or t.dim() != 2 or t.shape[0] != B or t.shape[1] < 1:
+                raise FlexAttnError(f"{n} must be int32 [B, n_docs + 1]")
+        if doc_offsets_kv is not None and tuple(doc_offsets_kv.shape) != tuple(doc_offsets.shape):
+            raise FlexAttnError("doc_offsets_kv must have the shape of doc_offsets")
+        oq = doc_offsets.data_ptr()
+        okv = None if doc_offsets_kv is None else doc_offsets_kv.data_ptr()
+        n_docs = doc_offsets.shape[1] - 1
+    mp = ModParams(int(window), int(offset), FLAG_TILE_MAP if tile_map is not None else 0,
+                   tile_map.data_ptr() if tile_map is not None else None, slopes_ptr, oq, okv, n_docs)
+    return mp, score
+
+
 def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
-        return_lse=True, out=None, lse_out=None, tile_map=None):
+        return_lse=True, out=None, lse_out=None, tile_map=None, alibi_slopes=None, doc_offsets=None,
+        doc_offsets_kv=None):
     """Flex-attention forward.  q [B,H,Sq,D], k/v [B,Hkv,Skv,D] (bf16 or f16, CUDA).
 
     Returns (O, LSE) (LSE is None when return_lse is False).  ``tile_map``: optional
     uint8 CUDA tensor of ceil(Sq/BM)*ceil(Skv/BN) bytes that receives the tile classes
-    of batch 0 / head 0.
+    of batch 0 / head 0.  Captured tensors: ``alibi_slopes`` (float32 [H], with
+    score_mod="alibi"); ``doc_offsets`` / ``doc_offsets_kv`` (int32 [B, n_docs + 1]
+    document boundaries, with mask_mod "document" or "document_causal").
     """
     lib = load_library()
     B, H, Hkv, Sq, Skv, D, scale, o, lse = _fwd_args(q, k, v, scale, return_lse, out, lse_out)
-    mp = ModParams(int(window), int(offset), FLAG_TILE_MAP if tile_map is not None else 0,
-                   tile_map.data_ptr() if tile_map is not None else None)
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
+                            doc_offsets_kv)
     rc = lib.flex_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
-                           scale, SCORE_MODS[score_mod], MASK_MODS[mask_mod], ctypes.byref(mp),
+                           scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
                            DTYPES[q.dtype], _stream(q.device))
     _check(rc, "flex_attn_fwd")
     return o, lse
@@ -150,7 +190,8 @@ def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset
 
 def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None, full_kv_indices=None,
                      scale=None, score_mod="none", mask_mod="none", window=0, offset=0, return_lse=True,
-                     out=None, lse_out=None, tile_map=None, block_size=128):
+                     out=None, lse_out=None, tile_map=None, block_size=128, alibi_slopes=None, doc_offsets=None,
+                     doc_offsets_kv=None):
     """Forward with a block mask (flex_attn_fwd_block_sparse).  The block lists are int32
     CUDA tensors: counts [Bm, Hm, ceil(Sq/128)], indices [Bm, Hm, ceil(Sq/128), max_blocks],
     Bm in {1, B}, Hm in {1, H}; either (counts, indices) pair may be None, not both.
@@ -179,10 +220,10 @@ def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None
                     shape[3], shape[0], shape[1], int(block_size), int(block_size))
     if shape[2] != -(-Sq // 128):
         raise FlexAttnError(f"block mask has {shape[2]} query tiles, Sq={Sq} needs {-(-Sq // 128)}")
-    mp = ModParams(int(window), int(offset), FLAG_TILE_MAP if tile_map is not None else 0,
-                   tile_map.data_ptr() if tile_map is not None else None)
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
+                            doc_offsets_kv)
     rc = lib.flex_attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
-                                        scale, SCORE_MODS[score_mod], MASK_MODS[mask_mod], ctypes.byref(mp),
+                                        scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
                                         ctypes.byref(bm), DTYPES[q.dtype], _stream(q.device))
     _check(rc, "flex_attn_fwd_block_sparse")
     return o, lse
@@ -243,11 +284,13 @@ def decode_noalloc(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_
     return o, lse
 
 
-def mask_eval(mask_mod, Sq, Skv, window=0, offset=0, device="cuda"):
-    """uint8 [Sq, Skv] CUDA tensor of the forward kernel's keep decisions."""
+def mask_eval(mask_mod, Sq, Skv, window=0, offset=0, device="cuda", doc_offsets=None, doc_offsets_kv=None):
+    """uint8 [Sq, Skv] CUDA tensor of the forward kernel's keep decisions (document
+    masks: the boundaries of batch 0, int32 [1, n_docs + 1] or [B, n_docs + 1])."""
     lib = load_library()
     keep = torch.empty((Sq, Skv), dtype=torch.uint8, device=device)
-    mp = ModParams(int(window), int(offset), 0, None)
+    B = 1 if doc_offsets is None else doc_offsets.shape[0]
+    mp, _ = _mod_params(B, 1, "none", mask_mod, window, offset, None, None, doc_offsets, doc_offsets_kv)
     rc = lib.flex_attn_mask_eval(MASK_MODS[mask_mod], ctypes.byref(mp), Sq, Skv, _ptr(keep), _stream(keep.device))
     _check(rc, "flex_attn_mask_eval")
     return keep

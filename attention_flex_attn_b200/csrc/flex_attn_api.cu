@@ -123,6 +123,38 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned* status) {
   mbar_wait(b, 0, status, kStatusSelftestTimeout, timeout_ns);
 }
 
+// Kernel mask kind of a flex_mask_mod_t, or -1.
+int mask_kind(int mask_mod_id) {
+  switch (mask_mod_id) {
+    case FLEX_MASK_NONE: return kMaskNone;
+    case FLEX_MASK_CAUSAL:
+    case FLEX_MASK_CAUSAL_FAST: return kMaskCausal;
+    case FLEX_MASK_SLIDING_WINDOW: return kMaskSliding;
+    case FLEX_MASK_KV_LE_Q_PLUS_OFFSET: return kMaskOffset;
+    case FLEX_MASK_DOCUMENT: return kMaskDocument;
+    case FLEX_MASK_DOCUMENT_CAUSAL: return kMaskDocumentCausal;
+  }
+  return -1;
+}
+
+// The document rules' captured boundaries: present, aligned, of a size that indexes in int64.
+flex_status_t check_documents(int mask, const flex_mod_params_t& mp) {
+  if (mask != kMaskDocument && mask != kMaskDocumentCausal) return FLEX_OK;
+  if (!mp.doc_offsets_q || mp.n_docs < 0 || mp.n_docs > (1 << 24)) return FLEX_ERR_INVALID_ARG;
+  if (!aligned4(mp.doc_offsets_q) || (mp.doc_offsets_kv && !aligned4(mp.doc_offsets_kv))) return FLEX_ERR_MISALIGNED;
+  return FLEX_OK;
+}
+
+MaskArgs mask_args(int mask, const flex_mod_params_t& mp, int Skv) {
+  MaskArgs m{Skv, mp.window, mp.offset};
+  if (mask == kMaskDocument || mask == kMaskDocumentCausal) {
+    m.off_q = mp.doc_offsets_q;
+    m.off_kv = mp.doc_offsets_kv ? mp.doc_offsets_kv : mp.doc_offsets_q;
+    m.n_docs = mp.n_docs;
+  }
+  return m;
+}
+
 // Shared body of flex_attn_fwd (bm == nullptr) and flex_attn_fwd_block_sparse.
 flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
                          int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
@@ -133,19 +165,21 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
   if (dtype != FLEX_DTYPE_BF16 && dtype != FLEX_DTYPE_F16) return FLEX_ERR_UNSUPPORTED;
-  if (score_mod_id != FLEX_SCORE_NONE && score_mod_id != FLEX_SCORE_ALIBI) return FLEX_ERR_INVALID_ARG;
-  int mask = -1;
-  switch (mask_mod_id) {
-    case FLEX_MASK_NONE: mask = kMaskNone; break;
-    case FLEX_MASK_CAUSAL:
-    case FLEX_MASK_CAUSAL_FAST: mask = kMaskCausal; break;
-    case FLEX_MASK_SLIDING_WINDOW: mask = kMaskSliding; break;
-    case FLEX_MASK_KV_LE_Q_PLUS_OFFSET: mask = kMaskOffset; break;
-    default: return FLEX_ERR_INVALID_ARG;
-  }
+  if (score_mod_id != FLEX_SCORE_NONE && score_mod_id != FLEX_SCORE_ALIBI && score_mod_id != FLEX_SCORE_ALIBI_SLOPES)
+    return FLEX_ERR_INVALID_ARG;
+  const int mask = mask_kind(mask_mod_id);
+  if (mask < 0) return FLEX_ERR_INVALID_ARG;
   const flex_mod_params_t zero{};
   const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
   if (mask == kMaskSliding && mp.window < 1) return FLEX_ERR_INVALID_ARG;
+  if (score_mod_id == FLEX_SCORE_ALIBI_SLOPES) {
+    if (!mp.alibi_slopes) return FLEX_ERR_INVALID_ARG;
+    if (!aligned4(mp.alibi_slopes)) return FLEX_ERR_MISALIGNED;
+  }
+  if (const flex_status_t ds = check_documents(mask, mp); ds != FLEX_OK) return ds;
+  // document masks walk per-CTA bitmaps of key tiles, like block masks
+  if ((mask == kMaskDocument || mask == kMaskDocumentCausal) && (Skv + kBN - 1) / kBN > kMaxBlockKeyTiles)
+    return FLEX_ERR_UNSUPPORTED;
   const bool want_map = (mp.flags & FLEX_FLAG_TILE_MAP) != 0;
   if (want_map && !mp.tile_map_out) return FLEX_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
@@ -192,7 +226,9 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   p.n_ktiles = (Skv + kBN - 1) / kBN;
   p.n_pairs = n_pairs;
   p.scale_log2 = scale * kLog2e;
-  p.mask = MaskArgs{Skv, mp.window, mp.offset};
+  p.mask = mask_args(mask, mp, Skv);
+  p.slopes = score_mod_id == FLEX_SCORE_ALIBI_SLOPES ? mp.alibi_slopes : nullptr;
+  const int score = score_mod_id == FLEX_SCORE_NONE ? kScoreNone : kScoreAlibi;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int units = static_cast<int>(n_units);
   if (bm) {
@@ -203,11 +239,11 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
     p.blk_max = bm->max_blocks;
     p.blk_b_stride = bm->batch == 1 ? 0 : bm->heads;
     p.blk_h_stride = bm->heads == 1 ? 0 : 1;
-    return D == 128 ? fwd_dispatch<128, true>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s)
-                    : fwd_dispatch<64, true>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s);
+    return D == 128 ? fwd_dispatch<128, true>(dtype, score, mask, mq, mk, mv, p, units, s)
+                    : fwd_dispatch<64, true>(dtype, score, mask, mq, mk, mv, p, units, s);
   }
-  return D == 128 ? fwd_dispatch<128, false>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s)
-                  : fwd_dispatch<64, false>(dtype, score_mod_id, mask, mq, mk, mv, p, units, s);
+  return D == 128 ? fwd_dispatch<128, false>(dtype, score, mask, mq, mk, mv, p, units, s)
+                  : fwd_dispatch<64, false>(dtype, score, mask, mq, mk, mv, p, units, s);
 }
 
 }  // namespace
@@ -303,7 +339,10 @@ flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_
   if (!keep || Sq < 1 || Skv < 1) return FLEX_ERR_INVALID_ARG;
   const flex_mod_params_t zero{};
   const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
-  MaskArgs m{Skv, mp.window, mp.offset};
+  const int mask = mask_kind(mask_mod_id);
+  if (mask < 0) return FLEX_ERR_INVALID_ARG;
+  if (const flex_status_t ds = check_documents(mask, mp); ds != FLEX_OK) return ds;
+  const MaskArgs m = mask_args(mask, mp, Skv);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t total = static_cast<int64_t>(Sq) * Skv;
   const int grid = static_cast<int>(total / 256 + 1 > 4096 ? 4096 : total / 256 + 1);
@@ -316,6 +355,10 @@ flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_
       mask_eval_kernel<kMaskSliding><<<grid, 256, 0, s>>>(m, Sq, Skv, keep);
       break;
     case FLEX_MASK_KV_LE_Q_PLUS_OFFSET: mask_eval_kernel<kMaskOffset><<<grid, 256, 0, s>>>(m, Sq, Skv, keep); break;
+    case FLEX_MASK_DOCUMENT: mask_eval_kernel<kMaskDocument><<<grid, 256, 0, s>>>(m, Sq, Skv, keep); break;
+    case FLEX_MASK_DOCUMENT_CAUSAL:
+      mask_eval_kernel<kMaskDocumentCausal><<<grid, 256, 0, s>>>(m, Sq, Skv, keep);
+      break;
     default: return FLEX_ERR_INVALID_ARG;
   }
   return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;

@@ -30,7 +30,7 @@ template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
 flex_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                          int n_units, cudaStream_t stream) {
   auto kern = flex_fwd_kernel<D, T, SCORE, MASK, BLOCKS>;
-  constexpr int kSmem = FwdSmem<D, BLOCKS>::kAlloc;
+  constexpr int kSmem = FwdSmem<D, BLOCKS, is_doc_mask(MASK)>::kAlloc;
   if (!ensure_smem_attr<D, T, SCORE, MASK, BLOCKS>(kern, kSmem)) return FLEX_ERR_CUDA;
   kern<<<n_units, kFwdThreads, kSmem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
@@ -44,6 +44,9 @@ flex_status_t dispatch_mask(int mask, const CUtensorMap& mq, const CUtensorMap& 
     case kMaskCausal: return launch_fwd<D, T, SCORE, kMaskCausal, BLOCKS>(mq, mk, mv, p, n_units, s);
     case kMaskSliding: return launch_fwd<D, T, SCORE, kMaskSliding, BLOCKS>(mq, mk, mv, p, n_units, s);
     case kMaskOffset: return launch_fwd<D, T, SCORE, kMaskOffset, BLOCKS>(mq, mk, mv, p, n_units, s);
+    case kMaskDocument: return launch_fwd<D, T, SCORE, kMaskDocument, BLOCKS>(mq, mk, mv, p, n_units, s);
+    case kMaskDocumentCausal:
+      return launch_fwd<D, T, SCORE, kMaskDocumentCausal, BLOCKS>(mq, mk, mv, p, n_units, s);
   }
   return FLEX_ERR_INVALID_ARG;
 }

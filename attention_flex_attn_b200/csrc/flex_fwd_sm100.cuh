@@ -92,7 +92,8 @@ struct FwdParams {
   int H, Hkv, G, Sq, Skv;
   int n_qtiles, n_ktiles, n_pairs;
   float scale_log2;    // scale * log2(e)
-  MaskArgs mask;
+  const float* slopes; // alibi: captured per-head slopes [H], or nullptr for 2^(-8(h+1)/H)
+  MaskArgs mask;       // document rules: boundaries of batch 0, advanced per batch below
   // Block mask (BLOCKS instantiations): [0] partial lists, [1] full lists; counts are
   // [rows x n_qtiles], indices [rows x n_qtiles x blk_max]; row of (b, h) =
   // b * blk_b_stride + h * blk_h_stride (a stride of 0 shares one row).
@@ -102,7 +103,11 @@ struct FwdParams {
   int blk_b_stride, blk_h_stride;
 };
 
-template <int D, bool BLOCKS = false>
+// Block-mask / document bitmaps: full0, full1, act0, act1, and with both a block mask
+// and a document mask the document sets doc0, doc1 (kBlkWords words each).
+constexpr int fwd_bitmaps(bool blocks, bool doc) { return blocks ? (doc ? 6 : 4) : (doc ? 4 : 0); }
+
+template <int D, bool BLOCKS = false, bool DOC = false>
 struct FwdSmem {
   static constexpr int kTileBytes = kBM * D * 2;          // one 128-row tile
   static constexpr int kChunkBytes = kBM * 128;           // one 64-element-wide chunk
@@ -119,9 +124,10 @@ struct FwdSmem {
   // step records (kRec*): one per key/value slot, plus the first step's
   static constexpr int kRecOff = kTmemPtrOff + 16;
   static constexpr int kRecBytes = ((kSlots + 1) * 4 + 15) / 16 * 16;
-  // block-mask bitmaps: full0, full1, act0, act1 (kBlkWords words each)
-  static constexpr int kBlkOff = kRecOff + kRecBytes;
-  static constexpr int kBytes = kBlkOff + (BLOCKS ? 4 * kBlkWords * 4 : 0);
+  // document rules: the documents of each tile's first and last row (4 ints)
+  static constexpr int kDocOff = kRecOff + kRecBytes;
+  static constexpr int kBlkOff = kDocOff + (DOC ? 16 : 0);
+  static constexpr int kBytes = kBlkOff + fwd_bitmaps(BLOCKS, DOC) * kBlkWords * 4;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
   static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
 };
@@ -189,11 +195,22 @@ struct RangeCursor {
 
 __device__ __forceinline__ bool bits_has(const uint32_t* w, int j) { return (w[j >> 5] >> (j & 31)) & 1u; }
 
+// Sets bits [u_lo, u_hi] of a bitmap (word-wise atomic ORs).
+__device__ __forceinline__ void bits_set_range(uint32_t* w, int u_lo, int u_hi) {
+  for (int wi = u_lo >> 5; wi <= (u_hi >> 5); ++wi) {
+    const int a = max(u_lo, wi << 5) & 31, b = min(u_hi, (wi << 5) + 31) & 31;
+    const uint32_t m = (b == 31 ? 0xffffffffu : ((2u << b) - 1u)) & ~((1u << a) - 1u);
+    atomicOr(w + wi, m);
+  }
+}
+
+constexpr bool is_doc_mask(int mask) { return mask == kMaskDocument || mask == kMaskDocumentCausal; }
+
 template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     flex_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using L = FwdSmem<D, BLOCKS>;
+  using L = FwdSmem<D, BLOCKS, is_doc_mask(MASK)>;
   constexpr int NS = L::kSlots;
   constexpr int kChunks = D / 64;
   constexpr uint32_t kTmemCols = 512;
@@ -230,62 +247,122 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // constant, so that no array is indexed at run time (that would put it in local memory).
   int q0[2], q1[2], lo[2], hi[2];
   auto sel = [](const int (&a)[2], int k) { return k ? a[1] : a[0]; };
+  constexpr bool kDoc = MASK == kMaskDocument || MASK == kMaskDocumentCausal;
+  MaskArgs mk = p.mask;
+  if constexpr (kDoc) {
+    mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
+    mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
+  }
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int qt = 2 * pair + k;
     q0[k] = qt * kBM;
     q1[k] = min(q0[k] + kBM, p.Sq);
     lo[k] = hi[k] = 0;
-    if (qt < p.n_qtiles) tile_range<MASK>(q0[k], q1[k], kBN, p.mask, lo[k], hi[k]);
+    if (qt < p.n_qtiles && !kDoc) tile_range<MASK>(q0[k], q1[k], kBN, mk, lo[k], hi[k]);
   }
 
-  // ---------------------------------------------------------------- block-mask bitmaps
-  // full_k: tiles listed full; act_k: every tile query tile k visits.  Complete at the
-  // setup barrier below.
+  // ---------------------------------------------------------------- visit bitmaps
+  // With a block mask or a document mask the key tiles a query tile visits are a set, not
+  // a range: full_k = tiles needing no element mask, act_k = every tile query tile k
+  // visits (complete at the setup barrier below).  Document masks build them from the
+  // documents; with a block mask as well, the document sets doc_k filter the lists.
+  constexpr bool kBits = BLOCKS || kDoc;
   uint32_t* blk = reinterpret_cast<uint32_t*>(sgen + L::kBlkOff);
   auto full_bits = [&](int k) { return blk + k * kBlkWords; };
   auto act_bits = [&](int k) { return blk + (2 + k) * kBlkWords; };
-  if constexpr (BLOCKS) {
-    for (int w = threadIdx.x; w < 4 * kBlkWords; w += kFwdThreads) blk[w] = 0u;
-    __syncthreads();
-    const int64_t row0 = static_cast<int64_t>(b) * p.blk_b_stride + static_cast<int64_t>(h) * p.blk_h_stride;
-    // list l = 2 * k + f: query tile 2 * pair + k, f = 0 partial / 1 full (selects, not
-    // indexing, so that nothing here is forced into local memory)
-    auto count = [&](int k, int f) {
-      const int qt = 2 * pair + k;
-      const int32_t* num = f ? p.blk_num[1] : p.blk_num[0];
-      const int c = (qt < p.n_qtiles && num != nullptr) ? num[row0 * p.n_qtiles + qt] : 0;
-      return c < 0 ? 0 : (c > p.blk_max ? p.blk_max : c);
-    };
-    const int c00 = count(0, 0), c01 = count(0, 1), c10 = count(1, 0), c11 = count(1, 1);
-    for (int e = threadIdx.x; e < 4 * p.blk_max; e += kFwdThreads) {
-      const int l = e / p.blk_max, c = e - l * p.blk_max;
-      const int k = l >> 1, f = l & 1;
-      const int cl = k ? (f ? c11 : c10) : (f ? c01 : c00);
-      if (c >= cl) continue;
-      const int32_t* idx = f ? p.blk_idx[1] : p.blk_idx[0];
-      const int u = idx[(row0 * p.n_qtiles + 2 * pair + k) * p.blk_max + c];
-      if (u < 0 || u >= p.n_ktiles) continue;
-      bool full = f == 1;
-      if (!full) {
-        // a partial tile outside the mask_mod range keeps nothing; one the mask keeps
-        // whole needs no per-element mask
-        if (u < sel(lo, k) || u >= sel(hi, k)) continue;
-        full = tile_class<MASK>(sel(q0, k), sel(q1, k), u * kBN, kBN, p.mask) == kTileFull;
+  auto doc_bits = [&](int k) { return BLOCKS ? blk + (4 + k) * kBlkWords : blk + (2 + k) * kBlkWords; };
+  int* doc_rows = reinterpret_cast<int*>(sgen + L::kDocOff);  // doc_floor of q0/q1-1 per tile
+  if constexpr (kBits) {
+    for (int w = threadIdx.x; w < fwd_bitmaps(BLOCKS, kDoc) * kBlkWords; w += kFwdThreads) blk[w] = 0u;
+    if constexpr (kDoc) {
+      if (threadIdx.x < 4) {  // four independent binary searches, one per lane
+        const int k = threadIdx.x >> 1, qt = 2 * pair + k;
+        doc_rows[threadIdx.x] = qt < p.n_qtiles ? doc_floor(mk.off_q, mk.n_docs,
+                                                            (threadIdx.x & 1) ? sel(q1, k) - 1 : sel(q0, k))
+                                                : -1;
       }
-      const uint32_t bit = 1u << (u & 31);
-      if (full) atomicOr(full_bits(k) + (u >> 5), bit);
-      atomicOr(act_bits(k) + (u >> 5), bit);
+    }
+    __syncthreads();
+    // Document rules: tile k's class bounds (the first row's last key, the last row's
+    // first key); FULL iff lo_last <= k0 and k1 - 1 <= hi_first.
+    int64_t lo_last[2] = {0, 0}, hi_first[2] = {-1, -1};
+    if constexpr (kDoc) {
+      constexpr bool kCausal = MASK == kMaskDocumentCausal;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (2 * pair + k >= p.n_qtiles) continue;
+        int64_t t;
+        doc_interval(mk, doc_rows[2 * k + 1], sel(q1, k) - 1, kCausal, lo_last[k], t);
+        doc_interval(mk, doc_rows[2 * k], sel(q0, k), kCausal, t, hi_first[k]);
+      }
+      // every document with rows in tile k: the key tiles those rows keep
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (2 * pair + k >= p.n_qtiles) continue;
+        const int d0 = max(doc_rows[2 * k], 0), d1 = min(doc_rows[2 * k + 1], mk.n_docs - 1);
+        for (int d = d0 + threadIdx.x; d <= d1; d += kFwdThreads) {
+          const int64_t r0 = max(static_cast<int64_t>(sel(q0, k)), static_cast<int64_t>(__ldg(mk.off_q + d)));
+          const int64_t r1 = min(static_cast<int64_t>(sel(q1, k)), static_cast<int64_t>(__ldg(mk.off_q + d + 1)));
+          if (r0 >= r1) continue;  // no row of this document in the tile
+          int64_t a, e;
+          doc_interval(mk, d, r1 - 1, kCausal, a, e);  // the union of its rows' intervals
+          if (a > e) continue;
+          bits_set_range(doc_bits(k), static_cast<int>(a / kBN), static_cast<int>(e / kBN));
+        }
+        if (!BLOCKS && threadIdx.x == 0) {
+          const int64_t f_lo = (lo_last[k] + kBN - 1) / kBN, f_hi = (hi_first[k] + 1) / kBN - 1;
+          if (f_lo <= f_hi) bits_set_range(full_bits(k), static_cast<int>(f_lo), static_cast<int>(f_hi));
+        }
+      }
+      if constexpr (BLOCKS) __syncthreads();  // the document sets filter the lists below
+    }
+    if constexpr (BLOCKS) {
+      const int64_t row0 = static_cast<int64_t>(b) * p.blk_b_stride + static_cast<int64_t>(h) * p.blk_h_stride;
+      // list l = 2 * k + f: query tile 2 * pair + k, f = 0 partial / 1 full (selects, not
+      // indexing, so that nothing here is forced into local memory)
+      auto count = [&](int k, int f) {
+        const int qt = 2 * pair + k;
+        const int32_t* num = f ? p.blk_num[1] : p.blk_num[0];
+        const int c = (qt < p.n_qtiles && num != nullptr) ? num[row0 * p.n_qtiles + qt] : 0;
+        return c < 0 ? 0 : (c > p.blk_max ? p.blk_max : c);
+      };
+      const int c00 = count(0, 0), c01 = count(0, 1), c10 = count(1, 0), c11 = count(1, 1);
+      for (int e = threadIdx.x; e < 4 * p.blk_max; e += kFwdThreads) {
+        const int l = e / p.blk_max, c = e - l * p.blk_max;
+        const int k = l >> 1, f = l & 1;
+        const int cl = k ? (f ? c11 : c10) : (f ? c01 : c00);
+        if (c >= cl) continue;
+        const int32_t* idx = f ? p.blk_idx[1] : p.blk_idx[0];
+        const int u = idx[(row0 * p.n_qtiles + 2 * pair + k) * p.blk_max + c];
+        if (u < 0 || u >= p.n_ktiles) continue;
+        bool full = f == 1;
+        if (!full) {
+          // a partial tile the mask_mod drops whole keeps nothing; one it keeps whole
+          // needs no per-element mask
+          if constexpr (kDoc) {
+            if (!bits_has(doc_bits(k), u)) continue;
+            full = tile_class_of(k ? lo_last[1] : lo_last[0], k ? hi_first[1] : hi_first[0], u * kBN, kBN,
+                                 p.Skv) == kTileFull;
+          } else {
+            if (u < sel(lo, k) || u >= sel(hi, k)) continue;
+            full = tile_class<MASK>(sel(q0, k), sel(q1, k), u * kBN, kBN, mk) == kTileFull;
+          }
+        }
+        const uint32_t bit = 1u << (u & 31);
+        if (full) atomicOr(full_bits(k) + (u >> 5), bit);
+        atomicOr(act_bits(k) + (u >> 5), bit);
+      }
     }
   }
   // The walk over query tile k's key tiles (valid after the setup barrier); the CTA's
   // steps are the union of both walks: j = max of the two cursors.
   auto cursor = [&](int k) {
-    if constexpr (BLOCKS) return BitCursor(act_bits(k), full_bits(k), p.n_ktiles);
+    if constexpr (kBits) return BitCursor(act_bits(k), full_bits(k), p.n_ktiles);
     else return RangeCursor(sel(lo, k), sel(hi, k));
   };
   auto has = [&](int k, int j) -> bool {  // debug tile map only
-    if constexpr (BLOCKS) return bits_has(act_bits(k), j);
+    if constexpr (kBits) return bits_has(act_bits(k), j);
     else return j >= sel(lo, k) && j < sel(hi, k);
   };
 
@@ -510,7 +587,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float l_sum = 0.f;
     const float sc = SCORE == kScoreAlibi ? 1.0f : p.scale_log2;
     float slope2 = 0.f;
-    if (SCORE == kScoreAlibi) slope2 = exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H)) * kLog2e;
+    if (SCORE == kScoreAlibi)
+      slope2 = (p.slopes ? __ldg(p.slopes + h) : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
+               kLog2e;
+    // Document rules: this row's kept interval, looked up once (a binary search over the
+    // boundaries); the tile classes come from the visit bitmaps.
+    int64_t row_lo = 0, row_hi = -1;
+    if constexpr (kDoc) row_interval<MASK>(qi, mk, row_lo, row_hi);
 
     bool ok = true;
     int n = 0;
@@ -532,7 +615,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tc_fence_after();
       const int k0 = j * kBN;
-      const int cls = BLOCKS ? cls_blk : tile_class<MASK>(q0k, q1k, k0, kBN, p.mask);
+      int cls;
+      if constexpr (kBits) cls = cls_blk;
+      else cls = tile_class<MASK>(q0k, q1k, k0, kBN, mk);
       if (write_map)
         p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] =
             static_cast<uint8_t>(cls == kTileFullRagged ? kTilePartial : cls);
@@ -547,10 +632,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (cls != kTileFull) {
         int c_lo, c_hi;
-        if (BLOCKS && cls == kTileFullRagged)
-          col_interval<kMaskNone>(qi, k0, p.mask, c_lo, c_hi);
+        if (kBits && cls == kTileFullRagged)
+          col_interval<kMaskNone>(qi, k0, mk, c_lo, c_hi);
         else
-          col_interval<MASK>(qi, k0, p.mask, c_lo, c_hi);
+          if constexpr (kDoc) col_interval_of(row_lo, row_hi, k0, c_lo, c_hi);
+          else col_interval<MASK>(qi, k0, mk, c_lo, c_hi);
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
           if (c < c_lo || c > c_hi) s[c] = -INFINITY;

@@ -10,7 +10,13 @@
 //   CAUSAL:          j <= i
 //   SLIDING_WINDOW:  j <= i  &&  i - j < W
 //   KV_LE_Q_PLUS_OFF j <= i + off
+//   DOCUMENT         i and j in the same document (captured per-batch boundaries
+//                    off_q / off_kv: position p is in document d iff off[d] <= p < off[d+1])
+//   DOCUMENT_CAUSAL  DOCUMENT && j <= i
 // and every rule also requires j < Skv (the pad rule for a ragged last key tile).
+// The document rules are tensor-capturing mask_mods (FlyDSL PR 931, Out of scope: a
+// later phase); with non-decreasing boundaries the keys of row i's document form one
+// interval, so they ride on the same interval machinery.
 //
 // For each rule the kept keys of row i form one interval [a(i), b(i)] with a and b
 // non-decreasing in i, so the kept keys of a query tile (rows q0..q1-1) form the
@@ -22,7 +28,14 @@
 
 namespace flexattn {
 
-enum MaskKind : int { kMaskNone = 0, kMaskCausal = 1, kMaskSliding = 2, kMaskOffset = 3 };
+enum MaskKind : int {
+  kMaskNone = 0,
+  kMaskCausal = 1,
+  kMaskSliding = 2,
+  kMaskOffset = 3,
+  kMaskDocument = 5,
+  kMaskDocumentCausal = 6
+};
 enum ScoreKind : int { kScoreNone = 0, kScoreAlibi = 1 };
 enum TileClass : int { kTileEmpty = 0, kTileFull = 1, kTilePartial = 2 };
 
@@ -30,7 +43,38 @@ struct MaskArgs {
   int Skv;
   int window;
   int offset;
+  // document rules: this batch's boundaries, n_docs + 1 entries each (device memory)
+  const int32_t* off_q = nullptr;
+  const int32_t* off_kv = nullptr;
+  int n_docs = 0;
 };
+
+// Largest d in [0, n] with off[d] <= i, or -1 when i < off[0] (binary search over
+// non-decreasing boundaries; reads only off[0..n]).
+__device__ __forceinline__ int doc_floor(const int32_t* off, int n, int64_t i) {
+  if (static_cast<int64_t>(__ldg(off)) > i) return -1;
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (static_cast<int64_t>(__ldg(off + mid)) <= i) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Kept key interval [lo, hi] of row i under the document rules, given d = its
+// doc_floor.  Rows outside every document keep nothing; their empty interval sits at the
+// boundary of the neighbouring documents so that both ends stay non-decreasing in i.
+__device__ __forceinline__ void doc_interval(const MaskArgs& m, int d, int64_t i, bool causal, int64_t& lo,
+                                             int64_t& hi) {
+  const int dk = d < 0 ? 0 : d;
+  const int64_t a = __ldg(m.off_kv + dk);
+  const int64_t e = (d < 0 || d >= m.n_docs) ? a : static_cast<int64_t>(__ldg(m.off_kv + d + 1));
+  lo = a > 0 ? a : 0;
+  hi = static_cast<int64_t>(m.Skv) - 1;
+  hi = e - 1 < hi ? e - 1 : hi;
+  if (causal) hi = i < hi ? i : hi;
+}
 
 // Kept key interval [lo, hi] (inclusive, may be empty: lo > hi) of query row i.
 template <int MASK>
@@ -47,6 +91,13 @@ __host__ __device__ __forceinline__ void row_interval(int64_t i, const MaskArgs&
   } else if (MASK == kMaskOffset) {
     const int64_t b = i + m.offset;
     hi = b < hi ? b : hi;
+  } else if (MASK == kMaskDocument || MASK == kMaskDocumentCausal) {
+#ifdef __CUDA_ARCH__
+    doc_interval(m, doc_floor(m.off_q, m.n_docs, i), i, MASK == kMaskDocumentCausal, lo, hi);
+#else
+    lo = 0;
+    hi = -1;
+#endif
   }
 }
 
@@ -80,12 +131,8 @@ __host__ __device__ __forceinline__ int tile_class(int q0, int q1, int k0, int B
   return (lo_last <= k0 && k1 - 1 <= hi_first) ? kTileFull : kTilePartial;
 }
 
-// Column interval [c_lo, c_hi] (relative to k0) kept in row i of a key tile at k0.
-template <int MASK>
-__host__ __device__ __forceinline__ void col_interval(int64_t i, int k0, const MaskArgs& m, int& c_lo,
-                                                      int& c_hi) {
-  int64_t lo, hi;
-  row_interval<MASK>(i, m, lo, hi);
+// Column interval [c_lo, c_hi] (relative to k0) of the kept keys [lo, hi] of one row.
+__host__ __device__ __forceinline__ void col_interval_of(int64_t lo, int64_t hi, int k0, int& c_lo, int& c_hi) {
   lo -= k0;
   hi -= k0;
   // clamp to a range that fits in int and keeps "lo > hi" meaning empty
@@ -95,6 +142,23 @@ __host__ __device__ __forceinline__ void col_interval(int64_t i, int k0, const M
     c_lo = 1;
     c_hi = 0;
   }
+}
+
+// Column interval [c_lo, c_hi] (relative to k0) kept in row i of a key tile at k0.
+template <int MASK>
+__host__ __device__ __forceinline__ void col_interval(int64_t i, int k0, const MaskArgs& m, int& c_lo,
+                                                      int& c_hi) {
+  int64_t lo, hi;
+  row_interval<MASK>(i, m, lo, hi);
+  col_interval_of(lo, hi, k0, c_lo, c_hi);
+}
+
+// FULL or PARTIAL for a key tile [k0, k0 + BN) from the kept intervals of the tile's
+// first row (hi_first) and last row (lo_last), as tile_class computes them.
+__host__ __device__ __forceinline__ int tile_class_of(int64_t lo_last, int64_t hi_first, int k0, int BN, int Skv) {
+  const int64_t k1 = static_cast<int64_t>(k0) + BN;
+  if (k1 > Skv) return kTilePartial;
+  return (lo_last <= k0 && k1 - 1 <= hi_first) ? kTileFull : kTilePartial;
 }
 
 }  // namespace flexattn

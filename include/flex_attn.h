@@ -62,7 +62,8 @@ typedef enum { FLEX_DTYPE_BF16 = 0, FLEX_DTYPE_F16 = 1 } flex_dtype_t;
 /* score_mod: applied to s = scale * q.k before any mask (FlyDSL PR 931, Summary). */
 typedef enum {
   FLEX_SCORE_NONE = 0,
-  FLEX_SCORE_ALIBI = 1 /* s += slope_h * (kv_idx - q_idx), slope_h = 2^(-8 (h+1) / H) */
+  FLEX_SCORE_ALIBI = 1,       /* s += slope_h * (kv_idx - q_idx), slope_h = 2^(-8 (h+1) / H) */
+  FLEX_SCORE_ALIBI_SLOPES = 2 /* tensor-capturing: slope_h = mod_params->alibi_slopes[h] */
 } flex_score_mod_t;
 
 /* mask_mod: keep (q_idx, kv_idx) iff the rule holds; indices are absolute (top-left). */
@@ -71,7 +72,16 @@ typedef enum {
   FLEX_MASK_CAUSAL = 1,                /* causal_via_mask: kv_idx <= q_idx                  */
   FLEX_MASK_SLIDING_WINDOW = 2,        /* kv_idx <= q_idx && q_idx - kv_idx < window        */
   FLEX_MASK_KV_LE_Q_PLUS_OFFSET = 3,   /* kv_idx <= q_idx + offset (offset may be negative) */
-  FLEX_MASK_CAUSAL_FAST = 4            /* causal=True: the same keep rule as CAUSAL          */
+  FLEX_MASK_CAUSAL_FAST = 4,           /* causal=True: the same keep rule as CAUSAL          */
+  /* Tensor-capturing mask_mods (FlyDSL PR 931, Out of scope: a later phase, not defined
+   * there).  Packed sequences: per batch b, mod_params->doc_offsets_q[b][0 .. n_docs]
+   * are the document boundaries of the query positions and doc_offsets_kv those of the
+   * keys; position p is in document d iff off[d] <= p < off[d+1] (in none otherwise).
+   * Boundaries must be non-decreasing; other values cannot make a kernel read out of
+   * bounds, but then the keys kept are unspecified.  The forward kernels skip exactly the
+   * key tiles no row keeps; Skv at most 2048 * 128 (FLEX_ERR_UNSUPPORTED beyond). */
+  FLEX_MASK_DOCUMENT = 5,              /* q_idx and kv_idx in the same document            */
+  FLEX_MASK_DOCUMENT_CAUSAL = 6        /* ... and kv_idx <= q_idx                           */
 } flex_mask_mod_t;
 
 /* Tile classification written by the debug tile map (one byte per tile). */
@@ -87,6 +97,14 @@ typedef struct {
    * set, the work units of batch 0 / head 0 write the class of every (q-tile, kv-tile)
    * they process (FULL or PARTIAL) and EMPTY for every tile they skip. */
   uint8_t* tile_map_out;
+  /* Captured tensors (device memory, 4-byte aligned, owned by the caller):
+   * FLEX_SCORE_ALIBI_SLOPES: alibi_slopes[H] fp32.
+   * FLEX_MASK_DOCUMENT*: doc_offsets_q [B, n_docs + 1] int32 and doc_offsets_kv of the
+   * same shape (NULL = the same boundaries as the queries); n_docs >= 0. */
+  const float* alibi_slopes;
+  const int32_t* doc_offsets_q;
+  const int32_t* doc_offsets_kv;
+  int32_t n_docs;
 } flex_mod_params_t;
 
 /*
@@ -211,7 +229,8 @@ flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const
 /*
  * flex_attn_mask_eval -- debug: evaluates the device mask rule the forward kernel uses
  * into keep[Sq * Skv] (uint8, device, 1 = kept) for element-exact comparison.
- * Covers mask_mod and the j < Skv pad rule.
+ * Covers mask_mod and the j < Skv pad rule; the document rules read the boundaries of
+ * batch 0 (the first n_docs + 1 entries of doc_offsets_q / doc_offsets_kv).
  */
 flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_params,
                                   int Sq, int Skv, uint8_t* keep, flex_stream_t stream);

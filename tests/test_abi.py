@@ -135,3 +135,23 @@ def test_block_sparse_rejects_bad_args_on_host(lib):
     assert bs(mask(), Skv=2048 * 128 + 1) == 2            # beyond what the bitmaps name
     assert bs(mask(num=34)) == 3                          # not 4-byte aligned
     assert bs(mask(fnum=32, fidx=66)) == 3
+
+
+def test_captured_mods_rejected_on_host(lib):
+    def fwd(score=0, mask=0, mp=None):
+        return lib.flex_attn_fwd(P(16), P(16), P(16), P(16), None, 2, 2, 1, 8, 8, 128, 0.1, score, mask,
+                                 ctypes.byref(mp) if mp is not None else None, 0, None)
+    mp = lambda **kw: fa.ModParams(kw.get("window", 0), 0, 0, None, kw.get("slopes"), kw.get("oq"), kw.get("okv"),
+                                   kw.get("n", 1))
+    assert fwd(score=2) == 1                                  # slope table missing
+    assert fwd(score=2, mp=mp(slopes=18)) == 3                # slope table misaligned
+    assert fwd(score=3) == 1                                  # no such score_mod
+    assert fwd(mask=5) == 1                                   # boundaries missing
+    assert fwd(mask=6, mp=mp(oq=32, n=-1)) == 1               # negative document count
+    assert fwd(mask=5, mp=mp(oq=34)) == 3                     # misaligned boundaries
+    assert fwd(mask=6, mp=mp(oq=32, okv=66)) == 3
+    assert fwd(mask=7) == 1                                   # no such mask_mod
+    big = lib.flex_attn_fwd(P(16), P(16), P(16), P(16), None, 2, 2, 1, 8, 2048 * 128 + 1, 128, 0.1, 0, 5,
+                            ctypes.byref(mp(oq=32)), 0, None)
+    assert big == 2                                           # beyond the key-tile bitmaps
+    assert lib.flex_attn_mask_eval(5, None, 4, 4, P(16), None) == 1
