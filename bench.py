@@ -389,7 +389,45 @@ def per_case(fa, q, k, v, scale, o, lse, args):
         if name.startswith("sliding"):
             out[name]["tflops_useful"] = useful_window / t / 1e12
     out.update(block_cases(fa, q, k, v, scale, o, lse))
+    out.update(captured_cases(fa, q, k, v, scale, o, lse))
     return out
+
+
+def captured_cases(fa, q, k, v, scale, o, lse):
+    """Tensor-capturing mods on the forward inputs: alibi with a captured slope tensor
+    (TFLOPS as no_mod), and packed documents whose boundaries fall off the 128 grid
+    (lengths 200..3000, per-batch draws, seed 4102), plain and causal; useful TFLOPS =
+    4 * D * kept pairs."""
+    import numpy as np
+    import torch
+    B, H, S, D = q.shape
+    dev = q.device
+    res = {}
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32, device=dev)
+    t = _time_fn(lambda: fa.fwd(q, k, v, scale=scale, score_mod="alibi", alibi_slopes=slopes, out=o, lse_out=lse),
+                 20, 3)
+    res["alibi_slope_tensor"] = {"us": t * 1e6, "tflops": fwd_flops(B, H, S, S, D) / t / 1e12}
+    rng = np.random.default_rng(4102)
+    bounds = []
+    for _ in range(B):
+        cuts, pos = [0], 0
+        while pos < S:
+            pos = min(S, pos + int(rng.integers(200, 3001)))
+            cuts.append(pos)
+        bounds.append(cuts)
+    n = max(len(c) for c in bounds)
+    off = np.array([c + [S] * (n - len(c)) for c in bounds], np.int32)  # repeats = empty documents
+    doff = torch.from_numpy(off).to(dev)
+    for mask in ("document", "document_causal"):
+        t = _time_fn(lambda: fa.fwd(q, k, v, scale=scale, mask_mod=mask, doc_offsets=doff, out=o, lse_out=lse), 20, 3)
+        pairs = 0.0
+        for b in range(B):
+            for a, e in zip(off[b, :-1], off[b, 1:]):
+                L = float(e - a)
+                pairs += L * (L + 1) / 2 if mask == "document_causal" else L * L
+        res[f"{mask}_packed"] = {"us": t * 1e6, "tflops_useful": 4.0 * D * H * pairs / t / 1e12,
+                                 "documents": [len(c) - 1 for c in bounds]}
+    return res
 
 
 def block_lists(sel):
