@@ -55,6 +55,8 @@ def _bind(lib):
     lib.oracle_fwd_block_sparse.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, I,
                                             P, P, P, P, I, I, I, P, I64, P, P, I]
     lib.oracle_fwd_block_sparse.restype = I
+    lib.oracle_bwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, I, P, I64, P, P, P, I]
+    lib.oracle_bwd.restype = I
     return lib
 
 
@@ -165,6 +167,42 @@ def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset
         if probs is not None:
             probs = probs.reshape(B, H, Sq, Skv)
     return (o, lse, probs) if want_probs else (o, lse)
+
+
+def bwd(q, k, v, dout, scale=None, score_mod="none", mask_mod="none", window=0, offset=0, groups=None,
+        threads=None, alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None):
+    """Oracle backward: gradients dQ, dK, dV of sum(dout * O) for the forward with the same
+    arguments.  groups: optional list of (b, hk) pairs (or flat b * Hkv + hk) to compute;
+    None computes all.  Returns float64 arrays: dq [B,H,Sq,D], dk/dv [B,Hkv,Skv,D] for all
+    groups, else dq [n, G, Sq, D] and dk/dv [n, Skv, D] in the order given."""
+    lib = _load()
+    B, H, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    assert tuple(dout.shape) == tuple(q.shape) and dout.dtype == q.dtype
+    slopes, oq, okv, n_docs = _captured(B, H, mask_mod, alibi_slopes, doc_offsets, doc_offsets_kv)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    G = H // Hkv
+    if groups is None:
+        g_arr, n = None, B * Hkv
+    else:
+        flat = [g[0] * Hkv + g[1] if isinstance(g, (tuple, list)) else int(g) for g in groups]
+        g_arr = np.ascontiguousarray(np.asarray(flat, dtype=np.int64))
+        n = int(g_arr.size)
+    dq = np.zeros((n, G, Sq, D))
+    dk = np.zeros((n, Skv, D))
+    dv = np.zeros((n, Skv, D))
+    qb, kb, vb, ob = _bits(q), _bits(k), _bits(v), _bits(dout)
+    rc = lib.oracle_bwd(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, ob.ctypes.data, _dtype_code(q),
+                        B, H, Hkv, Sq, Skv, D, float(scale), SCORE_MODS[score_mod], MASK_MODS[mask_mod],
+                        int(window), int(offset), _p(slopes), _p(oq), _p(okv), n_docs,
+                        None if g_arr is None else g_arr.ctypes.data, n,
+                        dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_bwd rejected its arguments (rc={rc})")
+    if groups is None:
+        return dq.reshape(B, H, Sq, D), dk.reshape(B, Hkv, Skv, D), dv.reshape(B, Hkv, Skv, D)
+    return dq, dk, dv
 
 
 def _i32(a):

@@ -1,5 +1,5 @@
 /*
- * flex_oracle.c -- plain fp64 CPU oracle for flex attention (forward + decode).
+ * flex_oracle.c -- plain fp64 CPU oracle for flex attention (forward, backward, decode).
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
  * benchmark's CPU-baseline leg may load this library.  It shares no code,
@@ -196,32 +196,50 @@ typedef struct {
   int64_t r0, r1;
 } fwd_job;
 
+/* Key/value head of query head h (GQA: contiguous groups of H / Hkv query heads). */
+static int kv_head(const fwd_job* J, int h) {
+  int G = J->H / J->Hkv;
+  int hk = h / G;
+  return hk;
+}
+
+/* x_ij = scale * q_i . k_j + score_mod bias, for row i of (b, h) and key j. */
+static double score_ij(const fwd_job* J, int b, int h, int64_t i, int64_t j) {
+  int D = J->D;
+  const int64_t qbase = (((int64_t)b * J->H + h) * J->Sq + i) * D;
+  const int64_t kvbase = ((int64_t)b * J->Hkv + kv_head(J, h)) * (int64_t)J->Skv * D;
+  double slope = 0.0;
+  if (J->score_mod == OR_SCORE_ALIBI) slope = J->cap.slopes ? J->cap.slopes[h] : oracle_alibi_slope(h, J->H);
+  double dot = 0.0;
+  for (int d = 0; d < D; ++d)
+    dot += elem(J->q, qbase + d, J->dtype) * elem(J->k, kvbase + j * D + d, J->dtype);
+  double s = J->scale * dot;
+  if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);
+  return s;
+}
+
+/* The keep decision of element (i, j) of (b, h): the block mask if any, else mask_mod. */
+static int keep_ij(const fwd_job* J, int b, int h, int64_t i, int64_t j) {
+  int64_t bh = (int64_t)b * J->H + h;
+  return J->blk ? block_keep(J->blk, bh, J->mask_mod, i, j, J->Skv, J->window, J->offset, &J->cap, b)
+                : keep_rule(J->mask_mod, J->window, J->offset, &J->cap, b, i, j);
+}
+
 static void fwd_row(const fwd_job* J, int64_t r, double* x, unsigned char* keep) {
   int64_t flat = J->rows ? J->rows[r] : r;
   int64_t i = flat % J->Sq;
   int64_t bh = flat / J->Sq;
   int h = (int)(bh % J->H);
   int b = (int)(bh / J->H);
-  int G = J->H / J->Hkv;
-  int hk = h / G;
   int D = J->D;
-  const int64_t qbase = flat * D;
-  const int64_t kvbase = ((int64_t)b * J->Hkv + hk) * (int64_t)J->Skv * D;
-  double slope = 0.0;
-  if (J->score_mod == OR_SCORE_ALIBI) slope = J->cap.slopes ? J->cap.slopes[h] : oracle_alibi_slope(h, J->H);
+  const int64_t kvbase = ((int64_t)b * J->Hkv + kv_head(J, h)) * (int64_t)J->Skv * D;
 
   double M = -INFINITY;
   int any = 0;
   for (int64_t j = 0; j < J->Skv; ++j) {
-    double dot = 0.0;
-    for (int d = 0; d < D; ++d)
-      dot += elem(J->q, qbase + d, J->dtype) * elem(J->k, kvbase + j * D + d, J->dtype);
-    double s = J->scale * dot;
-    if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);
+    double s = score_ij(J, b, h, i, j);
     x[j] = s;
-    keep[j] = (unsigned char)(J->blk ? block_keep(J->blk, bh, J->mask_mod, i, j, J->Skv, J->window, J->offset,
-                                                  &J->cap, b)
-                                     : keep_rule(J->mask_mod, J->window, J->offset, &J->cap, b, i, j));
+    keep[j] = (unsigned char)keep_ij(J, b, h, i, j);
     if (keep[j]) {
       any = 1;
       if (s > M) M = s;
@@ -305,6 +323,199 @@ int oracle_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int dtyp
   J.cap.slopes = slopes; J.cap.off_q = off_q; J.cap.off_kv = off_kv; J.cap.n_docs = n_docs;
   if ((mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) && (!off_q || !off_kv || n_docs < 0)) return -2;
   return run_jobs(&J, J.n_rows, nthreads, fwd_worker, sizeof J);
+}
+
+/* ---- backward ---------------------------------------------------------------
+ * Gradients of the forward above (FlyDSL PR 931, Out of scope: the backward pass as a
+ * later phase; xformers 1094 reports dq/dk/dv mean errors of its own backward).  With an
+ * upstream gradient dO, per query row i of (b, h) and kept key j:
+ *   P_ij  = exp(x_ij - M_i) / l_i            (the forward's probabilities, 0 if dropped)
+ *   O_i   = sum_j P_ij V_j,   delta_i = sum_d dO_id O_id
+ *   dP_ij = dO_i . V_j,       dS_ij = P_ij (dP_ij - delta_i)
+ *   dQ_i  = scale sum_j dS_ij K_j
+ *   dK_j  = scale sum_{h, i} dS_ij Q_i,   dV_j = sum_{h, i} P_ij dO_i
+ * where the sums over h run over the query heads that share key/value head hk (GQA).
+ * score_mod adds a bias that does not depend on Q or K, so it enters only through P.
+ * Two passes per (b, hk) group: rows (statistics, delta, dQ), then keys (dK, dV, with P
+ * and dS recomputed from the row statistics). */
+
+typedef struct {
+  fwd_job f;                 /* inputs, mods and the keep rule of the forward */
+  const uint16_t* dout;      /* dO [B, H, Sq, D] */
+  const int64_t* groups;     /* b * Hkv + hk of each group computed */
+  int64_t n_groups;
+  double *dq, *dk, *dv;      /* [n_groups, G, Sq, D], [n_groups, Skv, D] x 2 */
+  double *M, *l, *delta;     /* [n_groups, G, Sq] row statistics */
+  int pass;                  /* 1: rows, 2: keys */
+} bwd_job;
+
+static void* bwd_worker(void* arg) {
+  bwd_job* W = (bwd_job*)arg;
+  const fwd_job* J = &W->f;
+  const int D = J->D, G = J->H / J->Hkv;
+  const int64_t Sq = J->Sq, Skv = J->Skv;
+  double* x = (double*)malloc(sizeof(double) * (size_t)Skv);
+  unsigned char* keep = (unsigned char*)malloc((size_t)Skv);
+  double* acc = (double*)malloc(sizeof(double) * (size_t)D * 2);
+  if (x && keep && acc) {
+    for (int64_t t = J->r0; t < J->r1; ++t) {
+      if (W->pass == 1) {
+        /* task t = (group, head in group, row) */
+        int64_t gi = t / (G * Sq), rem = t % (G * Sq);
+        int hg = (int)(rem / Sq);
+        int64_t i = rem % Sq;
+        int64_t g = W->groups[gi];
+        int b = (int)(g / J->Hkv), hk = (int)(g % J->Hkv), h = hk * G + hg;  /* kv_head(J, h) == hk */
+        const int64_t kvbase = ((int64_t)b * J->Hkv + hk) * Skv * D;
+        const int64_t obase = (((int64_t)b * J->H + h) * Sq + i) * D;
+        for (int64_t j = 0; j < Skv; ++j) {
+          x[j] = score_ij(J, b, h, i, j);
+          keep[j] = (unsigned char)keep_ij(J, b, h, i, j);
+        }
+        double M = -INFINITY, l = 0.0;
+        for (int64_t j = 0; j < Skv; ++j)
+          if (keep[j] && x[j] > M) M = x[j];
+        double* dq = W->dq + ((gi * G + hg) * Sq + i) * D;
+        for (int d = 0; d < D; ++d) dq[d] = 0.0;
+        int64_t srow = (gi * G + hg) * Sq + i;
+        W->M[srow] = M;
+        if (M == -INFINITY) {  /* no kept key: no gradient through this row */
+          W->l[srow] = 0.0;
+          W->delta[srow] = 0.0;
+          continue;
+        }
+        for (int64_t j = 0; j < Skv; ++j)
+          if (keep[j]) l += exp(x[j] - M);
+        W->l[srow] = l;
+        /* O_i and delta_i */
+        for (int d = 0; d < D; ++d) acc[d] = 0.0;
+        for (int64_t j = 0; j < Skv; ++j) {
+          if (!keep[j]) continue;
+          double pij = exp(x[j] - M) / l;
+          for (int d = 0; d < D; ++d) acc[d] += pij * elem(J->v, kvbase + j * D + d, J->dtype);
+        }
+        double delta = 0.0;
+        for (int d = 0; d < D; ++d) delta += elem(W->dout, obase + d, J->dtype) * acc[d];
+        W->delta[srow] = delta;
+        /* dQ_i */
+        for (int64_t j = 0; j < Skv; ++j) {
+          if (!keep[j]) continue;
+          double pij = exp(x[j] - M) / l, dp = 0.0;
+          for (int d = 0; d < D; ++d) dp += elem(W->dout, obase + d, J->dtype) * elem(J->v, kvbase + j * D + d, J->dtype);
+          double ds = pij * (dp - delta);
+          for (int d = 0; d < D; ++d) dq[d] += J->scale * ds * elem(J->k, kvbase + j * D + d, J->dtype);
+        }
+      } else {
+        /* task t = (group, key) */
+        int64_t gi = t / Skv, j = t % Skv;
+        int64_t g = W->groups[gi];
+        int b = (int)(g / J->Hkv), hk = (int)(g % J->Hkv);
+        const int64_t kvbase = ((int64_t)b * J->Hkv + hk) * Skv * D;
+        double* dk = acc;
+        double* dv = acc + D;
+        for (int d = 0; d < 2 * D; ++d) acc[d] = 0.0;
+        for (int hg = 0; hg < G; ++hg) {
+          int h = hk * G + hg;
+          for (int64_t i = 0; i < Sq; ++i) {
+            int64_t srow = (gi * G + hg) * Sq + i;
+            if (W->M[srow] == -INFINITY) continue;
+            if (!keep_ij(J, b, h, i, j)) continue;
+            const int64_t qbase = (((int64_t)b * J->H + h) * Sq + i) * D;
+            double dp = 0.0;
+            for (int d = 0; d < D; ++d)
+              dp += elem(W->dout, qbase + d, J->dtype) * elem(J->v, kvbase + j * D + d, J->dtype);
+            double pij = exp(score_ij(J, b, h, i, j) - W->M[srow]) / W->l[srow];
+            double ds = pij * (dp - W->delta[srow]);
+            for (int d = 0; d < D; ++d) {
+              dk[d] += J->scale * ds * elem(J->q, qbase + d, J->dtype);
+              dv[d] += pij * elem(W->dout, qbase + d, J->dtype);
+            }
+          }
+        }
+        for (int d = 0; d < D; ++d) {
+          W->dk[(gi * Skv + j) * D + d] = dk[d];
+          W->dv[(gi * Skv + j) * D + d] = dv[d];
+        }
+      }
+    }
+  }
+  free(x);
+  free(keep);
+  free(acc);
+  return NULL;
+}
+
+static int run_bwd_pass(bwd_job* base, int64_t n_tasks, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if ((int64_t)nthreads > n_tasks) nthreads = (int)(n_tasks > 0 ? n_tasks : 1);
+  bwd_job* jobs = (bwd_job*)malloc(sizeof(bwd_job) * (size_t)nthreads);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  if (!jobs || !th) { free(jobs); free(th); return -3; }
+  for (int t = 0; t < nthreads; ++t) {
+    jobs[t] = *base;
+    jobs[t].f.r0 = n_tasks * t / nthreads;
+    jobs[t].f.r1 = n_tasks * (t + 1) / nthreads;
+  }
+  int started = 0;
+  for (int t = 1; t < nthreads; ++t) {
+    if (pthread_create(&th[t], NULL, bwd_worker, &jobs[t]) != 0) break;
+    started = t;
+  }
+  bwd_worker(&jobs[0]);
+  for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
+  for (int t = started + 1; t < nthreads; ++t) bwd_worker(&jobs[t]);
+  free(jobs);
+  free(th);
+  return 0;
+}
+
+/* Backward for the (b, hk) groups listed (groups == NULL: all B*Hkv).  dq: [n_groups, G,
+ * Sq, D]; dk, dv: [n_groups, Skv, D] (G = H / Hkv query heads per group, in order). */
+int oracle_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout, int dtype,
+               int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
+               int score_mod, int mask_mod, int window, int offset,
+               const double* slopes, const int32_t* off_q, const int32_t* off_kv, int n_docs,
+               const int64_t* groups, int64_t n_groups, double* dq, double* dk, double* dv, int nthreads) {
+  if (H <= 0 || Hkv <= 0 || H % Hkv != 0 || Sq <= 0 || Skv <= 0 || D <= 0) return -1;
+  if ((mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) && (!off_q || !off_kv || n_docs < 0)) return -2;
+  int64_t ng = groups ? n_groups : (int64_t)B * Hkv;
+  int64_t* all = NULL;
+  if (!groups) {
+    all = (int64_t*)malloc(sizeof(int64_t) * (size_t)ng);
+    if (!all) return -3;
+    for (int64_t g = 0; g < ng; ++g) all[g] = g;
+  }
+  const int G = H / Hkv;
+  bwd_job W;
+  memset(&W, 0, sizeof W);
+  fwd_job* J = &W.f;
+  J->q = q; J->k = k; J->v = v; J->dtype = dtype;
+  J->B = B; J->H = H; J->Hkv = Hkv; J->Sq = Sq; J->Skv = Skv; J->D = D;
+  J->scale = scale; J->score_mod = score_mod; J->mask_mod = mask_mod;
+  J->window = window; J->offset = offset;
+  J->cap.slopes = slopes; J->cap.off_q = off_q; J->cap.off_kv = off_kv; J->cap.n_docs = n_docs;
+  W.dout = dout;
+  W.groups = groups ? groups : all;
+  W.n_groups = ng;
+  W.dq = dq; W.dk = dk; W.dv = dv;
+  size_t nrows = (size_t)ng * G * Sq;
+  W.M = (double*)malloc(sizeof(double) * nrows);
+  W.l = (double*)malloc(sizeof(double) * nrows);
+  W.delta = (double*)malloc(sizeof(double) * nrows);
+  int rc = -3;
+  if (W.M && W.l && W.delta) {
+    W.pass = 1;
+    rc = run_bwd_pass(&W, ng * G * (int64_t)Sq, nthreads);
+    if (rc == 0) {
+      W.pass = 2;
+      rc = run_bwd_pass(&W, ng * (int64_t)Skv, nthreads);
+    }
+  }
+  free(W.M);
+  free(W.l);
+  free(W.delta);
+  free(all);
+  return rc;
 }
 
 /* ---- decode ---------------------------------------------------------------- */

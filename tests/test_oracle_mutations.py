@@ -1,5 +1,6 @@
 """Plants plausible mistakes in copies of the C oracle and checks that the pins in
-test_oracle_pins.py, test_oracle_block_pins.py and test_oracle_mods_pins.py catch every one (each mutant must fail at least one pin).
+test_oracle_pins.py, test_oracle_block_pins.py, test_oracle_mods_pins.py and
+test_oracle_bwd_pins.py catch every one (each mutant must fail at least one pin).
 Everything runs on the CPU against a temporary build; the real oracle is untouched.
 Mutants that leave the mathematics unchanged (e.g. dropping the fully-masked guard,
 which still yields p = 0 and log 0 = -inf) are not listed: no test could tell them apart."""
@@ -12,6 +13,7 @@ import torch
 
 import oracle
 import tests.test_oracle_block_pins as bpins
+import tests.test_oracle_bwd_pins as bwpins
 import tests.test_oracle_mods_pins as mpins
 import tests.test_oracle_pins as pins
 
@@ -19,16 +21,16 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "flex_oracle.c")
 
 # (name, text in flex_oracle.c, replacement)
 MUTANTS = [
-    ("scale dropped", "    double s = J->scale * dot;\n    if (J->score_mod", "    double s = dot;\n    if (J->score_mod"),
-    ("scale applied after alibi", "    double s = J->scale * dot;\n    if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);",
-     "    double s = dot;\n    if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);\n    s *= J->scale;"),
+    ("scale dropped", "  double s = J->scale * dot;\n  if (J->score_mod", "  double s = dot;\n  if (J->score_mod"),
+    ("scale applied after alibi", "  double s = J->scale * dot;\n  if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);",
+     "  double s = dot;\n  if (J->score_mod == OR_SCORE_ALIBI) s += slope * (double)(j - i);\n  s *= J->scale;"),
     ("alibi sign", "s += slope * (double)(j - i);", "s += slope * (double)(i - j);"),
     ("alibi slope index", "pow(2.0, -8.0 * (double)(h + 1) / (double)H)", "pow(2.0, -8.0 * (double)h / (double)H)"),
     ("causal strict", "case OR_MASK_CAUSAL: return j <= i;", "case OR_MASK_CAUSAL: return j < i;"),
     ("window off by one", "(i - j < (int64_t)window)", "(i - j <= (int64_t)window)"),
     ("window not causal", "return (j <= i) && (i - j < (int64_t)window);", "return (i - j < (int64_t)window);"),
     ("offset sign", "return j <= i + (int64_t)offset;", "return j <= i - (int64_t)offset;"),
-    ("GQA modulo mapping", "int hk = h / G;", "int hk = h % J->Hkv;"),
+    ("GQA modulo mapping", "  int hk = h / G;\n  return hk;", "  int hk = h % J->Hkv;\n  return hk;"),
     ("LSE in base 2", "  J->lse[r] = M + log(l);\n}\n\nstatic void* fwd_worker", "  J->lse[r] = M + log2(l);\n}\n\nstatic void* fwd_worker"),
     ("K used for V", "o[d] += p * elem(J->v, kvbase + j * D + d, J->dtype);", "o[d] += p * elem(J->k, kvbase + j * D + d, J->dtype);"),
     ("Q index transposed", "elem(J->q, qbase + d, J->dtype) * elem(J->k, kvbase + j * D + d, J->dtype)",
@@ -55,6 +57,14 @@ MUTANTS = [
      "const int32_t* oq = C->off_q;"),
     ("slope table ignored", "slope = J->cap.slopes ? J->cap.slopes[h] : oracle_alibi_slope(h, J->H);",
      "slope = oracle_alibi_slope(h, J->H);"),
+    ("bwd delta sign", "double ds = pij * (dp - delta);", "double ds = pij * (dp + delta);"),
+    ("bwd dK without scale", "dk[d] += J->scale * ds * elem(J->q, qbase + d, J->dtype);", "dk[d] += ds * elem(J->q, qbase + d, J->dtype);"),
+    ("bwd dV from dS", "dv[d] += pij * elem(W->dout, qbase + d, J->dtype);", "dv[d] += ds * elem(W->dout, qbase + d, J->dtype);"),
+    ("bwd dQ from V", "dq[d] += J->scale * ds * elem(J->k, kvbase + j * D + d, J->dtype);",
+     "dq[d] += J->scale * ds * elem(J->v, kvbase + j * D + d, J->dtype);"),
+    ("bwd one head per group", "for (int hg = 0; hg < G; ++hg) {", "for (int hg = 0; hg < 1; ++hg) {"),
+    ("bwd P unnormalised", "double pij = exp(score_ij(J, b, h, i, j) - W->M[srow]) / W->l[srow];",
+     "double pij = exp(score_ij(J, b, h, i, j) - W->M[srow]);"),
     ("bf16 decoded as truncated", "  uint32_t u = ((uint32_t)b) << 16;", "  uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
 ]
 
@@ -90,6 +100,10 @@ CHECKS = [
     (mpins.test_document_masks_equal_torch, {"case": "tail_unassigned", "causal": False}),
     (mpins.test_document_masks_equal_torch, {"case": "cross", "causal": False}),
     (mpins.test_document_mask_matrix_and_tile_map, {"causal": True}),
+    (bwpins.test_bwd_equals_torch_autograd, {"mask": "causal", "window": 0, "offset": 0, "score": "alibi",
+                                             "dtype": torch.bfloat16}),
+    (bwpins.test_bwd_single_key_closed_form, {}),
+    (bwpins.test_bwd_equals_finite_differences_of_forward, {}),
 ]
 
 
