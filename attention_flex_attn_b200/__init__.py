@@ -27,7 +27,8 @@ MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset":
 FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
-EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_decode_workspace_size", "flex_attn_decode",
+EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_bwd_workspace_size", "flex_attn_bwd",
+            "flex_attn_decode_workspace_size", "flex_attn_decode",
             "flex_attn_decode_noalloc", "flex_attn_mask_eval", "flex_attn_selftest_wait_timeout",
             "flex_attn_tile_sizes", "flex_attn_device_status", "flex_status_string"]
 
@@ -68,6 +69,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_fwd_block_sparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams),
                                                ctypes.POINTER(BlockMaskC), I, P]
     lib.flex_attn_fwd_block_sparse.restype = I
+    lib.flex_attn_bwd_workspace_size.argtypes = [I, I, I]
+    lib.flex_attn_bwd_workspace_size.restype = SZ
+    lib.flex_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams), I,
+                                  P, SZ, P]
+    lib.flex_attn_bwd.restype = I
     lib.flex_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.flex_attn_decode_workspace_size.restype = SZ
     lib.flex_attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, P]
@@ -227,6 +233,39 @@ def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None
                                         ctypes.byref(bm), DTYPES[q.dtype], _stream(q.device))
     _check(rc, "flex_attn_fwd_block_sparse")
     return o, lse
+
+
+def bwd_workspace_size(B, H, Sq) -> int:
+    return int(load_library().flex_attn_bwd_workspace_size(B, H, Sq))
+
+
+def bwd(q, k, v, o, lse, dout, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
+        alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None, dq=None, dk=None, dv=None, workspace=None):
+    """Flex-attention backward (flex_attn_bwd): gradients (dq, dk, dv) of sum(dout * o)
+    for the forward with the same arguments; o and lse are that forward's outputs.
+    dk/dv are [B, Hkv, Skv, D] (summed over the query heads of each group)."""
+    lib = load_library()
+    for t, n in ((o, "o"), (dout, "dout"), (lse, "lse")):
+        _cuda_tensor(t, n)
+    B, H, Hkv, Sq, Skv, D, scale, _, _ = _fwd_args(q, k, v, scale, False, q, None)
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape) or dout.dtype != q.dtype:
+        raise FlexAttnError("o and dout must match q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq):
+        raise FlexAttnError("lse must be float32 [B, H, Sq]")
+    dq = dq if dq is not None else torch.empty_like(q)
+    dk = dk if dk is not None else torch.empty_like(k)
+    dv = dv if dv is not None else torch.empty_like(v)
+    need = bwd_workspace_size(B, H, Sq)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, doc_offsets,
+                            doc_offsets_kv)
+    rc = lib.flex_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                           B, H, Hkv, Sq, Skv, D, scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
+                           DTYPES[q.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
+                           _stream(q.device))
+    _check(rc, "flex_attn_bwd")
+    return dq, dk, dv
 
 
 def decode_workspace_size(B, H, Hkv, cap, D) -> int:

@@ -270,6 +270,76 @@ flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const voi
                     block_mask, dtype, stream);
 }
 
+size_t flex_attn_bwd_workspace_size(int B, int H, int Sq) {
+  if (B < 1 || H < 1 || Sq < 1) return 0;
+  const size_t sq_pad = (static_cast<size_t>(Sq) + kBM - 1) / kBM * kBM;
+  return 2 * static_cast<size_t>(B) * H * sq_pad * sizeof(float);
+}
+
+flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, int B, int H, int Hkv, int Sq, int Skv,
+                            int D, float scale, int score_mod_id, int mask_mod_id, const flex_mod_params_t* mod_params,
+                            flex_dtype_t dtype, void* workspace, size_t workspace_bytes, flex_stream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FLEX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
+  if (dtype != FLEX_DTYPE_BF16 && dtype != FLEX_DTYPE_F16) return FLEX_ERR_UNSUPPORTED;
+  if (score_mod_id != FLEX_SCORE_NONE && score_mod_id != FLEX_SCORE_ALIBI && score_mod_id != FLEX_SCORE_ALIBI_SLOPES)
+    return FLEX_ERR_INVALID_ARG;
+  const int mask = mask_kind(mask_mod_id);
+  if (mask < 0) return FLEX_ERR_INVALID_ARG;
+  const flex_mod_params_t zero{};
+  const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
+  if (mask == kMaskSliding && mp.window < 1) return FLEX_ERR_INVALID_ARG;
+  if (score_mod_id == FLEX_SCORE_ALIBI_SLOPES) {
+    if (!mp.alibi_slopes) return FLEX_ERR_INVALID_ARG;
+    if (!aligned4(mp.alibi_slopes)) return FLEX_ERR_MISALIGNED;
+  }
+  if (const flex_status_t ds = check_documents(mask, mp); ds != FLEX_OK) return ds;
+  const size_t need = flex_attn_bwd_workspace_size(B, H, Sq);
+  if (!workspace || workspace_bytes < need) return FLEX_ERR_WORKSPACE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || !aligned4(lse))
+    return FLEX_ERR_MISALIGNED;
+  const int n_qtiles = (Sq + kBM - 1) / kBM, n_ktiles = (Skv + kBN - 1) / kBN;
+  const int64_t bh = static_cast<int64_t>(B) * H, bhkv = static_cast<int64_t>(B) * Hkv;
+  if (bh * n_qtiles > 0x7fffffff || bhkv * n_ktiles > 0x7fffffff) return FLEX_ERR_UNSUPPORTED;
+  unsigned* st = status_ptr();
+  if (!st) return FLEX_ERR_CUDA;
+  BwdMaps m;
+  if (!make_map(&m.q, q, dtype, D, Sq, bh) || !make_map(&m.o, dout, dtype, D, Sq, bh) ||
+      !make_map(&m.k, k, dtype, D, Skv, bhkv) || !make_map(&m.v, v, dtype, D, Skv, bhkv))
+    return FLEX_ERR_CUDA;
+  BwdParams p{};
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.Sq_pad = n_qtiles * kBM;
+  p.lse2 = static_cast<float*>(workspace);
+  p.delta = p.lse2 + bh * p.Sq_pad;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.status = st;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.D = D;
+  p.n_qtiles = n_qtiles;
+  p.n_ktiles = n_ktiles;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.slopes = score_mod_id == FLEX_SCORE_ALIBI_SLOPES ? mp.alibi_slopes : nullptr;
+  p.mask = mask_args(mask, mp, Skv);
+  const int score = score_mod_id == FLEX_SCORE_NONE ? kScoreNone : kScoreAlibi;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return D == 128 ? bwd_dispatch<128>(dtype, score, mask, m, p, s) : bwd_dispatch<64>(dtype, score, mask, m, p, s);
+}
+
 size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D) {
   if (B < 1 || H < 1 || Hkv < 1 || cap < 1 || D < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H;

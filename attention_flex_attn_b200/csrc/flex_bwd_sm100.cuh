@@ -1,0 +1,614 @@
+// flex_bwd_sm100.cuh -- flex-attention backward for sm_100a: dQ, dK, dV of sum(dO * O).
+//
+// The backward pass is named as a later phase on FlyDSL PR 931 "Add flex_attention
+// (score_mod / mask_mod) on the generic flash-attention kernel" (Out of scope); xformers
+// 1094 "Tiny upstream pr" reports dq/dk/dv errors of a backward against a reference.
+// With the forward's LSE (natural log) and O, per query row i and kept key j:
+//   P_ij = exp(x_ij - LSE_i),  delta_i = dO_i . O_i,  dP_ij = dO_i . V_j,
+//   dS_ij = P_ij (dP_ij - delta_i),
+//   dQ_i = scale sum_j dS_ij K_j,  dK_j = scale sum_i dS_ij Q_i,  dV_j = sum_i P_ij dO_i
+// (dK, dV summed over the query heads of a GQA group); x_ij is the forward's modded,
+// scaled score, so the mods enter through P and the masks zero P.
+//
+// Three kernels, no atomics (results do not depend on scheduling):
+//   bwd_prep_kernel   per row: delta_i and LSE_i * log2(e) into a padded workspace
+//   bwd_dq_kernel     one CTA per 128-row query tile: for each key tile, S = Q K^T and
+//                     dP = dO V^T (tcgen05, TMEM), dS on the CUDA cores (one row per
+//                     thread), dQ += dS K (tcgen05, dS read from TMEM); S alternates between
+//                     two TMEM buffers so S of the next key tile overlaps the dS work
+//   bwd_dkdv_kernel   one CTA per 128-key tile and kv head: for each query tile of each
+//                     query head of the group, S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
+//                     per key row, dV += P^T dO and dK += dS^T Q (TMEM accumulators)
+// Roles per CTA (256 threads): warp 0 issues the MMAs (one thread), warp 1 the TMA loads,
+// warps 4-7 do the element-wise work (thread = TMEM lane = row), warps 2-3 idle.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "flex_fwd_sm100.cuh"
+#include "mask_rules.cuh"
+#include "ptx_sm100.cuh"
+
+namespace flexattn {
+
+constexpr int kBwdThreads = 256;
+constexpr int kBwdWarp0 = 4;  // first element-wise warp
+constexpr unsigned kStatusBwdTimeout = 16u;
+
+struct BwdParams {
+  const void* o;          // forward output [B, H, Sq, D]
+  const void* dout;       // upstream gradient [B, H, Sq, D]
+  const float* lse;       // forward LSE [B, H, Sq] (natural log)
+  float* lse2;            // workspace [B*H, Sq_pad]: LSE * log2(e), +inf for rows without keys
+  float* delta;           // workspace [B*H, Sq_pad]: dO . O
+  void* dq;               // [B, H, Sq, D]
+  void* dk;               // [B, Hkv, Skv, D]
+  void* dv;               // [B, Hkv, Skv, D]
+  unsigned* status;
+  int B, H, Hkv, G, Sq, Skv, D, Sq_pad;
+  int n_qtiles, n_ktiles;
+  float scale;
+  float scale_log2;       // scale * log2(e)
+  const float* slopes;    // alibi slope tensor [H] or nullptr
+  MaskArgs mask;          // document rules: boundaries of batch 0, advanced per batch
+};
+
+// ---------------------------------------------------------------- prep
+
+// One warp per row (b, h, i) of the padded row space: delta = dO . O in fp32, and the
+// base-2 LSE; padding rows get lse2 = +inf and delta = 0 so that they contribute nothing.
+template <int D, typename T>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
+  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Sq_pad;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; r < rows;
+       r += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int64_t bh = r / p.Sq_pad;
+    const int i = static_cast<int>(r - bh * p.Sq_pad);
+    float acc = 0.f, l2 = INFINITY;
+    if (i < p.Sq) {
+      const int64_t base = (bh * p.Sq + i) * D;
+      const T* o = reinterpret_cast<const T*>(p.o) + base;
+      const T* g = reinterpret_cast<const T*>(p.dout) + base;
+      for (int d = lane; d < D; d += 32) acc = fmaf(static_cast<float>(o[d]), static_cast<float>(g[d]), acc);
+      const float l = p.lse[bh * p.Sq + i];
+      l2 = l == -INFINITY ? INFINITY : l * kLog2e;
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) {
+      p.delta[r] = i < p.Sq ? acc : 0.f;
+      p.lse2[r] = l2;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- shared memory
+
+template <int D>
+struct BwdDqSmem {
+  static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kChunkBytes = kBM * 128;
+  static constexpr int kSlots = D == 128 ? 4 : 10;  // K/V ring (K_t, V_t consecutive)
+  static constexpr int kQOff = 0;                   // Q, then dO
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
+  // barriers: q, full[NS], empty[NS], sdp, ds, done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 3;
+  static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kTmemPtrOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
+};
+
+template <int D>
+struct BwdDkvSmem {
+  static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kChunkBytes = kBM * 128;
+  static constexpr int kStatBytes = 2 * kBM * 4;                      // lse2[128], delta[128]
+  static constexpr int kSlotBytes = 2 * kTileBytes + kStatBytes;      // Q, dO, stats
+  static constexpr int kSlots = D == 128 ? 2 : 4;
+  static constexpr int kKOff = 0;                                     // K, then V
+  static constexpr int kSlotOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kSlotOff + kSlots * kSlotBytes;
+  // barriers: kv, full[NS], empty[NS], sdp, pds, done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 3;
+  static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kTmemPtrOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
+  static_assert(kSlotBytes % 1024 == 0, "slots must keep the 1024-byte swizzle alignment");
+};
+
+// Bounded wait that also gives up when another role of the CTA has given up.
+__device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const BwdParams& p, volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (!mbar_wait(bar, parity, p.status, kStatusBwdTimeout, kWaitTimeoutNs)) {
+    *abort_flag = 1;
+    return false;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------- dQ
+
+template <int D, typename T, int SCORE, int MASK>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const BwdParams p) {
+  using L = BwdDqSmem<D>;
+  constexpr int NS = L::kSlots;
+  constexpr int kChunks = D / 64;
+  constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);   // S, dP: K-major B
+  constexpr uint32_t kIdescDq = idesc_f16(DtypeBits<T>::kFmt, kBM, D, 1);    // dQ: B = K, N-major
+  constexpr bool kDoc = is_doc_mask(MASK);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw_addr);
+  const uint32_t bar_q = sbase + L::kBarOff;
+  auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
+  const uint32_t bar_sdp = sbase + L::kBarOff + 8u * (1 + 2 * NS);
+  const uint32_t bar_ds = bar_sdp + 8u;
+  const uint32_t bar_done = bar_sdp + 16u;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
+  const uint32_t q_smem = sbase + L::kQOff, o_smem = q_smem + L::kTileBytes;
+  auto kv_smem = [&](int s) { return sbase + static_cast<uint32_t>(L::kKVOff + s * L::kTileBytes); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x % p.n_qtiles;
+  const int bh = blockIdx.x / p.n_qtiles;
+  const int h = bh % p.H, b = bh / p.H;
+  const int bkv = b * p.Hkv + h / p.G;
+  const int q0 = qt * kBM, q1 = min(q0 + kBM, p.Sq);
+  MaskArgs mk = p.mask;
+  if constexpr (kDoc) {
+    mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
+    mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
+  }
+  int lo = 0, hi = 0;
+  tile_range<MASK>(q0, q1, kBN, mk, lo, hi);
+  const int n = hi - lo;  // key tiles lo .. hi-1, visited in ascending order
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    mbar_init(bar_sdp, 1);
+    mbar_init(bar_ds, kBM);
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_ptr), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  // TMEM columns: S buffers [0,128) and [128,256), dP [256,384), dQ [384, 384+D)
+  auto s_col = [](int t) { return 128u * static_cast<uint32_t>(t & 1); };
+  constexpr uint32_t kDpCol = 256, kDqCol = 384;
+
+  if (warp == 1 && lane == 0 && n > 0) {
+    // ============================================================ TMA producer
+    mbar_arrive_expect_tx(bar_q, 2 * L::kTileBytes);
+    for (int c = 0; c < kChunks; ++c) {
+      tma_load_3d(q_smem + c * L::kChunkBytes, &tmQ, bar_q, c * 64, q0, bh);
+      tma_load_3d(o_smem + c * L::kChunkBytes, &tmO, bar_q, c * 64, q0, bh);
+    }
+    int r = 0;
+    bool ok = true;
+    for (int t = 0; t < n && ok; ++t) {
+      for (int which = 0; which < 2 && ok; ++which, ++r) {
+        const int s = r % NS;
+        if (!bwd_wait(bar_empty(s), (static_cast<uint32_t>(r / NS) & 1u) ^ 1u, p, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(kv_smem(s) + c * L::kChunkBytes, which ? &tmV : &tmK, bar_full(s), c * 64, (lo + t) * kBN, bkv);
+      }
+    }
+    for (int e = r - NS < 0 ? 0 : r - NS; e < r; ++e)
+      mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+    mbar_wait(bar_q, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+  } else if (warp == 0 && lane == 0 && n > 0) {
+    // ============================================================ MMA issuer
+    bool ok = bwd_wait(bar_q, 0, p, abort_flag);
+    tc_fence_after();
+    const uint64_t dq0 = smem_desc(q_smem, 16, 1024, kSwizzle128B);
+    const uint64_t do0 = smem_desc(o_smem, 16, 1024, kSwizzle128B);
+    // S-type product: d = A (K-major, rows = queries) * B^T (K-major, rows = keys), K = D
+    auto issue_qk = [&](uint32_t d, uint64_t a0, int slot) {
+      const uint64_t bk = smem_desc(kv_smem(slot), 16, 1024, kSwizzle128B);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
+        mma_ss(d, a0 + off, bk + off, kIdescS, kk > 0 ? 1u : 0u);
+      }
+    };
+    if (ok && !bwd_wait(bar_full(0), 0, p, abort_flag)) ok = false;
+    if (ok) {
+      tc_fence_after();
+      issue_qk(tmem + s_col(0), dq0, 0);
+    }
+    for (int t = 0; t < n && ok; ++t) {
+      const int rK = 2 * t, rV = rK + 1;
+      if (!bwd_wait(bar_full(rV % NS), static_cast<uint32_t>(rV / NS) & 1u, p, abort_flag)) break;
+      tc_fence_after();
+      issue_qk(tmem + kDpCol, do0, rV % NS);  // dP = dO V^T
+      mma_commit(bar_sdp);
+      mma_commit(bar_empty(rV % NS));
+      if (t + 1 < n) {
+        const int rK2 = rK + 2;
+        if (!bwd_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p, abort_flag)) break;
+        tc_fence_after();
+        issue_qk(tmem + s_col(t + 1), dq0, rK2 % NS);  // S of the next key tile
+      }
+      if (!bwd_wait(bar_ds, static_cast<uint32_t>(t) & 1u, p, abort_flag)) break;
+      tc_fence_after();
+      // dQ += dS K: A = dS (bf16/f16 pairs in the first 64 columns of its S buffer)
+      const uint64_t bkn = smem_desc(kv_smem(rK % NS), L::kChunkBytes, 1024, kSwizzle128B);
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        mma_ts(tmem + kDqCol, tmem + s_col(t) + 8u * kk, bkn + static_cast<uint64_t>((kk * 2048) >> 4), kIdescDq,
+               (t > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(bar_empty(rK % NS));
+    }
+    mma_commit(bar_done);
+    mbar_wait(bar_done, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+  } else if (warp >= kBwdWarp0) {
+    // ============================================================ element-wise warps
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int i = q0 + row;
+    const bool row_valid = i < p.Sq;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int64_t srow = static_cast<int64_t>(bh) * p.Sq_pad + (row_valid ? i : 0);
+    const float lse2 = row_valid ? p.lse2[srow] : INFINITY;
+    const float delta = row_valid ? p.delta[srow] : 0.f;
+    float slope2 = 0.f;
+    if (SCORE == kScoreAlibi)
+      slope2 = (p.slopes ? __ldg(p.slopes + h) : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
+               kLog2e;
+    int64_t row_lo, row_hi, lo_last, hi_first, t0, t1;
+    row_interval<MASK>(i, mk, row_lo, row_hi);
+    row_interval<MASK>(q1 - 1, mk, lo_last, t1);
+    row_interval<MASK>(q0, mk, t0, hi_first);
+    bool ok = true;
+    for (int t = 0; t < n; ++t) {
+      const bool got = bwd_wait(bar_sdp, static_cast<uint32_t>(t) & 1u, p, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int k0 = (lo + t) * kBN;
+      const bool full = row_valid && tile_class_of(lo_last, hi_first, k0, kBN, p.Skv) == kTileFull;
+      int c_lo = 0, c_hi = kBN - 1;
+      if (!full) {
+        col_interval_of(row_lo, row_hi, k0, c_lo, c_hi);
+        if (!row_valid) {
+          c_lo = 1;
+          c_hi = 0;
+        }
+      }
+      const uint32_t tS = tmem + lane_off + s_col(t), tP = tmem + lane_off + kDpCol;
+      const float base = slope2 * static_cast<float>(k0 - i) - lse2;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sr[64], pr[64], w[32];
+        tmem_ld64(tS + 64u * half, sr);
+        tmem_ld64(tP + 64u * half, pr);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = 64 * half + 2 * e + u;
+            const float x = fmaf(__uint_as_float(sr[2 * e + u]), p.scale_log2, fmaf(slope2, static_cast<float>(c), base));
+            const bool keep = full || (c >= c_lo && c <= c_hi);
+            const float pe = keep ? ex2_approx(x) : 0.f;
+            ds[u] = keep ? pe * (__uint_as_float(pr[2 * e + u]) - delta) : 0.f;
+          }
+          w[e] = DtypeBits<T>::pack(ds[0], ds[1]);
+        }
+        tmem_st32(tS + 32u * half, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+    }
+    // epilogue: dQ row * scale
+    bool ran = ok && n > 0;
+    if (ran) {
+      const bool got = bwd_wait(bar_done, 0, p, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) ran = false;
+      tc_fence_after();
+    }
+    T* out = reinterpret_cast<T*>(p.dq) + (static_cast<int64_t>(bh) * p.Sq + i) * D;
+#pragma unroll 1
+    for (int c = 0; c < D; c += 32) {
+      uint32_t r[32];
+      if (ran) tmem_ld32(tmem + lane_off + kDqCol + c, r);
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        w[e] = DtypeBits<T>::pack(ran ? __uint_as_float(r[2 * e]) * p.scale : 0.f,
+                                  ran ? __uint_as_float(r[2 * e + 1]) * p.scale : 0.f);
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dK, dV
+
+template <int D, typename T, int SCORE, int MASK>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const BwdParams p) {
+  using L = BwdDkvSmem<D>;
+  constexpr int NS = L::kSlots;
+  constexpr int kChunks = D / 64;
+  constexpr uint32_t kIdescT = idesc_f16(DtypeBits<T>::kFmt, kBN, kBM, 0);  // S^T, dP^T: K-major B
+  constexpr uint32_t kIdescAcc = idesc_f16(DtypeBits<T>::kFmt, kBN, D, 1);  // dV, dK: N-major B
+  constexpr bool kDoc = is_doc_mask(MASK);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw_addr);
+  const uint32_t bar_kv = sbase + L::kBarOff;
+  auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
+  const uint32_t bar_sdp = sbase + L::kBarOff + 8u * (1 + 2 * NS);
+  const uint32_t bar_pds = bar_sdp + 8u;
+  const uint32_t bar_done = bar_sdp + 16u;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
+  const uint32_t k_smem = sbase + L::kKOff, v_smem = k_smem + L::kTileBytes;
+  auto slot_base = [&](int s) { return static_cast<uint32_t>(L::kSlotOff + s * L::kSlotBytes); };
+  auto q_slot = [&](int s) { return sbase + slot_base(s); };
+  auto o_slot = [&](int s) { return sbase + slot_base(s) + L::kTileBytes; };
+  auto stat_slot = [&](int s) { return slot_base(s) + 2 * L::kTileBytes; };  // byte offset from sbase
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x % p.n_ktiles;
+  const int bkv = blockIdx.x / p.n_ktiles;
+  const int hk = bkv % p.Hkv, b = bkv / p.Hkv;
+  const int k0 = kt * kBN;
+  MaskArgs mk = p.mask;
+  if constexpr (kDoc) {
+    mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
+    mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
+  }
+  // does query tile t see key tile kt?
+  auto active = [&](int t) {
+    int lo, hi;
+    tile_range<MASK>(t * kBM, min(t * kBM + kBM, p.Sq), kBN, mk, lo, hi);
+    return kt >= lo && kt < hi;
+  };
+  // steps: (query head of the group) x (active query tile); every role walks the same list
+  int n_active = 0;
+  for (int t = 0; t < p.n_qtiles; ++t) n_active += active(t) ? 1 : 0;
+  const int n = n_active * p.G;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    mbar_init(bar_sdp, 1);
+    mbar_init(bar_pds, kBN);
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_ptr), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  // TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256, 256+D), dK [256+D, 256+2D)
+  constexpr uint32_t kSCol = 0, kDpCol = 128, kDvCol = 256, kDkCol = 256 + D;
+
+  if (warp == 1 && lane == 0 && n > 0) {
+    // ============================================================ TMA producer
+    mbar_arrive_expect_tx(bar_kv, 2 * L::kTileBytes);
+    for (int c = 0; c < kChunks; ++c) {
+      tma_load_3d(k_smem + c * L::kChunkBytes, &tmK, bar_kv, c * 64, k0, bkv);
+      tma_load_3d(v_smem + c * L::kChunkBytes, &tmV, bar_kv, c * 64, k0, bkv);
+    }
+    int u = 0;
+    bool ok = true;
+    for (int hg = 0; hg < p.G && ok; ++hg) {
+      const int bh = b * p.H + hk * p.G + hg;
+      for (int t = 0; t < p.n_qtiles && ok; ++t) {
+        if (!active(t)) continue;
+        const int s = u % NS;
+        if (!bwd_wait(bar_empty(s), (static_cast<uint32_t>(u / NS) & 1u) ^ 1u, p, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar_full(s), 2 * L::kTileBytes + L::kStatBytes);
+        for (int c = 0; c < kChunks; ++c) {
+          tma_load_3d(q_slot(s) + c * L::kChunkBytes, &tmQ, bar_full(s), c * 64, t * kBM, bh);
+          tma_load_3d(o_slot(s) + c * L::kChunkBytes, &tmO, bar_full(s), c * 64, t * kBM, bh);
+        }
+        const int64_t srow = static_cast<int64_t>(bh) * p.Sq_pad + t * kBM;
+        bulk_load(sbase + stat_slot(s), p.lse2 + srow, kBM * 4, bar_full(s));
+        bulk_load(sbase + stat_slot(s) + kBM * 4, p.delta + srow, kBM * 4, bar_full(s));
+        ++u;
+      }
+    }
+    for (int e = u - NS < 0 ? 0 : u - NS; e < u; ++e)
+      mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+    mbar_wait(bar_kv, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+  } else if (warp == 0 && lane == 0 && n > 0) {
+    // ============================================================ MMA issuer
+    bool ok = bwd_wait(bar_kv, 0, p, abort_flag);
+    tc_fence_after();
+    const uint64_t dk0 = smem_desc(k_smem, 16, 1024, kSwizzle128B);
+    const uint64_t dv0 = smem_desc(v_smem, 16, 1024, kSwizzle128B);
+    for (int u = 0; u < n && ok; ++u) {
+      const int s = u % NS;
+      if (!bwd_wait(bar_full(s), static_cast<uint32_t>(u / NS) & 1u, p, abort_flag)) break;
+      tc_fence_after();
+      const uint64_t bq = smem_desc(q_slot(s), 16, 1024, kSwizzle128B);
+      const uint64_t bo = smem_desc(o_slot(s), 16, 1024, kSwizzle128B);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
+        mma_ss(tmem + kSCol, dk0 + off, bq + off, kIdescT, kk > 0 ? 1u : 0u);   // S^T = K Q^T
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
+        mma_ss(tmem + kDpCol, dv0 + off, bo + off, kIdescT, kk > 0 ? 1u : 0u);  // dP^T = V dO^T
+      }
+      mma_commit(bar_sdp);
+      if (!bwd_wait(bar_pds, static_cast<uint32_t>(u) & 1u, p, abort_flag)) break;
+      tc_fence_after();
+      const uint64_t bon = smem_desc(o_slot(s), L::kChunkBytes, 1024, kSwizzle128B);
+      const uint64_t bqn = smem_desc(q_slot(s), L::kChunkBytes, 1024, kSwizzle128B);
+#pragma unroll
+      for (int kk = 0; kk < kBM / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>((kk * 2048) >> 4);
+        mma_ts(tmem + kDvCol, tmem + kSCol + 8u * kk, bon + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
+        mma_ts(tmem + kDkCol, tmem + kDpCol + 8u * kk, bqn + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit(bar_empty(s));
+    }
+    mma_commit(bar_done);
+    mbar_wait(bar_done, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+  } else if (warp >= kBwdWarp0) {
+    // ============================================================ element-wise warps
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int j = k0 + row;  // this thread's key
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    int64_t key_lo, key_hi;
+    key_interval<MASK>(j, mk, p.Sq, key_lo, key_hi);
+    bool ok = true;
+    int u = 0;
+    for (int hg = 0; hg < p.G && ok; ++hg) {
+      const int h = hk * p.G + hg;
+      float slope2 = 0.f;
+      if (SCORE == kScoreAlibi)
+        slope2 = (p.slopes ? __ldg(p.slopes + h) : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
+                 kLog2e;
+      for (int t = 0; t < p.n_qtiles; ++t) {
+        if (!active(t)) continue;
+        const int s = u % NS;
+        // S^T / dP^T ready; the slot's statistics (written by the bulk copy) are read
+        // below, so observe the slot's own barrier too
+        const bool got = bwd_wait(bar_sdp, static_cast<uint32_t>(u) & 1u, p, abort_flag) &&
+                         bwd_wait(bar_full(s), static_cast<uint32_t>(u / NS) & 1u, p, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int q0 = t * kBM;
+        const bool full = tile_class<MASK>(q0, min(q0 + kBM, p.Sq), k0, kBN, mk) == kTileFull;
+        int c_lo = 0, c_hi = kBM - 1;
+        if (!full) col_interval_of(key_lo, key_hi, q0, c_lo, c_hi);
+        const float* stat = reinterpret_cast<const float*>(sgen + stat_slot(s));
+        const float base = slope2 * static_cast<float>(j - q0);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sr[64], pr[64], wp[32], wd[32];
+          tmem_ld64(tmem + lane_off + kSCol + 64u * half, sr);
+          tmem_ld64(tmem + lane_off + kDpCol + 64u * half, pr);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float pe[2], ds[2];
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const int c = 64 * half + 2 * e + v;  // query q0 + c
+              const float x = fmaf(__uint_as_float(sr[2 * e + v]), p.scale_log2,
+                                   fmaf(-slope2, static_cast<float>(c), base)) - stat[c];
+              const bool keep = full || (c >= c_lo && c <= c_hi);
+              pe[v] = keep ? ex2_approx(x) : 0.f;
+              ds[v] = keep ? pe[v] * (__uint_as_float(pr[2 * e + v]) - stat[kBM + c]) : 0.f;
+            }
+            wp[e] = DtypeBits<T>::pack(pe[0], pe[1]);
+            wd[e] = DtypeBits<T>::pack(ds[0], ds[1]);
+          }
+          tmem_st32(tmem + lane_off + kSCol + 32u * half, wp);
+          tmem_st32(tmem + lane_off + kDpCol + 32u * half, wd);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_pds);
+        ++u;
+      }
+    }
+    // epilogue: dK = scale * (dS^T Q), dV = P^T dO
+    bool ran = ok && n > 0;
+    if (ran) {
+      const bool got = bwd_wait(bar_done, 0, p, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) ran = false;
+      tc_fence_after();
+    }
+    const bool key_valid = j < p.Skv;
+    const int64_t orow = (static_cast<int64_t>(bkv) * p.Skv + j) * D;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      T* out = reinterpret_cast<T*>(which ? p.dk : p.dv) + orow;
+      const float mul = which ? p.scale : 1.0f;
+      const uint32_t col = which ? kDkCol : kDvCol;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        if (ran) tmem_ld32(tmem + lane_off + col + c, r);
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = DtypeBits<T>::pack(ran ? __uint_as_float(r[2 * e]) * mul : 0.f,
+                                    ran ? __uint_as_float(r[2 * e + 1]) * mul : 0.f);
+        if (key_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace flexattn

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "flex_attn.h"
+#include "flex_bwd_sm100.cuh"
 #include "flex_decode.cuh"
 #include "flex_fwd_sm100.cuh"
 
@@ -30,6 +31,21 @@ extern template flex_status_t fwd_dispatch<64, true>(flex_dtype_t, int, int, con
 extern template flex_status_t fwd_dispatch<128, true>(flex_dtype_t, int, int, const CUtensorMap&,
                                                       const CUtensorMap&, const CUtensorMap&, const FwdParams&,
                                                       int, cudaStream_t);
+
+// Tensor maps of the backward: Q and dO [D, Sq, B*H], K and V [D, Skv, B*Hkv].
+struct BwdMaps {
+  CUtensorMap q, o, k, v;
+};
+
+// Backward (prep, dQ, dK/dV) over every (dtype, score_mod, mask_mod) of one head dim.
+// Instantiated in flex_bwd_d{64,128}.cu.
+template <int D>
+flex_status_t bwd_dispatch(flex_dtype_t dtype, int score, int mask, const BwdMaps& m, const BwdParams& p,
+                           cudaStream_t s);
+extern template flex_status_t bwd_dispatch<64>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
+                                               cudaStream_t);
+extern template flex_status_t bwd_dispatch<128>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
+                                                cudaStream_t);
 
 // Split-KV decode + combine (flex_decode_launch.cu).
 flex_status_t decode_dispatch(int D, flex_dtype_t dtype, const DecodeParams& p, cudaStream_t s);

@@ -101,6 +101,41 @@ __host__ __device__ __forceinline__ void row_interval(int64_t i, const MaskArgs&
   }
 }
 
+// Kept query interval [lo, hi] (inclusive, may be empty) of key j, for kernels whose
+// rows are keys (the backward's dK/dV): keep(i, j) holds for i < Sq exactly when
+// lo <= i <= hi.  Keys at or beyond Skv keep nothing.
+template <int MASK>
+__device__ __forceinline__ void key_interval(int64_t j, const MaskArgs& m, int Sq, int64_t& lo, int64_t& hi) {
+  lo = 0;
+  hi = static_cast<int64_t>(Sq) - 1;
+  if (j >= m.Skv) {
+    lo = 1;
+    hi = 0;
+    return;
+  }
+  if (MASK == kMaskCausal) {
+    lo = j;
+  } else if (MASK == kMaskSliding) {
+    lo = j;
+    const int64_t b = j + m.window - 1;
+    hi = b < hi ? b : hi;
+  } else if (MASK == kMaskOffset) {
+    const int64_t a = j - m.offset;
+    lo = a > 0 ? a : 0;
+  } else if (MASK == kMaskDocument || MASK == kMaskDocumentCausal) {
+    const int d = doc_floor(m.off_kv, m.n_docs, j);
+    if (d < 0 || d >= m.n_docs) {
+      lo = 1;
+      hi = 0;
+      return;
+    }
+    const int64_t a = __ldg(m.off_q + d), e = static_cast<int64_t>(__ldg(m.off_q + d + 1)) - 1;
+    lo = a > 0 ? a : 0;
+    hi = e < hi ? e : hi;
+    if (MASK == kMaskDocumentCausal) lo = j > lo ? j : lo;
+  }
+}
+
 // Key-tile range [t_lo, t_hi) that rows [q0, q1) (q1 exclusive, already clipped to Sq)
 // must visit; empty (t_lo == t_hi == 0) when no key of these rows is kept.
 template <int MASK>

@@ -172,6 +172,33 @@ flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const voi
                                          flex_stream_t stream);
 
 /*
+ * flex_attn_bwd_workspace_size -- bytes of device workspace flex_attn_bwd needs
+ * (per query row: LSE in base 2 and delta = dO . O, rows padded to a multiple of 128).
+ */
+size_t flex_attn_bwd_workspace_size(int B, int H, int Sq);
+
+/*
+ * flex_attn_bwd -- gradients of sum(dout * O) for the forward with the same arguments
+ * (the backward pass, FlyDSL PR 931, Out of scope: a later phase; xformers 1094 "Tiny
+ * upstream pr" reports dq/dk/dv mean errors of a backward).  With P the forward's
+ * probabilities (recomputed from q, k and the forward's lse), delta_i = dout_i . o_i and
+ * dS = P * (dout V^T - delta):  dq = scale dS K,  dk = scale dS^T Q,  dv = P^T dout, where
+ * dk and dv sum over the H / Hkv query heads that share a key/value head.
+ *   q, o, dout, dq [B, H, Sq, D] dtype;  k, v, dk, dv [B, Hkv, Skv, D] dtype;
+ *   lse [B, H, Sq] fp32: the forward's LSE (natural log; -inf for rows without keys).
+ *   scale, score_mod_id, mask_mod_id, mod_params: those of the forward (any mod
+ *   flex_attn_fwd takes; no block mask).
+ *   workspace: at least flex_attn_bwd_workspace_size(B, H, Sq) bytes, 16-byte aligned.
+ * Accumulation is fp32; P and dS enter the matmuls rounded to dtype (round-to-nearest-
+ * even).  Rows without keys give no gradient.  Deterministic: no atomics.
+ */
+flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, int B, int H, int Hkv,
+                            int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
+                            const flex_mod_params_t* mod_params, flex_dtype_t dtype, void* workspace,
+                            size_t workspace_bytes, flex_stream_t stream);
+
+/*
  * flex_attn_decode_workspace_size -- bytes of device workspace flex_attn_decode needs
  * for these sizes (the split-KV partial outputs and their log-sum-exps).
  */
@@ -252,7 +279,8 @@ void flex_attn_tile_sizes(int D, int* bm, int* bn);
  * flex_attn_device_status -- reads (and, if reset != 0, clears) the device status
  * word on the current device.  Synchronises the device.  Bits:
  *   1 = a decode kv_len outside [0, cap];  2 = a forward-kernel wait ran out of time;
- *   4 = a decode-kernel wait ran out of time;  8 = the self-test wait ran out (expected).
+ *   4 = a decode-kernel wait ran out of time;  8 = the self-test wait ran out (expected);
+ *   16 = a backward-kernel wait ran out of time.
  */
 flex_status_t flex_attn_device_status(uint32_t* status_out, int reset);
 

@@ -155,3 +155,22 @@ def test_captured_mods_rejected_on_host(lib):
                             ctypes.byref(mp(oq=32)), 0, None)
     assert big == 2                                           # beyond the key-tile bitmaps
     assert lib.flex_attn_mask_eval(5, None, 4, 4, P(16), None) == 1
+
+
+def test_bwd_rejects_bad_args_on_host(lib):
+    def bwd(q=16, lse=32, ws=64, wsb=1 << 20, B=1, H=2, Hkv=1, Sq=8, Skv=8, D=128, scale=0.1, score=0, mask=0,
+            mp=None, dtype=0):
+        return lib.flex_attn_bwd(P(q), P(16), P(16), P(16), P(lse), P(16), P(16), P(16), P(16), B, H, Hkv, Sq, Skv, D,
+                                 scale, score, mask, ctypes.byref(mp) if mp is not None else None, dtype, P(ws), wsb,
+                                 None)
+    assert bwd(q=0) == 1
+    assert bwd(lse=0) == 1
+    assert bwd(H=3, Hkv=2) == 1
+    assert bwd(scale=-1.0) == 1
+    assert bwd(D=96) == 2
+    assert bwd(mask=9) == 1
+    assert bwd(ws=0) == 4
+    assert bwd(wsb=16) == 4
+    assert bwd(q=24) == 3
+    assert bwd(lse=34) == 3
+    assert fa.bwd_workspace_size(2, 4, 300) == 2 * 2 * 4 * 384 * 4
