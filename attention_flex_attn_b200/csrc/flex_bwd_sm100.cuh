@@ -19,8 +19,11 @@
 //   bwd_dkdv_kernel   one CTA per 128-key tile and kv head: for each query tile of each
 //                     query head of the group, S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
 //                     per key row, dV += P^T dO and dK += dS^T Q (TMEM accumulators)
-// Roles per CTA (256 threads): warp 0 issues the MMAs (one thread), warp 1 the TMA loads,
-// warps 4-7 do the element-wise work (thread = TMEM lane = row), warps 2-3 idle.
+// Roles per CTA (384 threads): warp 0 issues the MMAs (one thread), warp 1 the TMA loads,
+// warps 4-7 and 8-11 do the element-wise work on the two 64-column halves of each tile
+// (thread = TMEM lane = row), warps 2-3 idle.  Each half writes its 16-bit results into
+// its own quarter of the TMEM buffer it read (columns [0, 32) and [64, 96)), and signals
+// its own barrier, so the products that consume them start on the first finished half.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -34,8 +37,8 @@
 
 namespace flexattn {
 
-constexpr int kBwdThreads = 256;
-constexpr int kBwdWarp0 = 4;  // first element-wise warp
+constexpr int kBwdThreads = 384;
+constexpr int kBwdWarp0 = 4;  // warps 4-7: columns [0, 64) of each tile, warps 8-11: [64, 128)
 constexpr unsigned kStatusBwdTimeout = 16u;
 
 struct BwdParams {
@@ -96,8 +99,8 @@ struct BwdDqSmem {
   static constexpr int kQOff = 0;                   // Q, then dO
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  // barriers: q, full[NS], empty[NS], sdp, ds, done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 3;
+  // barriers: q, full[NS], empty[NS], sdp, ds[2], done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 4;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemPtrOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -114,8 +117,8 @@ struct BwdDkvSmem {
   static constexpr int kKOff = 0;                                     // K, then V
   static constexpr int kSlotOff = 2 * kTileBytes;
   static constexpr int kBarOff = kSlotOff + kSlots * kSlotBytes;
-  // barriers: kv, full[NS], empty[NS], sdp, pds, done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 3;
+  // barriers: kv, full[NS], empty[NS], sdp, pds[2], done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 4;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemPtrOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -155,8 +158,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
   auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
   const uint32_t bar_sdp = sbase + L::kBarOff + 8u * (1 + 2 * NS);
-  const uint32_t bar_ds = bar_sdp + 8u;
-  const uint32_t bar_done = bar_sdp + 16u;
+  auto bar_ds = [&](int half) { return bar_sdp + 8u * (1 + half); };
+  const uint32_t bar_done = bar_sdp + 24u;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
   const uint32_t q_smem = sbase + L::kQOff, o_smem = q_smem + L::kTileBytes;
@@ -184,7 +187,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar_empty(s), 1);
     }
     mbar_init(bar_sdp, 1);
-    mbar_init(bar_ds, kBM);
+    mbar_init(bar_ds(0), kBM);
+    mbar_init(bar_ds(1), kBM);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -258,14 +262,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         issue_qk(tmem + s_col(t + 1), dq0, rK2 % NS);  // S of the next key tile
       }
-      if (!bwd_wait(bar_ds, static_cast<uint32_t>(t) & 1u, p, abort_flag)) break;
-      tc_fence_after();
-      // dQ += dS K: A = dS (bf16/f16 pairs in the first 64 columns of its S buffer)
+      // dQ += dS K, one 64-key half per element-wise warpgroup: A = dS, 16-bit pairs in
+      // columns [0, 32) (keys 0-63) and [64, 96) (keys 64-127) of its S buffer
       const uint64_t bkn = smem_desc(kv_smem(rK % NS), L::kChunkBytes, 1024, kSwizzle128B);
+      bool got_ds = true;
+      for (int half = 0; half < 2 && got_ds; ++half) {
+        if (!bwd_wait(bar_ds(half), static_cast<uint32_t>(t) & 1u, p, abort_flag)) {
+          got_ds = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
-        mma_ts(tmem + kDqCol, tmem + s_col(t) + 8u * kk, bkn + static_cast<uint64_t>((kk * 2048) >> 4), kIdescDq,
-               (t > 0 || kk > 0) ? 1u : 0u);
+        for (int q = 0; q < 4; ++q) {
+          const int kk = 4 * half + q;
+          mma_ts(tmem + kDqCol, tmem + s_col(t) + 64u * half + 8u * q, bkn + static_cast<uint64_t>((kk * 2048) >> 4),
+                 kIdescDq, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      if (!got_ds) break;
       mma_commit(bar_empty(rK % NS));
     }
     mma_commit(bar_done);
@@ -273,6 +287,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp >= kBwdWarp0) {
     // ============================================================ element-wise warps
     const int wq = warp & 3;
+    const int wg = (warp - kBwdWarp0) >> 2;  // column half of this warpgroup
+    const uint32_t cb = 64u * static_cast<uint32_t>(wg);
     const int row = wq * 32 + lane;
     const int i = q0 + row;
     const bool row_valid = i < p.Sq;
@@ -306,31 +322,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           c_hi = 0;
         }
       }
-      const uint32_t tS = tmem + lane_off + s_col(t), tP = tmem + lane_off + kDpCol;
-      const float base = slope2 * static_cast<float>(k0 - i) - lse2;
+      const uint32_t tS = tmem + lane_off + s_col(t) + cb, tP = tmem + lane_off + kDpCol + cb;
+      const float base = slope2 * static_cast<float>(k0 + static_cast<int>(cb) - i) - lse2;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[64], pr[64], w[32];
-        tmem_ld64(tS + 64u * half, sr);
-        tmem_ld64(tP + 64u * half, pr);
+      for (int part = 0; part < 2; ++part) {  // 32 columns at a time
+        uint32_t sr[32], pr[32], w[16];
+        tmem_ld32(tS + 32u * part, sr);
+        tmem_ld32(tP + 32u * part, pr);
+        float* x = reinterpret_cast<float*>(sr);
+        const int c0 = static_cast<int>(cb) + 32 * part;  // column of x[0] within the tile
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float ds[2];
+        for (int c = 0; c < 32; ++c)
+          x[c] = fmaf(x[c], p.scale_log2, fmaf(slope2, static_cast<float>(32 * part + c), base));
+        if (!full) {  // warp-uniform: the mask pass runs on PARTIAL tiles only
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 64 * half + 2 * e + u;
-            const float x = fmaf(__uint_as_float(sr[2 * e + u]), p.scale_log2, fmaf(slope2, static_cast<float>(c), base));
-            const bool keep = full || (c >= c_lo && c <= c_hi);
-            const float pe = keep ? ex2_approx(x) : 0.f;
-            ds[u] = keep ? pe * (__uint_as_float(pr[2 * e + u]) - delta) : 0.f;
-          }
-          w[e] = DtypeBits<T>::pack(ds[0], ds[1]);
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c < c_lo || c0 + c > c_hi) x[c] = -INFINITY;
         }
-        tmem_st32(tS + 32u * half, w);
+        // branch-free: ex2(-inf) = 0 gives dS = 0 for dropped keys
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = DtypeBits<T>::pack(ex2_approx(x[2 * e]) * (__uint_as_float(pr[2 * e]) - delta),
+                                    ex2_approx(x[2 * e + 1]) * (__uint_as_float(pr[2 * e + 1]) - delta));
+        tmem_st16(tS + 16u * part, w);  // columns cb + [0, 32): read by this warpgroup already
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar_ds);
+      mbar_arrive(bar_ds(wg));
     }
     // epilogue: dQ row * scale
     bool ran = ok && n > 0;
@@ -341,7 +359,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     T* out = reinterpret_cast<T*>(p.dq) + (static_cast<int64_t>(bh) * p.Sq + i) * D;
 #pragma unroll 1
-    for (int c = 0; c < D; c += 32) {
+    for (int c = wg * (D / 2); c < (wg + 1) * (D / 2); c += 32) {  // each warpgroup half of the columns
       uint32_t r[32];
       if (ran) tmem_ld32(tmem + lane_off + kDqCol + c, r);
       uint32_t w[16];
@@ -386,8 +404,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
   auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
   const uint32_t bar_sdp = sbase + L::kBarOff + 8u * (1 + 2 * NS);
-  const uint32_t bar_pds = bar_sdp + 8u;
-  const uint32_t bar_done = bar_sdp + 16u;
+  auto bar_pds = [&](int half) { return bar_sdp + 8u * (1 + half); };
+  const uint32_t bar_done = bar_sdp + 24u;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
   const uint32_t k_smem = sbase + L::kKOff, v_smem = k_smem + L::kTileBytes;
@@ -424,7 +442,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar_empty(s), 1);
     }
     mbar_init(bar_sdp, 1);
-    mbar_init(bar_pds, kBN);
+    mbar_init(bar_pds(0), kBN);
+    mbar_init(bar_pds(1), kBN);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -495,16 +514,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_ss(tmem + kDpCol, dv0 + off, bo + off, kIdescT, kk > 0 ? 1u : 0u);  // dP^T = V dO^T
       }
       mma_commit(bar_sdp);
-      if (!bwd_wait(bar_pds, static_cast<uint32_t>(u) & 1u, p, abort_flag)) break;
-      tc_fence_after();
+      // dV += P^T dO and dK += dS^T Q, one 64-query half per element-wise warpgroup: A =
+      // 16-bit pairs in columns [0, 32) / [64, 96) of the S^T and dP^T buffers
       const uint64_t bon = smem_desc(o_slot(s), L::kChunkBytes, 1024, kSwizzle128B);
       const uint64_t bqn = smem_desc(q_slot(s), L::kChunkBytes, 1024, kSwizzle128B);
+      bool got_p = true;
+      for (int half = 0; half < 2; ++half) {
+        if (!bwd_wait(bar_pds(half), static_cast<uint32_t>(u) & 1u, p, abort_flag)) {
+          got_p = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < kBM / 16; ++kk) {
-        const uint64_t off = static_cast<uint64_t>((kk * 2048) >> 4);
-        mma_ts(tmem + kDvCol, tmem + kSCol + 8u * kk, bon + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
-        mma_ts(tmem + kDkCol, tmem + kDpCol + 8u * kk, bqn + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
+        for (int q = 0; q < 4; ++q) {
+          const int kk = 4 * half + q;
+          const uint64_t off = static_cast<uint64_t>((kk * 2048) >> 4);
+          const uint32_t acol = 64u * half + 8u * q;
+          mma_ts(tmem + kDvCol, tmem + kSCol + acol, bon + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + kDkCol, tmem + kDpCol + acol, bqn + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
+        }
       }
+      if (!got_p) break;
       mma_commit(bar_empty(s));
     }
     mma_commit(bar_done);
@@ -512,6 +542,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp >= kBwdWarp0) {
     // ============================================================ element-wise warps
     const int wq = warp & 3;
+    const int wg = (warp - kBwdWarp0) >> 2;  // column (query) half of this warpgroup
+    const int cb = 64 * wg;
     const int row = wq * 32 + lane;
     const int j = k0 + row;  // this thread's key
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -542,33 +574,50 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         int c_lo = 0, c_hi = kBM - 1;
         if (!full) col_interval_of(key_lo, key_hi, q0, c_lo, c_hi);
         const float* stat = reinterpret_cast<const float*>(sgen + stat_slot(s));
-        const float base = slope2 * static_cast<float>(j - q0);
+        const float base = slope2 * static_cast<float>(j - q0 - cb);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sr[64], pr[64], wp[32], wd[32];
-          tmem_ld64(tmem + lane_off + kSCol + 64u * half, sr);
-          tmem_ld64(tmem + lane_off + kDpCol + 64u * half, pr);
+        for (int part = 0; part < 2; ++part) {  // 32 columns (queries) at a time
+          const int c0 = cb + 32 * part;       // column of x[0] within the tile
+          uint32_t sr[32], pr[32], wp[16], wd[16];
+          tmem_ld32(tmem + lane_off + kSCol + c0, sr);
+          tmem_ld32(tmem + lane_off + kDpCol + c0, pr);
+          float* x = reinterpret_cast<float*>(sr);
+          const float4* st4 = reinterpret_cast<const float4*>(stat + c0);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float pe[2], ds[2];
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 l4 = st4[c4];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const int c = 64 * half + 2 * e + v;  // query q0 + c
-              const float x = fmaf(__uint_as_float(sr[2 * e + v]), p.scale_log2,
-                                   fmaf(-slope2, static_cast<float>(c), base)) - stat[c];
-              const bool keep = full || (c >= c_lo && c <= c_hi);
-              pe[v] = keep ? ex2_approx(x) : 0.f;
-              ds[v] = keep ? pe[v] * (__uint_as_float(pr[2 * e + v]) - stat[kBM + c]) : 0.f;
+            for (int v = 0; v < 4; ++v) {
+              const int c = 4 * c4 + v;
+              x[c] = fmaf(x[c], p.scale_log2, fmaf(-slope2, static_cast<float>(32 * part + c), base)) - lv[v];
             }
-            wp[e] = DtypeBits<T>::pack(pe[0], pe[1]);
-            wd[e] = DtypeBits<T>::pack(ds[0], ds[1]);
           }
-          tmem_st32(tmem + lane_off + kSCol + 32u * half, wp);
-          tmem_st32(tmem + lane_off + kDpCol + 32u * half, wd);
+          if (!full) {  // warp-uniform: the mask pass runs on PARTIAL tiles only
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c0 + c < c_lo || c0 + c > c_hi) x[c] = -INFINITY;
+          }
+          const float4* dl4 = reinterpret_cast<const float4*>(stat + kBM + c0);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 d4 = dl4[c4];
+            const float p0 = ex2_approx(x[4 * c4]), p1 = ex2_approx(x[4 * c4 + 1]);
+            const float p2 = ex2_approx(x[4 * c4 + 2]), p3 = ex2_approx(x[4 * c4 + 3]);
+            wp[2 * c4] = DtypeBits<T>::pack(p0, p1);
+            wp[2 * c4 + 1] = DtypeBits<T>::pack(p2, p3);
+            wd[2 * c4] = DtypeBits<T>::pack(p0 * (__uint_as_float(pr[4 * c4]) - d4.x),
+                                            p1 * (__uint_as_float(pr[4 * c4 + 1]) - d4.y));
+            wd[2 * c4 + 1] = DtypeBits<T>::pack(p2 * (__uint_as_float(pr[4 * c4 + 2]) - d4.z),
+                                                p3 * (__uint_as_float(pr[4 * c4 + 3]) - d4.w));
+          }
+          // columns cb + [0, 32) of each buffer, already read by this warpgroup
+          tmem_st16(tmem + lane_off + kSCol + cb + 16u * part, wp);
+          tmem_st16(tmem + lane_off + kDpCol + cb + 16u * part, wd);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar_pds);
+        mbar_arrive(bar_pds(wg));
         ++u;
       }
     }
@@ -581,8 +630,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     const bool key_valid = j < p.Skv;
     const int64_t orow = (static_cast<int64_t>(bkv) * p.Skv + j) * D;
-#pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
+    {
+      const int which = wg;  // warpgroup 0 writes dV, warpgroup 1 dK
       T* out = reinterpret_cast<T*>(which ? p.dk : p.dv) + orow;
       const float mul = which ? p.scale : 1.0f;
       const uint32_t col = which ? kDkCol : kDvCol;

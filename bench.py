@@ -390,7 +390,28 @@ def per_case(fa, q, k, v, scale, o, lse, args):
             out[name]["tflops_useful"] = useful_window / t / 1e12
     out.update(block_cases(fa, q, k, v, scale, o, lse))
     out.update(captured_cases(fa, q, k, v, scale, o, lse))
+    out.update(bwd_cases(fa, q, k, v, scale))
     return out
+
+
+def bwd_cases(fa, q, k, v, scale):
+    """Backward (flex_attn_bwd: prep + dQ + dK/dV launches) on the forward inputs, with
+    dO ~ N(0, 1) (seed 4103): TFLOPS count the five algorithmic products of the backward,
+    10 * B * H * Sq * Skv * D (halved for causal), not the two the kernels recompute."""
+    import torch
+    import synth
+    B, H, S, D = q.shape
+    res = {}
+    dout = synth.normal_tensor(tuple(q.shape), 4103, dtype="bf16", device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.bwd_workspace_size(B, H, S), dtype=torch.uint8, device=q.device)
+    for name, mods in (("bwd_no_mod", {}), ("bwd_causal", dict(mask_mod="causal"))):
+        o, lse = fa.fwd(q, k, v, scale=scale, **mods)
+        t = _time_fn(lambda: fa.bwd(q, k, v, o, lse, dout, scale=scale, dq=dq, dk=dk, dv=dv, workspace=ws, **mods),
+                     10, 2)
+        flops = 2.5 * fwd_flops(B, H, S, S, D) * (0.5 if "causal" in name else 1.0)
+        res[name] = {"us": t * 1e6, "tflops": flops / t / 1e12}
+    return res
 
 
 def captured_cases(fa, q, k, v, scale, o, lse):
