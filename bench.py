@@ -38,9 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram read+write bytes per launch from ncu, keyed by the hash of the kernel sources
 # they were measured on (a changed kernel reports null until it is captured again)
 MEASURED_TRAFFIC = {
-    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 402,740,480 B read +
-    # 116,575,744 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
-    "60a6582866216d8d": 519316224,
+    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 403,024,640 B read +
+    # 115,118,080 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
+    "0c78b41d8c4eb42c": 518142720,
 }
 # the forward kernel's sources: the roofline traffic below belongs to that kernel
 KERNEL_SOURCES = ["attention_flex_attn_b200/csrc/flex_fwd_sm100.cuh",
@@ -236,7 +236,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-case and e2e measurements")
-    ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "bwd", "decode"], default=None,
                     help="run only a few launches of one kernel (for ncu captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -572,13 +572,21 @@ def profile_case(which):
     """A few launches of one kernel on a case larger than L2 but a few GB at most:
     fwd = B2 H32 S4096 D128 bf16 no_mod (192 MiB of Q/K/V); fwd8192 = the full forward
     workload; fwd_blocks = the S4096 inputs with random per-head block lists, half of the
-    key blocks of every query tile full; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
+    key blocks of every query tile full; bwd = forward + backward at B2 H32 S4096 D128,
+    no_mod then causal; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
     import torch
     import synth
     import attention_flex_attn_b200 as fa
     fa.load_library()
     dev = torch.device("cuda", 0)
-    if which == "fwd_blocks":
+    if which == "bwd":
+        S = 4096
+        q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
+        dout = synth.normal_tensor(tuple(q.shape), 4103, dtype="bf16", device=dev)
+        for mask in ("none", "causal"):
+            o, lse = fa.fwd(q, k, v, mask_mod=mask)
+            fa.bwd(q, k, v, o, lse, dout, mask_mod=mask)
+    elif which == "fwd_blocks":
         import numpy as np
         S, nq = 4096, 32
         q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
