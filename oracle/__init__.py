@@ -52,6 +52,8 @@ def _bind(lib):
     lib.oracle_tile_map.restype = I
     lib.oracle_alibi_slope.argtypes = [I, I]
     lib.oracle_alibi_slope.restype = D
+    lib.oracle_e4m3_value.argtypes = [I]
+    lib.oracle_e4m3_value.restype = D
     lib.oracle_fwd_block_sparse.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, I,
                                             P, P, P, P, I, I, I, P, I64, P, P, I]
     lib.oracle_fwd_block_sparse.restype = I
@@ -81,11 +83,15 @@ def _dtype_code(t: torch.Tensor) -> int:
         return 0
     if t.dtype == torch.float16:
         return 1
-    raise TypeError(f"oracle takes bf16/f16 tensors, got {t.dtype}")
+    if t.dtype == torch.float8_e4m3fn:
+        return 2
+    raise TypeError(f"oracle takes bf16/f16/e4m3 tensors, got {t.dtype}")
 
 
 def _bits(t: torch.Tensor) -> np.ndarray:
-    """The raw 16-bit patterns of a CPU bf16/f16 tensor (contiguous copy)."""
+    """The raw bit patterns of a CPU bf16/f16 (16-bit) or e4m3 (8-bit) tensor (contiguous copy)."""
+    if t.dtype == torch.float8_e4m3fn:
+        return t.detach().cpu().contiguous().view(torch.uint8).numpy()
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
@@ -203,6 +209,21 @@ def bwd(q, k, v, dout, scale=None, score_mod="none", mask_mod="none", window=0, 
     if groups is None:
         return dq.reshape(B, H, Sq, D), dk.reshape(B, Hkv, Skv, D), dv.reshape(B, Hkv, Skv, D)
     return dq, dk, dv
+
+
+def e4m3_value(bits: int) -> float:
+    """The exact value of an 8-bit e4m3 (E4M3FN) code."""
+    return float(_load().oracle_e4m3_value(int(bits)))
+
+
+def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None, **kw):
+    """Oracle forward on e4m3 inputs with per-tensor descales: q = descale_q * q8 (and so
+    on) exactly; returns (O, LSE) of the plain definition on those values (P unrounded)."""
+    D = q8.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o, lse = fwd(q8, k8, v8, scale=float(scale) * float(descale_q) * float(descale_k), **kw)
+    return o * float(descale_v), lse
 
 
 def _i32(a):

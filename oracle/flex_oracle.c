@@ -72,6 +72,7 @@
 
 #define OR_DT_BF16 0
 #define OR_DT_F16 1
+#define OR_DT_E4M3 2  /* 8-bit e4m3 (OCP E4M3FN): the buffers hold bytes */
 
 /* ---- exact conversion of stored 16-bit values to double ---------------- */
 
@@ -97,7 +98,26 @@ static double f16_bits_to_double(uint16_t h) {
   return sign ? -v : v;
 }
 
+/* e4m3: sign, 4 exponent bits (bias 7), 3 mantissa bits; no infinities; S.1111.111 is NaN */
+static double e4m3_bits_to_double(uint8_t b) {
+  int sign = (b >> 7) & 1;
+  int e = (b >> 3) & 15;
+  int m = b & 7;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -9);              /* subnormal: m/8 * 2^-6 */
+  } else if (e == 15 && m == 7) {
+    v = NAN;
+  } else {
+    v = ldexp((double)(m + 8), e - 10);    /* (1 + m/8) * 2^(e-7) */
+  }
+  return sign ? -v : v;
+}
+
+double oracle_e4m3_value(int bits) { return e4m3_bits_to_double((uint8_t)bits); }
+
 static double elem(const uint16_t* p, int64_t idx, int dtype) {
+  if (dtype == OR_DT_E4M3) return e4m3_bits_to_double(((const uint8_t*)p)[idx]);
   return dtype == OR_DT_BF16 ? bf16_bits_to_double(p[idx]) : f16_bits_to_double(p[idx]);
 }
 

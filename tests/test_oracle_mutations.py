@@ -1,6 +1,6 @@
 """Plants plausible mistakes in copies of the C oracle and checks that the pins in
-test_oracle_pins.py, test_oracle_block_pins.py, test_oracle_mods_pins.py and
-test_oracle_bwd_pins.py catch every one (each mutant must fail at least one pin).
+test_oracle_pins.py, test_oracle_block_pins.py, test_oracle_mods_pins.py,
+test_oracle_bwd_pins.py and test_oracle_fp8_pins.py catch every one (each mutant must fail at least one pin).
 Everything runs on the CPU against a temporary build; the real oracle is untouched.
 Mutants that leave the mathematics unchanged (e.g. dropping the fully-masked guard,
 which still yields p = 0 and log 0 = -inf) are not listed: no test could tell them apart."""
@@ -14,6 +14,7 @@ import torch
 import oracle
 import tests.test_oracle_block_pins as bpins
 import tests.test_oracle_bwd_pins as bwpins
+import tests.test_oracle_fp8_pins as f8pins
 import tests.test_oracle_mods_pins as mpins
 import tests.test_oracle_pins as pins
 
@@ -65,6 +66,10 @@ MUTANTS = [
     ("bwd one head per group", "for (int hg = 0; hg < G; ++hg) {", "for (int hg = 0; hg < 1; ++hg) {"),
     ("bwd P unnormalised", "double pij = exp(score_ij(J, b, h, i, j) - W->M[srow]) / W->l[srow];",
      "double pij = exp(score_ij(J, b, h, i, j) - W->M[srow]);"),
+    ("e4m3 exponent bias", "v = ldexp((double)(m + 8), e - 10);    /* (1 + m/8) * 2^(e-7) */",
+     "v = ldexp((double)(m + 8), e - 11);    /* (1 + m/8) * 2^(e-7) */"),
+    ("e4m3 subnormal scale", "v = ldexp((double)m, -9);              /* subnormal: m/8 * 2^-6 */",
+     "v = ldexp((double)m, -10);              /* subnormal: m/8 * 2^-6 */"),
     ("bf16 decoded as truncated", "  uint32_t u = ((uint32_t)b) << 16;", "  uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
 ]
 
@@ -104,6 +109,7 @@ CHECKS = [
                                              "dtype": torch.bfloat16}),
     (bwpins.test_bwd_single_key_closed_form, {}),
     (bwpins.test_bwd_equals_finite_differences_of_forward, {}),
+    (f8pins.test_e4m3_decode_matches_torch, {}),
 ]
 
 
