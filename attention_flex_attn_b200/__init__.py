@@ -27,7 +27,8 @@ MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset":
 FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
-EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_bwd_workspace_size", "flex_attn_bwd",
+EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_fwd_fp8_workspace_size", "flex_attn_fwd_fp8",
+            "flex_attn_bwd_workspace_size", "flex_attn_bwd",
             "flex_attn_decode_workspace_size", "flex_attn_decode",
             "flex_attn_decode_noalloc", "flex_attn_mask_eval", "flex_attn_selftest_wait_timeout",
             "flex_attn_tile_sizes", "flex_attn_device_status", "flex_status_string"]
@@ -69,6 +70,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_fwd_block_sparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams),
                                                ctypes.POINTER(BlockMaskC), I, P]
     lib.flex_attn_fwd_block_sparse.restype = I
+    lib.flex_attn_fwd_fp8_workspace_size.argtypes = [I, I, I, I]
+    lib.flex_attn_fwd_fp8_workspace_size.restype = SZ
+    lib.flex_attn_fwd_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, F, F, F, I, I, ctypes.POINTER(ModParams),
+                                      P, SZ, P]
+    lib.flex_attn_fwd_fp8.restype = I
     lib.flex_attn_bwd_workspace_size.argtypes = [I, I, I]
     lib.flex_attn_bwd_workspace_size.restype = SZ
     lib.flex_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams), I,
@@ -232,6 +238,39 @@ def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None
                                         scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
                                         ctypes.byref(bm), DTYPES[q.dtype], _stream(q.device))
     _check(rc, "flex_attn_fwd_block_sparse")
+    return o, lse
+
+
+def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None, score_mod="none",
+            mask_mod="none", window=0, offset=0, alibi_slopes=None, return_lse=True, out=None, lse_out=None,
+            workspace=None):
+    """8-bit forward (flex_attn_fwd_fp8): q8/k8/v8 are torch.float8_e4m3fn CUDA tensors in
+    the layouts of fwd(); their values are descale_* times the codes.  Returns (O, LSE)
+    with O in bf16.  Head dim 128."""
+    lib = load_library()
+    for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _cuda_tensor(t, n)
+        if t.dtype != torch.float8_e4m3fn:
+            raise FlexAttnError(f"{n} must be torch.float8_e4m3fn")
+    B, H, Sq, D = q8.shape
+    Bk, Hkv, Skv, Dk = k8.shape
+    if Bk != B or Dk != D or tuple(v8.shape) != tuple(k8.shape):
+        raise FlexAttnError("shape mismatch between q8, k8, v8")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = out if out is not None else torch.empty((B, H, Sq, D), dtype=torch.bfloat16, device=q8.device)
+    lse = None
+    if return_lse:
+        lse = lse_out if lse_out is not None else torch.empty((B, H, Sq), dtype=torch.float32, device=q8.device)
+    need = int(lib.flex_attn_fwd_fp8_workspace_size(B, Hkv, Skv, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q8.device)
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, None, None)
+    rc = lib.flex_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D, float(scale),
+                               float(descale_q), float(descale_k), float(descale_v), score, MASK_MODS[mask_mod],
+                               ctypes.byref(mp), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(q8.device))
+    _check(rc, "flex_attn_fwd_fp8")
     return o, lse
 
 

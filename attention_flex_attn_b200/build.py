@@ -21,7 +21,7 @@ OBJ_DIR = os.path.join(PKG, "_build")
 # They compile in parallel and link into one shared library.
 SOURCES = [os.path.join(CSRC, f) for f in (
     "flex_fwd_d128.cu", "flex_fwd_d128_blocks.cu", "flex_fwd_d64.cu", "flex_fwd_d64_blocks.cu",
-    "flex_bwd_d128.cu", "flex_bwd_d64.cu", "flex_decode_launch.cu", "flex_attn_api.cu")]
+    "flex_bwd_d128.cu", "flex_bwd_d64.cu", "flex_fwd_fp8.cu", "flex_decode_launch.cu", "flex_attn_api.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, "flex_attn.h")]
 

@@ -56,6 +56,21 @@ bool make_map(CUtensorMap* map, const void* base, flex_dtype_t dt, int D, int ro
   return r == CUDA_SUCCESS;
 }
 
+// [outer x rows x inner] bytes, box = 128 bytes x 128 rows x 1, 128-byte swizzle (the
+// 8-bit forward's tiles; inner must be a multiple of 16).
+bool make_map_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(inner * rows)};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Scratch for flex_attn_decode_noalloc: compiled into the library so that callers who
 // cannot allocate device memory still get a workspace.  One copy per device, shared by
 // every call on that device.
@@ -268,6 +283,72 @@ flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const voi
   if (!block_mask) return FLEX_ERR_INVALID_ARG;
   return fwd_common(q, k, v, o, lse, B, H, Hkv, Sq, Skv, D, scale, score_mod_id, mask_mod_id, mod_params,
                     block_mask, dtype, stream);
+}
+
+size_t flex_attn_fwd_fp8_workspace_size(int B, int Hkv, int Skv, int D) {
+  if (B < 1 || Hkv < 1 || Skv < 1 || D != kFp8D) return 0;
+  const size_t skv_pad = (static_cast<size_t>(Skv) + 127) / 128 * 128;
+  return static_cast<size_t>(B) * Hkv * D * skv_pad;
+}
+
+flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int H,
+                                int Hkv, int Sq, int Skv, int D, float scale, float descale_q, float descale_k,
+                                float descale_v, int score_mod_id, int mask_mod_id,
+                                const flex_mod_params_t* mod_params, void* workspace, size_t workspace_bytes,
+                                flex_stream_t stream) {
+  if (!q8 || !k8 || !v8 || !o) return FLEX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
+  for (float f : {scale, descale_q, descale_k, descale_v})
+    if (!(f > 0.f) || !std::isfinite(f)) return FLEX_ERR_INVALID_ARG;
+  if (D != kFp8D) return FLEX_ERR_UNSUPPORTED;
+  if (score_mod_id != FLEX_SCORE_NONE && score_mod_id != FLEX_SCORE_ALIBI && score_mod_id != FLEX_SCORE_ALIBI_SLOPES)
+    return FLEX_ERR_INVALID_ARG;
+  const int mask = mask_kind(mask_mod_id);
+  if (mask < 0) return FLEX_ERR_INVALID_ARG;
+  if (mask == kMaskDocument || mask == kMaskDocumentCausal) return FLEX_ERR_UNSUPPORTED;
+  const flex_mod_params_t zero{};
+  const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
+  if (mask == kMaskSliding && mp.window < 1) return FLEX_ERR_INVALID_ARG;
+  if (mp.flags & FLEX_FLAG_TILE_MAP) return FLEX_ERR_UNSUPPORTED;
+  if (score_mod_id == FLEX_SCORE_ALIBI_SLOPES) {
+    if (!mp.alibi_slopes) return FLEX_ERR_INVALID_ARG;
+    if (!aligned4(mp.alibi_slopes)) return FLEX_ERR_MISALIGNED;
+  }
+  const size_t need = flex_attn_fwd_fp8_workspace_size(B, Hkv, Skv, D);
+  if (!workspace || workspace_bytes < need) return FLEX_ERR_WORKSPACE;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(workspace) ||
+      (lse && !aligned16(lse)))
+    return FLEX_ERR_MISALIGNED;
+  const int64_t bh = static_cast<int64_t>(B) * H, bhkv = static_cast<int64_t>(B) * Hkv;
+  const int n_qtiles = (Sq + kBM - 1) / kBM, n_pairs = (n_qtiles + 1) / 2;
+  const int skv_pad = (Skv + 127) / 128 * 128;
+  if (bh * n_pairs > 0x7fffffff || bhkv * (skv_pad / 128) > 0x7fffffff) return FLEX_ERR_UNSUPPORTED;
+  unsigned* st = status_ptr();
+  if (!st) return FLEX_ERR_CUDA;
+  Fp8Maps m;
+  if (!make_map_u8(&m.q, q8, D, Sq, bh) || !make_map_u8(&m.k, k8, D, Skv, bhkv) ||
+      !make_map_u8(&m.vt, workspace, skv_pad, D, bhkv))
+    return FLEX_ERR_CUDA;
+  Fp8Params p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.status = st;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.G = H / Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.Skv_pad = skv_pad;
+  p.n_qtiles = n_qtiles;
+  p.n_ktiles = (Skv + kBN - 1) / kBN;
+  p.n_pairs = n_pairs;
+  p.scale_log2 = scale * descale_q * descale_k * kLog2e;
+  p.descale_v = descale_v;
+  p.slopes = score_mod_id == FLEX_SCORE_ALIBI_SLOPES ? mp.alibi_slopes : nullptr;
+  p.mask = mask_args(mask, mp, Skv);
+  const int score = score_mod_id == FLEX_SCORE_NONE ? kScoreNone : kScoreAlibi;
+  return fp8_dispatch(score, mask, static_cast<const uint8_t*>(v8), static_cast<uint8_t*>(workspace), bhkv, m, p,
+                      static_cast<int>(bh * n_pairs), reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t flex_attn_bwd_workspace_size(int B, int H, int Sq) {

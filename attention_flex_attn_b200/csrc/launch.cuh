@@ -9,9 +9,21 @@
 #include "flex_attn.h"
 #include "flex_bwd_sm100.cuh"
 #include "flex_decode.cuh"
+#include "flex_fwd_fp8_sm100.cuh"
 #include "flex_fwd_sm100.cuh"
 
 namespace flexattn {
+
+// Tensor maps of the 8-bit forward: Q [128, Sq, B*H], K [128, Skv, B*Hkv] and the
+// transposed V^T [Skv_pad, 128, B*Hkv], all bytes, 128 x 128 boxes.
+struct Fp8Maps {
+  CUtensorMap q, k, vt;
+};
+
+// V transpose into vt, then the 8-bit forward over (score_mod, mask_mod)
+// (flex_fwd_fp8.cu).
+flex_status_t fp8_dispatch(int score, int mask, const uint8_t* v, uint8_t* vt, int64_t kv_rows, const Fp8Maps& m,
+                           const Fp8Params& p, int n_units, cudaStream_t s);
 
 // Forward over every (dtype, score_mod, mask_mod) instantiation of one head dim and
 // block-mask mode.  Instantiated in flex_fwd_d{64,128}{,_blocks}.cu.

@@ -174,3 +174,20 @@ def test_bwd_rejects_bad_args_on_host(lib):
     assert bwd(q=24) == 3
     assert bwd(lse=34) == 3
     assert fa.bwd_workspace_size(2, 4, 300) == 2 * 2 * 4 * 384 * 4
+
+
+def test_fp8_rejects_bad_args_on_host(lib):
+    def f8(q=16, ws=64, wsb=1 << 24, D=128, scale=0.1, dq=1.0, dk=1.0, dv=1.0, score=0, mask=0, mp=None):
+        return lib.flex_attn_fwd_fp8(P(q), P(16), P(16), P(16), None, 1, 2, 1, 8, 8, D, scale, dq, dk, dv, score,
+                                     mask, ctypes.byref(mp) if mp is not None else None, P(ws), wsb, None)
+    assert f8(q=0) == 1
+    assert f8(D=64) == 2
+    assert f8(dq=0.0) == 1
+    assert f8(dv=float("inf")) == 1
+    assert f8(mask=5) == 2                                   # document rules: not on the 8-bit path
+    assert f8(mp=fa.ModParams(0, 0, 1, 16, None, None, None, 0)) == 2   # tile map: not on the 8-bit path
+    assert f8(ws=0) == 4
+    assert f8(wsb=100) == 4
+    assert f8(q=8) == 3
+    assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 128) == 2 * 4 * 128 * 384
+    assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 64) == 0

@@ -1,0 +1,124 @@
+"""GPU parity of flex_attn_fwd_fp8 (e4m3 Q/K/V, per-tensor descales, bf16 O).
+
+FP8 flex paths are named as a later phase on FlyDSL PR 931 "Add flex_attention (score_mod
+/ mask_mod) on the generic flash-attention kernel" (Out of scope). The oracle computes the
+exact definition on the dequantized inputs (P unrounded); the kernel rounds P to e4m3 for
+the P.V product. Tolerance per element, derived from that rounding: P' = P * 2^(6..8)
+keeps a relative error of 2^-4 for normal e4m3 values and an absolute error of 2^-10 in
+P' (2^-16 in P) below them, so
+    |O - O_ref| <= descale_v * (2^-4 * (P |v8|) + 2^-16 * (keep |v8|)) * 1.05
+                   + 2^-8 |O_ref| + 1e-4            (bf16 output rounding, fp32 sums),
+checked element by element with the oracle's P; LSE (unaffected by the rounding of P)
+within 1e-2; rows without keys O = +0 and LSE = -inf exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _fa():
+    import attention_flex_attn_b200 as fa
+    fa.load_library()
+    return fa
+
+
+def _inputs(B, H, Hkv, Sq, Skv, seed, spread=1.0):
+    q, k, v = synth.qkv(B, H, Hkv, Sq, Skv, 128, seed=seed)
+    return tuple((t.float() * spread).to(torch.float8_e4m3fn) for t in (q, k, v))
+
+
+def _check(q8, k8, v8, o, lse, dq, dk, dv, scale, rows=None, **mods):
+    ro, rl = oracle.fwd_fp8(q8, k8, v8, descale_q=dq, descale_k=dk, descale_v=dv, scale=scale, rows=rows, **mods)
+    # the oracle's probabilities on the same values (every e4m3 value is exact in bf16)
+    bf = lambda t: t.to(torch.bfloat16)
+    _, _, P = oracle.fwd(bf(q8), bf(k8), bf(v8), scale=scale * dq * dk, rows=rows, want_probs=True, **mods)
+    B, H, Sq, D = q8.shape
+    G = H // k8.shape[1]
+    av = np.abs(v8.double().numpy())  # [B, Hkv, Skv, D]
+    if rows is None:
+        av_rows = np.repeat(av, G, axis=1)                      # [B, H, Skv, D]
+        Pm = P.reshape(B, H, Sq, -1)
+        bound = dv * (2.0 ** -4 * np.einsum("bhij,bhjd->bhid", Pm, av_rows)
+                      + 2.0 ** -16 * np.einsum("bhij,bhjd->bhid", (Pm > 0).astype(np.float64), av_rows))
+        got = o.float().cpu().numpy().astype(np.float64)
+        lg = lse.cpu().numpy().astype(np.float64)
+    else:
+        rows = np.asarray(rows)
+        b_idx = rows // (H * Sq)
+        h_idx = (rows // Sq) % H
+        av_rows = av[b_idx, h_idx // G]                         # [n, Skv, D]
+        bound = dv * (2.0 ** -4 * np.einsum("nj,njd->nd", P, av_rows)
+                      + 2.0 ** -16 * np.einsum("nj,njd->nd", (P > 0).astype(np.float64), av_rows))
+        got = o.reshape(-1, D)[torch.as_tensor(rows, device=o.device)].float().cpu().numpy().astype(np.float64)
+        lg = lse.reshape(-1)[torch.as_tensor(rows, device=lse.device)].cpu().numpy().astype(np.float64)
+        ro, rl = ro.reshape(got.shape), rl.reshape(lg.shape)
+    tol = 1.05 * bound + 2.0 ** -8 * np.abs(ro) + 1e-4
+    err = np.abs(got - ro)
+    assert not np.isnan(got).any()
+    worst = float((err / tol).max())
+    assert worst <= 1.0, f"O error exceeds the e4m3 bound (worst ratio {worst:.3f})"
+    dead = np.isneginf(rl)
+    assert np.array_equal(np.isneginf(lg), dead)
+    assert np.all(got[dead] == 0.0)
+    if (~dead).any():
+        assert float(np.abs(lg[~dead] - rl[~dead]).max()) <= 1e-2
+    return float(err.mean())
+
+
+MODS = [dict(), dict(mask_mod="causal"), dict(mask_mod="causal", score_mod="alibi"),
+        dict(mask_mod="sliding_window", window=150), dict(mask_mod="kv_le_q_plus_offset", offset=-60),
+        dict(score_mod="alibi", alibi_slopes=np.array([0.25, -0.125, 0.0625, 0.5], np.float32))]
+
+
+@pytest.mark.parametrize("mods", MODS, ids=lambda m: "-".join(f"{k}" for k in m) or "no_mod")
+@pytest.mark.parametrize("desc", [(1.0, 1.0, 1.0), (0.5, 2.0, 0.25), (0.37, 1.3, 0.71)])
+def test_ragged_gqa(mods, desc):
+    fa = _fa()
+    B, H, Hkv, Sq, Skv = 2, 4, 2, 300, 700
+    q8, k8, v8 = _inputs(B, H, Hkv, Sq, Skv, seed=97)
+    dq, dk, dv = desc
+    scale = 1.0 / math.sqrt(128)
+    m = dict(mods)
+    if m.get("alibi_slopes") is not None:
+        m["alibi_slopes"] = torch.from_numpy(m["alibi_slopes"]).cuda()
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), descale_q=dq, descale_k=dk, descale_v=dv, scale=scale, **m)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    _check(q8, k8, v8, o, lse, dq, dk, dv, scale, **mods)
+
+
+def test_rows_without_keys():
+    fa = _fa()
+    q8, k8, v8 = _inputs(1, 2, 2, 250, 1024, seed=98)
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), scale=0.1, mask_mod="kv_le_q_plus_offset", offset=-300)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_peaked_scores_wide_range():
+    """Larger scores (values spread x4): P concentrates on few keys, where the 8-bit
+    rounding of P matters most."""
+    fa = _fa()
+    q8, k8, v8 = _inputs(1, 4, 4, 256, 512, seed=99, spread=4.0)
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), scale=0.125, mask_mod="causal")
+    torch.cuda.synchronize()
+    _check(q8, k8, v8, o, lse, 1.0, 1.0, 1.0, 0.125, mask_mod="causal")
+
+
+def test_mha_2048_sampled():
+    fa = _fa()
+    B, H, S = 2, 32, 2048
+    q8, k8, v8 = _inputs(B, H, H, S, S, seed=100)
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), descale_q=0.5, descale_k=0.5, descale_v=2.0,
+                        mask_mod="causal")
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(101)
+    rows = np.sort(rng.choice(B * H * S, 96, replace=False))
+    _check(q8, k8, v8, o, lse, 0.5, 0.5, 2.0, 1.0 / math.sqrt(128), rows=rows, mask_mod="causal")
