@@ -33,6 +33,12 @@ namespace flexattn {
 constexpr int kFp8D = 128;
 constexpr float kP8Shift = 6.0f;      // log2 of the factor P carries into the 8-bit product
 constexpr float kP8Rescale = 2.0f;    // O rescale threshold (log2) for the 8-bit path
+#ifndef FLEX_FP8_EMU_PAIRS
+#define FLEX_FP8_EMU_PAIRS 0
+#endif
+// Of the 8 value pairs of each 16-key chunk, how many take 2^x from the polynomial on the
+// FMA pipe instead of MUFU ex2 (the 8-bit kernel is bound by MUFU, not the tensor core).
+constexpr int kFp8EmuPairs = FLEX_FP8_EMU_PAIRS;
 
 struct Fp8Params {
   __nv_bfloat16* o;
@@ -428,10 +434,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           float e[16];
 #pragma unroll
           for (int x = 0; x < 16; x += 2) {
-            float x0, x1;
-            unpack2(fma2(pack2(s[c0 + x], s[c0 + x + 1]), sc2, nm2), x0, x1);
-            e[x] = ex2_approx(x0);
-            e[x + 1] = ex2_approx(x1);
+            const uint64_t x2 = fma2(pack2(s[c0 + x], s[c0 + x + 1]), sc2, nm2);
+            if (x / 2 >= 8 - kFp8EmuPairs) {  // this pair on the FMA pipe
+              unpack2(exp2_poly2(x2), e[x], e[x + 1]);
+            } else {
+              float x0, x1;
+              unpack2(x2, x0, x1);
+              e[x] = ex2_approx(x0);
+              e[x + 1] = ex2_approx(x1);
+            }
             if (x & 2)
               acc_b = add2(acc_b, pack2(e[x], e[x + 1]));
             else

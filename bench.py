@@ -236,7 +236,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-case and e2e measurements")
-    ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "bwd", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "bwd", "fp8", "decode"], default=None,
                     help="run only a few launches of one kernel (for ncu captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -391,7 +391,26 @@ def per_case(fa, q, k, v, scale, o, lse, args):
     out.update(block_cases(fa, q, k, v, scale, o, lse))
     out.update(captured_cases(fa, q, k, v, scale, o, lse))
     out.update(bwd_cases(fa, q, k, v, scale))
+    out.update(fp8_cases(fa, q, k, v, scale))
     return out
+
+
+def fp8_cases(fa, q, k, v, scale):
+    """8-bit forward (flex_attn_fwd_fp8) on the forward inputs rounded to e4m3 (descales 1),
+    including its V transpose pre-pass; TFLOPS as for the 16-bit forward."""
+    import torch
+    B, H, S, D = q.shape
+    q8, k8, v8 = (t.float().to(torch.float8_e4m3fn) for t in (q, k, v))
+    ws = torch.empty(fa.load_library().flex_attn_fwd_fp8_workspace_size(B, k.shape[1], S, D), dtype=torch.uint8,
+                     device=q.device)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    res = {}
+    for name, mods in (("fp8_no_mod", {}), ("fp8_causal", dict(mask_mod="causal"))):
+        t = _time_fn(lambda: fa.fwd_fp8(q8, k8, v8, scale=scale, out=o, lse_out=lse, workspace=ws, **mods), 20, 3)
+        flops = fwd_flops(B, H, S, S, D) * (0.5 if "causal" in name else 1.0)
+        res[name] = {"us": t * 1e6, "tflops": flops / t / 1e12}
+    return res
 
 
 def bwd_cases(fa, q, k, v, scale):
@@ -573,13 +592,19 @@ def profile_case(which):
     fwd = B2 H32 S4096 D128 bf16 no_mod (192 MiB of Q/K/V); fwd8192 = the full forward
     workload; fwd_blocks = the S4096 inputs with random per-head block lists, half of the
     key blocks of every query tile full; bwd = forward + backward at B2 H32 S4096 D128,
-    no_mod then causal; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
+    no_mod then causal; fp8 = the S4096 inputs rounded to e4m3, 8-bit forward; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
     import torch
     import synth
     import attention_flex_attn_b200 as fa
     fa.load_library()
     dev = torch.device("cuda", 0)
-    if which == "bwd":
+    if which == "fp8":
+        S = 4096
+        q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
+        q8, k8, v8 = (t.float().to(torch.float8_e4m3fn) for t in (q, k, v))
+        for _ in range(4):
+            fa.fwd_fp8(q8, k8, v8)
+    elif which == "bwd":
         S = 4096
         q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
         dout = synth.normal_tensor(tuple(q.shape), 4103, dtype="bf16", device=dev)
