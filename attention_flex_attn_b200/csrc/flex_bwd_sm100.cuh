@@ -117,8 +117,8 @@ struct BwdDkvSmem {
   static constexpr int kKOff = 0;                                     // K, then V
   static constexpr int kSlotOff = 2 * kTileBytes;
   static constexpr int kBarOff = kSlotOff + kSlots * kSlotBytes;
-  // barriers: kv, full[NS], empty[NS], sdp, pds[2], done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 4;
+  // barriers: kv, full[NS], empty[NS], sdp[2], pds[2], done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 5;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemPtrOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   using L = BwdDkvSmem<D>;
   constexpr int NS = L::kSlots;
   constexpr int kChunks = D / 64;
-  constexpr uint32_t kIdescT = idesc_f16(DtypeBits<T>::kFmt, kBN, kBM, 0);  // S^T, dP^T: K-major B
+  constexpr uint32_t kIdescHalf = idesc_f16(DtypeBits<T>::kFmt, kBN, kBM / 2, 0);  // S^T, dP^T halves
   constexpr uint32_t kIdescAcc = idesc_f16(DtypeBits<T>::kFmt, kBN, D, 1);  // dV, dK: N-major B
   constexpr bool kDoc = is_doc_mask(MASK);
 
@@ -403,9 +403,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t bar_kv = sbase + L::kBarOff;
   auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
   auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
-  const uint32_t bar_sdp = sbase + L::kBarOff + 8u * (1 + 2 * NS);
-  auto bar_pds = [&](int half) { return bar_sdp + 8u * (1 + half); };
-  const uint32_t bar_done = bar_sdp + 24u;
+  const uint32_t bar_sdp0 = sbase + L::kBarOff + 8u * (1 + 2 * NS);
+  auto bar_sdp = [&](int half) { return bar_sdp0 + 8u * half; };
+  auto bar_pds = [&](int half) { return bar_sdp0 + 8u * (2 + half); };
+  const uint32_t bar_done = bar_sdp0 + 32u;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
   const uint32_t k_smem = sbase + L::kKOff, v_smem = k_smem + L::kTileBytes;
@@ -441,7 +442,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), 1);
     }
-    mbar_init(bar_sdp, 1);
+    mbar_init(bar_sdp(0), 1);
+    mbar_init(bar_sdp(1), 1);
     mbar_init(bar_pds(0), kBN);
     mbar_init(bar_pds(1), kBN);
     mbar_init(bar_done, 1);
@@ -497,45 +499,64 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     const uint64_t dk0 = smem_desc(k_smem, 16, 1024, kSwizzle128B);
     const uint64_t dv0 = smem_desc(v_smem, 16, 1024, kSwizzle128B);
-    for (int u = 0; u < n && ok; ++u) {
-      const int s = u % NS;
-      if (!bwd_wait(bar_full(s), static_cast<uint32_t>(u / NS) & 1u, p, abort_flag)) break;
-      tc_fence_after();
-      const uint64_t bq = smem_desc(q_slot(s), 16, 1024, kSwizzle128B);
-      const uint64_t bo = smem_desc(o_slot(s), 16, 1024, kSwizzle128B);
+    // S^T and dP^T for the query half `half` (64 queries: rows 64 * half.. of the Q / dO
+    // tiles, 8 KB into each 16 KB chunk) of step u's slot, into their half of the buffers
+    auto issue_sdp = [&](int s, int half) {
+      const uint64_t hoff = static_cast<uint64_t>((half * 64 * 128) >> 4);
+      const uint64_t bq = smem_desc(q_slot(s), 16, 1024, kSwizzle128B) + hoff;
+      const uint64_t bo = smem_desc(o_slot(s), 16, 1024, kSwizzle128B) + hoff;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
-        mma_ss(tmem + kSCol, dk0 + off, bq + off, kIdescT, kk > 0 ? 1u : 0u);   // S^T = K Q^T
+        mma_ss(tmem + kSCol + 64u * half, dk0 + off, bq + off, kIdescHalf, kk > 0 ? 1u : 0u);   // S^T = K Q^T
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
-        mma_ss(tmem + kDpCol, dv0 + off, bo + off, kIdescT, kk > 0 ? 1u : 0u);  // dP^T = V dO^T
+        mma_ss(tmem + kDpCol + 64u * half, dv0 + off, bo + off, kIdescHalf, kk > 0 ? 1u : 0u);  // dP^T = V dO^T
       }
-      mma_commit(bar_sdp);
-      // dV += P^T dO and dK += dS^T Q, one 64-query half per element-wise warpgroup: A =
-      // 16-bit pairs in columns [0, 32) / [64, 96) of the S^T and dP^T buffers
+      mma_commit(bar_sdp(half));
+    };
+    // dV += P^T dO and dK += dS^T Q over the query half `half` (A = 16-bit pairs in
+    // columns [64 * half, 64 * half + 32) of the S^T and dP^T buffers)
+    auto issue_acc = [&](int s, int u, int half) {
       const uint64_t bon = smem_desc(o_slot(s), L::kChunkBytes, 1024, kSwizzle128B);
       const uint64_t bqn = smem_desc(q_slot(s), L::kChunkBytes, 1024, kSwizzle128B);
-      bool got_p = true;
-      for (int half = 0; half < 2; ++half) {
-        if (!bwd_wait(bar_pds(half), static_cast<uint32_t>(u) & 1u, p, abort_flag)) {
-          got_p = false;
-          break;
-        }
-        tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int kk = 4 * half + q;
-          const uint64_t off = static_cast<uint64_t>((kk * 2048) >> 4);
-          const uint32_t acol = 64u * half + 8u * q;
-          mma_ts(tmem + kDvCol, tmem + kSCol + acol, bon + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tmem + kDkCol, tmem + kDpCol + acol, bqn + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
-        }
+      for (int q = 0; q < 4; ++q) {
+        const int kk = 4 * half + q;
+        const uint64_t off = static_cast<uint64_t>((kk * 2048) >> 4);
+        const uint32_t acol = 64u * half + 8u * q;
+        mma_ts(tmem + kDvCol, tmem + kSCol + acol, bon + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
+        mma_ts(tmem + kDkCol, tmem + kDpCol + acol, bqn + off, kIdescAcc, (u > 0 || kk > 0) ? 1u : 0u);
       }
-      if (!got_p) break;
+    };
+    // Software-pipelined by query half: as soon as warpgroup A has finished half A of step
+    // u, its products run and half A of step u + 1 is formed, while warpgroup B still works
+    // on half B of step u (the halves use disjoint TMEM columns).
+    if (ok && bwd_wait(bar_full(0), 0, p, abort_flag)) {
+      tc_fence_after();
+      issue_sdp(0, 0);
+      issue_sdp(0, 1);
+    } else {
+      ok = false;
+    }
+    for (int u = 0; u < n && ok; ++u) {
+      const int s = u % NS, s1 = (u + 1) % NS;
+      const bool more = u + 1 < n;
+      if (!bwd_wait(bar_pds(0), static_cast<uint32_t>(u) & 1u, p, abort_flag)) break;
+      tc_fence_after();
+      issue_acc(s, u, 0);
+      if (more) {
+        if (!bwd_wait(bar_full(s1), static_cast<uint32_t>((u + 1) / NS) & 1u, p, abort_flag)) break;
+        tc_fence_after();
+        issue_sdp(s1, 0);
+      }
+      if (!bwd_wait(bar_pds(1), static_cast<uint32_t>(u) & 1u, p, abort_flag)) break;
+      tc_fence_after();
+      issue_acc(s, u, 1);
       mma_commit(bar_empty(s));
+      if (more) issue_sdp(s1, 1);
     }
     mma_commit(bar_done);
     mbar_wait(bar_done, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
@@ -562,7 +583,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int s = u % NS;
         // S^T / dP^T ready; the slot's statistics (written by the bulk copy) are read
         // below, so observe the slot's own barrier too
-        const bool got = bwd_wait(bar_sdp, static_cast<uint32_t>(u) & 1u, p, abort_flag) &&
+        const bool got = bwd_wait(bar_sdp(wg), static_cast<uint32_t>(u) & 1u, p, abort_flag) &&
                          bwd_wait(bar_full(s), static_cast<uint32_t>(u / NS) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
