@@ -397,8 +397,8 @@ flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const v
   p.dout = dout;
   p.lse = lse;
   p.Sq_pad = n_qtiles * kBM;
-  p.lse2 = static_cast<float*>(workspace);
-  p.delta = p.lse2 + bh * p.Sq_pad;
+  p.nlse2 = static_cast<float*>(workspace);
+  p.ndelta = p.nlse2 + bh * p.Sq_pad;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;

@@ -11,7 +11,7 @@
 // scaled score, so the mods enter through P and the masks zero P.
 //
 // Three kernels, no atomics (results do not depend on scheduling):
-//   bwd_prep_kernel   per row: delta_i and LSE_i * log2(e) into a padded workspace
+//   bwd_prep_kernel   per row: -delta_i and -LSE_i * log2(e) into a padded workspace
 //   bwd_dq_kernel     one CTA per 128-row query tile: for each key tile, S = Q K^T and
 //                     dP = dO V^T (tcgen05, TMEM), dS on the CUDA cores (one row per
 //                     thread), dQ += dS K (tcgen05, dS read from TMEM); S alternates between
@@ -45,8 +45,8 @@ struct BwdParams {
   const void* o;          // forward output [B, H, Sq, D]
   const void* dout;       // upstream gradient [B, H, Sq, D]
   const float* lse;       // forward LSE [B, H, Sq] (natural log)
-  float* lse2;            // workspace [B*H, Sq_pad]: LSE * log2(e), +inf for rows without keys
-  float* delta;           // workspace [B*H, Sq_pad]: dO . O
+  float* nlse2;           // workspace [B*H, Sq_pad]: -LSE * log2(e), -inf for rows without keys
+  float* ndelta;          // workspace [B*H, Sq_pad]: -(dO . O)
   void* dq;               // [B, H, Sq, D]
   void* dk;               // [B, Hkv, Skv, D]
   void* dv;               // [B, Hkv, Skv, D]
@@ -62,7 +62,8 @@ struct BwdParams {
 // ---------------------------------------------------------------- prep
 
 // One warp per row (b, h, i) of the padded row space: delta = dO . O in fp32, and the
-// base-2 LSE; padding rows get lse2 = +inf and delta = 0 so that they contribute nothing.
+// base-2 LSE, both stored negated so that the element-wise passes add them with packed
+// f32x2 arithmetic; padding rows get -inf and 0 so that they contribute nothing.
 template <int D, typename T>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
   const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Sq_pad;
@@ -71,20 +72,20 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
        r += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
     const int64_t bh = r / p.Sq_pad;
     const int i = static_cast<int>(r - bh * p.Sq_pad);
-    float acc = 0.f, l2 = INFINITY;
+    float acc = 0.f, nl2 = -INFINITY;
     if (i < p.Sq) {
       const int64_t base = (bh * p.Sq + i) * D;
       const T* o = reinterpret_cast<const T*>(p.o) + base;
       const T* g = reinterpret_cast<const T*>(p.dout) + base;
       for (int d = lane; d < D; d += 32) acc = fmaf(static_cast<float>(o[d]), static_cast<float>(g[d]), acc);
       const float l = p.lse[bh * p.Sq + i];
-      l2 = l == -INFINITY ? INFINITY : l * kLog2e;
+      nl2 = l == -INFINITY ? -INFINITY : -l * kLog2e;
     }
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
     if (lane == 0) {
-      p.delta[r] = i < p.Sq ? acc : 0.f;
-      p.lse2[r] = l2;
+      p.ndelta[r] = i < p.Sq ? -acc : 0.f;
+      p.nlse2[r] = nl2;
     }
   }
 }
@@ -95,12 +96,12 @@ template <int D>
 struct BwdDqSmem {
   static constexpr int kTileBytes = kBM * D * 2;
   static constexpr int kChunkBytes = kBM * 128;
-  static constexpr int kSlots = D == 128 ? 4 : 10;  // K/V ring (K_t, V_t consecutive)
+  static constexpr int kSlots = D == 128 ? 5 : 10;  // K/V ring (K_t, V_t consecutive)
   static constexpr int kQOff = 0;                   // Q, then dO
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  // barriers: q, full[NS], empty[NS], sdp, ds[2], done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 4;
+  // barriers: q, full[NS], empty[NS], sdp[2], ds[2], done
+  static constexpr int kNumBars = 1 + 2 * kSlots + 5;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemPtrOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -111,7 +112,7 @@ template <int D>
 struct BwdDkvSmem {
   static constexpr int kTileBytes = kBM * D * 2;
   static constexpr int kChunkBytes = kBM * 128;
-  static constexpr int kStatBytes = 2 * kBM * 4;                      // lse2[128], delta[128]
+  static constexpr int kStatBytes = 2 * kBM * 4;                      // -lse2[128], -delta[128]
   static constexpr int kSlotBytes = 2 * kTileBytes + kStatBytes;      // Q, dO, stats
   static constexpr int kSlots = D == 128 ? 2 : 4;
   static constexpr int kKOff = 0;                                     // K, then V
@@ -146,7 +147,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   using L = BwdDqSmem<D>;
   constexpr int NS = L::kSlots;
   constexpr int kChunks = D / 64;
-  constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);   // S, dP: K-major B
+  constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);       // S: K-major B
+  constexpr uint32_t kIdescHalf = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN / 2, 0);  // dP halves
   constexpr uint32_t kIdescDq = idesc_f16(DtypeBits<T>::kFmt, kBM, D, 1);    // dQ: B = K, N-major
   constexpr bool kDoc = is_doc_mask(MASK);
 
@@ -157,9 +159,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t bar_q = sbase + L::kBarOff;
   auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
   auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
-  const uint32_t bar_sdp = sbase + L::kBarOff + 8u * (1 + 2 * NS);
-  auto bar_ds = [&](int half) { return bar_sdp + 8u * (1 + half); };
-  const uint32_t bar_done = bar_sdp + 24u;
+  const uint32_t bar_sdp0 = sbase + L::kBarOff + 8u * (1 + 2 * NS);
+  auto bar_sdp = [&](int half) { return bar_sdp0 + 8u * half; };
+  auto bar_ds = [&](int half) { return bar_sdp0 + 8u * (2 + half); };
+  const uint32_t bar_done = bar_sdp0 + 32u;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
   const uint32_t q_smem = sbase + L::kQOff, o_smem = q_smem + L::kTileBytes;
@@ -186,7 +189,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), 1);
     }
-    mbar_init(bar_sdp, 1);
+    mbar_init(bar_sdp(0), 1);
+    mbar_init(bar_sdp(1), 1);
     mbar_init(bar_ds(0), kBM);
     mbar_init(bar_ds(1), kBM);
     mbar_init(bar_done, 1);
@@ -244,43 +248,70 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_ss(d, a0 + off, bk + off, kIdescS, kk > 0 ? 1u : 0u);
       }
     };
-    if (ok && !bwd_wait(bar_full(0), 0, p, abort_flag)) ok = false;
-    if (ok) {
+    // dP over the key half `half` (V rows 64 * half.., 8 KB into each 16 KB chunk) into its
+    // half of the dP buffer
+    auto issue_dp = [&](int slot, int half) {
+      const uint64_t bv = smem_desc(kv_smem(slot), 16, 1024, kSwizzle128B) + static_cast<uint64_t>((half * 64 * 128) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
+        mma_ss(tmem + kDpCol + 64u * half, do0 + off, bv + off, kIdescHalf, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_sdp(half));
+    };
+    // dQ += dS K over the key half `half`: A = dS, 16-bit pairs in columns
+    // [64 * half, 64 * half + 32) of tile t's S buffer
+    auto issue_dq = [&](int t, int slotK, int half) {
+      const uint64_t bkn = smem_desc(kv_smem(slotK), L::kChunkBytes, 1024, kSwizzle128B);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int kk = 4 * half + q;
+        mma_ts(tmem + kDqCol, tmem + s_col(t) + 64u * half + 8u * q, bkn + static_cast<uint64_t>((kk * 2048) >> 4),
+               kIdescDq, (t > 0 || kk > 0) ? 1u : 0u);
+      }
+    };
+    auto pos_wait = [&](int r) {  // ring position r: K_t at 2t, V_t at 2t + 1
+      if (!bwd_wait(bar_full(r % NS), static_cast<uint32_t>(r / NS) & 1u, p, abort_flag)) return false;
       tc_fence_after();
-      issue_qk(tmem + s_col(0), dq0, 0);
+      return true;
+    };
+    // Software-pipelined by key half: once warpgroup A has finished half A of tile t, dQ
+    // over that half runs and dP half A of tile t + 1 is formed while warpgroup B still
+    // works on half B of tile t; S alternates between two buffers one tile ahead.
+    if (ok && pos_wait(0)) issue_qk(tmem + s_col(0), dq0, 0);
+    else ok = false;
+    if (ok && pos_wait(1)) {
+      issue_dp(1 % NS, 0);
+      issue_dp(1 % NS, 1);
+      mma_commit(bar_empty(1 % NS));
+    } else {
+      ok = false;
+    }
+    if (ok && n > 1) {
+      if (pos_wait(2)) issue_qk(tmem + s_col(1), dq0, 2 % NS);
+      else ok = false;
     }
     for (int t = 0; t < n && ok; ++t) {
-      const int rK = 2 * t, rV = rK + 1;
-      if (!bwd_wait(bar_full(rV % NS), static_cast<uint32_t>(rV / NS) & 1u, p, abort_flag)) break;
+      const int sK = (2 * t) % NS, rV1 = 2 * t + 3, rK2 = 2 * t + 4;
+      if (!bwd_wait(bar_ds(0), static_cast<uint32_t>(t) & 1u, p, abort_flag)) break;
       tc_fence_after();
-      issue_qk(tmem + kDpCol, do0, rV % NS);  // dP = dO V^T
-      mma_commit(bar_sdp);
-      mma_commit(bar_empty(rV % NS));
+      issue_dq(t, sK, 0);
       if (t + 1 < n) {
-        const int rK2 = rK + 2;
-        if (!bwd_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p, abort_flag)) break;
-        tc_fence_after();
-        issue_qk(tmem + s_col(t + 1), dq0, rK2 % NS);  // S of the next key tile
+        if (!pos_wait(rV1)) break;
+        issue_dp(rV1 % NS, 0);  // dP half A of tile t + 1 (S of t + 1 is already issued)
       }
-      // dQ += dS K, one 64-key half per element-wise warpgroup: A = dS, 16-bit pairs in
-      // columns [0, 32) (keys 0-63) and [64, 96) (keys 64-127) of its S buffer
-      const uint64_t bkn = smem_desc(kv_smem(rK % NS), L::kChunkBytes, 1024, kSwizzle128B);
-      bool got_ds = true;
-      for (int half = 0; half < 2 && got_ds; ++half) {
-        if (!bwd_wait(bar_ds(half), static_cast<uint32_t>(t) & 1u, p, abort_flag)) {
-          got_ds = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int kk = 4 * half + q;
-          mma_ts(tmem + kDqCol, tmem + s_col(t) + 64u * half + 8u * q, bkn + static_cast<uint64_t>((kk * 2048) >> 4),
-                 kIdescDq, (t > 0 || kk > 0) ? 1u : 0u);
-        }
+      if (!bwd_wait(bar_ds(1), static_cast<uint32_t>(t) & 1u, p, abort_flag)) break;
+      tc_fence_after();
+      issue_dq(t, sK, 1);
+      mma_commit(bar_empty(sK));
+      if (t + 1 < n) {
+        issue_dp(rV1 % NS, 1);
+        mma_commit(bar_empty(rV1 % NS));
       }
-      if (!got_ds) break;
-      mma_commit(bar_empty(rK % NS));
+      if (t + 2 < n) {
+        if (!pos_wait(rK2)) break;
+        issue_qk(tmem + s_col(t + 2), dq0, rK2 % NS);  // into tile t's buffer, whose dS is consumed
+      }
     }
     mma_commit(bar_done);
     mbar_wait(bar_done, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
@@ -294,8 +325,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool row_valid = i < p.Sq;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const int64_t srow = static_cast<int64_t>(bh) * p.Sq_pad + (row_valid ? i : 0);
-    const float lse2 = row_valid ? p.lse2[srow] : INFINITY;
-    const float delta = row_valid ? p.delta[srow] : 0.f;
+    const float nlse2 = row_valid ? p.nlse2[srow] : -INFINITY;
+    const uint64_t nd2 = pack2(row_valid ? p.ndelta[srow] : 0.f, row_valid ? p.ndelta[srow] : 0.f);
+    const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2);
     float slope2 = 0.f;
     if (SCORE == kScoreAlibi)
       slope2 = (p.slopes ? __ldg(p.slopes + h) : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
@@ -306,7 +338,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     row_interval<MASK>(q0, mk, t0, hi_first);
     bool ok = true;
     for (int t = 0; t < n; ++t) {
-      const bool got = bwd_wait(bar_sdp, static_cast<uint32_t>(t) & 1u, p, abort_flag);
+      const bool got = bwd_wait(bar_sdp(wg), static_cast<uint32_t>(t) & 1u, p, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -323,7 +355,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       const uint32_t tS = tmem + lane_off + s_col(t) + cb, tP = tmem + lane_off + kDpCol + cb;
-      const float base = slope2 * static_cast<float>(k0 + static_cast<int>(cb) - i) - lse2;
+      const float base = slope2 * static_cast<float>(k0 + static_cast<int>(cb) - i) + nlse2;
+      const uint64_t nl2 = pack2(nlse2, nlse2);
 #pragma unroll
       for (int part = 0; part < 2; ++part) {  // 32 columns at a time
         uint32_t sr[32], pr[32], w[16];
@@ -331,19 +364,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tP + 32u * part, pr);
         float* x = reinterpret_cast<float*>(sr);
         const int c0 = static_cast<int>(cb) + 32 * part;  // column of x[0] within the tile
+        // x = s * scale * log2(e) + bias - LSE * log2(e), two columns per instruction
 #pragma unroll
-        for (int c = 0; c < 32; ++c)
-          x[c] = fmaf(x[c], p.scale_log2, fmaf(slope2, static_cast<float>(32 * part + c), base));
+        for (int e = 0; e < 16; ++e) {
+          const int c = 2 * e;
+          const uint64_t b2 = SCORE == kScoreAlibi
+                                  ? pack2(fmaf(slope2, static_cast<float>(32 * part + c), base),
+                                          fmaf(slope2, static_cast<float>(32 * part + c + 1), base))
+                                  : nl2;
+          unpack2(fma2(pack2(x[c], x[c + 1]), sc2, b2), x[c], x[c + 1]);
+        }
         if (!full) {  // warp-uniform: the mask pass runs on PARTIAL tiles only
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             if (c0 + c < c_lo || c0 + c > c_hi) x[c] = -INFINITY;
         }
-        // branch-free: ex2(-inf) = 0 gives dS = 0 for dropped keys
+        // branch-free: ex2(-inf) = 0 gives dS = 0 for dropped keys; dS = P (dP - delta)
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = DtypeBits<T>::pack(ex2_approx(x[2 * e]) * (__uint_as_float(pr[2 * e]) - delta),
-                                    ex2_approx(x[2 * e + 1]) * (__uint_as_float(pr[2 * e + 1]) - delta));
+        for (int e = 0; e < 16; ++e) {
+          const uint64_t p2 = pack2(ex2_approx(x[2 * e]), ex2_approx(x[2 * e + 1]));
+          float d0, d1;
+          unpack2(mul2(p2, add2(pack2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])), nd2)), d0, d1);
+          w[e] = DtypeBits<T>::pack(d0, d1);
+        }
         tmem_st16(tS + 16u * part, w);  // columns cb + [0, 32): read by this warpgroup already
       }
       tmem_st_wait();
@@ -485,8 +528,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_3d(o_slot(s) + c * L::kChunkBytes, &tmO, bar_full(s), c * 64, t * kBM, bh);
         }
         const int64_t srow = static_cast<int64_t>(bh) * p.Sq_pad + t * kBM;
-        bulk_load(sbase + stat_slot(s), p.lse2 + srow, kBM * 4, bar_full(s));
-        bulk_load(sbase + stat_slot(s) + kBM * 4, p.delta + srow, kBM * 4, bar_full(s));
+        bulk_load(sbase + stat_slot(s), p.nlse2 + srow, kBM * 4, bar_full(s));
+        bulk_load(sbase + stat_slot(s) + kBM * 4, p.ndelta + srow, kBM * 4, bar_full(s));
         ++u;
       }
     }
@@ -570,6 +613,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     int64_t key_lo, key_hi;
     key_interval<MASK>(j, mk, p.Sq, key_lo, key_hi);
+    const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2);
     bool ok = true;
     int u = 0;
     for (int hg = 0; hg < p.G && ok; ++hg) {
@@ -603,34 +647,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32(tmem + lane_off + kSCol + c0, sr);
           tmem_ld32(tmem + lane_off + kDpCol + c0, pr);
           float* x = reinterpret_cast<float*>(sr);
-          const float4* st4 = reinterpret_cast<const float4*>(stat + c0);
+          const uint64_t* nl = reinterpret_cast<const uint64_t*>(stat + c0);  // -lse2 pairs
+          // x = s * scale * log2(e) + bias - LSE * log2(e), two columns per instruction
 #pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 l4 = st4[c4];
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int c = 4 * c4 + v;
-              x[c] = fmaf(x[c], p.scale_log2, fmaf(-slope2, static_cast<float>(32 * part + c), base)) - lv[v];
-            }
+          for (int e = 0; e < 16; ++e) {
+            const int c = 2 * e;
+            uint64_t b2 = nl[e];
+            if (SCORE == kScoreAlibi)
+              b2 = add2(b2, pack2(fmaf(-slope2, static_cast<float>(32 * part + c), base),
+                                  fmaf(-slope2, static_cast<float>(32 * part + c + 1), base)));
+            unpack2(fma2(pack2(x[c], x[c + 1]), sc2, b2), x[c], x[c + 1]);
           }
           if (!full) {  // warp-uniform: the mask pass runs on PARTIAL tiles only
 #pragma unroll
             for (int c = 0; c < 32; ++c)
               if (c0 + c < c_lo || c0 + c > c_hi) x[c] = -INFINITY;
           }
-          const float4* dl4 = reinterpret_cast<const float4*>(stat + kBM + c0);
+          const uint64_t* nd = reinterpret_cast<const uint64_t*>(stat + kBM + c0);  // -delta pairs
+          // dS = P (dP - delta), two columns per instruction
 #pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 d4 = dl4[c4];
-            const float p0 = ex2_approx(x[4 * c4]), p1 = ex2_approx(x[4 * c4 + 1]);
-            const float p2 = ex2_approx(x[4 * c4 + 2]), p3 = ex2_approx(x[4 * c4 + 3]);
-            wp[2 * c4] = DtypeBits<T>::pack(p0, p1);
-            wp[2 * c4 + 1] = DtypeBits<T>::pack(p2, p3);
-            wd[2 * c4] = DtypeBits<T>::pack(p0 * (__uint_as_float(pr[4 * c4]) - d4.x),
-                                            p1 * (__uint_as_float(pr[4 * c4 + 1]) - d4.y));
-            wd[2 * c4 + 1] = DtypeBits<T>::pack(p2 * (__uint_as_float(pr[4 * c4 + 2]) - d4.z),
-                                                p3 * (__uint_as_float(pr[4 * c4 + 3]) - d4.w));
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(x[2 * e]), p1 = ex2_approx(x[2 * e + 1]);
+            wp[e] = DtypeBits<T>::pack(p0, p1);
+            float d0, d1;
+            unpack2(mul2(pack2(p0, p1), add2(pack2(__uint_as_float(pr[2 * e]), __uint_as_float(pr[2 * e + 1])), nd[e])),
+                    d0, d1);
+            wd[e] = DtypeBits<T>::pack(d0, d1);
           }
           // columns cb + [0, 32) of each buffer, already read by this warpgroup
           tmem_st16(tmem + lane_off + kSCol + cb + 16u * part, wp);

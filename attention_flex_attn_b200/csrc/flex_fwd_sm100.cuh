@@ -625,10 +625,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint32_t sr[kBN];
       tmem_ld128(tS, sr);
       float* s = reinterpret_cast<float*>(sr);
+      // Alibi: the bias slope2 * c of column c comes from four packed chains (columns
+      // 8i + 2r, 8i + 2r + 1), each stepped by 8 * slope2; the part common to the tile,
+      // slope2 * (k0 - qi), joins the running max instead of every element.  The _rn
+      // operations are never fused, so every instantiation rounds them alike.
+      const float base = SCORE == kScoreAlibi ? __fmul_rn(slope2, static_cast<float>(k0 - qi)) : 0.f;
       if (SCORE == kScoreAlibi) {
-        const float base = slope2 * static_cast<float>(k0 - qi);
+        const uint64_t scl2 = pack2(p.scale_log2, p.scale_log2);
+        const uint64_t astep = pack2(__fmul_rn(8.f, slope2), __fmul_rn(8.f, slope2));
+        uint64_t b0 = pack2(0.f, slope2), b1 = pack2(__fmul_rn(2.f, slope2), __fmul_rn(3.f, slope2));
+        uint64_t b2 = pack2(__fmul_rn(4.f, slope2), __fmul_rn(5.f, slope2));
+        uint64_t b3 = pack2(__fmul_rn(6.f, slope2), __fmul_rn(7.f, slope2));
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) s[c] = fmaf(s[c], p.scale_log2, fmaf(slope2, static_cast<float>(c), base));
+        for (int c = 0; c < kBN; c += 8) {
+          unpack2(fma2(pack2(s[c], s[c + 1]), scl2, b0), s[c], s[c + 1]);
+          unpack2(fma2(pack2(s[c + 2], s[c + 3]), scl2, b1), s[c + 2], s[c + 3]);
+          unpack2(fma2(pack2(s[c + 4], s[c + 5]), scl2, b2), s[c + 4], s[c + 5]);
+          unpack2(fma2(pack2(s[c + 6], s[c + 7]), scl2, b3), s[c + 6], s[c + 7]);
+          b0 = add2(b0, astep);
+          b1 = add2(b1, astep);
+          b2 = add2(b2, astep);
+          b3 = add2(b3, astep);
+        }
       }
       if (cls != kTileFull) {
         int c_lo, c_hi;
@@ -652,7 +670,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       mx0 = max3f(mx0, s[kBN - 4], s[kBN - 3]);
       mx1 = max3f(mx1, s[kBN - 2], s[kBN - 1]);
-      const float mx = max3f(mx0, mx1, fmaxf(mx2, mx3)) * sc;
+      const float mx = __fadd_rn(max3f(mx0, mx1, fmaxf(mx2, mx3)) * sc, base);
       const bool need = mx > m_used + kRescaleThreshold;  // false while both are -inf
       if (__any_sync(0xffffffffu, need)) {
         float alpha = 1.0f;
@@ -679,7 +697,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       const float m_safe = m_used == -INFINITY ? 0.f : m_used;
       const uint64_t sc2 = pack2(sc, sc);
-      const uint64_t nm2 = pack2(-m_safe, -m_safe);
+      const float nm = __fsub_rn(base, m_safe);
+      const uint64_t nm2 = pack2(nm, nm);
       uint64_t acc2 = 0;  // two running partial sums (0.0f, 0.0f)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
