@@ -96,12 +96,15 @@ template <int D>
 struct BwdDqSmem {
   static constexpr int kTileBytes = kBM * D * 2;
   static constexpr int kChunkBytes = kBM * 128;
-  static constexpr int kSlots = D == 128 ? 5 : 10;  // K/V ring (K_t, V_t consecutive)
+  // Separate K and V rings: K_t is read from S(t) (two tiles ahead) to dQ(t), V_t only by
+  // dP(t), so each ring frees its slots in order and every load has an iteration of lead.
+  static constexpr int kKSlots = D == 128 ? 3 : 6;
+  static constexpr int kVSlots = D == 128 ? 2 : 4;
   static constexpr int kQOff = 0;                   // Q, then dO
-  static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  // barriers: q, full[NS], empty[NS], sdp[2], ds[2], done
-  static constexpr int kNumBars = 1 + 2 * kSlots + 5;
+  static constexpr int kKVOff = 2 * kTileBytes;     // K slots, then V slots
+  static constexpr int kBarOff = kKVOff + (kKSlots + kVSlots) * kTileBytes;
+  // barriers: q, full_k[KS], empty_k[KS], full_v[VS], empty_v[VS], sdp[2], ds[2], done
+  static constexpr int kNumBars = 1 + 2 * (kKSlots + kVSlots) + 5;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemPtrOff + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -127,8 +130,12 @@ struct BwdDkvSmem {
   static_assert(kSlotBytes % 1024 == 0, "slots must keep the 1024-byte swizzle alignment");
 };
 
-// Bounded wait that also gives up when another role of the CTA has given up.
+// Bounded wait that also gives up when another role of the CTA has given up.  The fast
+// path is a single probe of the barrier: on the MMA-issuing thread every shared-memory
+// access between two matmuls idles the tensor pipe for about 100 cycles, so the abort flag
+// is read only when the phase is not complete yet.
 __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const BwdParams& p, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
   if (*abort_flag) return false;
   if (!mbar_wait(bar, parity, p.status, kStatusBwdTimeout, kWaitTimeoutNs)) {
     *abort_flag = 1;
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const BwdParams p) {
   using L = BwdDqSmem<D>;
-  constexpr int NS = L::kSlots;
+  constexpr int KS = L::kKSlots, VS = L::kVSlots;
   constexpr int kChunks = D / 64;
   constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);       // S: K-major B
   constexpr uint32_t kIdescHalf = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN / 2, 0);  // dP halves
@@ -157,16 +164,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sbase - raw_addr);
   const uint32_t bar_q = sbase + L::kBarOff;
-  auto bar_full = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
-  auto bar_empty = [&](int s) { return sbase + L::kBarOff + 8u * (1 + NS + s); };
-  const uint32_t bar_sdp0 = sbase + L::kBarOff + 8u * (1 + 2 * NS);
+  auto full_k = [&](int s) { return sbase + L::kBarOff + 8u * (1 + s); };
+  auto empty_k = [&](int s) { return sbase + L::kBarOff + 8u * (1 + KS + s); };
+  auto full_v = [&](int s) { return sbase + L::kBarOff + 8u * (1 + 2 * KS + s); };
+  auto empty_v = [&](int s) { return sbase + L::kBarOff + 8u * (1 + 2 * KS + VS + s); };
+  const uint32_t bar_sdp0 = sbase + L::kBarOff + 8u * (1 + 2 * KS + 2 * VS);
   auto bar_sdp = [&](int half) { return bar_sdp0 + 8u * half; };
   auto bar_ds = [&](int half) { return bar_sdp0 + 8u * (2 + half); };
   const uint32_t bar_done = bar_sdp0 + 32u;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
   const uint32_t q_smem = sbase + L::kQOff, o_smem = q_smem + L::kTileBytes;
-  auto kv_smem = [&](int s) { return sbase + static_cast<uint32_t>(L::kKVOff + s * L::kTileBytes); };
+  auto k_smem = [&](int s) { return sbase + static_cast<uint32_t>(L::kKVOff + s * L::kTileBytes); };
+  auto v_smem = [&](int s) { return sbase + static_cast<uint32_t>(L::kKVOff + (KS + s) * L::kTileBytes); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x % p.n_qtiles;
@@ -185,9 +195,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(full_k(s), 1);
+      mbar_init(empty_k(s), 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(full_v(s), 1);
+      mbar_init(empty_v(s), 1);
     }
     mbar_init(bar_sdp(0), 1);
     mbar_init(bar_sdp(1), 1);
@@ -216,22 +230,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_load_3d(q_smem + c * L::kChunkBytes, &tmQ, bar_q, c * 64, q0, bh);
       tma_load_3d(o_smem + c * L::kChunkBytes, &tmO, bar_q, c * 64, q0, bh);
     }
-    int r = 0;
-    bool ok = true;
-    for (int t = 0; t < n && ok; ++t) {
-      for (int which = 0; which < 2 && ok; ++which, ++r) {
-        const int s = r % NS;
-        if (!bwd_wait(bar_empty(s), (static_cast<uint32_t>(r / NS) & 1u) ^ 1u, p, abort_flag)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(kv_smem(s) + c * L::kChunkBytes, which ? &tmV : &tmK, bar_full(s), c * 64, (lo + t) * kBN, bkv);
-      }
-    }
-    for (int e = r - NS < 0 ? 0 : r - NS; e < r; ++e)
-      mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+    // Loads in the order the products need them: K_0, V_0, K_1, then V_{t+1}, K_{t+2}.
+    int nk = 0, nv = 0;
+    auto load = [&](bool is_v, int tile) -> bool {
+      const int i = is_v ? nv : nk;
+      const int slot = i % (is_v ? VS : KS);
+      const uint32_t full = is_v ? full_v(slot) : full_k(slot);
+      const uint32_t empty = is_v ? empty_v(slot) : empty_k(slot);
+      if (!bwd_wait(empty, (static_cast<uint32_t>(i / (is_v ? VS : KS)) & 1u) ^ 1u, p, abort_flag)) return false;
+      mbar_arrive_expect_tx(full, L::kTileBytes);
+      const uint32_t dst = is_v ? v_smem(slot) : k_smem(slot);
+      for (int c = 0; c < kChunks; ++c)
+        tma_load_3d(dst + c * L::kChunkBytes, is_v ? &tmV : &tmK, full, c * 64, (lo + tile) * kBN, bkv);
+      if (is_v) ++nv;
+      else ++nk;
+      return true;
+    };
+    bool ok = load(false, 0) && load(true, 0) && (n < 2 || load(false, 1));
+    for (int t = 0; t + 1 < n && ok; ++t) ok = load(true, t + 1) && (t + 2 >= n || load(false, t + 2));
+    // wait for the copies still in flight before the CTA may exit
+    for (int e = nk - KS < 0 ? 0 : nk - KS; e < nk; ++e)
+      mbar_wait(full_k(e % KS), static_cast<uint32_t>(e / KS) & 1u, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
+    for (int e = nv - VS < 0 ? 0 : nv - VS; e < nv; ++e)
+      mbar_wait(full_v(e % VS), static_cast<uint32_t>(e / VS) & 1u, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
     mbar_wait(bar_q, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
   } else if (warp == 0 && lane == 0 && n > 0) {
     // ============================================================ MMA issuer
@@ -241,7 +262,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t do0 = smem_desc(o_smem, 16, 1024, kSwizzle128B);
     // S-type product: d = A (K-major, rows = queries) * B^T (K-major, rows = keys), K = D
     auto issue_qk = [&](uint32_t d, uint64_t a0, int slot) {
-      const uint64_t bk = smem_desc(kv_smem(slot), 16, 1024, kSwizzle128B);
+      const uint64_t bk = smem_desc(k_smem(slot), 16, 1024, kSwizzle128B);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
@@ -251,7 +272,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // dP over the key half `half` (V rows 64 * half.., 8 KB into each 16 KB chunk) into its
     // half of the dP buffer
     auto issue_dp = [&](int slot, int half) {
-      const uint64_t bv = smem_desc(kv_smem(slot), 16, 1024, kSwizzle128B) + static_cast<uint64_t>((half * 64 * 128) >> 4);
+      const uint64_t bv = smem_desc(v_smem(slot), 16, 1024, kSwizzle128B) + static_cast<uint64_t>((half * 64 * 128) >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
@@ -262,7 +283,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // dQ += dS K over the key half `half`: A = dS, 16-bit pairs in columns
     // [64 * half, 64 * half + 32) of tile t's S buffer
     auto issue_dq = [&](int t, int slotK, int half) {
-      const uint64_t bkn = smem_desc(kv_smem(slotK), L::kChunkBytes, 1024, kSwizzle128B);
+      const uint64_t bkn = smem_desc(k_smem(slotK), L::kChunkBytes, 1024, kSwizzle128B);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int kk = 4 * half + q;
@@ -270,47 +291,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                kIdescDq, (t > 0 || kk > 0) ? 1u : 0u);
       }
     };
-    auto pos_wait = [&](int r) {  // ring position r: K_t at 2t, V_t at 2t + 1
-      if (!bwd_wait(bar_full(r % NS), static_cast<uint32_t>(r / NS) & 1u, p, abort_flag)) return false;
+    auto k_wait = [&](int tile) {  // K_tile is in slot tile % KS
+      if (!bwd_wait(full_k(tile % KS), static_cast<uint32_t>(tile / KS) & 1u, p, abort_flag)) return false;
+      tc_fence_after();
+      return true;
+    };
+    auto v_wait = [&](int tile) {
+      if (!bwd_wait(full_v(tile % VS), static_cast<uint32_t>(tile / VS) & 1u, p, abort_flag)) return false;
       tc_fence_after();
       return true;
     };
     // Software-pipelined by key half: once warpgroup A has finished half A of tile t, dQ
     // over that half runs and dP half A of tile t + 1 is formed while warpgroup B still
     // works on half B of tile t; S alternates between two buffers one tile ahead.
-    if (ok && pos_wait(0)) issue_qk(tmem + s_col(0), dq0, 0);
+    if (ok && k_wait(0)) issue_qk(tmem + s_col(0), dq0, 0);
     else ok = false;
-    if (ok && pos_wait(1)) {
-      issue_dp(1 % NS, 0);
-      issue_dp(1 % NS, 1);
-      mma_commit(bar_empty(1 % NS));
+    if (ok && v_wait(0)) {
+      issue_dp(0, 0);
+      issue_dp(0, 1);
+      mma_commit(empty_v(0));
     } else {
       ok = false;
     }
     if (ok && n > 1) {
-      if (pos_wait(2)) issue_qk(tmem + s_col(1), dq0, 2 % NS);
+      if (k_wait(1)) issue_qk(tmem + s_col(1), dq0, 1 % KS);
       else ok = false;
     }
     for (int t = 0; t < n && ok; ++t) {
-      const int sK = (2 * t) % NS, rV1 = 2 * t + 3, rK2 = 2 * t + 4;
+      const int sK = t % KS, sV1 = (t + 1) % VS;
       if (!bwd_wait(bar_ds(0), static_cast<uint32_t>(t) & 1u, p, abort_flag)) break;
       tc_fence_after();
       issue_dq(t, sK, 0);
       if (t + 1 < n) {
-        if (!pos_wait(rV1)) break;
-        issue_dp(rV1 % NS, 0);  // dP half A of tile t + 1 (S of t + 1 is already issued)
+        if (!v_wait(t + 1)) break;
+        issue_dp(sV1, 0);  // dP half A of tile t + 1 (S of t + 1 is already issued)
       }
       if (!bwd_wait(bar_ds(1), static_cast<uint32_t>(t) & 1u, p, abort_flag)) break;
       tc_fence_after();
       issue_dq(t, sK, 1);
-      mma_commit(bar_empty(sK));
+      mma_commit(empty_k(sK));
       if (t + 1 < n) {
-        issue_dp(rV1 % NS, 1);
-        mma_commit(bar_empty(rV1 % NS));
+        issue_dp(sV1, 1);
+        mma_commit(empty_v(sV1));
       }
       if (t + 2 < n) {
-        if (!pos_wait(rK2)) break;
-        issue_qk(tmem + s_col(t + 2), dq0, rK2 % NS);  // into tile t's buffer, whose dS is consumed
+        if (!k_wait(t + 2)) break;
+        issue_qk(tmem + s_col(t + 2), dq0, (t + 2) % KS);  // into tile t's buffer, whose dS is consumed
       }
     }
     mma_commit(bar_done);
