@@ -38,9 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram read+write bytes per launch from ncu, keyed by the hash of the kernel sources
 # they were measured on (a changed kernel reports null until it is captured again)
 MEASURED_TRAFFIC = {
-    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 403,024,640 B read +
-    # 115,118,080 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
-    "0c78b41d8c4eb42c": 518142720,
+    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 402,840,064 B read +
+    # 115,957,248 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
+    "ec937b6aa1d4e760": 518797312,
 }
 # the forward kernel's sources: the roofline traffic below belongs to that kernel
 KERNEL_SOURCES = ["attention_flex_attn_b200/csrc/flex_fwd_sm100.cuh",

@@ -121,3 +121,11 @@ def test_mha_2048_sampled_groups(mods):
 
 def test_gqa_4096_sampled_group():
     _case(1, 8, 2, 4096, 4096, 128, "bf16", 86, 1.0 / math.sqrt(128), groups=[(0, 1)], mask_mod="causal")
+
+
+@pytest.mark.parametrize("dtype,mods", [("bf16", dict(mask_mod="none")), ("f16", dict(mask_mod="causal")),
+                                        ("bf16", dict(mask_mod="sliding_window", window=300))])
+def test_d64_ring_wrap_sampled_group(dtype, mods):
+    """D=64 at Sq = Skv = 1500: 12 key tiles (ragged), so both of the dQ kernel's key and
+    value rings and the dK/dV kernel's query ring wrap several times."""
+    _case(1, 4, 2, 1500, 1500, 64, dtype, 87, 0.125, groups=[(0, 1)], **mods)
