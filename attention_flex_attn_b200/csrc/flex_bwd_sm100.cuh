@@ -15,7 +15,8 @@
 //   bwd_dq_kernel     one CTA per 128-row query tile: for each key tile, S = Q K^T and
 //                     dP = dO V^T (tcgen05, TMEM), dS on the CUDA cores (one row per
 //                     thread), dQ += dS K (tcgen05, dS read from TMEM); S alternates between
-//                     two TMEM buffers so S of the next key tile overlaps the dS work
+//                     two TMEM buffers so S of the next key tile overlaps the dS work, and
+//                     K and V stream through rings of their own, each freed in order
 //   bwd_dkdv_kernel   one CTA per 128-key tile and kv head: for each query tile of each
 //                     query head of the group, S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
 //                     per key row, dV += P^T dO and dK += dS^T Q (TMEM accumulators)
