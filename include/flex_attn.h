@@ -200,7 +200,8 @@ flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, 
 
 /*
  * flex_attn_bwd_workspace_size -- bytes of device workspace flex_attn_bwd needs
- * (per query row: LSE in base 2 and delta = dO . O, rows padded to a multiple of 128).
+ * (per query row: -LSE in base 2 and -delta with delta = dO . O, rows padded to a multiple
+ * of 128).  The contents are private to one call.
  */
 size_t flex_attn_bwd_workspace_size(int B, int H, int Sq);
 
