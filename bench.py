@@ -203,7 +203,7 @@ def run_reference(args, rank, world):
     t0 = time.perf_counter()
     oracle.fwd(q, k, v, scale=1 / math.sqrt(D), rows=probe, threads=threads)
     per_row = (time.perf_counter() - t0) / probe.size
-    budget = 120.0 / (args.steps + args.warmup)
+    budget = args.ref_seconds / (args.steps + args.warmup)
     n = int(max(threads, min(B * H * S, budget / max(per_row, 1e-6))))
     times = []
     for i in range(args.warmup + args.steps):
@@ -234,6 +234,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="reference arm: host seconds of oracle work over all warm-up and timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-case and e2e measurements")
     ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "bwd", "fp8", "decode"], default=None,
