@@ -191,3 +191,30 @@ def test_fp8_rejects_bad_args_on_host(lib):
     assert f8(q=8) == 3
     assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 128) == 2 * 4 * 128 * 384
     assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 64) == 0
+
+
+def _declared_arity():
+    """Parameter count of every function the header declares (void-parameter lists count 0)."""
+    txt = open(os.path.join(ROOT, "include", "flex_attn.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    txt = re.sub(r"//[^\n]*", "", txt)
+    out = {}
+    for m in re.finditer(r"\b(flex_\w+)\s*\(([^;{]*?)\)\s*;", txt):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_header(lib):
+    """Every argtypes list the binding sets has exactly as many entries as the header's
+    declaration has parameters, so a changed signature cannot be called with a stale one."""
+    arity = _declared_arity()
+    assert set(arity) == set(fa.EXPORTED)
+    checked = 0
+    for name, n in arity.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+        checked += 1
+    assert checked >= len(arity) // 2
