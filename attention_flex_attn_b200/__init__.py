@@ -42,7 +42,13 @@ class ModParams(ctypes.Structure):
     _fields_ = [("window", ctypes.c_int32), ("offset", ctypes.c_int32),
                 ("flags", ctypes.c_uint32), ("tile_map_out", ctypes.c_void_p),
                 ("alibi_slopes", ctypes.c_void_p), ("doc_offsets_q", ctypes.c_void_p),
-                ("doc_offsets_kv", ctypes.c_void_p), ("n_docs", ctypes.c_int32)]
+                ("doc_offsets_kv", ctypes.c_void_p), ("n_docs", ctypes.c_int32),
+                ("status_out", ctypes.c_void_p)]
+
+
+class DecodeParamsC(ctypes.Structure):
+    """flex_decode_params_t of include/flex_attn.h."""
+    _fields_ = [("split_size", ctypes.c_int32), ("status_out", ctypes.c_void_p)]
 
 
 class BlockMaskC(ctypes.Structure):
@@ -82,9 +88,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_bwd.restype = I
     lib.flex_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.flex_attn_decode_workspace_size.restype = SZ
-    lib.flex_attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ, P]
+    lib.flex_attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ,
+                                     ctypes.POINTER(DecodeParamsC), P]
     lib.flex_attn_decode.restype = I
-    lib.flex_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P]
+    lib.flex_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I,
+                                             ctypes.POINTER(DecodeParamsC), P]
     lib.flex_attn_decode_noalloc.restype = I
     lib.flex_attn_mask_eval.argtypes = [I, ctypes.POINTER(ModParams), I, I, P, P]
     lib.flex_attn_mask_eval.restype = I
@@ -127,15 +135,44 @@ def tile_sizes(D: int = 128):
     return bm.value, bn.value
 
 
-def _fwd_args(q, k, v, scale, return_lse, out, lse_out):
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _cuda_tensor(t, n)
+def _expect(t, name, shape, dtype, device):
+    """Checks a tensor argument's shape, dtype and device (a wrong size would make the
+    kernels read or write past the allocation)."""
+    if not isinstance(t, torch.Tensor):
+        raise FlexAttnError(f"{name} must be a tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise FlexAttnError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise FlexAttnError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise FlexAttnError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise FlexAttnError(f"{name} must be contiguous")
+
+
+def _check_fwd_shapes(q, k, v, out=None, lse_out=None):
+    """Shapes and dtypes of a forward's tensors (no device work)."""
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise FlexAttnError("q, k, v must be 4-D [B, H, S, D]")
     B, H, Sq, D = q.shape
     Bk, Hkv, Skv, Dk = k.shape
     if Bk != B or Dk != D or tuple(v.shape) != tuple(k.shape) or not (q.dtype == k.dtype == v.dtype):
         raise FlexAttnError("shape/dtype mismatch between q, k, v")
+    if q.device != k.device or q.device != v.device:
+        raise FlexAttnError("q, k, v must be on one device")
     if q.dtype not in DTYPES:
         raise FlexAttnError(f"unsupported dtype {q.dtype}")
+    if out is not None:
+        _expect(out, "out", q.shape, q.dtype, q.device)
+    if lse_out is not None:
+        _expect(lse_out, "lse_out", (B, H, Sq), torch.float32, q.device)
+    return B, H, Hkv, Sq, Skv, D
+
+
+def _fwd_args(q, k, v, scale, return_lse, out, lse_out):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda_tensor(t, n)
+    B, H, Hkv, Sq, Skv, D = _check_fwd_shapes(q, k, v, out, lse_out if return_lse else None)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     o = out if out is not None else torch.empty_like(q)
@@ -145,8 +182,19 @@ def _fwd_args(q, k, v, scale, return_lse, out, lse_out):
     return B, H, Hkv, Sq, Skv, D, float(scale), o, lse
 
 
+def _status_word(status, device):
+    """Pointer of a caller's per-call status word: an int32 (or uint32) CUDA tensor of one
+    element on the call's device, or None for the shared per-device word."""
+    if status is None:
+        return None
+    _cuda_tensor(status, "status")
+    if status.numel() != 1 or status.dtype not in (torch.int32, torch.uint32) or status.device != device:
+        raise FlexAttnError("status must be a one-element int32 tensor on the call's device")
+    return status.data_ptr()
+
+
 def _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
-                doc_offsets_kv):
+                doc_offsets_kv, status_ptr=None):
     """ModParams and the score_mod id; the captured tensors are checked, not copied."""
     score = SCORE_MODS[score_mod]
     slopes_ptr = None
@@ -174,25 +222,26 @@ def _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slope
         okv = None if doc_offsets_kv is None else doc_offsets_kv.data_ptr()
         n_docs = doc_offsets.shape[1] - 1
     mp = ModParams(int(window), int(offset), FLAG_TILE_MAP if tile_map is not None else 0,
-                   tile_map.data_ptr() if tile_map is not None else None, slopes_ptr, oq, okv, n_docs)
+                   tile_map.data_ptr() if tile_map is not None else None, slopes_ptr, oq, okv, n_docs, status_ptr)
     return mp, score
 
 
 def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
         return_lse=True, out=None, lse_out=None, tile_map=None, alibi_slopes=None, doc_offsets=None,
-        doc_offsets_kv=None):
+        doc_offsets_kv=None, status=None):
     """Flex-attention forward.  q [B,H,Sq,D], k/v [B,Hkv,Skv,D] (bf16 or f16, CUDA).
 
     Returns (O, LSE) (LSE is None when return_lse is False).  ``tile_map``: optional
     uint8 CUDA tensor of ceil(Sq/BM)*ceil(Skv/BN) bytes that receives the tile classes
     of batch 0 / head 0.  Captured tensors: ``alibi_slopes`` (float32 [H], with
     score_mod="alibi"); ``doc_offsets`` / ``doc_offsets_kv`` (int32 [B, n_docs + 1]
-    document boundaries, with mask_mod "document" or "document_causal").
+    document boundaries, with mask_mod "document" or "document_causal").  ``status``:
+    optional one-element int32 CUDA tensor that receives this call's device status bits.
     """
     lib = load_library()
     B, H, Hkv, Sq, Skv, D, scale, o, lse = _fwd_args(q, k, v, scale, return_lse, out, lse_out)
     mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
-                            doc_offsets_kv)
+                            doc_offsets_kv, _status_word(status, q.device))
     rc = lib.flex_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
                            scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
                            DTYPES[q.dtype], _stream(q.device))
@@ -203,7 +252,7 @@ def fwd(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset
 def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None, full_kv_indices=None,
                      scale=None, score_mod="none", mask_mod="none", window=0, offset=0, return_lse=True,
                      out=None, lse_out=None, tile_map=None, block_size=128, alibi_slopes=None, doc_offsets=None,
-                     doc_offsets_kv=None):
+                     doc_offsets_kv=None, status=None):
     """Forward with a block mask (flex_attn_fwd_block_sparse).  The block lists are int32
     CUDA tensors: counts [Bm, Hm, ceil(Sq/128)], indices [Bm, Hm, ceil(Sq/128), max_blocks],
     Bm in {1, B}, Hm in {1, H}; either (counts, indices) pair may be None, not both.
@@ -233,7 +282,7 @@ def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None
     if shape[2] != -(-Sq // 128):
         raise FlexAttnError(f"block mask has {shape[2]} query tiles, Sq={Sq} needs {-(-Sq // 128)}")
     mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
-                            doc_offsets_kv)
+                            doc_offsets_kv, _status_word(status, q.device))
     rc = lib.flex_attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
                                         scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
                                         ctypes.byref(bm), DTYPES[q.dtype], _stream(q.device))
@@ -243,7 +292,7 @@ def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None
 
 def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None, score_mod="none",
             mask_mod="none", window=0, offset=0, alibi_slopes=None, return_lse=True, out=None, lse_out=None,
-            workspace=None):
+            workspace=None, status=None):
     """8-bit forward (flex_attn_fwd_fp8): q8/k8/v8 are torch.float8_e4m3fn CUDA tensors in
     the layouts of fwd(); their values are descale_* times the codes.  Returns (O, LSE)
     with O in bf16.  Head dim 128."""
@@ -252,10 +301,18 @@ def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None,
         _cuda_tensor(t, n)
         if t.dtype != torch.float8_e4m3fn:
             raise FlexAttnError(f"{n} must be torch.float8_e4m3fn")
+    if q8.dim() != 4 or k8.dim() != 4:
+        raise FlexAttnError("q8, k8, v8 must be 4-D [B, H, S, D]")
     B, H, Sq, D = q8.shape
     Bk, Hkv, Skv, Dk = k8.shape
     if Bk != B or Dk != D or tuple(v8.shape) != tuple(k8.shape):
         raise FlexAttnError("shape mismatch between q8, k8, v8")
+    if k8.device != q8.device or v8.device != q8.device:
+        raise FlexAttnError("q8, k8, v8 must be on one device")
+    if out is not None:
+        _expect(out, "out", (B, H, Sq, D), torch.bfloat16, q8.device)
+    if return_lse and lse_out is not None:
+        _expect(lse_out, "lse_out", (B, H, Sq), torch.float32, q8.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     o = out if out is not None else torch.empty((B, H, Sq, D), dtype=torch.bfloat16, device=q8.device)
@@ -265,7 +322,10 @@ def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None,
     need = int(lib.flex_attn_fwd_fp8_workspace_size(B, Hkv, Skv, D))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q8.device)
-    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, None, None)
+    elif workspace.device != q8.device or not workspace.is_contiguous():
+        raise FlexAttnError("workspace must be a contiguous tensor on q8's device")
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, None, None,
+                            _status_word(status, q8.device))
     rc = lib.flex_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D, float(scale),
                                float(descale_q), float(descale_k), float(descale_v), score, MASK_MODS[mask_mod],
                                ctypes.byref(mp), _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -279,7 +339,8 @@ def bwd_workspace_size(B, H, Sq) -> int:
 
 
 def bwd(q, k, v, o, lse, dout, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
-        alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None, dq=None, dk=None, dv=None, workspace=None):
+        alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None, dq=None, dk=None, dv=None, workspace=None,
+        status=None):
     """Flex-attention backward (flex_attn_bwd): gradients (dq, dk, dv) of sum(dout * o)
     for the forward with the same arguments; o and lse are that forward's outputs.
     dk/dv are [B, Hkv, Skv, D] (summed over the query heads of each group)."""
@@ -287,18 +348,22 @@ def bwd(q, k, v, o, lse, dout, scale=None, score_mod="none", mask_mod="none", wi
     for t, n in ((o, "o"), (dout, "dout"), (lse, "lse")):
         _cuda_tensor(t, n)
     B, H, Hkv, Sq, Skv, D, scale, _, _ = _fwd_args(q, k, v, scale, False, q, None)
-    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape) or dout.dtype != q.dtype:
-        raise FlexAttnError("o and dout must match q")
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq):
-        raise FlexAttnError("lse must be float32 [B, H, Sq]")
+    _expect(o, "o", q.shape, q.dtype, q.device)
+    _expect(dout, "dout", q.shape, q.dtype, q.device)
+    _expect(lse, "lse", (B, H, Sq), torch.float32, q.device)
+    for t, n, like in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        if t is not None:
+            _expect(t, n, like.shape, like.dtype, like.device)
     dq = dq if dq is not None else torch.empty_like(q)
     dk = dk if dk is not None else torch.empty_like(k)
     dv = dv if dv is not None else torch.empty_like(v)
     need = bwd_workspace_size(B, H, Sq)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    elif workspace.device != q.device or not workspace.is_contiguous():
+        raise FlexAttnError("workspace must be a contiguous tensor on q's device")
     mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, doc_offsets,
-                            doc_offsets_kv)
+                            doc_offsets_kv, _status_word(status, q.device))
     rc = lib.flex_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                            B, H, Hkv, Sq, Skv, D, scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
                            DTYPES[q.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -311,26 +376,60 @@ def decode_workspace_size(B, H, Hkv, cap, D) -> int:
     return int(load_library().flex_attn_decode_workspace_size(B, H, Hkv, cap, D))
 
 
-def decode(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None, workspace=None):
-    """Decode attention.  q [B,H,1,D]; caches [B,Hkv,cap,D]; kv_len [B] int32 (CUDA);
-    mask optional [B,H,1,cap] of q's dtype.  Returns (O [B,H,1,D], LSE [B,H,1])."""
-    lib = load_library()
+def _check_decode_shapes(q, k_cache, v_cache, kv_len, mask=None, out=None, lse_out=None):
+    """Shapes, dtypes and devices of a decode's tensors (no device work): a short kv_len
+    or mask, a smaller v_cache or a small out would make the kernels read or write past
+    the allocation."""
+    if q.dim() != 4 or q.shape[2] != 1:
+        raise FlexAttnError("decode takes q [B, H, 1, D]")
+    B, H, _, D = q.shape
+    if q.dtype not in DTYPES:
+        raise FlexAttnError(f"unsupported dtype {q.dtype}")
+    if k_cache.dim() != 4 or k_cache.shape[0] != B or k_cache.shape[3] != D:
+        raise FlexAttnError(f"k_cache must be [B={B}, Hkv, cap, D={D}], got {tuple(k_cache.shape)}")
+    Hkv, cap = k_cache.shape[1], k_cache.shape[2]
+    _expect(k_cache, "k_cache", (B, Hkv, cap, D), q.dtype, q.device)
+    _expect(v_cache, "v_cache", (B, Hkv, cap, D), q.dtype, q.device)
+    _expect(kv_len, "kv_len", (B,), torch.int32, q.device)
+    if mask is not None:
+        _expect(mask, "mask", (B, H, 1, cap), q.dtype, q.device)
+    if out is not None:
+        _expect(out, "out", (B, H, 1, D), q.dtype, q.device)
+    if lse_out is not None:
+        _expect(lse_out, "lse_out", (B, H, 1), torch.float32, q.device)
+    return B, H, Hkv, cap, D
+
+
+def _decode_prep(q, k_cache, v_cache, kv_len, mask, out, lse_out, split_size, status):
     for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (kv_len, "kv_len")):
         _cuda_tensor(t, n)
     if mask is not None:
         _cuda_tensor(mask, "mask")
-    B, H, one, D = q.shape
-    _, Hkv, cap, _ = k_cache.shape
-    if one != 1 or kv_len.dtype != torch.int32:
-        raise FlexAttnError("decode takes q [B,H,1,D] and int32 kv_len")
+    B, H, Hkv, cap, D = _check_decode_shapes(q, k_cache, v_cache, kv_len, mask, out, lse_out)
     o = out if out is not None else torch.empty_like(q)
     lse = lse_out if lse_out is not None else torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    dp = DecodeParamsC(int(split_size), _status_word(status, q.device))
+    return B, H, Hkv, cap, D, o, lse, dp
+
+
+def decode(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None, workspace=None, split_size=0,
+           status=None):
+    """Decode attention.  q [B,H,1,D]; caches [B,Hkv,cap,D] of q's dtype; kv_len [B] int32
+    (CUDA); mask optional [B,H,1,cap] of q's dtype.  ``split_size``: cache positions per
+    split (0 = the library's choice, 128 or 256).  ``status``: optional one-element int32
+    CUDA tensor that receives this call's device status bits.  Returns (O [B,H,1,D],
+    LSE [B,H,1])."""
+    lib = load_library()
+    B, H, Hkv, cap, D, o, lse, dp = _decode_prep(q, k_cache, v_cache, kv_len, mask, out, lse_out, split_size,
+                                                 status)
     need = decode_workspace_size(B, H, Hkv, cap, D)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    elif workspace.device != q.device or not workspace.is_contiguous():
+        raise FlexAttnError("workspace must be a contiguous tensor on q's device")
     rc = lib.flex_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_len), _ptr(mask), _ptr(o), _ptr(lse),
                               B, H, Hkv, cap, D, float(scale), DTYPES[q.dtype], _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _stream(q.device))
+                              workspace.numel() * workspace.element_size(), ctypes.byref(dp), _stream(q.device))
     _check(rc, "flex_attn_decode")
     return o, lse
 
@@ -339,25 +438,18 @@ def decode(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None
 DECODE_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
-def decode_noalloc(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None):
+def decode_noalloc(q, k_cache, v_cache, kv_len, scale, mask=None, out=None, lse_out=None, split_size=0,
+                   status=None):
     """Decode through flex_attn_decode_noalloc: no workspace argument and no device
     allocation inside the library; it uses the scratch array compiled into the library
     (shared by all calls on a device, so calls must not overlap on the GPU).  Outputs
     are allocated here only when ``out`` / ``lse_out`` are not given."""
     lib = load_library()
-    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (kv_len, "kv_len")):
-        _cuda_tensor(t, n)
-    if mask is not None:
-        _cuda_tensor(mask, "mask")
-    B, H, one, D = q.shape
-    _, Hkv, cap, _ = k_cache.shape
-    if one != 1 or kv_len.dtype != torch.int32:
-        raise FlexAttnError("decode takes q [B,H,1,D] and int32 kv_len")
-    o = out if out is not None else torch.empty_like(q)
-    lse = lse_out if lse_out is not None else torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    B, H, Hkv, cap, D, o, lse, dp = _decode_prep(q, k_cache, v_cache, kv_len, mask, out, lse_out, split_size,
+                                                 status)
     rc = lib.flex_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kv_len), _ptr(mask), _ptr(o),
                                       _ptr(lse), B, H, Hkv, cap, D, float(scale), DTYPES[q.dtype],
-                                      _stream(q.device))
+                                      ctypes.byref(dp), _stream(q.device))
     _check(rc, "flex_attn_decode_noalloc")
     return o, lse
 

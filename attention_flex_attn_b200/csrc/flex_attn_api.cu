@@ -76,24 +76,71 @@ bool make_map_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows
 // every call on that device.
 __device__ __align__(256) unsigned char g_decode_scratch[FLEX_DECODE_STATIC_SCRATCH_BYTES];
 
-// Device address of g_decode_scratch on the current device, looked up once per device
-// (host code only sees a host-side stand-in under that name, never usable on the GPU).
-void* decode_scratch_ptr() {
+// Id of the context current on this thread (driver entry points, so the runtime does not
+// create a context just to answer), or false when none is current.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(a);
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(b);
+    }
+  });
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device addresses of the library's __device__ symbols (host code sees only host-side
+// stand-ins under those names).  Looked up once per device and context: a context that
+// was destroyed and created again (cudaDeviceReset) loads the module anew, at a new
+// address, so the cache is keyed on the context's id.
+enum Symbol { kSymStatus = 0, kSymScratch = 1 };
+
+void* symbol_ptr(Symbol which) {
   constexpr int kMaxDevices = 64;
-  static std::atomic<void*> cache[kMaxDevices];
+  struct Entry {
+    unsigned long long ctx;
+    void* addr[2];
+  };
+  static Entry cache[kMaxDevices] = {};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void* p = cache[dev].load(std::memory_order_acquire);
-  if (p) return p;
-  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
-  cache[dev].store(p, std::memory_order_release);
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
+  if (have_id) {
+    std::lock_guard<std::mutex> g(mu);
+    if (cache[dev].ctx == id && cache[dev].addr[which]) return cache[dev].addr[which];
+  }
+  void* p = nullptr;
+  const cudaError_t e = which == kSymStatus ? cudaGetSymbolAddress(&p, g_status)
+                                            : cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr) return nullptr;
+  if (!have_id) have_id = current_context_id(&id);  // the lookup made the context current
+  if (have_id) {
+    std::lock_guard<std::mutex> g(mu);
+    if (cache[dev].ctx != id) cache[dev] = Entry{id, {nullptr, nullptr}};
+    cache[dev].addr[which] = p;
+  }
   return p;
 }
 
-unsigned* status_ptr() {
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-  return static_cast<unsigned*>(p);
+void* decode_scratch_ptr() { return symbol_ptr(kSymScratch); }
+
+// The status word a call's kernels report into: the caller's own, or the shared one.
+unsigned* status_for(uint32_t* status_out) {
+  if (status_out) return reinterpret_cast<unsigned*>(status_out);
+  return static_cast<unsigned*>(symbol_ptr(kSymStatus));
 }
 
 // ---------------------------------------------------------------- mask evaluation (debug)
@@ -124,7 +171,22 @@ __global__ void mask_eval_kernel(MaskArgs m, int Sq, int Skv, uint8_t* keep) {
   }
 }
 
-int decode_splits(int cap) { return (cap + kChunk - 1) / kChunk; }
+int decode_splits(int cap, int split) { return (cap + split - 1) / split; }
+
+// Workspace bytes of a decode with splits of `split` positions: partial outputs
+// [B*H, n_splits, D] fp32 (rounded up to 256 bytes), then their LSEs [B*H, n_splits].
+size_t decode_ws_bytes(int B, int H, int cap, int D, int split) {
+  const size_t rows = static_cast<size_t>(B) * H;
+  const size_t ns = static_cast<size_t>(decode_splits(cap, split));
+  const size_t o_bytes = rows * ns * D * sizeof(float);
+  return ((o_bytes + 255) & ~static_cast<size_t>(255)) + rows * ns * sizeof(float);
+}
+
+// The split size a decode uses: the caller's, or the library's choice.
+int decode_split_for(const flex_decode_params_t* dp) {
+  if (dp && dp->split_size != 0) return dp->split_size;
+  return kChunkDefault;
+}
 
 constexpr unsigned kStatusSelftestTimeout = 8u;
 
@@ -220,7 +282,8 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   const int64_t n_units = bh * n_pairs;
   if (n_units > 0x7fffffff || static_cast<int64_t>(B) * Hkv > 0x7fffffff) return FLEX_ERR_UNSUPPORTED;
 
-  unsigned* st = status_ptr();
+  if (mp.status_out && !aligned4(mp.status_out)) return FLEX_ERR_MISALIGNED;
+  unsigned* st = status_for(mp.status_out);
   if (!st) return FLEX_ERR_CUDA;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, dtype, D, Sq, bh) || !make_map(&mk, k, dtype, D, Skv, static_cast<int64_t>(B) * Hkv) ||
@@ -323,7 +386,8 @@ flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, 
   const int n_qtiles = (Sq + kBM - 1) / kBM, n_pairs = (n_qtiles + 1) / 2;
   const int skv_pad = (Skv + 127) / 128 * 128;
   if (bh * n_pairs > 0x7fffffff || bhkv * (skv_pad / 128) > 0x7fffffff) return FLEX_ERR_UNSUPPORTED;
-  unsigned* st = status_ptr();
+  if (mp.status_out && !aligned4(mp.status_out)) return FLEX_ERR_MISALIGNED;
+  unsigned* st = status_for(mp.status_out);
   if (!st) return FLEX_ERR_CUDA;
   Fp8Maps m;
   if (!make_map_u8(&m.q, q8, D, Sq, bh) || !make_map_u8(&m.k, k8, D, Skv, bhkv) ||
@@ -386,7 +450,8 @@ flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const v
   const int n_qtiles = (Sq + kBM - 1) / kBM, n_ktiles = (Skv + kBN - 1) / kBN;
   const int64_t bh = static_cast<int64_t>(B) * H, bhkv = static_cast<int64_t>(B) * Hkv;
   if (bh * n_qtiles > 0x7fffffff || bhkv * n_ktiles > 0x7fffffff) return FLEX_ERR_UNSUPPORTED;
-  unsigned* st = status_ptr();
+  if (mp.status_out && !aligned4(mp.status_out)) return FLEX_ERR_MISALIGNED;
+  unsigned* st = status_for(mp.status_out);
   if (!st) return FLEX_ERR_CUDA;
   BwdMaps m;
   if (!make_map(&m.q, q, dtype, D, Sq, bh) || !make_map(&m.o, dout, dtype, D, Sq, bh) ||
@@ -423,29 +488,28 @@ flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const v
 
 size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D) {
   if (B < 1 || H < 1 || Hkv < 1 || cap < 1 || D < 1) return 0;
-  const size_t rows = static_cast<size_t>(B) * H;
-  const size_t ns = static_cast<size_t>(decode_splits(cap));
-  const size_t o_bytes = rows * ns * D * sizeof(float);
-  const size_t o_round = (o_bytes + 255) & ~static_cast<size_t>(255);
-  return o_round + rows * ns * sizeof(float);
+  return decode_ws_bytes(B, H, cap, D, kChunkMin);
 }
 
 flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_len,
                                const void* additive_mask, void* o, float* lse, int B, int H, int Hkv, int cap, int D,
                                float scale, flex_dtype_t dtype, void* workspace, size_t workspace_bytes,
-                               flex_stream_t stream) {
+                               const flex_decode_params_t* dp, flex_stream_t stream) {
   if (!q || !k_cache || !v_cache || !kv_len || !o) return FLEX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Hkv < 1 || cap < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
+  const int split = decode_split_for(dp);
+  if (split != 128 && split != 256) return FLEX_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
   if (dtype != FLEX_DTYPE_BF16 && dtype != FLEX_DTYPE_F16) return FLEX_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * Hkv * (H / Hkv) > 65535LL * 8) return FLEX_ERR_UNSUPPORTED;
-  const size_t need = flex_attn_decode_workspace_size(B, H, Hkv, cap, D);
+  const size_t need = decode_ws_bytes(B, H, cap, D, split);
   if (!workspace || workspace_bytes < need) return FLEX_ERR_WORKSPACE;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(workspace) ||
       (lse && !aligned16(lse)) || (additive_mask && !aligned16(additive_mask)) || !aligned16(kv_len))
     return FLEX_ERR_MISALIGNED;
-  unsigned* st = status_ptr();
+  if (dp && dp->status_out && !aligned4(dp->status_out)) return FLEX_ERR_MISALIGNED;
+  unsigned* st = status_for(dp ? dp->status_out : nullptr);
   if (!st) return FLEX_ERR_CUDA;
   DecodeParams p{};
   p.q = q;
@@ -460,7 +524,8 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
   p.Hkv = Hkv;
   p.G = H / Hkv;
   p.cap = cap;
-  p.n_splits = decode_splits(cap);
+  p.split = split;
+  p.n_splits = decode_splits(cap, split);
   const size_t rows = static_cast<size_t>(B) * H;
   const size_t o_bytes = rows * p.n_splits * D * sizeof(float);
   p.part_o = static_cast<float*>(workspace);
@@ -475,14 +540,20 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
 flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                        const int32_t* kv_len, const void* additive_mask, void* o, float* lse,
                                        int B, int H, int Hkv, int cap, int D, float scale, flex_dtype_t dtype,
-                                       flex_stream_t stream) {
-  const size_t need = flex_attn_decode_workspace_size(B, H, Hkv, cap, D);
-  if (need == 0) return FLEX_ERR_INVALID_ARG;
-  if (need > FLEX_DECODE_STATIC_SCRATCH_BYTES) return FLEX_ERR_WORKSPACE;
+                                       const flex_decode_params_t* dp, flex_stream_t stream) {
+  if (B < 1 || H < 1 || Hkv < 1 || cap < 1 || D < 1) return FLEX_ERR_INVALID_ARG;
+  // 256-position splits unless the caller asks otherwise (the smaller workspace)
+  flex_decode_params_t use{kChunkMax, nullptr};
+  if (dp) {
+    use = *dp;
+    if (use.split_size == 0) use.split_size = kChunkMax;
+  }
+  if (use.split_size != 128 && use.split_size != 256) return FLEX_ERR_INVALID_ARG;
+  if (decode_ws_bytes(B, H, cap, D, use.split_size) > FLEX_DECODE_STATIC_SCRATCH_BYTES) return FLEX_ERR_WORKSPACE;
   void* scratch = decode_scratch_ptr();
   if (!scratch) return FLEX_ERR_CUDA;
   return flex_attn_decode(q, k_cache, v_cache, kv_len, additive_mask, o, lse, B, H, Hkv, cap, D, scale, dtype,
-                          scratch, FLEX_DECODE_STATIC_SCRATCH_BYTES, stream);
+                          scratch, FLEX_DECODE_STATIC_SCRATCH_BYTES, &use, stream);
 }
 
 flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_params, int Sq, int Skv,
@@ -517,7 +588,7 @@ flex_status_t flex_attn_mask_eval(int mask_mod_id, const flex_mod_params_t* mod_
 
 flex_status_t flex_attn_selftest_wait_timeout(uint32_t timeout_us, flex_stream_t stream) {
   if (timeout_us < 1 || timeout_us > 2000000u) return FLEX_ERR_INVALID_ARG;
-  unsigned* st = status_ptr();
+  unsigned* st = status_for(nullptr);
   if (!st) return FLEX_ERR_CUDA;
   selftest_wait_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(timeout_us) * 1000ull, st);

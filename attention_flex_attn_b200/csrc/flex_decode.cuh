@@ -4,8 +4,8 @@
 // additive mask [B,H,1,?], f32 accumulation).
 //
 // Split-KV ("flash decoding"): the cache of each (b, kv head) is cut into chunks of
-// kChunk positions.  decode_split_kernel handles one chunk for GT query heads that share
-// a kv head: it streams the chunk's K rows with 16-byte read-only loads, forms the scores
+// CH positions (128 or 256, a run-time choice between two instantiations).
+// decode_split_kernel handles one chunk for GT query heads that share a kv head: it streams the chunk's K rows with 16-byte read-only loads, forms the scores
 // (scale * q.k + mask) in base 2, takes the chunk-local softmax and streams V for
 // sum_j p_j V_j.  Each chunk writes its normalised partial output and its base-2
 // log-sum-exp to the workspace.  decode_combine_kernel merges the chunks of each
@@ -24,7 +24,9 @@
 
 namespace flexattn {
 
-constexpr int kChunk = 256;           // cache positions per split
+constexpr int kChunkMin = 128;        // cache positions per split: the two sizes built
+constexpr int kChunkMax = 256;
+constexpr int kChunkDefault = 256;
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr unsigned kStatusBadKvLen = 1u;
@@ -41,7 +43,7 @@ struct DecodeParams {
   float* part_o;      // [B*H, n_splits, D]
   float* part_lse;    // [B*H, n_splits]
   unsigned* status;
-  int B, H, Hkv, G, cap, n_splits;
+  int B, H, Hkv, G, cap, split, n_splits;  // split: positions per chunk (CH of the kernels)
   float scale_log2;
 };
 
@@ -85,14 +87,14 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int b) {
   return (L < 0 || L > p.cap) ? -1 : L;
 }
 
-template <int D, typename T, int GT>
+template <int D, typename T, int GT, int CH>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeParams p) {
   constexpr int LPR = D / 8;            // lanes per cache row (8 elements = 16 bytes each)
   constexpr int RPW = 32 / LPR;         // rows per warp per load instruction
   constexpr int ROWS_PER_PASS = kDecWarps * RPW;
   constexpr int U = 8;                  // loads in flight per lane
 
-  __shared__ float s_sc[GT][kChunk];
+  __shared__ float s_sc[GT][CH];
   __shared__ float s_red[kDecWarps][GT][D];
   __shared__ float s_m[GT], s_l[GT];
 
@@ -105,9 +107,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   const int h0 = hkv * p.G + gt * GT;
 
   const int L = checked_len(p, b);
-  const int j0 = split * kChunk;
+  const int j0 = split * CH;
   if (L <= 0 || j0 >= L) return;
-  const int n = min(kChunk, L - j0);
+  const int n = min(CH, L - j0);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane % LPR, rsub = lane / LPR;
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   }
 
   // ---- scores: s = scale*log2(e) * q.k over the chunk
-  for (int base = 0; base < kChunk; base += ROWS_PER_PASS * U) {
+  for (int base = 0; base < CH; base += ROWS_PER_PASS * U) {
     uint4 kr[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
         for (int e = 0; e < 8; ++e) acc = fmaf(qf[g][e], kf[e], acc);
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (sub == 0 && row < kChunk) s_sc[g][row] = acc;
+        if (sub == 0 && row < CH) s_sc[g][row] = acc;
       }
     }
   }
@@ -155,10 +157,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   for (int g = warp; g < GT; g += kDecWarps) {
     const T* mrow = p.mask ? reinterpret_cast<const T*>(p.mask) + (static_cast<int64_t>(b) * p.H + h0 + g) * p.cap + j0
                            : nullptr;
-    float vals[kChunk / 32];
+    float vals[CH / 32];
     float mx = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < kChunk / 32; ++t) {
+    for (int t = 0; t < CH / 32; ++t) {
       const int e = lane + 32 * t;
       float x = -INFINITY;
       if (e < n) {
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
     const float ms = mx == -INFINITY ? 0.f : mx;
     float sum = 0.f;
 #pragma unroll
-    for (int t = 0; t < kChunk / 32; ++t) {
+    for (int t = 0; t < CH / 32; ++t) {
       const float e2 = ex2_approx(vals[t] - ms);
       s_sc[g][lane + 32 * t] = e2;
       sum += e2;
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   for (int g = 0; g < GT; ++g)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-  for (int base = 0; base < kChunk; base += ROWS_PER_PASS * U) {
+  for (int base = 0; base < CH; base += ROWS_PER_PASS * U) {
     uint4 vr[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -248,7 +250,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 // K/V byte, so the per-byte arithmetic grows with G.  This kernel puts up to 16 heads in
 // the 16 rows of warp-level tensor-core MMAs (mma.sync m16n8k16, fp32 accumulate), which
 // makes the arithmetic per byte independent of G and leaves the kernel bound by HBM.
-// Each warp owns 64 keys of the 256-key chunk:
+// Each warp owns CH / 4 keys (64 or 32) of the chunk:
 //  * S = Q K^T: K rows are loaded straight into B fragments, 16 bytes per lane.  Within
 //    each 32-wide slice of the head dimension the contraction index is permuted the same
 //    way in the Q (A) and K (B) fragments, so each lane reads 8 consecutive elements.
@@ -260,7 +262,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
 // The four warps' partial results are merged through shared memory into one (O, LSE)
 // partial per chunk, in the same workspace format as decode_split_kernel.
 constexpr int kGqaRows = 16;
-constexpr int kGqaKeysPerWarp = kChunk / kDecWarps;  // 64
 
 template <typename T>
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -300,9 +301,13 @@ __device__ __forceinline__ uint32_t u4_at(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-template <int D, typename T>
+template <int D, typename T, int CH>
 __global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const DecodeParams p) {
   constexpr int KC = D / 32;  // 32-wide slices of the head dimension
+  constexpr int KPW = CH / kDecWarps;  // keys per warp
+  constexpr int NT = KPW / 8;          // 8-key tiles of S per warp
+  constexpr int KS = KPW / 16;         // 16-key steps of P V per warp
+  static_assert(NT % 2 == 0 && KS >= 1, "chunk too small for the warp tiling");
   __shared__ float s_m[kDecWarps][kGqaRows], s_l[kDecWarps][kGqaRows];
   __shared__ __align__(16) float s_o[kDecWarps][kGqaRows][D];
 
@@ -316,13 +321,13 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const Decode
   const int gt = min(kGqaRows, p.G - grp * kGqaRows);  // valid MMA rows (query heads)
 
   const int L = checked_len(p, b);
-  const int j0 = split * kChunk;
+  const int j0 = split * CH;
   if (L <= 0 || j0 >= L) return;
-  const int n = min(kChunk, L - j0);
+  const int n = min(CH, L - j0);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int kw0 = warp * kGqaKeysPerWarp;
+  const int kw0 = warp * KPW;
   const T* kbase = reinterpret_cast<const T*>(p.k) + ((static_cast<int64_t>(b) * p.Hkv + hkv) * p.cap + j0) * D;
   const T* vbase = reinterpret_cast<const T*>(p.v) + ((static_cast<int64_t>(b) * p.Hkv + hkv) * p.cap + j0) * D;
 
@@ -338,10 +343,10 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const Decode
                            : make_uint4(0, 0, 0, 0);
     }
 
-  // ---- S = Q K^T over this warp's 64 keys (8 tiles of 8 keys)
-  float sc[8][4];
+  // ---- S = Q K^T over this warp's KPW keys (NT tiles of 8 keys)
+  float sc[NT][4];
 #pragma unroll
-  for (int nt = 0; nt < 8; nt += 2) {
+  for (int nt = 0; nt < NT; nt += 2) {
     uint4 kr[2][KC];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
@@ -375,7 +380,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const Decode
   }
   float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int key = kw0 + nt * 8 + 2 * q + (e & 1);
@@ -398,9 +403,9 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const Decode
   }
   const float ms0 = m0 == -INFINITY ? 0.f : m0, ms1 = m1 == -INFINITY ? 0.f : m1;
   float l0 = 0.f, l1 = 0.f;
-  uint32_t pa[4][4];  // A fragments of P for the four 16-key steps
+  uint32_t pa[KS][4];  // A fragments of P for the KS 16-key steps
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
+  for (int nt = 0; nt < NT; ++nt) {
     const float p0 = ex2_approx(sc[nt][0] - ms0), p1 = ex2_approx(sc[nt][1] - ms0);
     const float p2 = ex2_approx(sc[nt][2] - ms1), p3 = ex2_approx(sc[nt][3] - ms1);
     l0 += p0 + p1;
@@ -423,7 +428,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_gqa_kernel(const Decode
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[c][r][e] = 0.f;
 #pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
+  for (int ks = 0; ks < KS; ++ks) {
     const int keyA = kw0 + 16 * ks + g, keyB = keyA + 8;
     uint4 va[KC], vb[KC];
 #pragma unroll
@@ -495,7 +500,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_combine_kernel(const Decod
     if (lane == 0 && row % p.H == 0) atomicOr(p.status, kStatusBadKvLen);
     L = 0;
   }
-  const int ns = (L + kChunk - 1) / kChunk;
+  const int ns = (L + p.split - 1) / p.split;
   const float* plse = p.part_lse + static_cast<int64_t>(row) * p.n_splits;
   float M = -INFINITY;
   for (int s = lane; s < ns; s += 32) M = fmaxf(M, plse[s]);

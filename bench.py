@@ -340,6 +340,9 @@ def main():
                                 "unit": "GB/s", "frac": dbytes / dec_avg_s / 1e9 / peaks["hbm_gbs"],
                                 "peak_source": peak_kind}},
         "fwd_ms": fwd_avg_s * 1e3,
+        "fwd_stats": _spread(fwd_ms), "decode_stats": _spread(dec_ms),
+        "protocol": "headline step: per-step CUDA events over the K timed steps; cases: "
+                    f"{PROTOCOL['warmup']} warm-up, {PROTOCOL['samples']} samples x {PROTOCOL['iters']} iterations",
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
         "kernel_hash": kernel_hash(),
@@ -359,18 +362,48 @@ def main():
     return 0
 
 
-def _time_fn(fn, iters, warm):
+# The pages' timing protocol (FlyDSL PR 931, Performance Report header): 10 warm-up runs,
+# then 12 samples of 100 back-to-back iterations each; mean +- std over the samples.
+PROTOCOL = dict(warmup=10, samples=12, iters=100)
+
+
+def _time_stats(fn, samples=None, iters=None, warm=None):
+    """Seconds per call: mean, std and coefficient of variation over `samples` samples,
+    each the CUDA-event time of `iters` back-to-back calls divided by `iters`."""
     import torch
+    samples = samples or PROTOCOL["samples"]
+    iters = iters or PROTOCOL["iters"]
+    warm = PROTOCOL["warmup"] if warm is None else warm
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(iters):
-        fn()
-    b.record()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(samples + 1)]
+    ev[0].record()
+    for s in range(samples):
+        for _ in range(iters):
+            fn()
+        ev[s + 1].record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / iters / 1e3
+    per = [ev[s].elapsed_time(ev[s + 1]) / iters / 1e3 for s in range(samples)]
+    mean = statistics.fmean(per)
+    std = statistics.stdev(per) if len(per) > 1 else 0.0
+    return {"mean": mean, "std": std, "cv_pct": 100.0 * std / mean if mean > 0 else 0.0, "samples": samples,
+            "iters": iters}
+
+
+def _case_row(st, flops=None, key="tflops"):
+    """A per-case row: time in us with its spread, and TFLOPS from the mean time."""
+    row = {"us": st["mean"] * 1e6, "std_us": st["std"] * 1e6, "cv_pct": st["cv_pct"]}
+    if flops is not None:
+        row[key] = flops / st["mean"] / 1e12
+    return row
+
+
+def _spread(ms):
+    """mean, std and CV% of per-step times in ms (this rank's steps)."""
+    mean = statistics.fmean(ms)
+    std = statistics.stdev(ms) if len(ms) > 1 else 0.0
+    return {"mean_ms": mean, "std_ms": std, "cv_pct": 100.0 * std / mean if mean > 0 else 0.0, "steps": len(ms)}
 
 
 def per_case(fa, q, k, v, scale, o, lse, args):
@@ -384,10 +417,11 @@ def per_case(fa, q, k, v, scale, o, lse, args):
              "causal_via_mask": dict(mask_mod="causal"), "causal_fast": dict(mask_mod="causal_fast")}
     out = {}
     for name, mods in cases.items():
-        t = _time_fn(lambda: fa.fwd(q, k, v, scale=scale, out=o, lse_out=lse, **mods), 20, 3)
+        st = _time_stats(lambda: fa.fwd(q, k, v, scale=scale, out=o, lse_out=lse, **mods))
+        t = st["mean"]
         causal = "causal" in name
-        out[name] = {"us": t * 1e6, "tflops": (dense * (0.5 if causal else 1.0)) / t / 1e12,
-                     "tflops_dense_equiv": dense / t / 1e12}
+        out[name] = _case_row(st, dense * (0.5 if causal else 1.0))
+        out[name]["tflops_dense_equiv"] = dense / t / 1e12
         if name.startswith("sliding"):
             out[name]["tflops_useful"] = useful_window / t / 1e12
     out.update(block_cases(fa, q, k, v, scale, o, lse))
@@ -409,9 +443,8 @@ def fp8_cases(fa, q, k, v, scale):
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     res = {}
     for name, mods in (("fp8_no_mod", {}), ("fp8_causal", dict(mask_mod="causal"))):
-        t = _time_fn(lambda: fa.fwd_fp8(q8, k8, v8, scale=scale, out=o, lse_out=lse, workspace=ws, **mods), 20, 3)
-        flops = fwd_flops(B, H, S, S, D) * (0.5 if "causal" in name else 1.0)
-        res[name] = {"us": t * 1e6, "tflops": flops / t / 1e12}
+        st = _time_stats(lambda: fa.fwd_fp8(q8, k8, v8, scale=scale, out=o, lse_out=lse, workspace=ws, **mods))
+        res[name] = _case_row(st, fwd_flops(B, H, S, S, D) * (0.5 if "causal" in name else 1.0))
     return res
 
 
@@ -428,10 +461,9 @@ def bwd_cases(fa, q, k, v, scale):
     ws = torch.empty(fa.bwd_workspace_size(B, H, S), dtype=torch.uint8, device=q.device)
     for name, mods in (("bwd_no_mod", {}), ("bwd_causal", dict(mask_mod="causal"))):
         o, lse = fa.fwd(q, k, v, scale=scale, **mods)
-        t = _time_fn(lambda: fa.bwd(q, k, v, o, lse, dout, scale=scale, dq=dq, dk=dk, dv=dv, workspace=ws, **mods),
-                     10, 2)
-        flops = 2.5 * fwd_flops(B, H, S, S, D) * (0.5 if "causal" in name else 1.0)
-        res[name] = {"us": t * 1e6, "tflops": flops / t / 1e12}
+        st = _time_stats(lambda: fa.bwd(q, k, v, o, lse, dout, scale=scale, dq=dq, dk=dk, dv=dv, workspace=ws,
+                                        **mods))
+        res[name] = _case_row(st, 2.5 * fwd_flops(B, H, S, S, D) * (0.5 if "causal" in name else 1.0))
     return res
 
 
@@ -446,9 +478,9 @@ def captured_cases(fa, q, k, v, scale, o, lse):
     dev = q.device
     res = {}
     slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32, device=dev)
-    t = _time_fn(lambda: fa.fwd(q, k, v, scale=scale, score_mod="alibi", alibi_slopes=slopes, out=o, lse_out=lse),
-                 20, 3)
-    res["alibi_slope_tensor"] = {"us": t * 1e6, "tflops": fwd_flops(B, H, S, S, D) / t / 1e12}
+    st = _time_stats(lambda: fa.fwd(q, k, v, scale=scale, score_mod="alibi", alibi_slopes=slopes, out=o,
+                                    lse_out=lse))
+    res["alibi_slope_tensor"] = _case_row(st, fwd_flops(B, H, S, S, D))
     rng = np.random.default_rng(4102)
     bounds = []
     for _ in range(B):
@@ -461,14 +493,14 @@ def captured_cases(fa, q, k, v, scale, o, lse):
     off = np.array([c + [S] * (n - len(c)) for c in bounds], np.int32)  # repeats = empty documents
     doff = torch.from_numpy(off).to(dev)
     for mask in ("document", "document_causal"):
-        t = _time_fn(lambda: fa.fwd(q, k, v, scale=scale, mask_mod=mask, doc_offsets=doff, out=o, lse_out=lse), 20, 3)
+        st = _time_stats(lambda: fa.fwd(q, k, v, scale=scale, mask_mod=mask, doc_offsets=doff, out=o, lse_out=lse))
         pairs = 0.0
         for b in range(B):
             for a, e in zip(off[b, :-1], off[b, 1:]):
                 L = float(e - a)
                 pairs += L * (L + 1) / 2 if mask == "document_causal" else L * L
-        res[f"{mask}_packed"] = {"us": t * 1e6, "tflops_useful": 4.0 * D * H * pairs / t / 1e12,
-                                 "documents": [len(c) - 1 for c in bounds]}
+        res[f"{mask}_packed"] = _case_row(st, 4.0 * D * H * pairs, "tflops_useful")
+        res[f"{mask}_packed"]["documents"] = [len(c) - 1 for c in bounds]
     return res
 
 
@@ -497,9 +529,9 @@ def block_cases(fa, q, k, v, scale, o, lse):
     kn, ki = block_lists(np.broadcast_to(diag, (1, 1, nq, nk)))
     fn, fi = block_lists(np.broadcast_to(below, (1, 1, nq, nk)))
     lists = [torch.from_numpy(a).to(dev) for a in (kn, ki, fn, fi)]
-    t = _time_fn(lambda: fa.fwd_block_sparse(q, k, v, *lists, scale=scale, mask_mod="causal", out=o,
-                                             lse_out=lse), 20, 3)
-    res["block_causal_lists"] = {"us": t * 1e6, "tflops": 0.5 * fwd_flops(B, H, S, S, D) / t / 1e12}
+    st = _time_stats(lambda: fa.fwd_block_sparse(q, k, v, *lists, scale=scale, mask_mod="causal", out=o,
+                                                 lse_out=lse))
+    res["block_causal_lists"] = _case_row(st, 0.5 * fwd_flops(B, H, S, S, D))
     # documents of 4..24 whole tiles (512..3072 tokens), causal inside each document:
     # the diagonal block partial, earlier blocks of the same document full
     rng = np.random.default_rng(4101)
@@ -518,22 +550,22 @@ def block_cases(fa, q, k, v, scale, o, lse):
     kn, ki = block_lists(part)
     fn, fi = block_lists(full)
     lists = [torch.from_numpy(a).to(dev) for a in (kn, ki, fn, fi)]
-    t = _time_fn(lambda: fa.fwd_block_sparse(q, k, v, *lists, scale=scale, mask_mod="causal", out=o,
-                                             lse_out=lse), 20, 3)
+    st = _time_stats(lambda: fa.fwd_block_sparse(q, k, v, *lists, scale=scale, mask_mod="causal", out=o,
+                                                 lse_out=lse))
     pairs = 0.0  # kept (query, key) pairs per (b, h)
     ends = starts[1:] + [nq]
     for s0, e0 in zip(starts, ends):
         n = (e0 - s0) * 128
         pairs += n * (n + 1) / 2
-    res["block_document_causal"] = {"us": t * 1e6, "tflops_useful": 4.0 * D * B * H * pairs / t / 1e12,
-                                    "documents": len(starts)}
+    res["block_document_causal"] = _case_row(st, 4.0 * D * B * H * pairs, "tflops_useful")
+    res["block_document_causal"]["documents"] = len(starts)
     rng = np.random.default_rng(4100)
     sel = rng.random((B, H, nq, nk)) < 0.5
     fn, fi = block_lists(sel)
     lists = [torch.from_numpy(a).to(dev) for a in (fn, fi)]
-    t = _time_fn(lambda: fa.fwd_block_sparse(q, k, v, None, None, *lists, scale=scale, out=o, lse_out=lse), 20, 3)
-    flops = 4.0 * D * 128 * 128 * float(sel.sum())
-    res["block_random_half_full"] = {"us": t * 1e6, "tflops": flops / t / 1e12, "density": float(sel.mean())}
+    st = _time_stats(lambda: fa.fwd_block_sparse(q, k, v, None, None, *lists, scale=scale, out=o, lse_out=lse))
+    res["block_random_half_full"] = _case_row(st, 4.0 * D * 128 * 128 * float(sel.sum()))
+    res["block_random_half_full"]["density"] = float(sel.mean())
     return res
 
 
@@ -556,11 +588,11 @@ def decode_cases(fa, dev, args):
             ws = torch.empty(fa.decode_workspace_size(d["B"], d["H"], Hkv, d["cap"], d["D"]), dtype=torch.uint8,
                              device=dev)
             for with_mask in (False, True):
-                t = _time_fn(lambda: fa.decode(qd, kc, vc, lens_d, d["scale"], mask=mask if with_mask else None,
-                                               workspace=ws), 20, 3)
+                st = _time_stats(lambda: fa.decode(qd, kc, vc, lens_d, d["scale"], mask=mask if with_mask else None,
+                                                   workspace=ws))
                 by = decode_bytes(lens.tolist(), d["H"], Hkv, d["D"], with_mask)
                 key = f"Hkv{Hkv}_{'long' if long_kv else 'random'}_{'mask' if with_mask else 'nomask'}"
-                res[key] = {"us": t * 1e6, "gbs": by / t / 1e9}
+                res[key] = _case_row(st, by * 1e3, "gbs")  # bytes / s / 1e9 = (by * 1e3) / s / 1e12
             del qd, kc, vc, mask, ws
     return res
 
@@ -581,12 +613,14 @@ def e2e(fa, q, k, v, scale, args, dev, world):
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
-    iters = max(3, min(args.steps, 10))
-    t = _time_fn(once, iters, 2)
+    # each call moves 512 MiB over PCIe: 4 samples of up to 5 calls
+    st = _time_stats(once, samples=4, iters=max(2, min(args.steps, 5)), warm=2)
+    t = st["mean"]
     h2d = 3 * q.numel() * q.element_size()
     d2h = q.numel() * q.element_size() + hl.numel() * 4
     return {"value": world * flops / t / 1e12, "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "what": "forward with host Q/K/V in pinned memory, copies included"}
+            "d2h_bytes_per_step": d2h, "cv_pct": st["cv_pct"],
+            "what": "forward with host Q/K/V in pinned memory, copies included"}
 
 
 def profile_case(which):

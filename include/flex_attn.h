@@ -32,8 +32,13 @@
  *    error code and launches nothing.  Work is enqueued on `stream` and the call
  *    returns without synchronising.
  *  - Problems that only the device can see (a kv_len outside [0, cap], a wait that
- *    ran out of time) set bits in a device status word instead of trapping; read it
- *    with flex_attn_device_status().
+ *    ran out of time) set bits in a device status word instead of trapping.  Each call
+ *    can name its own word (status_out in flex_mod_params_t / flex_decode_params_t:
+ *    a caller-owned device uint32, OR-ed into, never cleared by the library), so that
+ *    calls on different streams can tell whose problem a bit is and read it with a
+ *    stream-ordered copy.  Calls that name none report into one word per device that
+ *    all such calls share; flex_attn_device_status() reads it (and synchronises the
+ *    device to do so).  The bits are listed with flex_attn_device_status().
  */
 #ifndef FLEX_ATTN_H_
 #define FLEX_ATTN_H_
@@ -105,6 +110,10 @@ typedef struct {
   const int32_t* doc_offsets_q;
   const int32_t* doc_offsets_kv;
   int32_t n_docs;
+  /* Per-call device status word (device memory, 4-byte aligned, owned by the caller):
+   * the kernels of this call OR their status bits into it.  NULL = the shared per-device
+   * word read by flex_attn_device_status(). */
+  uint32_t* status_out;
 } flex_mod_params_t;
 
 /*
@@ -227,8 +236,23 @@ flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const v
                             size_t workspace_bytes, flex_stream_t stream);
 
 /*
+ * flex_decode_params_t -- optional settings of one decode call (NULL = all defaults).
+ *   split_size: cache positions per split of the split-KV decode: 0 = the library's
+ *     choice, else 128 or 256 (FLEX_ERR_INVALID_ARG otherwise).  The result does not
+ *     depend on it beyond rounding (the combine is exact in real arithmetic); smaller
+ *     splits give more parallel work for short sequences and need more workspace.
+ *   status_out: per-call device status word, as in flex_mod_params_t (NULL = the shared
+ *     per-device word).
+ */
+typedef struct {
+  int32_t split_size;
+  uint32_t* status_out;
+} flex_decode_params_t;
+
+/*
  * flex_attn_decode_workspace_size -- bytes of device workspace flex_attn_decode needs
- * for these sizes (the split-KV partial outputs and their log-sum-exps).
+ * for these sizes (the split-KV partial outputs and their log-sum-exps), whatever split
+ * size the call uses (it is the size for the smallest split, 128 positions).
  */
 size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D);
 
@@ -245,14 +269,18 @@ size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D);
  *            -inf drops a position.
  *   o        [B, H, 1, D] dtype (out);  lse [B, H, 1] fp32 (out, NULL allowed).
  *   workspace: device buffer of at least flex_attn_decode_workspace_size() bytes,
- *            16-byte aligned; its contents on entry do not matter.
+ *            16-byte aligned; its contents on entry do not matter.  (A smaller buffer
+ *            is accepted when it holds the partials of the split size actually used:
+ *            B * H * ceil(cap / split) * (D + 1) * 4 bytes, the first part rounded up
+ *            to 256 bytes.)
  *   scale: finite and > 0.  D in {64, 128}; dtype in {BF16, F16}.
+ *   params: NULL or the split size and per-call status word (flex_decode_params_t).
  */
 flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                                const int32_t* kv_len, const void* additive_mask, void* o,
                                float* lse, int B, int H, int Hkv, int cap, int D, float scale,
                                flex_dtype_t dtype, void* workspace, size_t workspace_bytes,
-                               flex_stream_t stream);
+                               const flex_decode_params_t* params, flex_stream_t stream);
 
 /*
  * flex_attn_decode_noalloc -- flex_attn_decode without a caller-supplied workspace.
@@ -264,10 +292,12 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
  * needs no workspace: it uses a scratch array of FLEX_DECODE_STATIC_SCRATCH_BYTES
  * compiled into the library, which every GPU that loads the library keeps until the
  * process exits.  It calls no allocator of any kind.
- *   Arguments, layouts and errors are those of flex_attn_decode.  Sizes whose workspace
- *   (flex_attn_decode_workspace_size) exceeds FLEX_DECODE_STATIC_SCRATCH_BYTES return
- *   FLEX_ERR_WORKSPACE and launch nothing.
- *   The first call on a device looks up the device address of the scratch array
+ *   Arguments, layouts and errors are those of flex_attn_decode.  This variant splits
+ *   the cache into 256-position splits unless params->split_size asks for 128; sizes
+ *   whose partials at that split size (B * H * ceil(cap / split) * (D + 1) * 4 bytes)
+ *   exceed FLEX_DECODE_STATIC_SCRATCH_BYTES return FLEX_ERR_WORKSPACE and launch nothing.
+ *   The first call on a device (and the first after that device's context was destroyed
+ *   and created again) looks up the device address of the scratch array
  *   (cudaGetSymbolAddress, with that device current); make that first call before any
  *   stream capture on the device.
  *   All calls on a device share the one array and it keeps the last call's contents;
@@ -279,7 +309,8 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
 flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                        const int32_t* kv_len, const void* additive_mask, void* o,
                                        float* lse, int B, int H, int Hkv, int cap, int D, float scale,
-                                       flex_dtype_t dtype, flex_stream_t stream);
+                                       flex_dtype_t dtype, const flex_decode_params_t* params,
+                                       flex_stream_t stream);
 
 /*
  * flex_attn_mask_eval -- debug: evaluates the device mask rule the forward kernel uses
@@ -304,8 +335,10 @@ flex_status_t flex_attn_selftest_wait_timeout(uint32_t timeout_us, flex_stream_t
 void flex_attn_tile_sizes(int D, int* bm, int* bn);
 
 /*
- * flex_attn_device_status -- reads (and, if reset != 0, clears) the device status
- * word on the current device.  Synchronises the device.  Bits:
+ * flex_attn_device_status -- reads (and, if reset != 0, clears) the shared status word
+ * of the current device: the bits of every call that named no status_out of its own,
+ * whichever stream it ran on.  Synchronises the device.  (A per-call status_out holds
+ * the same bits for that call alone.)  Bits:
  *   1 = a decode kv_len outside [0, cap];  2 = a forward-kernel wait ran out of time;
  *   4 = a decode-kernel wait ran out of time;  8 = the self-test wait ran out (expected);
  *   16 = a backward-kernel wait ran out of time.

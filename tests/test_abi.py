@@ -44,9 +44,10 @@ def test_tile_sizes(lib):
 
 
 def test_workspace_size(lib):
-    # ceil(8192/256) = 32 splits; o part [16*32, 32, 128] fp32 + lse part
+    # sized for the smallest split (128 positions): ceil(8192/128) = 64 splits;
+    # o part [16*32, 64, 128] fp32 + lse part
     n = fa.decode_workspace_size(16, 32, 8, 8192, 128)
-    assert n == 16 * 32 * 32 * 128 * 4 + 16 * 32 * 32 * 4
+    assert n == 16 * 32 * 64 * 128 * 4 + 16 * 32 * 64 * 4
     assert fa.decode_workspace_size(0, 32, 8, 8192, 128) == 0
 
 
@@ -74,13 +75,16 @@ def test_fwd_rejects_bad_args_on_host(lib):
     assert _fwd(lib, mp=fa.ModParams(1, 0, 1, None)) == 1              # tile map without buffer
     assert _fwd(lib, q=17) == 3
     assert _fwd(lib, lse=20) == 3
+    st = fa.ModParams(0, 0, 0, None, None, None, None, 0, 18)         # status word not 4-byte aligned
+    assert _fwd(lib, mp=st) == 3
 
 
 def test_decode_rejects_bad_args_on_host(lib):
     def dec(q=16, k=16, v=16, kl=16, m=None, o=16, lse=None, B=2, H=4, Hkv=2, cap=64, D=128, scale=0.1,
-            dtype=1, ws=16, wsb=1 << 20):
+            dtype=1, ws=16, wsb=1 << 20, split=0, status=None):
+        dp = fa.DecodeParamsC(split, status)
         return lib.flex_attn_decode(P(q), P(k), P(v), P(kl), P(m), P(o), P(lse), B, H, Hkv, cap, D, scale,
-                                    dtype, P(ws), wsb, None)
+                                    dtype, P(ws), wsb, ctypes.byref(dp), None)
     assert dec(kl=0) == 1
     assert dec(H=3) == 1
     assert dec(cap=0) == 1
@@ -89,6 +93,16 @@ def test_decode_rejects_bad_args_on_host(lib):
     assert dec(wsb=16) == 4
     assert dec(m=18) == 3
     assert dec(kl=4) == 3
+    assert dec(split=64) == 1                 # split sizes are 128 and 256
+    assert dec(split=512) == 1
+    assert dec(status=6) == 3                 # status word not 4-byte aligned
+    # a workspace that holds the 256-split partials only is enough for split 256
+    small = 2 * 4 * 1 * 128 * 4 + 2 * 4 * 1 * 4  # B*H*ceil(64/256)*D*4 (a multiple of 256) + lse part
+    assert dec(wsb=small - 1, split=256) == 4
+    nalloc = lib.flex_attn_decode_noalloc
+    dp = fa.DecodeParamsC(96, None)
+    assert nalloc(P(16), P(16), P(16), P(16), None, P(16), None, 2, 4, 2, 64, 128, 0.1, 1, ctypes.byref(dp),
+                  None) == 1
 
 
 def test_mask_eval_rejects_bad_args(lib):
@@ -218,3 +232,97 @@ def test_binding_argument_counts_match_header(lib):
         assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
         checked += 1
     assert checked >= len(arity) // 2
+
+
+def _c_offsets():
+    """offsetof/sizeof of the header's parameter structs, from a C compiler."""
+    import subprocess
+    import tempfile
+    src = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "flex_attn.h"
+#define F(T, m) printf(#T "." #m " %zu\n", offsetof(T, m))
+int main(void) {
+  F(flex_mod_params_t, window); F(flex_mod_params_t, offset); F(flex_mod_params_t, flags);
+  F(flex_mod_params_t, tile_map_out); F(flex_mod_params_t, alibi_slopes); F(flex_mod_params_t, doc_offsets_q);
+  F(flex_mod_params_t, doc_offsets_kv); F(flex_mod_params_t, n_docs); F(flex_mod_params_t, status_out);
+  F(flex_decode_params_t, split_size); F(flex_decode_params_t, status_out);
+  F(flex_block_mask_t, kv_num_blocks); F(flex_block_mask_t, kv_indices); F(flex_block_mask_t, full_kv_num_blocks);
+  F(flex_block_mask_t, full_kv_indices); F(flex_block_mask_t, max_blocks); F(flex_block_mask_t, batch);
+  F(flex_block_mask_t, heads); F(flex_block_mask_t, q_block_size); F(flex_block_mask_t, kv_block_size);
+  printf("sizeof.flex_mod_params_t %zu\nsizeof.flex_decode_params_t %zu\nsizeof.flex_block_mask_t %zu\n",
+         sizeof(flex_mod_params_t), sizeof(flex_decode_params_t), sizeof(flex_block_mask_t));
+  return 0;
+}
+"""
+    with tempfile.TemporaryDirectory() as d:
+        c, exe = os.path.join(d, "layout.c"), os.path.join(d, "layout")
+        with open(c, "w") as f:
+            f.write(src)
+        subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), "-o", exe, c])
+        out = subprocess.check_output([exe]).decode()
+    return {k: int(v) for k, v in (line.split() for line in out.splitlines())}
+
+
+def test_struct_layouts_match_header():
+    """The binding's ctypes structures have the C layout of the header's structs (field
+    offsets and sizes), so a field added on one side cannot shift the other's."""
+    c = _c_offsets()
+    for name, cls in (("flex_mod_params_t", fa.ModParams), ("flex_decode_params_t", fa.DecodeParamsC),
+                      ("flex_block_mask_t", fa.BlockMaskC)):
+        assert ctypes.sizeof(cls) == c[f"sizeof.{name}"], name
+        for field, _ in cls._fields_:
+            assert getattr(cls, field).offset == c[f"{name}.{field}"], (name, field)
+
+
+def test_decode_shape_checks_on_cpu():
+    """decode()/decode_noalloc() validate every tensor before anything launches: each
+    mismatch below would otherwise make a kernel read or write past an allocation."""
+    import torch
+    B, H, Hkv, cap, D = 2, 4, 2, 64, 128
+    f16 = torch.float16
+
+    def args(**over):
+        a = dict(q=torch.zeros(B, H, 1, D, dtype=f16), k_cache=torch.zeros(B, Hkv, cap, D, dtype=f16),
+                 v_cache=torch.zeros(B, Hkv, cap, D, dtype=f16), kv_len=torch.zeros(B, dtype=torch.int32),
+                 mask=torch.zeros(B, H, 1, cap, dtype=f16), out=torch.zeros(B, H, 1, D, dtype=f16),
+                 lse_out=torch.zeros(B, H, 1, dtype=torch.float32))
+        a.update(over)
+        return a
+    assert fa._check_decode_shapes(**args()) == (B, H, Hkv, cap, D)
+    bad = [dict(kv_len=torch.zeros(B - 1, dtype=torch.int32)),              # short kv_len
+           dict(kv_len=torch.zeros(B, dtype=torch.int64)),                  # wrong kv_len dtype
+           dict(v_cache=torch.zeros(B, Hkv, cap // 2, D, dtype=f16)),       # smaller v_cache
+           dict(v_cache=torch.zeros(B, Hkv, cap, D, dtype=torch.bfloat16)),
+           dict(k_cache=torch.zeros(B + 1, Hkv, cap, D, dtype=f16)),        # batch mismatch
+           dict(k_cache=torch.zeros(B, Hkv, cap, 64, dtype=f16)),           # head dim mismatch
+           dict(mask=torch.zeros(B, H, 1, cap - 1, dtype=f16)),             # short mask
+           dict(mask=torch.zeros(B, H, 1, cap, dtype=torch.float32)),       # fp32 mask
+           dict(out=torch.zeros(B, H, 1, D // 2, dtype=f16)),               # small out
+           dict(out=torch.zeros(B, H, 1, D, dtype=torch.bfloat16)),
+           dict(lse_out=torch.zeros(B, H, dtype=torch.float32)),
+           dict(lse_out=torch.zeros(B, H, 1, dtype=f16)),
+           dict(q=torch.zeros(B, H, 2, D, dtype=f16)),                      # not one query row
+           dict(q=torch.zeros(B, H, 1, D, dtype=torch.float32))]
+    for over in bad:
+        with pytest.raises(fa.FlexAttnError):
+            fa._check_decode_shapes(**args(**over))
+
+
+def test_fwd_shape_checks_on_cpu():
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros(2, 4, 100, 64, dtype=bf)
+    k = torch.zeros(2, 2, 80, 64, dtype=bf)
+    assert fa._check_fwd_shapes(q, k, k) == (2, 4, 2, 100, 80, 64)
+    with pytest.raises(fa.FlexAttnError):
+        fa._check_fwd_shapes(q, k, torch.zeros(2, 2, 81, 64, dtype=bf))
+    with pytest.raises(fa.FlexAttnError):
+        fa._check_fwd_shapes(q, k, k, out=torch.zeros(2, 4, 99, 64, dtype=bf))
+    with pytest.raises(fa.FlexAttnError):
+        fa._check_fwd_shapes(q, k, k, out=torch.zeros(2, 4, 100, 64, dtype=torch.float16))
+    with pytest.raises(fa.FlexAttnError):
+        fa._check_fwd_shapes(q, k, k, lse_out=torch.zeros(2, 4, 100, dtype=bf))
+    with pytest.raises(fa.FlexAttnError):
+        fa._check_fwd_shapes(q, k, k, lse_out=torch.zeros(2, 4, 101, dtype=torch.float32))

@@ -129,3 +129,22 @@ def test_d64_ring_wrap_sampled_group(dtype, mods):
     """D=64 at Sq = Skv = 1500: 12 key tiles (ragged), so both of the dQ kernel's key and
     value rings and the dK/dV kernel's query ring wrap several times."""
     _case(1, 4, 2, 1500, 1500, 64, dtype, 87, 0.125, groups=[(0, 1)], **mods)
+
+
+@pytest.mark.parametrize("mods", [dict(mask_mod="none"), dict(mask_mod="causal")], ids=["no_mod", "causal"])
+def test_long_8192_sampled_groups(mods):
+    """The size the bench times: B2 H32 S8192 D128 bf16 with the bench's inputs
+    (N(0, 0.5^2), dO ~ N(0, 1)); the oracle computes two whole (b, head) groups, the
+    first and the last, in full."""
+    fa = _fa()
+    B, H, S, D = 2, 32, 8192, 128
+    q, k, v = synth.qkv(B, H, H, S, S, D, seed=4000, sigma=0.5, device="cuda")
+    dout = synth.normal_tensor((B, H, S, D), 4103, dtype="bf16", device="cuda")
+    scale = 1.0 / math.sqrt(D)
+    dq, dk, dv = _run(q, k, v, dout, scale, **mods)
+    groups = [(0, 0), (1, 31)]
+    rq, rk, rv = oracle.bwd(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), scale=scale, groups=groups, **mods)
+    dq = torch.stack([dq[b, hk:hk + 1] for b, hk in groups])
+    dk = torch.stack([dk[b, hk] for b, hk in groups])
+    dv = torch.stack([dv[b, hk] for b, hk in groups])
+    _check("dq", dq, rq), _check("dk", dk, rk), _check("dv", dv, rv)

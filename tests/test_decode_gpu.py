@@ -27,11 +27,11 @@ def _inputs(B, H, Hkv, cap, D, seed, dtype="f16", lens=None, mask_p=None):
     return q, kc, vc, kv_len, mask
 
 
-def _check(q, kc, vc, kv_len, mask, scale=SCALE):
+def _check(q, kc, vc, kv_len, mask, scale=SCALE, split=0):
     fa = _fa()
     d = torch.device("cuda")
     o, lse = fa.decode(q.to(d), kc.to(d), vc.to(d), kv_len.to(d), scale,
-                       mask=None if mask is None else mask.to(d))
+                       mask=None if mask is None else mask.to(d), split_size=split)
     torch.cuda.synchronize()
     assert fa.device_status() == 0
     ro, rl = oracle.decode(q, kc, vc, kv_len, scale, mask=mask)
@@ -40,10 +40,12 @@ def _check(q, kc, vc, kv_len, mask, scale=SCALE):
 
 @pytest.mark.parametrize("Hkv", [32, 8])
 @pytest.mark.parametrize("with_mask", [False, True])
-def test_decode_config(Hkv, with_mask):
-    """B=16, H=32, D=128, f16, kv_len ~ U[1, 8192], caches padded to 8192."""
+@pytest.mark.parametrize("split", [0, 128, 256])
+def test_decode_config(Hkv, with_mask, split):
+    """B=16, H=32, D=128, f16, kv_len ~ U[1, 8192], caches padded to 8192; the library's
+    split size and both explicit ones, every row against the oracle."""
     args = _inputs(16, 32, Hkv, 8192, 128, seed=3000 + Hkv, mask_p=0.1 if with_mask else None)
-    _check(*args)
+    _check(*args, split=split)
 
 
 @pytest.mark.parametrize("Hkv", [32, 8])
@@ -52,11 +54,35 @@ def test_decode_long_kv(Hkv):
     _check(*args)
 
 
-@pytest.mark.parametrize("lens", [[1, 255, 256, 257], [512, 0, 3, 1000], [0, 0, 0, 0]])
+@pytest.mark.parametrize("lens", [[1, 255, 256, 257], [512, 0, 3, 1000], [0, 0, 0, 0], [127, 128, 129, 383]])
 @pytest.mark.parametrize("D,dtype", [(128, "f16"), (64, "bf16"), (128, "bf16")])
-def test_decode_split_boundaries(lens, D, dtype):
+@pytest.mark.parametrize("split", [128, 256])
+def test_decode_split_boundaries(lens, D, dtype, split):
     args = _inputs(4, 8, 2, 1024, D, seed=3200 + D, dtype=dtype, lens=lens)
-    _check(*args)
+    _check(*args, split=split)
+    args = _inputs(4, 8, 8, 1024, D, seed=3250 + D, dtype=dtype, lens=lens)  # one query head per kv head
+    _check(*args, split=split)
+
+
+@pytest.mark.parametrize("Hkv", [32, 8])
+def test_decode_split_size_independence(Hkv):
+    """The combine merges chunk partials exactly in real arithmetic, so 128- and
+    256-position splits give the same rows up to rounding: both against the oracle and
+    against each other (O within 4e-3, LSE within 1e-3)."""
+    fa = _fa()
+    q, kc, vc, kv_len, mask = _inputs(16, 32, Hkv, 8192, 128, seed=3700 + Hkv, mask_p=0.1)
+    d = torch.device("cuda")
+    args = (q.to(d), kc.to(d), vc.to(d), kv_len.to(d), SCALE)
+    o1, l1 = fa.decode(*args, mask=mask.to(d), split_size=128)
+    o2, l2 = fa.decode(*args, mask=mask.to(d), split_size=256)
+    torch.cuda.synchronize()
+    ro, rl = oracle.decode(q, kc, vc, kv_len, SCALE, mask=mask)
+    compare(o1, l1, ro, rl, "split 128")
+    compare(o2, l2, ro, rl, "split 256")
+    assert torch.equal(torch.isneginf(l1), torch.isneginf(l2))
+    fin = ~torch.isneginf(l1)
+    assert (o1.float() - o2.float()).abs().max().item() <= 4e-3
+    assert (l1[fin] - l2[fin]).abs().max().item() <= 1e-3
 
 
 @pytest.mark.parametrize("H,Hkv", [(6, 2), (12, 4), (5, 5), (16, 2), (32, 2), (40, 2), (64, 4)])
@@ -82,6 +108,34 @@ def test_decode_bad_kv_len_sets_status():
     assert fa.device_status() & 1
     assert torch.all(o[0] == 0) and torch.all(torch.isneginf(lse[0]))
     assert fa.device_status() == 0  # cleared by the read
+
+
+def test_decode_per_call_status_on_two_streams():
+    """A bad kv_len on one stream and a clean decode on another, each with its own status
+    word: only the first caller's word gets bit 1, and the shared word stays clear."""
+    fa = _fa()
+    assert fa.device_status() == 0
+    q, kc, vc, _, _ = _inputs(2, 8, 2, 512, 128, seed=3550, lens=[1, 1])
+    q, kc, vc = q.cuda(), kc.cuda(), vc.cuda()
+    bad = torch.tensor([513, 100], dtype=torch.int32, device="cuda")
+    good = torch.tensor([512, 100], dtype=torch.int32, device="cuda")
+    st_a = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st_b = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(sa):
+        oa, la = fa.decode(q, kc, vc, bad, SCALE, status=st_a)
+    with torch.cuda.stream(sb):
+        ob, lb = fa.decode(q, kc, vc, good, SCALE, status=st_b)
+        fwd_st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        fa.fwd(q, kc, vc, status=fwd_st)
+    torch.cuda.synchronize()
+    assert int(st_a.item()) == 1
+    assert int(st_b.item()) == 0 and int(fwd_st.item()) == 0
+    assert fa.device_status() == 0
+    assert torch.all(oa[0] == 0) and torch.all(torch.isneginf(la[0]))
+    ro, rl = oracle.decode(q.cpu(), kc.cpu(), vc.cpu(), good.cpu(), SCALE)
+    compare(ob, lb, ro, rl, "clean stream")
 
 
 def test_decode_matches_forward_single_row():

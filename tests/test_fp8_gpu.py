@@ -29,9 +29,9 @@ def _fa():
     return fa
 
 
-def _inputs(B, H, Hkv, Sq, Skv, seed, spread=1.0):
-    q, k, v = synth.qkv(B, H, Hkv, Sq, Skv, 128, seed=seed)
-    return tuple((t.float() * spread).to(torch.float8_e4m3fn) for t in (q, k, v))
+def _inputs(B, H, Hkv, Sq, Skv, seed, spread=1.0, sigma=1.0, device="cpu"):
+    q, k, v = synth.qkv(B, H, Hkv, Sq, Skv, 128, seed=seed, sigma=sigma, device=device)
+    return tuple((t.float() * spread).to(torch.float8_e4m3fn).cpu() for t in (q, k, v))
 
 
 def _check(q8, k8, v8, o, lse, dq, dk, dv, scale, rows=None, **mods):
@@ -52,10 +52,13 @@ def _check(q8, k8, v8, o, lse, dq, dk, dv, scale, rows=None, **mods):
     else:
         rows = np.asarray(rows)
         b_idx = rows // (H * Sq)
-        h_idx = (rows // Sq) % H
-        av_rows = av[b_idx, h_idx // G]                         # [n, Skv, D]
-        bound = dv * (2.0 ** -4 * np.einsum("nj,njd->nd", P, av_rows)
-                      + 2.0 ** -16 * np.einsum("nj,njd->nd", (P > 0).astype(np.float64), av_rows))
+        hk_idx = ((rows // Sq) % H) // G
+        bound = np.zeros((rows.size, D))
+        for b in np.unique(b_idx):                              # one product per (batch, kv head)
+            for hk in np.unique(hk_idx[b_idx == b]):
+                sel = (b_idx == b) & (hk_idx == hk)
+                Pg = P[sel]
+                bound[sel] = dv * (2.0 ** -4 * (Pg @ av[b, hk]) + 2.0 ** -16 * ((Pg > 0).astype(np.float64) @ av[b, hk]))
         got = o.reshape(-1, D)[torch.as_tensor(rows, device=o.device)].float().cpu().numpy().astype(np.float64)
         lg = lse.reshape(-1)[torch.as_tensor(rows, device=lse.device)].cpu().numpy().astype(np.float64)
         ro, rl = ro.reshape(got.shape), rl.reshape(lg.shape)
@@ -112,13 +115,43 @@ def test_peaked_scores_wide_range():
     _check(q8, k8, v8, o, lse, 1.0, 1.0, 1.0, 0.125, mask_mod="causal")
 
 
-def test_mha_2048_sampled():
+def _sampled_rows(B, H, S, n, seed, fixed):
+    """n seeded random rows plus the fixed (b, h, i) rows, as flat indices."""
+    rng = np.random.default_rng(seed)
+    pick = set(rng.choice(B * H * S, n, replace=False).tolist())
+    pick.update((b * H + h) * S + i for b, h, i in fixed if i < S)
+    return np.array(sorted(pick), dtype=np.int64)
+
+
+@pytest.mark.parametrize("mods", [dict(mask_mod="causal"), dict()], ids=["causal", "no_mod"])
+def test_mha_2048_sampled(mods):
+    """B2 H32 S2048: 2048 seeded rows plus the first and last rows of the first and last
+    query-tile pairs."""
     fa = _fa()
     B, H, S = 2, 32, 2048
-    q8, k8, v8 = _inputs(B, H, H, S, S, seed=100)
-    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), descale_q=0.5, descale_k=0.5, descale_v=2.0,
-                        mask_mod="causal")
+    q8, k8, v8 = _inputs(B, H, H, S, S, seed=100, device="cuda")
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), descale_q=0.5, descale_k=0.5, descale_v=2.0, **mods)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(101)
-    rows = np.sort(rng.choice(B * H * S, 96, replace=False))
-    _check(q8, k8, v8, o, lse, 0.5, 0.5, 2.0, 1.0 / math.sqrt(128), rows=rows, mask_mod="causal")
+    fixed = [(0, 0, 0), (0, 0, 127), (0, 0, 128), (0, 0, 255), (0, 0, 256), (1, 31, 1792), (1, 31, 2047),
+             (1, 7, 1023), (1, 7, 1024)]
+    rows = _sampled_rows(B, H, S, 2048, 101, fixed)
+    _check(q8, k8, v8, o, lse, 0.5, 0.5, 2.0, 1.0 / math.sqrt(128), rows=rows, **mods)
+
+
+@pytest.mark.parametrize("mods", [dict(), dict(mask_mod="causal"), dict(score_mod="alibi"),
+                                  dict(mask_mod="sliding_window", window=1024)],
+                         ids=["no_mod", "causal", "alibi", "window1024"])
+def test_long_8192_sampled(mods):
+    """The long-context shape (B2 H32 S8192, N(0, 0.5^2) rounded to e4m3) on 2048 seeded
+    rows plus rows 0, 127, 128, 8191, the window edges and the first/last tile pairs."""
+    fa = _fa()
+    B, H, S = 2, 32, 8192
+    q8, k8, v8 = _inputs(B, H, H, S, S, seed=102, sigma=0.5, device="cuda")
+    scale = 1.0 / math.sqrt(128)
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), scale=scale, **mods)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    fixed = [(0, 0, 0), (0, 0, 127), (0, 0, 128), (0, 0, 255), (0, 0, 256), (1, 31, 8191), (1, 31, 7936),
+             (0, 17, 1023), (0, 17, 1024), (0, 17, 1025), (1, 2, 4095)]
+    rows = _sampled_rows(B, H, S, 2048, 103, fixed)
+    _check(q8, k8, v8, o, lse, 1.0, 1.0, 1.0, scale, rows=rows, **mods)

@@ -59,8 +59,9 @@ def test_mha_2048(case):
     B, H, S, D = 2, 32, 2048, 128
     q, k, v = synth.qkv(B, H, H, S, S, D, seed=synth.case_seed(1, 0), device="cuda")
     mods = CASES.get(case, dict(score_mod="none", mask_mod="sliding_window", window=256))
-    rows = sample_rows(B, H, S, 384, seed=7, must=[(0, 0, 0), (0, 0, 127), (0, 0, 128), (1, 31, 2047),
-                                                    (1, 5, 255), (1, 5, 256), (0, 9, 1000)])
+    rows = sample_rows(B, H, S, 2048, seed=7, must=[(0, 0, 0), (0, 0, 127), (0, 0, 128), (1, 31, 2047),
+                                                     (1, 5, 255), (1, 5, 256), (0, 9, 1000), (1, 31, 1792),
+                                                     (0, 4, 1023), (0, 4, 1024)])
     _run(q, k, v, 1.0 / math.sqrt(D), rows=rows, **mods)
 
 
@@ -118,8 +119,12 @@ def test_long_8192(case):
     B, H, S, D = 2, 32, 8192, 128
     q, k, v = synth.qkv(B, H, H, S, S, D, seed=synth.case_seed(4, 0), sigma=0.5, device="cuda")
     mods = CASES.get(case, dict(score_mod="none", mask_mod="sliding_window", window=1024))
-    rows = sample_rows(B, H, S, 96, seed=44, must=[(0, 0, 0), (0, 0, 127), (0, 0, 128), (1, 31, 8191),
-                                                   (0, 17, 1023), (0, 17, 1024), (1, 2, 4095)])
+    # 2048 seeded rows plus rows 0, 127, 128, 8191, the window edges (1023/1024/1025 for
+    # W = 1024), and the first and last rows of the first and last query-tile pairs
+    rows = sample_rows(B, H, S, 2048, seed=44, must=[(0, 0, 0), (0, 0, 127), (0, 0, 128), (0, 0, 255),
+                                                     (0, 0, 256), (1, 31, 8191), (1, 31, 7936), (1, 31, 8064),
+                                                     (0, 17, 1023), (0, 17, 1024), (0, 17, 1025),
+                                                     (1, 2, 4095), (1, 2, 4096)])
     _run(q, k, v, 1.0 / math.sqrt(D), rows=rows, **mods)
 
 
