@@ -182,10 +182,12 @@ size_t decode_ws_bytes(int B, int H, int cap, int D, int split) {
   return ((o_bytes + 255) & ~static_cast<size_t>(255)) + rows * ns * sizeof(float);
 }
 
-// The split size a decode uses: the caller's, or the library's choice.
-int decode_split_for(const flex_decode_params_t* dp) {
+// The split size a decode uses: the caller's, or the library's choice.  Measured on B200
+// (B16 H32 cap 8192 D128 f16): 128-position splits stream 1.5-2 % faster with one query
+// head per kv head; with grouped heads the tensor-core kernel is 2-16 % slower at 128.
+int decode_split_for(const flex_decode_params_t* dp, int G) {
   if (dp && dp->split_size != 0) return dp->split_size;
-  return kChunkDefault;
+  return G == 1 ? kChunkMin : kChunkMax;
 }
 
 constexpr unsigned kStatusSelftestTimeout = 8u;
@@ -498,7 +500,7 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
   if (!q || !k_cache || !v_cache || !kv_len || !o) return FLEX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Hkv < 1 || cap < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
-  const int split = decode_split_for(dp);
+  const int split = decode_split_for(dp, H / Hkv);
   if (split != 128 && split != 256) return FLEX_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
   if (dtype != FLEX_DTYPE_BF16 && dtype != FLEX_DTYPE_F16) return FLEX_ERR_UNSUPPORTED;

@@ -26,7 +26,6 @@ namespace flexattn {
 
 constexpr int kChunkMin = 128;        // cache positions per split: the two sizes built
 constexpr int kChunkMax = 256;
-constexpr int kChunkDefault = 256;
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr unsigned kStatusBadKvLen = 1u;

@@ -12,6 +12,8 @@
 //   warp 0      MMA issuer (one thread): S_k = Q_k K_j^T and O_k += P_k V_j with tcgen05,
 //               accumulators in tensor memory.  It is warp 0 so that the warp scheduler of
 //               its sub-partition, shared with two busy softmax warps, serves it first.
+//               Block-mask kernels have a second issuer in warp 2: warp 0 then issues for
+//               query tile 0 only and warp 2 for tile 1 (fwd_two_issuers below).
 //   warp 1      TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory slots
 //   warps 2-3   idle (they only give their registers to the softmax warpgroups)
 //   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1: each thread owns one
@@ -28,7 +30,11 @@
 // that query tile.  The sets live in shared memory as bitmaps built at the start.
 // Key tiles are visited from the last to the first.  With t counting steps, the MMA order
 // S0(t0) S1(t0) | PV0(t) S0(t+1) PV1(t) S1(t+1) | ... lets one softmax warpgroup work
-// while the tensor core runs the other tile's matmuls.
+// while the tensor core runs the other tile's matmuls.  With two issuers each runs
+// S_k(t0) | PV_k(t) S_k(t+1) | ... for its tile; a K/V slot is then freed when both have
+// arrived on its empty barrier (count 2), and an issuer whose tile skips a step still
+// waits for that step's slots to be filled before it arrives, so it can never arrive for
+// a slot's next use before the other issuer has arrived for the current one.
 //
 // Tensor memory (512 columns x 128 lanes): S0 [0,128) S1 [128,256) O0 [256,256+D)
 // O1 [384,384+D); P_k aliases the first 64 columns of S_k (two 16-bit values per column).
@@ -51,7 +57,8 @@ namespace flexattn {
 constexpr int kBM = 128;        // query rows per tile (tcgen05 M)
 constexpr int kBN = 128;        // keys per tile
 constexpr int kFwdThreads = 384;
-constexpr int kMmaWarp = 0;
+constexpr int kMmaWarp = 0;   // issuer of query tile 0
+constexpr int kMmaWarp1 = 2;  // issuer of query tile 1
 constexpr int kTmaWarp = 1;
 constexpr int kSoftmaxWarp0 = 4;        // warps 4-7: query tile 0, warps 8-11: query tile 1
 constexpr uint32_t kSoftmaxRegs = 200;  // per thread, softmax warpgroups after setmaxnreg
@@ -61,7 +68,26 @@ constexpr uint32_t kAuxRegs = 96;       // per thread, producer/MMA warpgroup af
 static_assert(256 * kSoftmaxRegs + 128 * kAuxRegs <= (65536 / kFwdThreads) / 8 * 8 * kFwdThreads,
               "setmaxnreg split exceeds the registers the block is launched with");
 static_assert(2 * kSoftmaxRegs + kAuxRegs <= 512, "per sub-partition register file exceeded");
-constexpr int kEmuPairsPerHalf = 0;     // of 32 column pairs per 64-column half run on the FMA pipe
+// Of the 32 column pairs of each 64-column half, how many take 2^x from the polynomial on
+// the FMA pipe instead of MUFU ex2 (spread evenly over the half).
+#ifndef FLEX_FWD_EMU_PAIRS
+#define FLEX_FWD_EMU_PAIRS 0
+#endif
+constexpr int kEmuPairsPerHalf = FLEX_FWD_EMU_PAIRS;
+__host__ __device__ constexpr bool emu_pair(int i) { return (i * kEmuPairsPerHalf) % 32 < kEmuPairsPerHalf; }
+// MMA issuers: one thread for both query tiles, or one per tile.  One issuer finishes a
+// tile's P.V and its next S back to back, which keeps each softmax warpgroup's wait for
+// its next S short; two issuers interleave both tiles' products and hide each other's
+// barrier probes, which pays when steps often visit one tile only (block masks).
+// Measured on B200: one issuer 1.45x faster on dense work, two 1.2x faster on random
+// half-dense block masks.  0 = one issuer everywhere, 1 = two for block-mask kernels,
+// 2 = two everywhere.
+#ifndef FLEX_FWD_TWO_ISSUERS
+#define FLEX_FWD_TWO_ISSUERS 1
+#endif
+constexpr bool fwd_two_issuers(bool blocks) {
+  return FLEX_FWD_TWO_ISSUERS == 2 || (FLEX_FWD_TWO_ISSUERS == 1 && blocks);
+}
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
@@ -118,8 +144,8 @@ struct FwdSmem {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  // barriers: q, full[NS], empty[NS], s_full[2], p_half[2][2], o_full[2], drain; then tmem addr
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 4 + 2 + 1;
+  // barriers: q, full[NS], empty[NS], s_full[2], p_half[2][2], o_full[2], drain[2]; then tmem addr
+  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 4 + 2 + 2;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   // step records (kRec*): one per key/value slot, plus the first step's
   static constexpr int kRecOff = kTmemPtrOff + 16;
@@ -212,6 +238,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using L = FwdSmem<D, BLOCKS, is_doc_mask(MASK)>;
   constexpr int NS = L::kSlots;
+  constexpr bool kTwoIssuers = fwd_two_issuers(BLOCKS);
   constexpr int kChunks = D / 64;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);
@@ -228,7 +255,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   auto bar_s = [&](int k) { return sbase + L::kBarOff + 8u * (1 + 2 * NS + k); };
   auto bar_p = [&](int k, int half) { return sbase + L::kBarOff + 8u * (3 + 2 * NS + 2 * k + half); };
   auto bar_o = [&](int k) { return sbase + L::kBarOff + 8u * (7 + 2 * NS + k); };
-  const uint32_t bar_drain = sbase + L::kBarOff + 8u * (9 + 2 * NS);
+  auto bar_drain = [&](int k) { return sbase + L::kBarOff + 8u * (9 + 2 * NS + k); };
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
   uint32_t* rec_smem = reinterpret_cast<uint32_t*>(sgen + L::kRecOff);  // [NS] per V slot, [NS] first
@@ -371,7 +398,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(bar_q, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
+      mbar_init(bar_empty(s), kTwoIssuers ? 2 : 1);  // one arrival per issuer and use
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar_s(k), 1);
@@ -379,7 +406,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar_p(k, 1), kBM);
       mbar_init(bar_o(k), 1);
     }
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_drain(0), 1);
+    mbar_init(bar_drain(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -458,8 +486,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusFwdTimeout,
                   kWaitTimeoutNs);
       mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
-    } else if (warp == kMmaWarp && lane == 0 && any_work) {
-      // ============================================================ MMA issuer
+    } else if (!kTwoIssuers && warp == kMmaWarp && lane == 0 && any_work) {
+      // ============================================================ MMA issuer (both tiles)
       bool ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
       tc_fence_after();
       int np[2] = {0, 0};
@@ -559,8 +587,109 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) *abort_flag = 1;
       // Drain: all MMAs this thread issued have completed before TMEM is released.
-      mma_commit(bar_drain);
-      mbar_wait(bar_drain, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+      mma_commit(bar_drain(0));
+      mbar_wait(bar_drain(0), 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+    } else if (kTwoIssuers && (warp == kMmaWarp || warp == kMmaWarp1) && lane == 0 && any_work) {
+      // ============================================================ MMA issuer of tile k
+      // (k a compile-time constant in each of the two copies below)
+      auto issuer = [&](auto kc) {
+      constexpr int k = decltype(kc)::value;
+      constexpr uint32_t in_bit = k ? kRecIn1 : kRecIn0, pre_bit = k ? kRecPre1 : kRecPre0;
+      constexpr uint32_t last_bit = k ? kRecLast1 : kRecLast0;
+      bool ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+      tc_fence_after();
+      // descriptor of chunk 0 / k-step 0; k-step kk adds ((kk/4)*chunk + (kk%4)*32) >> 4
+      const uint64_t aq = smem_desc(q_smem(k), 16, 1024, kSwizzle128B);
+      const uint32_t t_s = tmem + 128u * k, t_o = tmem + 256u + 128u * k;
+      auto issue_s = [&](int slot) {
+        const uint64_t bk = smem_desc(kv_smem(slot), 16, 1024, kSwizzle128B);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk / 4) * L::kChunkBytes + (kk % 4) * 32) >> 4);
+          mma_ss(t_s, aq + off, bk + off, kIdescS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int slot, bool acc, int kk0, int kk1) {
+        const uint64_t bv = smem_desc(kv_smem(slot), L::kChunkBytes, 1024, kSwizzle128B);
+#pragma unroll
+        for (int kk = kk0; kk < kk1; ++kk)
+          mma_ts(t_o, t_s + 8u * kk, bv + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      // s_ready: S_k of this step was issued during the previous one (its K already
+      // waited for: k_ready); np: P.V steps done (the parity of the P barriers).
+      bool s_ready = false, k_ready = false, started = false;
+      int np = 0;
+      uint32_t rec = rec_smem[NS];  // published with the Q barrier
+      for (int t = 0; !(rec & kRecEnd) && ok; ++t) {
+        const int rK = 2 * t, rV = rK + 1;
+        const int sK = rK % NS, sV = rV % NS;
+        const bool in = rec & in_bit;
+        if (!k_ready && !mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+                                   kStatusFwdTimeout, kWaitTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        k_ready = false;
+        if (in) {
+          tc_fence_after();
+          if (!s_ready) {
+            issue_s(sK);
+            mma_commit(bar_s(k));
+          }
+          s_ready = false;
+          mma_commit(bar_empty(sK));  // K_j is free once this thread's S_k(j) has run
+        } else {
+          mbar_arrive(bar_empty(sK));  // this tile skips the step: the slot was filled, release it
+        }
+        if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status, kStatusFwdTimeout,
+                       kWaitTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
+        if (!in) {
+          mbar_arrive(bar_empty(sV));
+          rec = next_rec;
+          continue;
+        }
+        const uint32_t par = static_cast<uint32_t>(np) & 1u;
+        for (int half = 0; half < 2 && ok; ++half) {
+          if (!mbar_wait(bar_p(k, half), par, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(sV, started, 4 * half, 4 * half + 4);
+        }
+        if (!ok) break;
+        started = true;
+        ++np;
+        if (rec & pre_bit) {
+          const int rK2 = rK + 2;  // K of the next step
+          if (!mbar_wait(bar_full(rK2 % NS), static_cast<uint32_t>(rK2 / NS) & 1u, p.status, kStatusFwdTimeout,
+                         kWaitTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          k_ready = true;
+          issue_s(rK2 % NS);
+          mma_commit(bar_s(k));
+          s_ready = true;
+        } else if (rec & last_bit) {
+          mma_commit(bar_o(k));
+        }
+        mma_commit(bar_empty(sV));
+        rec = next_rec;
+      }
+      if (!ok) *abort_flag = 1;
+      // Drain: all MMAs this thread issued have completed before TMEM is released.
+      mma_commit(bar_drain(k));
+      mbar_wait(bar_drain(k), 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+      };
+      if (warp == kMmaWarp) issuer(std::integral_constant<int, 0>{});
+      else issuer(std::integral_constant<int, 1>{});
     }
   } else {
     regs_inc<kSoftmaxRegs>();
@@ -708,7 +837,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const int c = 64 * half + 2 * i;
           const uint64_t x2 = fma2(pack2(s[c], s[c + 1]), sc2, nm2);
           uint64_t e2;
-          if (i >= 32 - kEmuPairsPerHalf) {
+          if (emu_pair(i)) {
             e2 = exp2_poly2(x2);
           } else {
             float x0, x1;

@@ -367,10 +367,60 @@ def main():
 PROTOCOL = dict(warmup=10, samples=12, iters=100)
 
 
+class NvmlClockPoll:
+    """SM clock of this process's GPU, read through NVML by a background thread every
+    10 ms while a measurement runs (median over the samples; None without NVML)."""
+
+    def __init__(self):
+        self.handle, self.vals, self.thread, self.stop_flag = None, [], None, False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        except Exception:  # NVML missing or the device not found: no clock record
+            self.handle = None
+
+    def _run(self):
+        while not self.stop_flag:
+            try:
+                self.vals.append(self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM))
+            except Exception:
+                return
+            time.sleep(0.01)
+
+    def __enter__(self):
+        import threading
+        if self.handle is not None:
+            self.vals, self.stop_flag = [], False
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join()
+            self.thread = None
+
+    def median(self):
+        return statistics.median(self.vals) if self.vals else None
+
+
+_CLOCKS = None
+
+
 def _time_stats(fn, samples=None, iters=None, warm=None):
     """Seconds per call: mean, std and coefficient of variation over `samples` samples,
-    each the CUDA-event time of `iters` back-to-back calls divided by `iters`."""
+    each the CUDA-event time of `iters` back-to-back calls divided by `iters`; plus the
+    median SM clock seen meanwhile (long runs settle under the board's power cap)."""
     import torch
+    global _CLOCKS
+    if _CLOCKS is None:
+        _CLOCKS = NvmlClockPoll()
     samples = samples or PROTOCOL["samples"]
     iters = iters or PROTOCOL["iters"]
     warm = PROTOCOL["warmup"] if warm is None else warm
@@ -378,22 +428,24 @@ def _time_stats(fn, samples=None, iters=None, warm=None):
         fn()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(samples + 1)]
-    ev[0].record()
-    for s in range(samples):
-        for _ in range(iters):
-            fn()
-        ev[s + 1].record()
-    torch.cuda.synchronize()
+    with _CLOCKS:
+        ev[0].record()
+        for s in range(samples):
+            for _ in range(iters):
+                fn()
+            ev[s + 1].record()
+        torch.cuda.synchronize()
     per = [ev[s].elapsed_time(ev[s + 1]) / iters / 1e3 for s in range(samples)]
     mean = statistics.fmean(per)
     std = statistics.stdev(per) if len(per) > 1 else 0.0
     return {"mean": mean, "std": std, "cv_pct": 100.0 * std / mean if mean > 0 else 0.0, "samples": samples,
-            "iters": iters}
+            "iters": iters, "sm_mhz": _CLOCKS.median(), "min_us": min(per) * 1e6}
 
 
 def _case_row(st, flops=None, key="tflops"):
     """A per-case row: time in us with its spread, and TFLOPS from the mean time."""
-    row = {"us": st["mean"] * 1e6, "std_us": st["std"] * 1e6, "cv_pct": st["cv_pct"]}
+    row = {"us": st["mean"] * 1e6, "std_us": st["std"] * 1e6, "cv_pct": st["cv_pct"], "min_us": st["min_us"],
+           "sm_mhz": st["sm_mhz"]}
     if flops is not None:
         row[key] = flops / st["mean"] / 1e12
     return row

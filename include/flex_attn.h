@@ -238,7 +238,8 @@ flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const v
 /*
  * flex_decode_params_t -- optional settings of one decode call (NULL = all defaults).
  *   split_size: cache positions per split of the split-KV decode: 0 = the library's
- *     choice, else 128 or 256 (FLEX_ERR_INVALID_ARG otherwise).  The result does not
+ *     choice (128 when H == Hkv, else 256), else 128 or 256 (FLEX_ERR_INVALID_ARG
+ *     otherwise).  The result does not
  *     depend on it beyond rounding (the combine is exact in real arithmetic); smaller
  *     splits give more parallel work for short sequences and need more workspace.
  *   status_out: per-call device status word, as in flex_mod_params_t (NULL = the shared

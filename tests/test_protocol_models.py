@@ -2,15 +2,15 @@
 
 Each model restates, role by role, the waits, arrivals, commits, tensor-core products and
 copies of one kernel as written in csrc/flex_fwd_sm100.cuh (flex_fwd_kernel: TMA producer,
-one MMA-issuing thread, two softmax warpgroups) and csrc/flex_bwd_sm100.cuh (bwd_dq_kernel
+one MMA-issuing thread per query tile, two softmax warpgroups) and csrc/flex_bwd_sm100.cuh (bwd_dq_kernel
 with its separate K and V rings; bwd_dkdv_kernel with its query-half pipelining).
 tests/protocol_model.py runs them under many random schedules with the hardware's
 phase-parity rule for mbarrier waits and checks that no schedule deadlocks and that every
 product and every element-wise pass reads the tile it expects (a slot or tensor-memory
 region overwritten too early shows up as a stale tag).  Planted mistakes (a K slot
 released before dQ has read it, a Q/dO slot released after the first query half, a
-second issuer releasing skipped slots without waiting) must be caught, which pins the
-checker.  The models check ordering only, not memory visibility between proxies.
+second issuer releasing skipped slots without waiting, slots released by the first of two
+issuers) must be caught, which pins the checker.  The models check ordering only, not memory visibility between proxies.
 """
 import random
 
@@ -32,15 +32,18 @@ class _Model:
 
 # ----------------------------------------------------------------------------- forward
 
-def fwd_roles(sets, NS, issuers="one"):
+def fwd_roles(sets, NS, issuers="two"):
     """Two query tiles with key-tile sets `sets` (descending), an NS-slot K/V ring.
-    issuers: "one" (the kernel), or "two_naive" (one issuer per tile, a skipped step's
-    slots released without waiting for them: a planted mistake)."""
+    issuers: "two" (the kernel: one MMA-issuing thread per query tile, each waiting for
+    every use of a slot before releasing it, even on steps its tile skips), "one" (the
+    earlier single issuer), or the planted mistakes "two_naive" (a skipped step's slots
+    released without waiting for them) and "two_count1" (slots released by whichever
+    issuer finishes first: empty barriers expecting one arrival)."""
     m = _Model()
     two = issuers != "one"
     bar_q = m.bar("q")
     full = [m.bar(f"full{s}") for s in range(NS)]
-    empty = [m.bar(f"empty{s}", 2 if two else 1) for s in range(NS)]
+    empty = [m.bar(f"empty{s}", 2 if two and issuers != "two_count1" else 1) for s in range(NS)]
     bar_s = [m.bar("s0"), m.bar("s1")]
     bar_p = [[m.bar(f"p{k}{h}") for h in range(2)] for k in range(2)]
     bar_o = [m.bar("o0"), m.bar("o1")]
@@ -58,13 +61,16 @@ def fwd_roles(sets, NS, issuers="one"):
         return r
 
     def producer():
+        yield ("write", {("rec", NS): ("rec", 0)})  # the first step's record, with Q
         yield ("expect", bar_q, TB)
         yield ("tma", ("Q",), "Q", bar_q, TB)
         r = 0
-        for j in steps:
+        for t, j in enumerate(steps):
             for which in ("K", "V"):
                 s = r % NS
                 yield ("wait", empty[s], ((r // NS) & 1) ^ 1)
+                if which == "V":  # the next step's record travels with V of this step
+                    yield ("write", {("rec", s): ("rec", t + 1)})
                 yield ("expect", full[s], TB)
                 yield ("tma", ("slot", s), (which, j), full[s], TB)
                 r += 1
@@ -83,6 +89,7 @@ def fwd_roles(sets, NS, issuers="one"):
 
     def issuer_one():
         yield ("wait", bar_q, 0)
+        yield ("read", [(("rec", NS), ("rec", 0))])
         s_ready, np_ = [False, False], [0, 0]
         for t, j in enumerate(steps):
             rK, rV = 2 * t, 2 * t + 1
@@ -97,6 +104,7 @@ def fwd_roles(sets, NS, issuers="one"):
                         yield ("commit", bar_s[k])
             yield ("commit", empty[sK])
             yield ("wait", full[sV], (rV // NS) & 1)
+            yield ("read", [(("rec", sV), ("rec", t + 1))])
             next_k_ready = False
             for k in range(2):
                 if k not in r:
@@ -119,6 +127,50 @@ def fwd_roles(sets, NS, issuers="one"):
             yield ("commit", empty[sV])
         yield ("commit", drain[0])
         yield ("wait", drain[0], 0)
+
+    def issuer_two(k):
+        """One issuer per query tile.  On a step its tile skips it still waits for the fill of
+        both slots (and reads the record) before arriving on their empty barriers, so it can
+        never arrive for a slot's next use before the other issuer has arrived for this one."""
+        yield ("wait", bar_q, 0)
+        yield ("read", [(("rec", NS), ("rec", 0))])
+        s_ready, k_ready, np_ = False, False, 0
+        for t, j in enumerate(steps):
+            rK, rV = 2 * t, 2 * t + 1
+            sK, sV = rK % NS, rV % NS
+            r = rec(t)
+            visit = k in r
+            if not k_ready:
+                yield ("wait", full[sK], (rK // NS) & 1)
+            k_ready = False
+            if visit:
+                if not s_ready:
+                    yield S(k, j, sK)
+                    yield ("commit", bar_s[k])
+                s_ready = False
+                yield ("commit", empty[sK])
+            else:
+                yield ("arrive", empty[sK])
+            yield ("wait", full[sV], (rV // NS) & 1)
+            yield ("read", [(("rec", sV), ("rec", t + 1))])
+            if not visit:
+                yield ("arrive", empty[sV])
+                continue
+            for half in range(2):
+                yield ("wait", bar_p[k][half], np_ & 1)
+                yield PV(k, j, half, sV, 2 * np_ + half)
+            np_ += 1
+            if r[k] == "pre":
+                yield ("wait", full[(rK + 2) % NS], ((rK + 2) // NS) & 1)
+                k_ready = True
+                yield S(k, steps[t + 1], (rK + 2) % NS)
+                yield ("commit", bar_s[k])
+                s_ready = True
+            elif r[k] == "last":
+                yield ("commit", bar_o[k])
+            yield ("commit", empty[sV])
+        yield ("commit", drain[k])
+        yield ("wait", drain[k], 0)
 
     def issuer_naive(k):
         yield ("wait", bar_q, 0)
@@ -167,8 +219,10 @@ def fwd_roles(sets, NS, issuers="one"):
             yield ("read", [(("O", k), 2 * len(sets[k]))])
 
     roles = {"producer": producer(), "sm0": softmax(0), "sm1": softmax(1)}
-    if two:
+    if issuers == "two_naive":
         roles["I0"], roles["I1"] = issuer_naive(0), issuer_naive(1)
+    elif two:
+        roles["I0"], roles["I1"] = issuer_two(0), issuer_two(1)
     else:
         roles["I"] = issuer_one()
     return roles, m.bars
@@ -197,18 +251,25 @@ def _schedules(make, n, seed0=0):
     return bad
 
 
+@pytest.mark.parametrize("issuers", ["two", "one"])
 @pytest.mark.parametrize("NS", [5, 12])
 @pytest.mark.parametrize("kind", ["dense", "causal", "one_empty", "random"])
-def test_forward_protocol(NS, kind):
+def test_forward_protocol(NS, kind, issuers):
     rng = random.Random(NS * 31 + len(kind))
     cases = [_sets(rng, rng.choice([1, 2, 3, 5, 8]), kind) for _ in range(40)]
-    assert _schedules(lambda i: fwd_roles(cases[i], NS), len(cases)) == 0
+    assert _schedules(lambda i: fwd_roles(cases[i], NS, issuers), len(cases)) == 0
 
 
 def test_forward_naive_second_issuer_is_caught():
     rng = random.Random(5)
     cases = [_sets(rng, rng.choice([5, 8, 12]), "one_empty") for _ in range(60)]
     assert _schedules(lambda i: fwd_roles(cases[i], 5, issuers="two_naive"), len(cases)) > 0
+
+
+def test_forward_single_arrival_release_is_caught():
+    rng = random.Random(6)
+    cases = [_sets(rng, rng.choice([3, 5, 8]), "random") for _ in range(60)]
+    assert _schedules(lambda i: fwd_roles(cases[i], 5, issuers="two_count1"), len(cases)) > 0
 
 
 # ----------------------------------------------------------------------------- dQ
