@@ -12,8 +12,9 @@
 //   warp 0      MMA issuer (one thread): S_k = Q_k K_j^T and O_k += P_k V_j with tcgen05,
 //               accumulators in tensor memory.  It is warp 0 so that the warp scheduler of
 //               its sub-partition, shared with two busy softmax warps, serves it first.
-//               Block-mask kernels have a second issuer in warp 2: warp 0 then issues for
-//               query tile 0 only and warp 2 for tile 1 (fwd_two_issuers below).
+//               A block-mask CTA whose steps often visit one query tile only takes a
+//               second issuer in warp 2: warp 0 then issues for query tile 0 and warp 2
+//               for tile 1 (kTwoIssuerShare below).
 //   warp 1      TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory slots
 //   warps 2-3   idle (they only give their registers to the softmax warpgroups)
 //   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1: each thread owns one
@@ -69,7 +70,8 @@ static_assert(256 * kSoftmaxRegs + 128 * kAuxRegs <= (65536 / kFwdThreads) / 8 *
               "setmaxnreg split exceeds the registers the block is launched with");
 static_assert(2 * kSoftmaxRegs + kAuxRegs <= 512, "per sub-partition register file exceeded");
 // Of the 32 column pairs of each 64-column half, how many take 2^x from the polynomial on
-// the FMA pipe instead of MUFU ex2 (spread evenly over the half).
+// the FMA pipe instead of MUFU ex2 (spread evenly over the half).  Measured on B200 at
+// D = 128: 4 of 32 cost 13 %, 8 of 32 cost 19 % on dense work, so none by default.
 #ifndef FLEX_FWD_EMU_PAIRS
 #define FLEX_FWD_EMU_PAIRS 0
 #endif
@@ -78,16 +80,12 @@ __host__ __device__ constexpr bool emu_pair(int i) { return (i * kEmuPairsPerHal
 // MMA issuers: one thread for both query tiles, or one per tile.  One issuer finishes a
 // tile's P.V and its next S back to back, which keeps each softmax warpgroup's wait for
 // its next S short; two issuers interleave both tiles' products and hide each other's
-// barrier probes, which pays when steps often visit one tile only (block masks).
-// Measured on B200: one issuer 1.45x faster on dense work, two 1.2x faster on random
-// half-dense block masks.  0 = one issuer everywhere, 1 = two for block-mask kernels,
-// 2 = two everywhere.
-#ifndef FLEX_FWD_TWO_ISSUERS
-#define FLEX_FWD_TWO_ISSUERS 1
-#endif
-constexpr bool fwd_two_issuers(bool blocks) {
-  return FLEX_FWD_TWO_ISSUERS == 2 || (FLEX_FWD_TWO_ISSUERS == 1 && blocks);
-}
+// barrier probes, which pays when many steps visit one tile only.  Measured on B200 (B2
+// H32 S8192): two issuers are 35 % slower on dense work and 21 % slower on causal block
+// lists, 10-20 % faster on random half-dense block lists.  So analytic masks always use
+// one issuer, and a block-mask CTA takes two when at least a third of its steps visit
+// only one of its two query tiles (decided per CTA from its visit bitmaps).
+constexpr int kTwoIssuerShare = 3;  // two issuers iff kTwoIssuerShare * single-tile steps >= steps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows > 2^8
@@ -238,7 +236,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using L = FwdSmem<D, BLOCKS, is_doc_mask(MASK)>;
   constexpr int NS = L::kSlots;
-  constexpr bool kTwoIssuers = fwd_two_issuers(BLOCKS);
+
   constexpr int kChunks = D / 64;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);
@@ -394,11 +392,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   };
 
   // ---------------------------------------------------------------- setup
+  // Block masks: one MMA issuer or two for this CTA (see kTwoIssuerShare), from the
+  // complete visit bitmaps; the empty barriers count one arrival per issuer and use.
+  volatile int* two_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 8);
+  if constexpr (BLOCKS) __syncthreads();
   if (threadIdx.x == 0) {
+    bool two = false;
+    if constexpr (BLOCKS) {
+      int single = 0, steps = 0;
+      for (int w = 0; w < (p.n_ktiles + 31) / 32; ++w) {
+        const uint32_t a = act_bits(0)[w], c = act_bits(1)[w];
+        single += __popc(a ^ c);
+        steps += __popc(a | c);
+      }
+      two = kTwoIssuerShare * single >= steps && steps > 0;
+    }
+    *two_flag = two ? 1 : 0;
     mbar_init(bar_q, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), kTwoIssuers ? 2 : 1);  // one arrival per issuer and use
+      mbar_init(bar_empty(s), two ? 2 : 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar_s(k), 1);
@@ -424,6 +437,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
+  const bool two_issuers = BLOCKS && *two_flag != 0;
   const bool act0 = cursor(0).cur >= 0, act1 = cursor(1).cur >= 0;
   const bool any_work = act0 || act1;
 
@@ -486,7 +500,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusFwdTimeout,
                   kWaitTimeoutNs);
       mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
-    } else if (!kTwoIssuers && warp == kMmaWarp && lane == 0 && any_work) {
+    } else if (!two_issuers && warp == kMmaWarp && lane == 0 && any_work) {
       // ============================================================ MMA issuer (both tiles)
       bool ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
       tc_fence_after();
@@ -589,7 +603,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // Drain: all MMAs this thread issued have completed before TMEM is released.
       mma_commit(bar_drain(0));
       mbar_wait(bar_drain(0), 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
-    } else if (kTwoIssuers && (warp == kMmaWarp || warp == kMmaWarp1) && lane == 0 && any_work) {
+    } else if (two_issuers && (warp == kMmaWarp || warp == kMmaWarp1) && lane == 0 && any_work) {
       // ============================================================ MMA issuer of tile k
       // (k a compile-time constant in each of the two copies below)
       auto issuer = [&](auto kc) {
