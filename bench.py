@@ -38,19 +38,28 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram read+write bytes per launch from ncu, keyed by the hash of the kernel sources
 # they were measured on (a changed kernel reports null until it is captured again)
 MEASURED_TRAFFIC = {
-    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 402,840,064 B read +
-    # 115,957,248 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192_dram.md)
-    "ec937b6aa1d4e760": 518797312,
+    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 402,710,784 B read +
+    # 113,622,272 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192.md)
+    "54190ee8878a9ab1": 516333056,
+}
+MEASURED_DECODE_TRAFFIC = {
+    # decode_split_kernel<128,f16,1,128>, B16 H32 Hkv32 cap8192, the bench's lengths and
+    # mask: 868,650,496 B read + 5,636,608 B written
+    # (profiles/decode_split_kernel_f16_hkv32_bench.md)
+    "cfc6ae7c1e23a6be": 874287104,
 }
 # the forward kernel's sources: the roofline traffic below belongs to that kernel
 KERNEL_SOURCES = ["attention_flex_attn_b200/csrc/flex_fwd_sm100.cuh",
                   "attention_flex_attn_b200/csrc/ptx_sm100.cuh",
                   "attention_flex_attn_b200/csrc/mask_rules.cuh"]
+DECODE_SOURCES = ["attention_flex_attn_b200/csrc/flex_decode.cuh",
+                  "attention_flex_attn_b200/csrc/flex_decode_launch.cu",
+                  "attention_flex_attn_b200/csrc/ptx_sm100.cuh"]
 
 
-def kernel_hash() -> str:
+def kernel_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -238,7 +247,8 @@ def main():
                     help="reference arm: host seconds of oracle work over all warm-up and timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the per-case and e2e measurements")
-    ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "bwd", "fp8", "decode"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "fwd8192", "fwd_blocks", "bwd", "fp8", "decode", "decode_bench"],
+                    default=None,
                     help="run only a few launches of one kernel (for ncu captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -338,7 +348,8 @@ def main():
         "decode": {"gbs": dbytes / dec_avg_s / 1e9, "ms": dec_avg_s * 1e3, "bytes": dbytes,
                    "roofline": {"bound": "hbm", "achieved": dbytes / dec_avg_s / 1e9, "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": dbytes / dec_avg_s / 1e9 / peaks["hbm_gbs"],
-                                "peak_source": peak_kind}},
+                                "traffic": MEASURED_DECODE_TRAFFIC.get(kernel_hash(DECODE_SOURCES)),
+                                "peak_source": peak_kind, "kernel": "decode_split_kernel<128,f16,1,128>"}},
         "fwd_ms": fwd_avg_s * 1e3,
         "fwd_stats": _spread(fwd_ms), "decode_stats": _spread(dec_ms),
         "protocol": "headline step: per-step CUDA events over the K timed steps; cases: "
@@ -680,7 +691,9 @@ def profile_case(which):
     fwd = B2 H32 S4096 D128 bf16 no_mod (192 MiB of Q/K/V); fwd8192 = the full forward
     workload; fwd_blocks = the S4096 inputs with random per-head block lists, half of the
     key blocks of every query tile full; bwd = forward + backward at B2 H32 S4096 D128,
-    no_mod then causal; fp8 = the S4096 inputs rounded to e4m3, 8-bit forward; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache)."""
+    no_mod then causal; fp8 = the S4096 inputs rounded to e4m3, 8-bit forward; decode = B16 H32 Hkv8 cap8192 all-full f16 with mask (537 MB of cache);
+    decode_bench = the benchmark step's decode (B16 H32 Hkv32 cap8192, kv_len ~ U[1, 8192],
+    10 % -inf mask; 2.1 GB of cache)."""
     import torch
     import synth
     import attention_flex_attn_b200 as fa
@@ -712,6 +725,11 @@ def profile_case(which):
         q, k, v = synth.qkv(2, 32, 32, S, S, 128, seed=4000, sigma=0.5, device=dev)
         for _ in range(4):
             fa.fwd(q, k, v)
+    elif which == "decode_bench":
+        _, (qd, kc, vc, lens, mask) = make_inputs(dev)
+        ws = torch.empty(fa.decode_workspace_size(16, 32, 32, 8192, 128), dtype=torch.uint8, device=dev)
+        for _ in range(4):
+            fa.decode(qd, kc, vc, lens, DEC["scale"], mask=mask, workspace=ws)
     else:
         qd = synth.normal_tensor((16, 32, 1, 128), 11, dtype="f16", device=dev)
         kc = synth.normal_tensor((16, 8, 8192, 128), 12, dtype="f16", device=dev)
