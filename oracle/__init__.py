@@ -59,6 +59,9 @@ def _bind(lib):
     lib.oracle_fwd_block_sparse.restype = I
     lib.oracle_bwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, I, P, I64, P, P, P, I]
     lib.oracle_bwd.restype = I
+    lib.oracle_bwd_block_sparse.argtypes = [P, P, P, P, I, I, I, I, I, I, I, D, I, I, I, I, P, P, P, I,
+                                            P, P, P, P, I, I, I, P, I64, P, P, P, I]
+    lib.oracle_bwd_block_sparse.restype = I
     return lib
 
 
@@ -206,6 +209,55 @@ def bwd(q, k, v, dout, scale=None, score_mod="none", mask_mod="none", window=0, 
                         dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(threads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_bwd rejected its arguments (rc={rc})")
+    if groups is None:
+        return dq.reshape(B, H, Sq, D), dk.reshape(B, Hkv, Skv, D), dv.reshape(B, Hkv, Skv, D)
+    return dq, dk, dv
+
+
+def _block_arrays(kv_num, kv_idx, full_num, full_idx, B, H, nq):
+    """The lists broadcast to [B, H, nq(, max_blocks)] int32 (either pair may be None)."""
+    kn, ki, fn, fi = _i32(kv_num), _i32(kv_idx), _i32(full_num), _i32(full_idx)
+    if kn is None and fn is None:
+        raise ValueError("a block mask needs at least one of the partial / full lists")
+    max_blocks = (ki if ki is not None else fi).shape[-1]
+
+    def expand(a, tail):
+        return None if a is None else np.ascontiguousarray(np.broadcast_to(a, (B, H, nq) + tail))
+    return expand(kn, ()), expand(ki, (max_blocks,)), expand(fn, ()), expand(fi, (max_blocks,)), max_blocks
+
+
+def bwd_block_sparse(q, k, v, dout, kv_num, kv_idx, full_num=None, full_idx=None, scale=None,
+                     score_mod="none", mask_mod="none", window=0, offset=0, bm=128, bn=128, groups=None,
+                     threads=None, alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None):
+    """Oracle backward of the block-sparse forward: bwd() with the keep rule of
+    fwd_block_sparse() (lists as there).  Returns (dq, dk, dv) like bwd()."""
+    lib = _load()
+    B, H, Sq, D = q.shape
+    _, Hkv, Skv, _ = k.shape
+    assert tuple(dout.shape) == tuple(q.shape) and dout.dtype == q.dtype
+    slopes, oq, okv, n_docs = _captured(B, H, mask_mod, alibi_slopes, doc_offsets, doc_offsets_kv)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    kn, ki, fn, fi, max_blocks = _block_arrays(kv_num, kv_idx, full_num, full_idx, B, H, -(-Sq // bm))
+    G = H // Hkv
+    if groups is None:
+        g_arr, n = None, B * Hkv
+    else:
+        flat = [g[0] * Hkv + g[1] if isinstance(g, (tuple, list)) else int(g) for g in groups]
+        g_arr = np.ascontiguousarray(np.asarray(flat, dtype=np.int64))
+        n = int(g_arr.size)
+    dq = np.zeros((n, G, Sq, D))
+    dk = np.zeros((n, Skv, D))
+    dv = np.zeros((n, Skv, D))
+    qb, kb, vb, ob = _bits(q), _bits(k), _bits(v), _bits(dout)
+    rc = lib.oracle_bwd_block_sparse(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, ob.ctypes.data, _dtype_code(q),
+                                     B, H, Hkv, Sq, Skv, D, float(scale), SCORE_MODS[score_mod], MASK_MODS[mask_mod],
+                                     int(window), int(offset), _p(slopes), _p(oq), _p(okv), n_docs,
+                                     _p(kn), _p(ki), _p(fn), _p(fi), int(max_blocks), int(bm), int(bn),
+                                     None if g_arr is None else g_arr.ctypes.data, n,
+                                     dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_bwd_block_sparse rejected its arguments (rc={rc})")
     if groups is None:
         return dq.reshape(B, H, Sq, D), dk.reshape(B, Hkv, Skv, D), dv.reshape(B, Hkv, Skv, D)
     return dq, dk, dv

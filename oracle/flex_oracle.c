@@ -43,7 +43,8 @@
  * PyTorch BlockMask convention.  For query tile t = i / BM of (b, h), a key j with
  * block u = j / BN is kept iff j < Skv and (u is in the full list of t, or u is in
  * the partial list of t and mask_mod(i, j) holds).  Unlisted blocks are dropped.
- * Everything else (scale, score_mod, softmax, 0/-inf rows) is the forward above.
+ * Everything else (scale, score_mod, softmax, 0/-inf rows) is the forward above, and
+ * the block-sparse backward is the backward below with this keep rule.
  *
  * Tile map: for a BM x BN grid over (query, key) positions, a tile is
  *   EMPTY(0)   if no element with i < Sq has keep && j < Skv,
@@ -489,13 +490,15 @@ static int run_bwd_pass(bwd_job* base, int64_t n_tasks, int nthreads) {
   return 0;
 }
 
-/* Backward for the (b, hk) groups listed (groups == NULL: all B*Hkv).  dq: [n_groups, G,
- * Sq, D]; dk, dv: [n_groups, Skv, D] (G = H / Hkv query heads per group, in order). */
-int oracle_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout, int dtype,
-               int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
-               int score_mod, int mask_mod, int window, int offset,
-               const double* slopes, const int32_t* off_q, const int32_t* off_kv, int n_docs,
-               const int64_t* groups, int64_t n_groups, double* dq, double* dk, double* dv, int nthreads) {
+/* Backward for the (b, hk) groups listed (groups == NULL: all B*Hkv), with the keep rule
+ * of mask_mod, or of the block lists when blk is given.  dq: [n_groups, G, Sq, D]; dk, dv:
+ * [n_groups, Skv, D] (G = H / Hkv query heads per group, in order). */
+static int bwd_run(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout, int dtype,
+                   int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
+                   int score_mod, int mask_mod, int window, int offset,
+                   const double* slopes, const int32_t* off_q, const int32_t* off_kv, int n_docs,
+                   const block_lists* blk, const int64_t* groups, int64_t n_groups, double* dq, double* dk,
+                   double* dv, int nthreads) {
   if (H <= 0 || Hkv <= 0 || H % Hkv != 0 || Sq <= 0 || Skv <= 0 || D <= 0) return -1;
   if ((mask_mod == OR_MASK_DOC || mask_mod == OR_MASK_DOC_CAUSAL) && (!off_q || !off_kv || n_docs < 0)) return -2;
   int64_t ng = groups ? n_groups : (int64_t)B * Hkv;
@@ -514,6 +517,7 @@ int oracle_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const ui
   J->scale = scale; J->score_mod = score_mod; J->mask_mod = mask_mod;
   J->window = window; J->offset = offset;
   J->cap.slopes = slopes; J->cap.off_q = off_q; J->cap.off_kv = off_kv; J->cap.n_docs = n_docs;
+  J->blk = blk;
   W.dout = dout;
   W.groups = groups ? groups : all;
   W.n_groups = ng;
@@ -536,6 +540,33 @@ int oracle_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const ui
   free(W.delta);
   free(all);
   return rc;
+}
+
+int oracle_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout, int dtype,
+               int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
+               int score_mod, int mask_mod, int window, int offset,
+               const double* slopes, const int32_t* off_q, const int32_t* off_kv, int n_docs,
+               const int64_t* groups, int64_t n_groups, double* dq, double* dk, double* dv, int nthreads) {
+  return bwd_run(q, k, v, dout, dtype, B, H, Hkv, Sq, Skv, D, scale, score_mod, mask_mod, window, offset, slopes,
+                 off_q, off_kv, n_docs, NULL, groups, n_groups, dq, dk, dv, nthreads);
+}
+
+/* Backward of the block-sparse forward: the gradients of the forward whose keep rule is
+ * the block lists' (oracle_fwd_block_sparse).  The lists are laid out as there. */
+int oracle_bwd_block_sparse(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                            int dtype, int B, int H, int Hkv, int Sq, int Skv, int D, double scale,
+                            int score_mod, int mask_mod, int window, int offset,
+                            const double* slopes, const int32_t* off_q, const int32_t* off_kv, int n_docs,
+                            const int32_t* kv_num, const int32_t* kv_idx, const int32_t* full_num,
+                            const int32_t* full_idx, int max_blocks, int BM, int BN,
+                            const int64_t* groups, int64_t n_groups, double* dq, double* dk, double* dv,
+                            int nthreads) {
+  if (BM <= 0 || BN <= 0 || max_blocks < 0 || Sq <= 0) return -1;
+  block_lists L;
+  L.kv_num = kv_num; L.kv_idx = kv_idx; L.full_num = full_num; L.full_idx = full_idx;
+  L.max_blocks = max_blocks; L.BM = BM; L.BN = BN; L.n_qtiles = (Sq + BM - 1) / BM;
+  return bwd_run(q, k, v, dout, dtype, B, H, Hkv, Sq, Skv, D, scale, score_mod, mask_mod, window, offset, slopes,
+                 off_q, off_kv, n_docs, &L, groups, n_groups, dq, dk, dv, nthreads);
 }
 
 /* ---- decode ---------------------------------------------------------------- */

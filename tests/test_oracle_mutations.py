@@ -1,6 +1,6 @@
 """Plants plausible mistakes in copies of the C oracle and checks that the pins in
 test_oracle_pins.py, test_oracle_block_pins.py, test_oracle_mods_pins.py,
-test_oracle_bwd_pins.py and test_oracle_fp8_pins.py catch every one (each mutant must fail at least one pin).
+test_oracle_bwd_pins.py, test_oracle_block_bwd_pins.py and test_oracle_fp8_pins.py catch every one (each mutant must fail at least one pin).
 Everything runs on the CPU against a temporary build; the real oracle is untouched.
 Mutants that leave the mathematics unchanged (e.g. dropping the fully-masked guard,
 which still yields p = 0 and log 0 = -inf) are not listed: no test could tell them apart."""
@@ -12,6 +12,7 @@ import pytest
 import torch
 
 import oracle
+import tests.test_oracle_block_bwd_pins as bbpins
 import tests.test_oracle_block_pins as bpins
 import tests.test_oracle_bwd_pins as bwpins
 import tests.test_oracle_fp8_pins as f8pins
@@ -70,6 +71,7 @@ MUTANTS = [
      "v = ldexp((double)(m + 8), e - 11);    /* (1 + m/8) * 2^(e-7) */"),
     ("e4m3 subnormal scale", "v = ldexp((double)m, -9);              /* subnormal: m/8 * 2^-6 */",
      "v = ldexp((double)m, -10);              /* subnormal: m/8 * 2^-6 */"),
+    ("bwd ignores the block mask", "  J->blk = blk;\n  W.dout = dout;", "  W.dout = dout;"),
     ("bf16 decoded as truncated", "  uint32_t u = ((uint32_t)b) << 16;", "  uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
 ]
 
@@ -110,6 +112,8 @@ CHECKS = [
     (bwpins.test_bwd_single_key_closed_form, {}),
     (bwpins.test_bwd_equals_finite_differences_of_forward, {}),
     (f8pins.test_e4m3_decode_matches_torch, {}),
+    (bbpins.test_block_bwd_equals_autograd, {"mask": "causal", "window": 0, "offset": 0, "score": "alibi",
+                                              "dtype": torch.bfloat16}),
 ]
 
 
