@@ -29,6 +29,7 @@ FLAG_TILE_MAP = 1
 # The symbols include/flex_attn.h declares.
 EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_fwd_fp8_workspace_size", "flex_attn_fwd_fp8",
             "flex_attn_bwd_workspace_size", "flex_attn_bwd",
+            "flex_attn_bwd_block_sparse_workspace_size", "flex_attn_bwd_block_sparse",
             "flex_attn_decode_workspace_size", "flex_attn_decode",
             "flex_attn_decode_noalloc", "flex_attn_mask_eval", "flex_attn_selftest_wait_timeout",
             "flex_attn_tile_sizes", "flex_attn_device_status", "flex_status_string"]
@@ -86,6 +87,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams), I,
                                   P, SZ, P]
     lib.flex_attn_bwd.restype = I
+    lib.flex_attn_bwd_block_sparse_workspace_size.argtypes = [I, I, I, I, I]
+    lib.flex_attn_bwd_block_sparse_workspace_size.restype = SZ
+    lib.flex_attn_bwd_block_sparse.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I,
+                                               ctypes.POINTER(ModParams), ctypes.POINTER(BlockMaskC), I, P, SZ, P]
+    lib.flex_attn_bwd_block_sparse.restype = I
     lib.flex_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
     lib.flex_attn_decode_workspace_size.restype = SZ
     lib.flex_attn_decode.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, I, P, SZ,
@@ -259,6 +265,18 @@ def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None
     Partial blocks apply mask_mod, full blocks only the key-length rule."""
     lib = load_library()
     B, H, Hkv, Sq, Skv, D, scale, o, lse = _fwd_args(q, k, v, scale, return_lse, out, lse_out)
+    bm = _block_mask(kv_num_blocks, kv_indices, full_kv_num_blocks, full_kv_indices, Sq, block_size)
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
+                            doc_offsets_kv, _status_word(status, q.device))
+    rc = lib.flex_attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
+                                        scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
+                                        ctypes.byref(bm), DTYPES[q.dtype], _stream(q.device))
+    _check(rc, "flex_attn_fwd_block_sparse")
+    return o, lse
+
+
+def _block_mask(kv_num_blocks, kv_indices, full_kv_num_blocks, full_kv_indices, Sq, block_size):
+    """BlockMaskC of the lists (int32 CUDA tensors, checked here)."""
     pairs = [(kv_num_blocks, kv_indices, "kv"), (full_kv_num_blocks, full_kv_indices, "full_kv")]
     shape = None
     for num, idx, name in pairs:
@@ -281,13 +299,7 @@ def fwd_block_sparse(q, k, v, kv_num_blocks, kv_indices, full_kv_num_blocks=None
                     shape[3], shape[0], shape[1], int(block_size), int(block_size))
     if shape[2] != -(-Sq // 128):
         raise FlexAttnError(f"block mask has {shape[2]} query tiles, Sq={Sq} needs {-(-Sq // 128)}")
-    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
-                            doc_offsets_kv, _status_word(status, q.device))
-    rc = lib.flex_attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
-                                        scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
-                                        ctypes.byref(bm), DTYPES[q.dtype], _stream(q.device))
-    _check(rc, "flex_attn_fwd_block_sparse")
-    return o, lse
+    return bm
 
 
 def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None, score_mod="none",
@@ -344,6 +356,23 @@ def bwd(q, k, v, o, lse, dout, scale=None, score_mod="none", mask_mod="none", wi
     """Flex-attention backward (flex_attn_bwd): gradients (dq, dk, dv) of sum(dout * o)
     for the forward with the same arguments; o and lse are that forward's outputs.
     dk/dv are [B, Hkv, Skv, D] (summed over the query heads of each group)."""
+    return _bwd(None, q, k, v, o, lse, dout, scale, score_mod, mask_mod, window, offset, alibi_slopes, doc_offsets,
+                doc_offsets_kv, dq, dk, dv, workspace, status)
+
+
+def bwd_block_sparse(q, k, v, o, lse, dout, kv_num_blocks, kv_indices, full_kv_num_blocks=None,
+                     full_kv_indices=None, scale=None, score_mod="none", mask_mod="none", window=0, offset=0,
+                     alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None, dq=None, dk=None, dv=None,
+                     workspace=None, status=None, block_size=128):
+    """Backward of fwd_block_sparse (flex_attn_bwd_block_sparse): the lists and the other
+    arguments as there, o and lse that forward's outputs."""
+    bm = _block_mask(kv_num_blocks, kv_indices, full_kv_num_blocks, full_kv_indices, q.shape[2], block_size)
+    return _bwd(bm, q, k, v, o, lse, dout, scale, score_mod, mask_mod, window, offset, alibi_slopes, doc_offsets,
+                doc_offsets_kv, dq, dk, dv, workspace, status)
+
+
+def _bwd(bm, q, k, v, o, lse, dout, scale, score_mod, mask_mod, window, offset, alibi_slopes, doc_offsets,
+         doc_offsets_kv, dq, dk, dv, workspace, status):
     lib = load_library()
     for t, n in ((o, "o"), (dout, "dout"), (lse, "lse")):
         _cuda_tensor(t, n)
@@ -357,18 +386,21 @@ def bwd(q, k, v, o, lse, dout, scale=None, score_mod="none", mask_mod="none", wi
     dq = dq if dq is not None else torch.empty_like(q)
     dk = dk if dk is not None else torch.empty_like(k)
     dv = dv if dv is not None else torch.empty_like(v)
-    need = bwd_workspace_size(B, H, Sq)
+    need = bwd_workspace_size(B, H, Sq) if bm is None else int(
+        lib.flex_attn_bwd_block_sparse_workspace_size(B, H, Hkv, Sq, Skv))
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     elif workspace.device != q.device or not workspace.is_contiguous():
         raise FlexAttnError("workspace must be a contiguous tensor on q's device")
     mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, doc_offsets,
                             doc_offsets_kv, _status_word(status, q.device))
-    rc = lib.flex_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                           B, H, Hkv, Sq, Skv, D, scale, score, MASK_MODS[mask_mod], ctypes.byref(mp),
-                           DTYPES[q.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(),
-                           _stream(q.device))
-    _check(rc, "flex_attn_bwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+            B, H, Hkv, Sq, Skv, D, scale, score, MASK_MODS[mask_mod], ctypes.byref(mp))
+    tail = (DTYPES[q.dtype], _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(q.device))
+    if bm is None:
+        _check(lib.flex_attn_bwd(*args, *tail), "flex_attn_bwd")
+    else:
+        _check(lib.flex_attn_bwd_block_sparse(*args, ctypes.byref(bm), *tail), "flex_attn_bwd_block_sparse")
     return dq, dk, dv
 
 

@@ -234,6 +234,38 @@ MaskArgs mask_args(int mask, const flex_mod_params_t& mp, int Skv) {
   return m;
 }
 
+// A block mask's lists: present in pairs, shapes that broadcast over (B, H), 128 x 128
+// blocks, key tiles the per-CTA bitmaps can name, 4-byte aligned.
+flex_status_t check_block_mask(const flex_block_mask_t& bm, int B, int H, int Sq, int Skv) {
+  const bool has_part = bm.kv_num_blocks != nullptr, has_full = bm.full_kv_num_blocks != nullptr;
+  if (has_part != (bm.kv_indices != nullptr) || has_full != (bm.full_kv_indices != nullptr))
+    return FLEX_ERR_INVALID_ARG;
+  if (!has_part && !has_full) return FLEX_ERR_INVALID_ARG;
+  if (bm.max_blocks < 1 || (bm.batch != 1 && bm.batch != B) || (bm.heads != 1 && bm.heads != H))
+    return FLEX_ERR_INVALID_ARG;
+  if (bm.q_block_size != kBM || bm.kv_block_size != kBN) return FLEX_ERR_UNSUPPORTED;
+  if ((Skv + kBN - 1) / kBN > kMaxBlockKeyTiles) return FLEX_ERR_UNSUPPORTED;
+  const int64_t idx_elems = static_cast<int64_t>(bm.batch) * bm.heads * ((Sq + kBM - 1) / kBM) * bm.max_blocks;
+  if (idx_elems > 0x7fffffffLL) return FLEX_ERR_UNSUPPORTED;
+  if (!aligned4(bm.kv_num_blocks) || !aligned4(bm.kv_indices) || !aligned4(bm.full_kv_num_blocks) ||
+      !aligned4(bm.full_kv_indices))
+    return FLEX_ERR_MISALIGNED;
+  return FLEX_OK;
+}
+
+// Backward workspace: -LSE*log2(e) and -delta per row (rows padded to 128), then, with a
+// block mask, the transposed bitmaps (B * Hkv * n_ktiles rows of 2 * tb_words words).
+size_t bwd_ws_bytes(int B, int H, int Hkv, int Sq, int Skv, bool blocks) {
+  const size_t sq_pad = (static_cast<size_t>(Sq) + kBM - 1) / kBM * kBM;
+  size_t bytes = 2 * static_cast<size_t>(B) * H * sq_pad * sizeof(float);
+  if (blocks) {
+    const size_t nq = (static_cast<size_t>(Sq) + kBM - 1) / kBM, nk = (static_cast<size_t>(Skv) + kBN - 1) / kBN;
+    const size_t words = (static_cast<size_t>(H / Hkv) * nq + 31) / 32;
+    bytes += static_cast<size_t>(B) * Hkv * nk * 2 * words * sizeof(uint32_t);
+  }
+  return bytes;
+}
+
 // Shared body of flex_attn_fwd (bm == nullptr) and flex_attn_fwd_block_sparse.
 flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
                          int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
@@ -264,19 +296,7 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
     return FLEX_ERR_MISALIGNED;
   if (bm) {
-    const bool has_part = bm->kv_num_blocks != nullptr, has_full = bm->full_kv_num_blocks != nullptr;
-    if (has_part != (bm->kv_indices != nullptr) || has_full != (bm->full_kv_indices != nullptr))
-      return FLEX_ERR_INVALID_ARG;
-    if (!has_part && !has_full) return FLEX_ERR_INVALID_ARG;
-    if (bm->max_blocks < 1 || (bm->batch != 1 && bm->batch != B) || (bm->heads != 1 && bm->heads != H))
-      return FLEX_ERR_INVALID_ARG;
-    if (bm->q_block_size != kBM || bm->kv_block_size != kBN) return FLEX_ERR_UNSUPPORTED;
-    if ((Skv + kBN - 1) / kBN > kMaxBlockKeyTiles) return FLEX_ERR_UNSUPPORTED;
-    const int64_t idx_elems = static_cast<int64_t>(bm->batch) * bm->heads * ((Sq + kBM - 1) / kBM) * bm->max_blocks;
-    if (idx_elems > 0x7fffffffLL) return FLEX_ERR_UNSUPPORTED;
-    if (!aligned4(bm->kv_num_blocks) || !aligned4(bm->kv_indices) || !aligned4(bm->full_kv_num_blocks) ||
-        !aligned4(bm->full_kv_indices))
-      return FLEX_ERR_MISALIGNED;
+    if (const flex_status_t bs = check_block_mask(*bm, B, H, Sq, Skv); bs != FLEX_OK) return bs;
   }
   const int64_t bh = static_cast<int64_t>(B) * H;
   const int n_qtiles = (Sq + kBM - 1) / kBM;
@@ -419,14 +439,25 @@ flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, 
 
 size_t flex_attn_bwd_workspace_size(int B, int H, int Sq) {
   if (B < 1 || H < 1 || Sq < 1) return 0;
-  const size_t sq_pad = (static_cast<size_t>(Sq) + kBM - 1) / kBM * kBM;
-  return 2 * static_cast<size_t>(B) * H * sq_pad * sizeof(float);
+  return bwd_ws_bytes(B, H, H, Sq, 1, false);
 }
 
-flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                            const void* dout, void* dq, void* dk, void* dv, int B, int H, int Hkv, int Sq, int Skv,
-                            int D, float scale, int score_mod_id, int mask_mod_id, const flex_mod_params_t* mod_params,
-                            flex_dtype_t dtype, void* workspace, size_t workspace_bytes, flex_stream_t stream) {
+size_t flex_attn_bwd_block_sparse_workspace_size(int B, int H, int Hkv, int Sq, int Skv) {
+  if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return 0;
+  return bwd_ws_bytes(B, H, Hkv, Sq, Skv, true);
+}
+
+}  // extern "C"
+
+namespace flexattn {
+namespace {
+
+// Shared body of flex_attn_bwd (bm == nullptr) and flex_attn_bwd_block_sparse.
+flex_status_t bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, int B, int H, int Hkv, int Sq, int Skv,
+                         int D, float scale, int score_mod_id, int mask_mod_id, const flex_mod_params_t* mod_params,
+                         const flex_block_mask_t* bm, flex_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                         flex_stream_t stream) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FLEX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
@@ -444,7 +475,10 @@ flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const v
     if (!aligned4(mp.alibi_slopes)) return FLEX_ERR_MISALIGNED;
   }
   if (const flex_status_t ds = check_documents(mask, mp); ds != FLEX_OK) return ds;
-  const size_t need = flex_attn_bwd_workspace_size(B, H, Sq);
+  if (bm) {
+    if (const flex_status_t bs = check_block_mask(*bm, B, H, Sq, Skv); bs != FLEX_OK) return bs;
+  }
+  const size_t need = bwd_ws_bytes(B, H, Hkv, Sq, Skv, bm != nullptr);
   if (!workspace || workspace_bytes < need) return FLEX_ERR_WORKSPACE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || !aligned4(lse))
@@ -485,7 +519,45 @@ flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const v
   p.mask = mask_args(mask, mp, Skv);
   const int score = score_mod_id == FLEX_SCORE_NONE ? kScoreNone : kScoreAlibi;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return D == 128 ? bwd_dispatch<128>(dtype, score, mask, m, p, s) : bwd_dispatch<64>(dtype, score, mask, m, p, s);
+  if (bm) {
+    p.blk_num[0] = bm->kv_num_blocks;
+    p.blk_idx[0] = bm->kv_indices;
+    p.blk_num[1] = bm->full_kv_num_blocks;
+    p.blk_idx[1] = bm->full_kv_indices;
+    p.blk_max = bm->max_blocks;
+    p.blk_b_stride = bm->batch == 1 ? 0 : bm->heads;
+    p.blk_h_stride = bm->heads == 1 ? 0 : 1;
+    p.tbits = reinterpret_cast<uint32_t*>(p.ndelta + bh * p.Sq_pad);
+    p.tb_words = (p.G * n_qtiles + 31) / 32;
+    return D == 128 ? bwd_dispatch<128, true>(dtype, score, mask, m, p, s)
+                    : bwd_dispatch<64, true>(dtype, score, mask, m, p, s);
+  }
+  return D == 128 ? bwd_dispatch<128, false>(dtype, score, mask, m, p, s)
+                  : bwd_dispatch<64, false>(dtype, score, mask, m, p, s);
+}
+
+}  // namespace
+}  // namespace flexattn
+
+extern "C" {
+
+flex_status_t flex_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, int B, int H, int Hkv, int Sq, int Skv,
+                            int D, float scale, int score_mod_id, int mask_mod_id, const flex_mod_params_t* mod_params,
+                            flex_dtype_t dtype, void* workspace, size_t workspace_bytes, flex_stream_t stream) {
+  return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, B, H, Hkv, Sq, Skv, D, scale, score_mod_id, mask_mod_id,
+                    mod_params, nullptr, dtype, workspace, workspace_bytes, stream);
+}
+
+flex_status_t flex_attn_bwd_block_sparse(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                         const void* dout, void* dq, void* dk, void* dv, int B, int H, int Hkv, int Sq,
+                                         int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
+                                         const flex_mod_params_t* mod_params, const flex_block_mask_t* block_mask,
+                                         flex_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                         flex_stream_t stream) {
+  if (!block_mask) return FLEX_ERR_INVALID_ARG;
+  return bwd_common(q, k, v, o, lse, dout, dq, dk, dv, B, H, Hkv, Sq, Skv, D, scale, score_mod_id, mask_mod_id,
+                    mod_params, block_mask, dtype, workspace, workspace_bytes, stream);
 }
 
 size_t flex_attn_decode_workspace_size(int B, int H, int Hkv, int cap, int D) {

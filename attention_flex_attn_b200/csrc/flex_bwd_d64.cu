@@ -2,5 +2,6 @@
 #include "flex_bwd_inst.cuh"
 
 namespace flexattn {
-template flex_status_t bwd_dispatch<64>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&, cudaStream_t);
+template flex_status_t bwd_dispatch<64, false>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
+                                               cudaStream_t);
 }  // namespace flexattn

@@ -20,6 +20,14 @@
 //   bwd_dkdv_kernel   one CTA per 128-key tile and kv head: for each query tile of each
 //                     query head of the group, S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
 //                     per key row, dV += P^T dO and dK += dS^T Q (TMEM accumulators)
+// With a block mask (BLOCKS instantiations; BlockMask, named with the backward as later
+// phases on FlyDSL PR 931, Out of scope) the keep rule is the block-sparse forward's: a
+// key tile on a query tile's full list keeps every key below Skv, one on its partial list
+// the keys mask_mod keeps.  The dQ kernel walks its query tile's listed key tiles from
+// bitmaps it builds in shared memory; the dK/dV kernel walks the (query head, query tile)
+// pairs that list its key tile, from transposed bitmaps that bwd_block_transpose_kernel
+// writes into the workspace first (one atomicOr per listed block, so the transpose costs
+// the size of the lists, not a scan per key tile).
 // Roles per CTA (384 threads): warp 0 issues the MMAs (one thread), warp 1 the TMA loads,
 // warps 4-7 and 8-11 do the element-wise work on the two 64-column halves of each tile
 // (thread = TMEM lane = row), warps 2-3 idle.  Each half writes its 16-bit results into
@@ -58,7 +66,114 @@ struct BwdParams {
   float scale_log2;       // scale * log2(e)
   const float* slopes;    // alibi slope tensor [H] or nullptr
   MaskArgs mask;          // document rules: boundaries of batch 0, advanced per batch
+  // Block mask (BLOCKS instantiations), as in FwdParams: [0] partial, [1] full lists.
+  const int32_t* blk_num[2];
+  const int32_t* blk_idx[2];
+  int blk_max, blk_b_stride, blk_h_stride;
+  // Transposed block mask in the workspace: per (b, kv head, key tile) two bitmaps of
+  // tb_words words over the (query head in group, query tile) pairs hg * n_qtiles + t:
+  // tbits[row * 2 * tb_words + w] (pairs that visit the key tile) and
+  // tbits[row * 2 * tb_words + tb_words + w] (those whose visit is FULL).
+  uint32_t* tbits;
+  int tb_words;
 };
+
+// Block-mask bitmap words a dQ CTA keeps in shared memory (key tiles <= 32 * kBwdBlkWords).
+constexpr int kBwdBlkWords = kBlkWords;
+
+// Ascending walk over the set bits of a bitmap (words read through `load`), with the
+// companion bitmap's bit of each position in cur_full; cur = -1 once the walk is over.
+template <typename Load>
+struct AscBits {
+  Load load;
+  int n_words, wi;
+  uint32_t bits, cword;
+  int cur;
+  bool cur_full;
+  __device__ __forceinline__ AscBits(Load l, int nw) : load(l), n_words(nw), wi(-1), bits(0), cword(0), cur(-1),
+                                                        cur_full(false) {
+    advance();
+  }
+  __device__ __forceinline__ void advance() {
+    while (bits == 0) {
+      if (++wi >= n_words) {
+        cur = -1;
+        return;
+      }
+      bits = load(wi, 0);
+      cword = load(wi, 1);
+    }
+    const int bit = __ffs(bits) - 1;
+    bits &= bits - 1u;
+    cur = (wi << 5) + bit;
+    cur_full = (cword >> bit) & 1u;
+  }
+};
+template <typename Load>
+__device__ __forceinline__ AscBits<Load> asc_bits(Load l, int n_words) {
+  return AscBits<Load>(l, n_words);
+}
+
+// The class a block mask gives key tile u of query tile [q0, q1): -1 (the tile keeps
+// nothing), kTileFull (every key below Skv kept) or kTilePartial (mask_mod per element).
+// A block on the full list is FULL; a partial block that mask_mod drops whole keeps
+// nothing and one it keeps whole is FULL, as in the forward (document rules: partial).
+template <int MASK>
+__device__ __forceinline__ int block_tile_class(bool listed_full, int q0, int q1, int u, const MaskArgs& m) {
+  if (listed_full) return kTileFull;
+  if constexpr (MASK == kMaskDocument || MASK == kMaskDocumentCausal) {
+    return kTilePartial;
+  } else {
+    int lo, hi;
+    tile_range<MASK>(q0, q1, kBN, m, lo, hi);
+    if (u < lo || u >= hi) return -1;
+    return tile_class<MASK>(q0, q1, u * kBN, kBN, m) == kTileFull ? kTileFull : kTilePartial;
+  }
+}
+
+// ---------------------------------------------------------------- block-mask transpose
+
+// One warp per list row (b, h, t): every key tile u the row lists sets bit hg * n_qtiles
+// + t of the (b, kv head, u) bitmaps in the workspace (zeroed before the launch), and of
+// the FULL bitmap when the visit needs no element mask.  Counts are clamped and indices
+// range-checked as in the forward.
+template <int MASK>
+__global__ void __launch_bounds__(256) bwd_block_transpose_kernel(const BwdParams p) {
+  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.n_qtiles;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; r < rows;
+       r += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+    const int t = static_cast<int>(r % p.n_qtiles);
+    const int64_t bh = r / p.n_qtiles;
+    const int h = static_cast<int>(bh % p.H), b = static_cast<int>(bh / p.H);
+    const int hk = h / p.G, hg = h % p.G;
+    const int q0 = t * kBM, q1 = min(q0 + kBM, p.Sq);
+    MaskArgs mk = p.mask;
+    if constexpr (MASK == kMaskDocument || MASK == kMaskDocumentCausal) {
+      mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
+      mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
+    }
+    const int64_t lrow = (static_cast<int64_t>(b) * p.blk_b_stride + static_cast<int64_t>(h) * p.blk_h_stride) *
+                             p.n_qtiles + t;
+    const int pair = hg * p.n_qtiles + t;
+    for (int f = 0; f < 2; ++f) {
+      const int32_t* num = f ? p.blk_num[1] : p.blk_num[0];
+      const int32_t* idx = f ? p.blk_idx[1] : p.blk_idx[0];
+      if (num == nullptr) continue;
+      int cnt = num[lrow];
+      cnt = cnt < 0 ? 0 : (cnt > p.blk_max ? p.blk_max : cnt);
+      for (int c = lane; c < cnt; c += 32) {
+        const int u = idx[lrow * p.blk_max + c];
+        if (u < 0 || u >= p.n_ktiles) continue;
+        const int cls = block_tile_class<MASK>(f == 1, q0, q1, u, mk);
+        if (cls < 0) continue;
+        uint32_t* row = p.tbits + ((static_cast<int64_t>(b) * p.Hkv + hk) * p.n_ktiles + u) * 2 * p.tb_words;
+        atomicOr(row + (pair >> 5), 1u << (pair & 31));
+        if (cls == kTileFull) atomicOr(row + p.tb_words + (pair >> 5), 1u << (pair & 31));
+      }
+    }
+  }
+}
 
 // ---------------------------------------------------------------- prep
 
@@ -93,7 +208,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
 
 // ---------------------------------------------------------------- shared memory
 
-template <int D>
+template <int D, bool BLOCKS = false>
 struct BwdDqSmem {
   static constexpr int kTileBytes = kBM * D * 2;
   static constexpr int kChunkBytes = kBM * 128;
@@ -107,7 +222,9 @@ struct BwdDqSmem {
   // barriers: q, full_k[KS], empty_k[KS], full_v[VS], empty_v[VS], sdp[2], ds[2], done
   static constexpr int kNumBars = 1 + 2 * (kKSlots + kVSlots) + 5;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kTmemPtrOff + 16;
+  // block mask: the visit and FULL bitmaps of this query tile's key tiles
+  static constexpr int kBlkOff = kTmemPtrOff + 16;
+  static constexpr int kBytes = kBlkOff + (BLOCKS ? 2 * kBwdBlkWords * 4 : 0);
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
 };
@@ -147,12 +264,12 @@ __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity, const Bw
 
 // ---------------------------------------------------------------- dQ
 
-template <int D, typename T, int SCORE, int MASK>
+template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const BwdParams p) {
-  using L = BwdDqSmem<D>;
+  using L = BwdDqSmem<D, BLOCKS>;
   constexpr int KS = L::kKSlots, VS = L::kVSlots;
   constexpr int kChunks = D / 64;
   constexpr uint32_t kIdescS = idesc_f16(DtypeBits<T>::kFmt, kBM, kBN, 0);       // S: K-major B
@@ -192,7 +309,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   int lo = 0, hi = 0;
   tile_range<MASK>(q0, q1, kBN, mk, lo, hi);
-  const int n = hi - lo;  // key tiles lo .. hi-1, visited in ascending order
+  // Block mask: the key tiles this query tile visits (act) and those it keeps whole
+  // (full), as bitmaps built from its two lists; the walk is their set bits in ascending
+  // order.  Otherwise: key tiles lo .. hi-1 in ascending order.
+  uint32_t* act_bits = reinterpret_cast<uint32_t*>(sgen + L::kBlkOff);
+  uint32_t* full_bits = act_bits + kBwdBlkWords;
+  const int n_words = (p.n_ktiles + 31) >> 5;
+  if constexpr (BLOCKS) {
+    for (int w = threadIdx.x; w < 2 * kBwdBlkWords; w += kBwdThreads) act_bits[w] = 0u;
+    __syncthreads();
+    const int64_t lrow = (static_cast<int64_t>(b) * p.blk_b_stride + static_cast<int64_t>(h) * p.blk_h_stride) *
+                             p.n_qtiles + qt;
+    for (int e = threadIdx.x; e < 2 * p.blk_max; e += kBwdThreads) {
+      const int f = e >= p.blk_max ? 1 : 0, c = e - f * p.blk_max;
+      const int32_t* num = f ? p.blk_num[1] : p.blk_num[0];
+      const int32_t* idx = f ? p.blk_idx[1] : p.blk_idx[0];
+      if (num == nullptr) continue;
+      const int cnt = num[lrow];
+      if (c >= (cnt < 0 ? 0 : (cnt > p.blk_max ? p.blk_max : cnt))) continue;
+      const int u = idx[lrow * p.blk_max + c];
+      if (u < 0 || u >= p.n_ktiles) continue;
+      const int cls = block_tile_class<MASK>(f == 1, q0, q1, u, mk);
+      if (cls < 0) continue;
+      atomicOr(act_bits + (u >> 5), 1u << (u & 31));
+      if (cls == kTileFull) atomicOr(full_bits + (u >> 5), 1u << (u & 31));
+    }
+    __syncthreads();
+    int cnt = 0;
+    for (int w = 0; w < n_words; ++w) cnt += __popc(act_bits[w]);
+    lo = 0;
+    hi = cnt;
+  }
+  const int n = hi - lo;  // steps
+  auto smem_words = [act_bits, full_bits](int w, int which) { return which ? full_bits[w] : act_bits[w]; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -232,7 +381,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_load_3d(o_smem + c * L::kChunkBytes, &tmO, bar_q, c * 64, q0, bh);
     }
     // Loads in the order the products need them: K_0, V_0, K_1, then V_{t+1}, K_{t+2}.
+    // Block mask: the key tile of each load comes from a walk of the visit bitmap (one
+    // walk for the K loads, one for the V loads).
     int nk = 0, nv = 0;
+    auto walk_k = asc_bits(smem_words, BLOCKS ? n_words : 0);
+    auto walk_v = asc_bits(smem_words, BLOCKS ? n_words : 0);
     auto load = [&](bool is_v, int tile) -> bool {
       const int i = is_v ? nv : nk;
       const int slot = i % (is_v ? VS : KS);
@@ -241,8 +394,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!bwd_wait(empty, (static_cast<uint32_t>(i / (is_v ? VS : KS)) & 1u) ^ 1u, p, abort_flag)) return false;
       mbar_arrive_expect_tx(full, L::kTileBytes);
       const uint32_t dst = is_v ? v_smem(slot) : k_smem(slot);
+      int key_tile = lo + tile;
+      if constexpr (BLOCKS) {
+        auto& w = is_v ? walk_v : walk_k;
+        key_tile = w.cur;
+        w.advance();
+      }
       for (int c = 0; c < kChunks; ++c)
-        tma_load_3d(dst + c * L::kChunkBytes, is_v ? &tmV : &tmK, full, c * 64, (lo + tile) * kBN, bkv);
+        tma_load_3d(dst + c * L::kChunkBytes, is_v ? &tmV : &tmK, full, c * 64, key_tile * kBN, bkv);
       if (is_v) ++nv;
       else ++nk;
       return true;
@@ -364,6 +523,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     row_interval<MASK>(q1 - 1, mk, lo_last, t1);
     row_interval<MASK>(q0, mk, t0, hi_first);
     bool ok = true;
+    auto walk = asc_bits(smem_words, BLOCKS ? n_words : 0);
     for (int t = 0; t < n; ++t) {
       const bool got = bwd_wait(bar_sdp(wg), static_cast<uint32_t>(t) & 1u, p, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
@@ -371,11 +531,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       }
       tc_fence_after();
-      const int k0 = (lo + t) * kBN;
-      const bool full = row_valid && tile_class_of(lo_last, hi_first, k0, kBN, p.Skv) == kTileFull;
+      const int k0 = (BLOCKS ? walk.cur : lo + t) * kBN;
+      bool full;
+      int64_t keep_lo = row_lo, keep_hi = row_hi;
+      if constexpr (BLOCKS) {
+        if (walk.cur_full) {  // a FULL block keeps every key below Skv
+          keep_lo = 0;
+          keep_hi = p.Skv - 1;
+        }
+        full = row_valid && walk.cur_full && k0 + kBN <= p.Skv;
+        walk.advance();
+      } else {
+        full = row_valid && tile_class_of(lo_last, hi_first, k0, kBN, p.Skv) == kTileFull;
+      }
       int c_lo = 0, c_hi = kBN - 1;
       if (!full) {
-        col_interval_of(row_lo, row_hi, k0, c_lo, c_hi);
+        col_interval_of(keep_lo, keep_hi, k0, c_lo, c_hi);
         if (!row_valid) {
           c_lo = 1;
           c_hi = 0;
@@ -454,7 +625,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---------------------------------------------------------------- dK, dV
 
-template <int D, typename T, int SCORE, int MASK>
+template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -501,10 +672,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tile_range<MASK>(t * kBM, min(t * kBM + kBM, p.Sq), kBN, mk, lo, hi);
     return kt >= lo && kt < hi;
   };
-  // steps: (query head of the group) x (active query tile); every role walks the same list
-  int n_active = 0;
-  for (int t = 0; t < p.n_qtiles; ++t) n_active += active(t) ? 1 : 0;
-  const int n = n_active * p.G;
+  // steps: (query head of the group) x (active query tile); every role walks the same list.
+  // Block mask: the steps are the set bits of this key tile's transposed bitmap (pairs
+  // hg * n_qtiles + t in ascending order, hg major), with the FULL bitmap alongside.
+  const uint32_t* tb_row =
+      BLOCKS ? p.tbits + ((static_cast<int64_t>(b) * p.Hkv + hk) * p.n_ktiles + kt) * 2 * p.tb_words : nullptr;
+  const int tb_words = p.tb_words;
+  auto tb_load = [tb_row, tb_words](int w, int which) { return __ldg(tb_row + which * tb_words + w); };
+  int n = 0;
+  if constexpr (BLOCKS) {
+    for (int w = 0; w < p.tb_words; ++w) n += __popc(tb_load(w, 0));
+  } else {
+    int n_active = 0;
+    for (int t = 0; t < p.n_qtiles; ++t) n_active += active(t) ? 1 : 0;
+    n = n_active * p.G;
+  }
+  // calls f(hg, t, listed_full) for every step in order; f returns false to stop
+  auto for_steps = [&](auto&& f) {
+    if constexpr (BLOCKS) {
+      for (auto w = asc_bits(tb_load, p.tb_words); w.cur >= 0; w.advance())
+        if (!f(w.cur / p.n_qtiles, w.cur % p.n_qtiles, w.cur_full)) return;
+    } else {
+      for (int hg = 0; hg < p.G; ++hg)
+        for (int t = 0; t < p.n_qtiles; ++t)
+          if (active(t) && !f(hg, t, false)) return;
+    }
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -539,27 +732,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_load_3d(v_smem + c * L::kChunkBytes, &tmV, bar_kv, c * 64, k0, bkv);
     }
     int u = 0;
-    bool ok = true;
-    for (int hg = 0; hg < p.G && ok; ++hg) {
+    for_steps([&](int hg, int t, bool) -> bool {
       const int bh = b * p.H + hk * p.G + hg;
-      for (int t = 0; t < p.n_qtiles && ok; ++t) {
-        if (!active(t)) continue;
-        const int s = u % NS;
-        if (!bwd_wait(bar_empty(s), (static_cast<uint32_t>(u / NS) & 1u) ^ 1u, p, abort_flag)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(bar_full(s), 2 * L::kTileBytes + L::kStatBytes);
-        for (int c = 0; c < kChunks; ++c) {
-          tma_load_3d(q_slot(s) + c * L::kChunkBytes, &tmQ, bar_full(s), c * 64, t * kBM, bh);
-          tma_load_3d(o_slot(s) + c * L::kChunkBytes, &tmO, bar_full(s), c * 64, t * kBM, bh);
-        }
-        const int64_t srow = static_cast<int64_t>(bh) * p.Sq_pad + t * kBM;
-        bulk_load(sbase + stat_slot(s), p.nlse2 + srow, kBM * 4, bar_full(s));
-        bulk_load(sbase + stat_slot(s) + kBM * 4, p.ndelta + srow, kBM * 4, bar_full(s));
-        ++u;
+      const int s = u % NS;
+      if (!bwd_wait(bar_empty(s), (static_cast<uint32_t>(u / NS) & 1u) ^ 1u, p, abort_flag)) return false;
+      mbar_arrive_expect_tx(bar_full(s), 2 * L::kTileBytes + L::kStatBytes);
+      for (int c = 0; c < kChunks; ++c) {
+        tma_load_3d(q_slot(s) + c * L::kChunkBytes, &tmQ, bar_full(s), c * 64, t * kBM, bh);
+        tma_load_3d(o_slot(s) + c * L::kChunkBytes, &tmO, bar_full(s), c * 64, t * kBM, bh);
       }
-    }
+      const int64_t srow = static_cast<int64_t>(bh) * p.Sq_pad + t * kBM;
+      bulk_load(sbase + stat_slot(s), p.nlse2 + srow, kBM * 4, bar_full(s));
+      bulk_load(sbase + stat_slot(s) + kBM * 4, p.ndelta + srow, kBM * 4, bar_full(s));
+      ++u;
+      return true;
+    });
     for (int e = u - NS < 0 ? 0 : u - NS; e < u; ++e)
       mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
     mbar_wait(bar_kv, 0, p.status, kStatusBwdTimeout, kWaitTimeoutNs);
@@ -643,14 +830,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t sc2 = pack2(p.scale_log2, p.scale_log2);
     bool ok = true;
     int u = 0;
-    for (int hg = 0; hg < p.G && ok; ++hg) {
-      const int h = hk * p.G + hg;
-      float slope2 = 0.f;
-      if (SCORE == kScoreAlibi)
-        slope2 = (p.slopes ? __ldg(p.slopes + h) : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
-                 kLog2e;
-      for (int t = 0; t < p.n_qtiles; ++t) {
-        if (!active(t)) continue;
+    int slope_h = -1;
+    float slope2 = 0.f;
+    for_steps([&](int hg, int t, bool listed_full) -> bool {
+      {
+        const int h = hk * p.G + hg;
+        if (SCORE == kScoreAlibi && h != slope_h) {
+          slope_h = h;
+          slope2 = (p.slopes ? __ldg(p.slopes + h)
+                             : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
+                   kLog2e;
+        }
         const int s = u % NS;
         // S^T / dP^T ready; the slot's statistics (written by the bulk copy) are read
         // below, so observe the slot's own barrier too
@@ -658,11 +848,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                          bwd_wait(bar_full(s), static_cast<uint32_t>(u / NS) & 1u, p, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
-          break;
+          return false;
         }
         tc_fence_after();
         const int q0 = t * kBM;
-        const bool full = tile_class<MASK>(q0, min(q0 + kBM, p.Sq), k0, kBN, mk) == kTileFull;
+        // a FULL block keeps every query (rows past Sq have P = 0 through their -inf LSE)
+        const bool full = BLOCKS ? listed_full : tile_class<MASK>(q0, min(q0 + kBM, p.Sq), k0, kBN, mk) == kTileFull;
         int c_lo = 0, c_hi = kBM - 1;
         if (!full) col_interval_of(key_lo, key_hi, q0, c_lo, c_hi);
         const float* stat = reinterpret_cast<const float*>(sgen + stat_slot(s));
@@ -710,7 +901,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(bar_pds(wg));
         ++u;
       }
-    }
+      return true;
+    });
     // epilogue: dK = scale * (dS^T Q), dV = P^T dO
     bool ran = ok && n > 0;
     if (ran) {

@@ -49,15 +49,20 @@ struct BwdMaps {
   CUtensorMap q, o, k, v;
 };
 
-// Backward (prep, dQ, dK/dV) over every (dtype, score_mod, mask_mod) of one head dim.
-// Instantiated in flex_bwd_d{64,128}.cu.
-template <int D>
+// Backward (prep, dQ, dK/dV; with a block mask also the transposed bitmaps) over every
+// (dtype, score_mod, mask_mod) of one head dim and block-mask mode.  Instantiated in
+// flex_bwd_d{64,128}{,_blocks}.cu.
+template <int D, bool BLOCKS>
 flex_status_t bwd_dispatch(flex_dtype_t dtype, int score, int mask, const BwdMaps& m, const BwdParams& p,
                            cudaStream_t s);
-extern template flex_status_t bwd_dispatch<64>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
-                                               cudaStream_t);
-extern template flex_status_t bwd_dispatch<128>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
-                                                cudaStream_t);
+extern template flex_status_t bwd_dispatch<64, false>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
+                                                      cudaStream_t);
+extern template flex_status_t bwd_dispatch<128, false>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
+                                                       cudaStream_t);
+extern template flex_status_t bwd_dispatch<64, true>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
+                                                     cudaStream_t);
+extern template flex_status_t bwd_dispatch<128, true>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
+                                                      cudaStream_t);
 
 // Split-KV decode + combine (flex_decode_launch.cu).
 flex_status_t decode_dispatch(int D, flex_dtype_t dtype, const DecodeParams& p, cudaStream_t s);

@@ -224,7 +224,7 @@ size_t flex_attn_bwd_workspace_size(int B, int H, int Sq);
  *   q, o, dout, dq [B, H, Sq, D] dtype;  k, v, dk, dv [B, Hkv, Skv, D] dtype;
  *   lse [B, H, Sq] fp32: the forward's LSE (natural log; -inf for rows without keys).
  *   scale, score_mod_id, mask_mod_id, mod_params: those of the forward (any mod
- *   flex_attn_fwd takes; no block mask).
+ *   flex_attn_fwd takes; with a block mask see flex_attn_bwd_block_sparse).
  *   workspace: at least flex_attn_bwd_workspace_size(B, H, Sq) bytes, 16-byte aligned.
  * Accumulation is fp32; P and dS enter the matmuls rounded to dtype (round-to-nearest-
  * even).  Rows without keys give no gradient.  Deterministic: no atomics.
@@ -249,6 +249,35 @@ typedef struct {
   int32_t split_size;
   uint32_t* status_out;
 } flex_decode_params_t;
+
+/*
+ * flex_attn_bwd_block_sparse_workspace_size -- bytes of device workspace
+ * flex_attn_bwd_block_sparse needs: flex_attn_bwd's per-row statistics plus the block
+ * mask transposed to key tiles (per batch, kv head and key tile, two bitmaps over the
+ * (query head of the group, query tile) pairs).  0 for invalid sizes.
+ */
+size_t flex_attn_bwd_block_sparse_workspace_size(int B, int H, int Hkv, int Sq, int Skv);
+
+/*
+ * flex_attn_bwd_block_sparse -- gradients of the block-sparse forward
+ * (flex_attn_fwd_block_sparse) with the same arguments: flex_attn_bwd with the keep rule
+ * of the block mask (block sparsity and the backward are both named as later phases on
+ * FlyDSL PR 931, Out of scope).  A key block on a query tile's full list keeps every key
+ * below Skv, one on its partial list the keys mask_mod keeps; every other key is dropped
+ * and takes no gradient.  Arguments, layouts and errors are those of flex_attn_bwd and of
+ * flex_attn_fwd_block_sparse (the block_mask rules and limits), plus:
+ *   workspace: at least flex_attn_bwd_block_sparse_workspace_size(B, H, Hkv, Sq, Skv)
+ *   bytes, 16-byte aligned; overwritten.
+ * Deterministic: the transposed bitmaps are built with atomic ORs, whose result does
+ * not depend on their order; the gradients use no atomics.
+ */
+flex_status_t flex_attn_bwd_block_sparse(const void* q, const void* k, const void* v, const void* o,
+                                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                         int B, int H, int Hkv, int Sq, int Skv, int D, float scale,
+                                         int score_mod_id, int mask_mod_id,
+                                         const flex_mod_params_t* mod_params,
+                                         const flex_block_mask_t* block_mask, flex_dtype_t dtype,
+                                         void* workspace, size_t workspace_bytes, flex_stream_t stream);
 
 /*
  * flex_attn_decode_workspace_size -- bytes of device workspace flex_attn_decode needs

@@ -326,3 +326,25 @@ def test_fwd_shape_checks_on_cpu():
         fa._check_fwd_shapes(q, k, k, lse_out=torch.zeros(2, 4, 100, dtype=bf))
     with pytest.raises(fa.FlexAttnError):
         fa._check_fwd_shapes(q, k, k, lse_out=torch.zeros(2, 4, 101, dtype=torch.float32))
+
+
+def test_bwd_block_sparse_rejects_bad_args_on_host(lib):
+    def bb(bm, ws=64, wsb=1 << 20, Skv=8):
+        return lib.flex_attn_bwd_block_sparse(P(16), P(16), P(16), P(16), P(32), P(16), P(16), P(16), P(16), 1, 2, 1,
+                                              8, Skv, 128, 0.1, 0, 0, None,
+                                              ctypes.byref(bm) if bm is not None else None, 0, P(ws), wsb, None)
+
+    def mask(num=32, idx=64, fnum=None, fidx=None, maxb=1, batch=1, heads=1, qb=128, kb=128):
+        return fa.BlockMaskC(num, idx, fnum, fidx, maxb, batch, heads, qb, kb)
+    assert bb(None) == 1
+    assert bb(mask(num=None, idx=None)) == 1
+    assert bb(mask(heads=3)) == 1
+    assert bb(mask(qb=64)) == 2
+    assert bb(mask(), Skv=2048 * 128 + 1) == 2
+    assert bb(mask(num=34)) == 3
+    assert bb(mask(), ws=0) == 4
+    assert bb(mask(), wsb=100) == 4
+    # statistics [2 * B * H * Sq_pad] floats, then per (b, kv head, key tile) 2 words per
+    # ceil(G * n_qtiles / 32): B=2 H=4 Hkv=2 Sq=300 Skv=700 -> 3 query tiles, 6 key tiles
+    assert lib.flex_attn_bwd_block_sparse_workspace_size(2, 4, 2, 300, 700) == 2 * 2 * 4 * 384 * 4 + 2 * 2 * 6 * 2 * 4
+    assert lib.flex_attn_bwd_block_sparse_workspace_size(2, 3, 2, 300, 700) == 0
