@@ -41,18 +41,34 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows3 x rows x D] 16-bit tensor, box = 64 elements x 128 rows x 1, 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, flex_dtype_t dt, int D, int rows, int64_t outer) {
+// [rows3 x rows x D] 16-bit tensor, box = 64 elements x box_rows rows x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, flex_dtype_t dt, int D, int rows, int64_t outer,
+              int box_rows = kBM) {
   auto fn = encode_fn();
   if (!fn) return false;
   const CUtensorMapDataType t = dt == FLEX_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(outer)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(D) * 2 * rows};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBM), 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The decode's additive mask [B, H, 1, cap] as a [cap, H, B] 16-bit tensor, box = 64
+// positions x `rows` heads x 1, no swizzle (cap must be a multiple of 8: 16-byte strides).
+bool make_map_mask(CUtensorMap* map, const void* base, flex_dtype_t dt, int cap, int H, int B, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const CUtensorMapDataType t = dt == FLEX_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cap), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cap) * 2, static_cast<cuuint64_t>(cap) * 2 * H};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kDtKeys), static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -136,6 +152,19 @@ void* symbol_ptr(Symbol which) {
 }
 
 void* decode_scratch_ptr() { return symbol_ptr(kSymScratch); }
+
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 // The status word a call's kernels report into: the caller's own, or the shared one.
 unsigned* status_for(uint32_t* status_out) {
@@ -606,9 +635,28 @@ flex_status_t flex_attn_decode(const void* q, const void* k_cache, const void* v
   p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ((o_bytes + 255) & ~static_cast<size_t>(255)));
   p.status = st;
   p.scale_log2 = scale * kLog2e;
+  if (p.G >= 2 && B <= kDtMaxBatch) {
+    // grouped heads: the persistent kernel streams the caches in 64-position TMA tiles
+    DecodeMaps m;
+    if (!make_map(&m.k, k_cache, dtype, D, cap, static_cast<int64_t>(B) * Hkv, kDtKeys) ||
+        !make_map(&m.v, v_cache, dtype, D, cap, static_cast<int64_t>(B) * Hkv, kDtKeys))
+      return FLEX_ERR_CUDA;
+    // the mask tile rides with each K tile through TMA when its rows can be mapped
+    m.mask_rows = 0;
+    m.m = m.k;
+    if (additive_mask != nullptr && cap % 8 == 0) {
+      m.mask_rows = p.G < kGqaRows ? p.G : kGqaRows;
+      if (!make_map_mask(&m.m, additive_mask, dtype, cap, H, B, m.mask_rows)) return FLEX_ERR_CUDA;
+    }
+    const int sms = sm_count();
+    if (sms < 1) return FLEX_ERR_CUDA;
+    const int64_t chunks = static_cast<int64_t>(B) * Hkv * ((p.G + kGqaRows - 1) / kGqaRows) * p.n_splits;
+    m.grid = static_cast<int>(chunks < sms ? chunks : sms);
+    return decode_dispatch(D, dtype, p, &m, reinterpret_cast<cudaStream_t>(stream));
+  }
   const int64_t grid_y = static_cast<int64_t>(B) * Hkv * (p.G >= 2 ? (p.G + kGqaRows - 1) / kGqaRows : 1);
   if (grid_y > 65535) return FLEX_ERR_UNSUPPORTED;
-  return decode_dispatch(D, dtype, p, reinterpret_cast<cudaStream_t>(stream));
+  return decode_dispatch(D, dtype, p, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 flex_status_t flex_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -9,6 +9,7 @@
 #include "flex_attn.h"
 #include "flex_bwd_sm100.cuh"
 #include "flex_decode.cuh"
+#include "flex_decode_gqa_tma.cuh"
 #include "flex_fwd_fp8_sm100.cuh"
 #include "flex_fwd_sm100.cuh"
 
@@ -64,7 +65,18 @@ extern template flex_status_t bwd_dispatch<64, true>(flex_dtype_t, int, int, con
 extern template flex_status_t bwd_dispatch<128, true>(flex_dtype_t, int, int, const BwdMaps&, const BwdParams&,
                                                       cudaStream_t);
 
-// Split-KV decode + combine (flex_decode_launch.cu).
-flex_status_t decode_dispatch(int D, flex_dtype_t dtype, const DecodeParams& p, cudaStream_t s);
+// Tensor maps of the caches ([D, cap, B*Hkv], 64 x 64 boxes) and of the additive mask
+// ([cap, H, B], 64 x mask_rows boxes; mask_rows = 0: the mask is read directly), and the
+// persistent grid of the grouped-query decode.
+struct DecodeMaps {
+  CUtensorMap k, v, m;
+  int mask_rows;
+  int grid;
+};
+
+// Split-KV decode + combine (flex_decode_launch.cu).  maps: the grouped-query decode's
+// tensor maps (G >= 2), or nullptr for the register-streaming kernels.
+flex_status_t decode_dispatch(int D, flex_dtype_t dtype, const DecodeParams& p, const DecodeMaps* maps,
+                              cudaStream_t s);
 
 }  // namespace flexattn

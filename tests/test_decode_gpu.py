@@ -86,8 +86,18 @@ def test_decode_split_size_independence(Hkv):
 
 
 @pytest.mark.parametrize("H,Hkv", [(6, 2), (12, 4), (5, 5), (16, 2), (32, 2), (40, 2), (64, 4)])
-def test_decode_group_sizes(H, Hkv):
-    args = _inputs(3, H, Hkv, 700, 128, seed=3300 + H, mask_p=0.3)
+@pytest.mark.parametrize("cap", [700, 704])
+def test_decode_group_sizes(H, Hkv, cap):
+    """Grouped heads: 2..20 query heads per kv head (up to two 16-row groups).  cap = 704
+    streams the mask tiles with TMA, cap = 700 (rows not a multiple of 16 bytes) reads them
+    directly."""
+    args = _inputs(3, H, Hkv, cap, 128, seed=3300 + H, mask_p=0.3)
+    _check(*args)
+
+
+def test_decode_large_batch():
+    """B above the grouped-query kernel's batch table (1024): the register-streaming kernel."""
+    args = _inputs(1030, 4, 2, 64, 64, seed=3350, dtype="bf16", mask_p=0.2)
     _check(*args)
 
 

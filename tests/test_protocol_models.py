@@ -453,3 +453,84 @@ def test_dkdv_protocol(n, NS):
 
 def test_dkdv_early_slot_release_is_caught():
     assert _schedules(lambda i: dkdv_roles(6, 2, early_release=True), 80) > 0
+
+
+# ----------------------------------------------------------------------------- decode
+
+def decode_roles(chunk_tiles, NS, consumers=4, shared_ring=False):
+    """decode_gqa_tma_kernel: one TMA producer, `consumers` warps taking the CTA's chunks
+    round-robin (warp w: chunks w, w + consumers, ...); each chunk is a list of tiles, each
+    tile a K then a V load.  The kernel gives every consumer a ring of NS slots of its
+    own, which the producer fills in that consumer's order (polling the rings, so one full
+    ring does not hold back the others).  shared_ring plants the mistake of one ring of
+    consumers * NS slots shared in global order: a consumer whose chunk lies more than a
+    ring cycle ahead waits with a parity that an earlier phase of the slot already shows."""
+    m = _Model()
+    n_slots = consumers * NS
+    full = [m.bar(f"full{s}") for s in range(n_slots)]
+    empty = [m.bar(f"empty{s}") for s in range(n_slots)]
+    own = [[k for k in range(len(chunk_tiles)) if k % consumers == w] for w in range(consumers)]
+    loads = {w: [(k, t, which) for k in own[w] for t in range(chunk_tiles[k]) for which in ("K", "V")]
+             for w in range(consumers)}
+    order = [(k, t, which) for k in range(len(chunk_tiles)) for t in range(chunk_tiles[k]) for which in ("K", "V")]
+    gpos = {ld: r for r, ld in enumerate(order)}
+
+    def slot_of(w, i, ld):
+        if shared_ring:
+            r = gpos[ld]
+            return r % n_slots, r // n_slots
+        return w * NS + i % NS, i // NS
+
+    def producer():
+        if shared_ring:
+            for ld in order:
+                w = ld[0] % consumers
+                s, cyc = slot_of(w, None, ld)
+                if cyc > 0:
+                    yield ("wait", empty[s], (cyc & 1) ^ 1)
+                yield ("expect", full[s], TB)
+                yield ("tma", ("slot", s), ld, full[s], TB)
+            return
+        nxt = [0] * consumers
+        while any(nxt[w] < len(loads[w]) for w in range(consumers)):
+            progressed = False
+            for w in range(consumers):
+                i = nxt[w]
+                if i >= len(loads[w]):
+                    continue
+                s, cyc = slot_of(w, i, loads[w][i])
+                if cyc > 0 and not empty[s].passes((cyc & 1) ^ 1):
+                    continue  # a non-blocking probe: this ring is full, try the next one
+                yield ("expect", full[s], TB)
+                yield ("tma", ("slot", s), loads[w][i], full[s], TB)
+                nxt[w] += 1
+                progressed = True
+            if not progressed:  # every ring full: block on the oldest pending one
+                w = min((w for w in range(consumers) if nxt[w] < len(loads[w])), key=lambda w: nxt[w])
+                s, cyc = slot_of(w, nxt[w], loads[w][nxt[w]])
+                yield ("wait", empty[s], (cyc & 1) ^ 1)
+
+    def consumer(w):
+        for i, ld in enumerate(loads[w]):
+            s, cyc = slot_of(w, i, ld)
+            yield ("wait", full[s], cyc & 1)
+            yield ("read", [(("slot", s), ld)])
+            yield ("arrive", empty[s])
+
+    roles = {"producer": producer()}
+    for w in range(consumers):
+        roles[f"c{w}"] = consumer(w)
+    return roles, m.bars
+
+
+@pytest.mark.parametrize("NS", [3, 6])
+def test_decode_ring_protocol(NS):
+    rng = random.Random(NS)
+    cases = [[rng.choice([1, 2, 3, 4]) for _ in range(rng.randint(1, 13))] for _ in range(50)]
+    assert _schedules(lambda i: decode_roles(cases[i], NS), len(cases)) == 0
+
+
+def test_decode_shared_ring_is_caught():
+    rng = random.Random(9)
+    cases = [[4] * rng.randint(6, 12) for _ in range(40)]
+    assert _schedules(lambda i: decode_roles(cases[i], 3, shared_ring=True), len(cases)) > 0
