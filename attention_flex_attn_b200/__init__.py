@@ -28,6 +28,7 @@ FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
 EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_fwd_fp8_workspace_size", "flex_attn_fwd_fp8",
+            "flex_attn_fwd_fp8_block_sparse",
             "flex_attn_bwd_workspace_size", "flex_attn_bwd",
             "flex_attn_bwd_block_sparse_workspace_size", "flex_attn_bwd_block_sparse",
             "flex_attn_decode_workspace_size", "flex_attn_decode",
@@ -82,6 +83,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_fwd_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, F, F, F, I, I, ctypes.POINTER(ModParams),
                                       P, SZ, P]
     lib.flex_attn_fwd_fp8.restype = I
+    lib.flex_attn_fwd_fp8_block_sparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, F, F, F, I, I,
+                                                   ctypes.POINTER(ModParams), ctypes.POINTER(BlockMaskC), P, SZ, P]
+    lib.flex_attn_fwd_fp8_block_sparse.restype = I
     lib.flex_attn_bwd_workspace_size.argtypes = [I, I, I]
     lib.flex_attn_bwd_workspace_size.restype = SZ
     lib.flex_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams), I,
@@ -304,10 +308,28 @@ def _block_mask(kv_num_blocks, kv_indices, full_kv_num_blocks, full_kv_indices, 
 
 def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None, score_mod="none",
             mask_mod="none", window=0, offset=0, alibi_slopes=None, return_lse=True, out=None, lse_out=None,
-            workspace=None, status=None):
+            workspace=None, status=None, tile_map=None, doc_offsets=None, doc_offsets_kv=None):
     """8-bit forward (flex_attn_fwd_fp8): q8/k8/v8 are torch.float8_e4m3fn CUDA tensors in
     the layouts of fwd(); their values are descale_* times the codes.  Returns (O, LSE)
-    with O in bf16.  Head dim 128."""
+    with O in bf16.  Head dim 64 or 128.  Mods, captured tensors and tile_map as fwd()."""
+    return _fp8(None, q8, k8, v8, descale_q, descale_k, descale_v, scale, score_mod, mask_mod, window, offset,
+                alibi_slopes, return_lse, out, lse_out, workspace, status, tile_map, doc_offsets, doc_offsets_kv)
+
+
+def fwd_fp8_block_sparse(q8, k8, v8, kv_num_blocks, kv_indices, full_kv_num_blocks=None, full_kv_indices=None,
+                         descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None, score_mod="none", mask_mod="none",
+                         window=0, offset=0, alibi_slopes=None, return_lse=True, out=None, lse_out=None,
+                         workspace=None, status=None, tile_map=None, doc_offsets=None, doc_offsets_kv=None,
+                         block_size=128):
+    """fwd_fp8 with a block mask (flex_attn_fwd_fp8_block_sparse); the lists as for
+    fwd_block_sparse()."""
+    bm = _block_mask(kv_num_blocks, kv_indices, full_kv_num_blocks, full_kv_indices, q8.shape[2], block_size)
+    return _fp8(bm, q8, k8, v8, descale_q, descale_k, descale_v, scale, score_mod, mask_mod, window, offset,
+                alibi_slopes, return_lse, out, lse_out, workspace, status, tile_map, doc_offsets, doc_offsets_kv)
+
+
+def _fp8(bm, q8, k8, v8, descale_q, descale_k, descale_v, scale, score_mod, mask_mod, window, offset, alibi_slopes,
+         return_lse, out, lse_out, workspace, status, tile_map, doc_offsets, doc_offsets_kv):
     lib = load_library()
     for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
         _cuda_tensor(t, n)
@@ -336,13 +358,15 @@ def fwd_fp8(q8, k8, v8, descale_q=1.0, descale_k=1.0, descale_v=1.0, scale=None,
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q8.device)
     elif workspace.device != q8.device or not workspace.is_contiguous():
         raise FlexAttnError("workspace must be a contiguous tensor on q8's device")
-    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, None, None,
-                            _status_word(status, q8.device))
-    rc = lib.flex_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D, float(scale),
-                               float(descale_q), float(descale_k), float(descale_v), score, MASK_MODS[mask_mod],
-                               ctypes.byref(mp), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                               _stream(q8.device))
-    _check(rc, "flex_attn_fwd_fp8")
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, tile_map, alibi_slopes, doc_offsets,
+                            doc_offsets_kv, _status_word(status, q8.device))
+    args = (_ptr(q8), _ptr(k8), _ptr(v8), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D, float(scale),
+            float(descale_q), float(descale_k), float(descale_v), score, MASK_MODS[mask_mod], ctypes.byref(mp))
+    tail = (_ptr(workspace), workspace.numel() * workspace.element_size(), _stream(q8.device))
+    if bm is None:
+        _check(lib.flex_attn_fwd_fp8(*args, *tail), "flex_attn_fwd_fp8")
+    else:
+        _check(lib.flex_attn_fwd_fp8_block_sparse(*args, ctypes.byref(bm), *tail), "flex_attn_fwd_fp8_block_sparse")
     return o, lse
 
 

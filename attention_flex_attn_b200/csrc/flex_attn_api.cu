@@ -73,7 +73,8 @@ bool make_map_mask(CUtensorMap* map, const void* base, flex_dtype_t dt, int cap,
 }
 
 // [outer x rows x inner] bytes, box = 128 bytes x 128 rows x 1, 128-byte swizzle (the
-// 8-bit forward's tiles; inner must be a multiple of 16).
+// 8-bit forward's tiles; inner must be a multiple of 16; a box past inner or rows reads
+// zeros, which pads 64-byte rows and 64-row V^T tiles to the 128-byte tile width).
 bool make_map_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t outer) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -400,34 +401,45 @@ flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const voi
 }
 
 size_t flex_attn_fwd_fp8_workspace_size(int B, int Hkv, int Skv, int D) {
-  if (B < 1 || Hkv < 1 || Skv < 1 || D != kFp8D) return 0;
+  if (B < 1 || Hkv < 1 || Skv < 1 || (D != 64 && D != 128)) return 0;
   const size_t skv_pad = (static_cast<size_t>(Skv) + 127) / 128 * 128;
   return static_cast<size_t>(B) * Hkv * D * skv_pad;
 }
 
-flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int H,
-                                int Hkv, int Sq, int Skv, int D, float scale, float descale_q, float descale_k,
-                                float descale_v, int score_mod_id, int mask_mod_id,
-                                const flex_mod_params_t* mod_params, void* workspace, size_t workspace_bytes,
-                                flex_stream_t stream) {
+}  // extern "C"
+
+namespace flexattn {
+namespace {
+
+// Shared body of flex_attn_fwd_fp8 (bm == nullptr) and flex_attn_fwd_fp8_block_sparse.
+flex_status_t fp8_common(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int H, int Hkv,
+                         int Sq, int Skv, int D, float scale, float descale_q, float descale_k, float descale_v,
+                         int score_mod_id, int mask_mod_id, const flex_mod_params_t* mod_params,
+                         const flex_block_mask_t* bm, void* workspace, size_t workspace_bytes, flex_stream_t stream) {
   if (!q8 || !k8 || !v8 || !o) return FLEX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
   for (float f : {scale, descale_q, descale_k, descale_v})
     if (!(f > 0.f) || !std::isfinite(f)) return FLEX_ERR_INVALID_ARG;
-  if (D != kFp8D) return FLEX_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
   if (score_mod_id != FLEX_SCORE_NONE && score_mod_id != FLEX_SCORE_ALIBI && score_mod_id != FLEX_SCORE_ALIBI_SLOPES)
     return FLEX_ERR_INVALID_ARG;
   const int mask = mask_kind(mask_mod_id);
   if (mask < 0) return FLEX_ERR_INVALID_ARG;
-  if (mask == kMaskDocument || mask == kMaskDocumentCausal) return FLEX_ERR_UNSUPPORTED;
   const flex_mod_params_t zero{};
   const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
   if (mask == kMaskSliding && mp.window < 1) return FLEX_ERR_INVALID_ARG;
-  if (mp.flags & FLEX_FLAG_TILE_MAP) return FLEX_ERR_UNSUPPORTED;
   if (score_mod_id == FLEX_SCORE_ALIBI_SLOPES) {
     if (!mp.alibi_slopes) return FLEX_ERR_INVALID_ARG;
     if (!aligned4(mp.alibi_slopes)) return FLEX_ERR_MISALIGNED;
   }
+  if (const flex_status_t ds = check_documents(mask, mp); ds != FLEX_OK) return ds;
+  if ((mask == kMaskDocument || mask == kMaskDocumentCausal) && (Skv + kBN - 1) / kBN > kMaxBlockKeyTiles)
+    return FLEX_ERR_UNSUPPORTED;
+  if (bm) {
+    if (const flex_status_t bs = check_block_mask(*bm, B, H, Sq, Skv); bs != FLEX_OK) return bs;
+  }
+  const bool want_map = (mp.flags & FLEX_FLAG_TILE_MAP) != 0;
+  if (want_map && !mp.tile_map_out) return FLEX_ERR_INVALID_ARG;
   const size_t need = flex_attn_fwd_fp8_workspace_size(B, Hkv, Skv, D);
   if (!workspace || workspace_bytes < need) return FLEX_ERR_WORKSPACE;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(workspace) ||
@@ -447,6 +459,7 @@ flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, 
   Fp8Params p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
+  p.tile_map = want_map ? mp.tile_map_out : nullptr;
   p.status = st;
   p.H = H;
   p.Hkv = Hkv;
@@ -454,6 +467,7 @@ flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, 
   p.Sq = Sq;
   p.Skv = Skv;
   p.Skv_pad = skv_pad;
+  p.D = D;
   p.n_qtiles = n_qtiles;
   p.n_ktiles = (Skv + kBN - 1) / kBN;
   p.n_pairs = n_pairs;
@@ -461,9 +475,38 @@ flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, 
   p.descale_v = descale_v;
   p.slopes = score_mod_id == FLEX_SCORE_ALIBI_SLOPES ? mp.alibi_slopes : nullptr;
   p.mask = mask_args(mask, mp, Skv);
+  if (bm) {
+    p.blocks = VisitLists{{bm->kv_num_blocks, bm->full_kv_num_blocks}, {bm->kv_indices, bm->full_kv_indices},
+                          bm->max_blocks, bm->batch == 1 ? 0 : bm->heads, bm->heads == 1 ? 0 : 1};
+  }
   const int score = score_mod_id == FLEX_SCORE_NONE ? kScoreNone : kScoreAlibi;
-  return fp8_dispatch(score, mask, static_cast<const uint8_t*>(v8), static_cast<uint8_t*>(workspace), bhkv, m, p,
-                      static_cast<int>(bh * n_pairs), reinterpret_cast<cudaStream_t>(stream));
+  return fp8_dispatch(score, mask, bm != nullptr, static_cast<const uint8_t*>(v8), static_cast<uint8_t*>(workspace),
+                      bhkv, m, p, static_cast<int>(bh * n_pairs), reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace flexattn
+
+extern "C" {
+
+flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse, int B, int H,
+                                int Hkv, int Sq, int Skv, int D, float scale, float descale_q, float descale_k,
+                                float descale_v, int score_mod_id, int mask_mod_id,
+                                const flex_mod_params_t* mod_params, void* workspace, size_t workspace_bytes,
+                                flex_stream_t stream) {
+  return fp8_common(q8, k8, v8, o, lse, B, H, Hkv, Sq, Skv, D, scale, descale_q, descale_k, descale_v, score_mod_id,
+                    mask_mod_id, mod_params, nullptr, workspace, workspace_bytes, stream);
+}
+
+flex_status_t flex_attn_fwd_fp8_block_sparse(const void* q8, const void* k8, const void* v8, void* o, float* lse,
+                                             int B, int H, int Hkv, int Sq, int Skv, int D, float scale,
+                                             float descale_q, float descale_k, float descale_v, int score_mod_id,
+                                             int mask_mod_id, const flex_mod_params_t* mod_params,
+                                             const flex_block_mask_t* block_mask, void* workspace,
+                                             size_t workspace_bytes, flex_stream_t stream) {
+  if (!block_mask) return FLEX_ERR_INVALID_ARG;
+  return fp8_common(q8, k8, v8, o, lse, B, H, Hkv, Sq, Skv, D, scale, descale_q, descale_k, descale_v, score_mod_id,
+                    mask_mod_id, mod_params, block_mask, workspace, workspace_bytes, stream);
 }
 
 size_t flex_attn_bwd_workspace_size(int B, int H, int Sq) {

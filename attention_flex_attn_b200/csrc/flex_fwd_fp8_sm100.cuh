@@ -7,7 +7,8 @@
 //   S = q8 k8^T (tcgen05 kind::f8f6f4, fp32 in TMEM) * (scale * descale_q * descale_k),
 //   P rounded to e4m3 for the P.V product, O = descale_v * (P v8) / l.
 // The structure is the 16-bit kernel's (two 128-row query tiles per CTA, one MMA-issuing
-// thread, a TMA producer that publishes step records, two softmax warpgroups), with two
+// thread, a TMA producer that publishes step records, two softmax warpgroups, the same
+// visit sets for block masks and document masks, the same debug tile map), with two
 // differences that keep both operands of every product K-major, the form every tcgen05
 // kind accepts:
 //   - P goes through shared memory (each softmax thread writes its row's 128 e4m3 values
@@ -16,7 +17,10 @@
 //     fp8_transpose_v_kernel writes first (keys padded to a multiple of 128 with zeros).
 // P is computed as 2^(x - m + 6) with the O rescale threshold at 2^2, so its largest value
 // is 2^8 <= 448 (the e4m3 maximum) and values down to 2^-15 of the row maximum survive the
-// 8-bit rounding; the factor 2^6 cancels between O and l.  Head dim 128.
+// 8-bit rounding; the factor 2^6 cancels between O and l.  Head dim 128 or 64: tiles are
+// always 128 bytes wide; at D = 64 the TMA boxes of Q and K run past the 64-byte rows and
+// the V^T box past its 64 rows, and TMA fills those bytes with zeros, so S gains only zero
+// products and O's columns 64..127 stay zero (they are not stored).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -30,7 +34,7 @@
 
 namespace flexattn {
 
-constexpr int kFp8D = 128;
+constexpr int kFp8D = 128;  // width of every 8-bit tile in bytes (head dims 64 and 128 fit)
 constexpr float kP8Shift = 6.0f;      // log2 of the factor P carries into the 8-bit product
 constexpr float kP8Rescale = 2.0f;    // O rescale threshold (log2) for the 8-bit path
 #ifndef FLEX_FP8_EMU_PAIRS
@@ -43,15 +47,18 @@ constexpr int kFp8EmuPairs = FLEX_FP8_EMU_PAIRS;
 struct Fp8Params {
   __nv_bfloat16* o;
   float* lse;
+  uint8_t* tile_map;  // debug tile map or nullptr
   unsigned* status;
-  int H, Hkv, G, Sq, Skv, Skv_pad;
+  int H, Hkv, G, Sq, Skv, Skv_pad, D;
   int n_qtiles, n_ktiles, n_pairs;
   float scale_log2;   // scale * descale_q * descale_k * log2(e)
   float descale_v;
   const float* slopes;
-  MaskArgs mask;
+  MaskArgs mask;      // document rules: boundaries of batch 0, advanced per batch
+  VisitLists blocks;  // block mask (BLOCKS instantiations)
 };
 
+template <bool BLOCKS = false, bool DOC = false>
 struct Fp8Smem {
   static constexpr int kTileBytes = kBM * kFp8D;  // 128 rows x 128 bytes
   static constexpr int kSlots = 10;               // K / V^T ring
@@ -64,7 +71,10 @@ struct Fp8Smem {
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   static constexpr int kRecOff = kTmemPtrOff + 16;
   static constexpr int kRecBytes = ((kSlots + 1) * 4 + 15) / 16 * 16;
-  static constexpr int kBytes = kRecOff + kRecBytes;
+  // document rules: the documents of each tile's first and last row; then the visit sets
+  static constexpr int kDocOff = kRecOff + kRecBytes;
+  static constexpr int kBlkOff = kDocOff + (DOC ? 16 : 0);
+  static constexpr int kBytes = kBlkOff + fwd_bitmaps(BLOCKS, DOC) * kBlkWords * 4;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 227 * 1024, "shared memory per CTA exceeded");
 };
@@ -91,28 +101,29 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
-// V [rows, Skv, 128] bytes -> V^T [rows, 128, Skv_pad] bytes (keys past Skv are zero).
+// V [rows, Skv, D] bytes -> V^T [rows, D, Skv_pad] bytes (keys past Skv are zero).
 // One CTA per (row, 128-key tile), 256 threads.  (A template so that every translation
 // unit that sees this header shares one definition.)
 template <int D>
 __global__ void __launch_bounds__(256) fp8_transpose_v_kernel(const uint8_t* v, uint8_t* vt, int Skv, int Skv_pad,
                                                               int n_tiles) {
-  static_assert(D == kFp8D, "the 8-bit path has head dim 128");
-  __shared__ uint8_t tile[128][128 + 16];
+  static_assert(D == 64 || D == 128, "the 8-bit path has head dim 64 or 128");
+  constexpr int kPieces = D / 16;  // 16-byte pieces of one key row
+  __shared__ uint8_t tile[128][D + 16];
   const int64_t row = blockIdx.x / n_tiles;
   const int j0 = (blockIdx.x % n_tiles) * 128;
-  const uint8_t* src = v + row * static_cast<int64_t>(Skv) * kFp8D;
-  for (int e = threadIdx.x; e < 128 * 8; e += 256) {  // 16-byte pieces of 128 key rows
-    const int jj = e >> 3, piece = e & 7;
+  const uint8_t* src = v + row * static_cast<int64_t>(Skv) * D;
+  for (int e = threadIdx.x; e < 128 * kPieces; e += 256) {  // 16-byte pieces of 128 key rows
+    const int jj = e / kPieces, piece = e % kPieces;
     uint4 val = make_uint4(0, 0, 0, 0);
-    if (j0 + jj < Skv) val = *reinterpret_cast<const uint4*>(src + static_cast<int64_t>(j0 + jj) * kFp8D + piece * 16);
+    if (j0 + jj < Skv) val = *reinterpret_cast<const uint4*>(src + static_cast<int64_t>(j0 + jj) * D + piece * 16);
     const uint8_t* b = reinterpret_cast<const uint8_t*>(&val);
 #pragma unroll
     for (int x = 0; x < 16; ++x) tile[jj][piece * 16 + x] = b[x];
   }
   __syncthreads();
-  uint8_t* dst = vt + row * static_cast<int64_t>(kFp8D) * Skv_pad;
-  for (int e = threadIdx.x; e < 128 * 8; e += 256) {  // dim d, 16 consecutive keys
+  uint8_t* dst = vt + row * static_cast<int64_t>(D) * Skv_pad;
+  for (int e = threadIdx.x; e < D * 8; e += 256) {  // dim d, 16 consecutive keys
     const int d = e >> 3, piece = e & 7;
     alignas(16) uint8_t b[16];
 #pragma unroll
@@ -122,11 +133,13 @@ __global__ void __launch_bounds__(256) fp8_transpose_v_kernel(const uint8_t* v, 
   }
 }
 
-template <int SCORE, int MASK>
+template <int SCORE, int MASK, bool BLOCKS>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     flex_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmVt, const Fp8Params p) {
-  using L = Fp8Smem;
+  constexpr bool kDoc = is_doc_mask(MASK);
+  constexpr bool kBits = BLOCKS || kDoc;
+  using L = Fp8Smem<BLOCKS, kDoc>;
   constexpr int NS = L::kSlots;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kIdesc = idesc_f16(0, kBM, kBN, 0);  // e4m3 x e4m3 -> f32, both K-major
@@ -156,15 +169,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int bkv = b * p.Hkv + h / p.G;
   int q0[2], q1[2], lo[2], hi[2];
   auto sel = [](const int (&a)[2], int k) { return k ? a[1] : a[0]; };
+  MaskArgs mk = p.mask;
+  if constexpr (kDoc) {
+    mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
+    mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
+  }
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int qt = 2 * pair + k;
     q0[k] = qt * kBM;
     q1[k] = min(q0[k] + kBM, p.Sq);
     lo[k] = hi[k] = 0;
-    if (qt < p.n_qtiles) tile_range<MASK>(q0[k], q1[k], kBN, p.mask, lo[k], hi[k]);
+    if (qt < p.n_qtiles && !kDoc) tile_range<MASK>(q0[k], q1[k], kBN, mk, lo[k], hi[k]);
   }
-  auto cursor = [&](int k) { return RangeCursor(sel(lo, k), sel(hi, k)); };
+  // visit sets of the two query tiles (block masks, document masks), as in the 16-bit kernel
+  uint32_t* blk = reinterpret_cast<uint32_t*>(sgen + L::kBlkOff);
+  if constexpr (kBits)
+    build_visit_sets<MASK, BLOCKS>(blk, reinterpret_cast<int*>(sgen + L::kDocOff), p.blocks, pair, b, h, q0, q1, lo,
+                                   hi, mk, p.n_qtiles, p.n_ktiles, p.Skv);
+  auto cursor = [&](int k) {
+    if constexpr (kBits) return BitCursor(visit_act_bits(blk, k), visit_full_bits(blk, k), p.n_ktiles);
+    else return RangeCursor(sel(lo, k), sel(hi, k));
+  };
+  auto has = [&](int k, int j) -> bool {  // debug tile map only
+    if constexpr (kBits) return bits_has(visit_act_bits(blk, k), j);
+    else return j >= sel(lo, k) && j < sel(hi, k);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -190,7 +220,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
-  const bool act0 = lo[0] < hi[0], act1 = lo[1] < hi[1];
+  const bool act0 = cursor(0).cur >= 0, act1 = cursor(1).cur >= 0;
   const bool any_work = act0 || act1;
 
   if (warp < kSoftmaxWarp0) {
@@ -200,7 +230,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int r = 0;
       bool ok = true;
       auto c0 = cursor(0), c1 = cursor(1);
-      auto make_rec = [](RangeCursor a0, RangeCursor a1) -> uint32_t {
+      auto make_rec = [](auto a0, auto a1) -> uint32_t {
         const int j = max(a0.cur, a1.cur);
         if (j < 0) return kRecEnd;
         const bool i0 = a0.cur == j, i1 = a1.cur == j;
@@ -346,6 +376,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tO = tmem + lane_off + 256u + 128u * k;
     const bool tile_valid = (2 * pair + k) < p.n_qtiles;
     const bool act_k = k == 0 ? act0 : act1;
+    const int qt = 2 * pair + k;
+    const bool write_map = p.tile_map != nullptr && bh == 0 && tile_valid && threadIdx.x % 128 == 0;
+    if (write_map) {
+      for (int u = 0; u < p.n_ktiles; ++u)
+        if (!act_k || !has(k, u)) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + u] = kTileEmpty;
+    }
+    // Document rules: this row's kept interval, looked up once.
+    int64_t row_lo = 0, row_hi = -1;
+    if constexpr (kDoc) row_interval<MASK>(qi, mk, row_lo, row_hi);
     // this thread's row of P in the 128-byte-swizzled tile: chunk c lives at chunk c ^ (row % 8)
     uint8_t* prow = sgen + L::kPOff + k * L::kTileBytes + row * 128;
     const int swz = row & 7;
@@ -360,6 +399,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int n = 0;
     auto cur = cursor(k);
     for (int j = act_k ? cur.cur : -1; j >= 0; j = cur.cur, ++n) {
+      // with block masks and document masks the class comes from the walk
+      const int cls_blk = cur.cur_full ? (j * kBN + kBN > p.Skv ? kTileFullRagged : kTileFull) : kTilePartial;
       cur.advance();
       const bool got = mbar_wait(bar_s(k), static_cast<uint32_t>(n) & 1u, p.status, kStatusFwdTimeout,
                                  kWaitTimeoutNs) &&
@@ -370,7 +411,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tc_fence_after();
       const int k0 = j * kBN;
-      const int cls = tile_class<MASK>(q0k, q1k, k0, kBN, p.mask);
+      int cls;
+      if constexpr (kBits) cls = cls_blk;
+      else cls = tile_class<MASK>(q0k, q1k, k0, kBN, mk);
+      if (write_map)
+        p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] =
+            static_cast<uint8_t>(cls == kTileFullRagged ? kTilePartial : cls);
       uint32_t sr[kBN];
       tmem_ld128(tS, sr);
       float* s = reinterpret_cast<float*>(sr);
@@ -381,7 +427,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (cls != kTileFull) {
         int c_lo, c_hi;
-        col_interval<MASK>(qi, k0, p.mask, c_lo, c_hi);
+        if (kBits && cls == kTileFullRagged)
+          col_interval<kMaskNone>(qi, k0, mk, c_lo, c_hi);
+        else if constexpr (kDoc)
+          col_interval_of(row_lo, row_hi, k0, c_lo, c_hi);
+        else
+          col_interval<MASK>(qi, k0, mk, c_lo, c_hi);
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
           if (c < c_lo || c > c_hi) s[c] = -INFINITY;
@@ -475,9 +526,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool row_ok = qi < p.Sq;
       const bool has_mass = ran && m_used != -INFINITY && l_sum > 0.f;
       const float inv = has_mass ? p.descale_v / l_sum : 0.f;
-      __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * p.Sq + qi) * kFp8D;
+      __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * p.Sq + qi) * p.D;
 #pragma unroll 1
-      for (int c = 0; c < kFp8D; c += 32) {
+      for (int c = 0; c < p.D; c += 32) {
         uint32_t r[32];
         if (ran) tmem_ld32(tO + c, r);
         uint32_t w[16];

@@ -230,6 +230,121 @@ __device__ __forceinline__ void bits_set_range(uint32_t* w, int u_lo, int u_hi) 
 
 constexpr bool is_doc_mask(int mask) { return mask == kMaskDocument || mask == kMaskDocumentCausal; }
 
+// Block lists as the forward kernels take them: [0] partial, [1] full; counts
+// [rows x n_qtiles], indices [rows x n_qtiles x max]; the row of (b, h) is
+// b * b_stride + h * h_stride (a stride of 0 shares one row).
+struct VisitLists {
+  const int32_t* num[2];
+  const int32_t* idx[2];
+  int max, b_stride, h_stride;
+};
+
+// Bitmaps of the visit sets in shared memory (kBlkWords words each): full_k = the key tiles
+// query tile k (= 2 * pair + k) keeps whole, act_k = every key tile it visits, and with a
+// block mask and a document mask both, doc_k = the tiles its documents reach.
+__device__ __forceinline__ uint32_t* visit_full_bits(uint32_t* blk, int k) { return blk + k * kBlkWords; }
+__device__ __forceinline__ uint32_t* visit_act_bits(uint32_t* blk, int k) { return blk + (2 + k) * kBlkWords; }
+
+// The visit sets of a CTA's two query tiles (all threads of the CTA call it; it ends
+// with the sets complete after a barrier of the caller's).  Document masks build them
+// from the documents the tiles' rows span; block masks from the tiles' two lists (with
+// a document mask as well, filtered by the document sets); a partial block the mask_mod
+// drops whole is left out and one it keeps whole counts as full, so lists read off the
+// analytic tile map reproduce the analytic kernel exactly.  lo/hi: the analytic key-tile
+// ranges (mask rules other than the document ones).
+template <int MASK, bool BLOCKS>
+__device__ __forceinline__ void build_visit_sets(uint32_t* blk, int* doc_rows, const VisitLists& bl, int pair,
+                                                 int b, int h, const int (&q0)[2], const int (&q1)[2],
+                                                 const int (&lo)[2], const int (&hi)[2], const MaskArgs& mk,
+                                                 int n_qtiles, int n_ktiles, int Skv) {
+  constexpr bool kDoc = MASK == kMaskDocument || MASK == kMaskDocumentCausal;
+  auto sel = [](const int (&a)[2], int k) { return k ? a[1] : a[0]; };
+  auto full_bits = [&](int k) { return visit_full_bits(blk, k); };
+  auto act_bits = [&](int k) { return visit_act_bits(blk, k); };
+  auto doc_bits = [&](int k) { return BLOCKS ? blk + (4 + k) * kBlkWords : blk + (2 + k) * kBlkWords; };
+  {
+    for (int w = threadIdx.x; w < fwd_bitmaps(BLOCKS, kDoc) * kBlkWords; w += kFwdThreads) blk[w] = 0u;
+    if constexpr (kDoc) {
+      if (threadIdx.x < 4) {  // four independent binary searches, one per lane
+        const int k = threadIdx.x >> 1, qt = 2 * pair + k;
+        doc_rows[threadIdx.x] =
+            qt < n_qtiles ? doc_floor(mk.off_q, mk.n_docs, (threadIdx.x & 1) ? sel(q1, k) - 1 : sel(q0, k)) : -1;
+      }
+    }
+    __syncthreads();
+    // Document rules: tile k's class bounds (the first row's last key, the last row's
+    // first key); FULL iff lo_last <= k0 and k1 - 1 <= hi_first.
+    int64_t lo_last[2] = {0, 0}, hi_first[2] = {-1, -1};
+    if constexpr (kDoc) {
+      constexpr bool kCausal = MASK == kMaskDocumentCausal;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (2 * pair + k >= n_qtiles) continue;
+        int64_t t;
+        doc_interval(mk, doc_rows[2 * k + 1], sel(q1, k) - 1, kCausal, lo_last[k], t);
+        doc_interval(mk, doc_rows[2 * k], sel(q0, k), kCausal, t, hi_first[k]);
+      }
+      // every document with rows in tile k: the key tiles those rows keep
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (2 * pair + k >= n_qtiles) continue;
+        const int d0 = max(doc_rows[2 * k], 0), d1 = min(doc_rows[2 * k + 1], mk.n_docs - 1);
+        for (int d = d0 + threadIdx.x; d <= d1; d += kFwdThreads) {
+          const int64_t r0 = max(static_cast<int64_t>(sel(q0, k)), static_cast<int64_t>(__ldg(mk.off_q + d)));
+          const int64_t r1 = min(static_cast<int64_t>(sel(q1, k)), static_cast<int64_t>(__ldg(mk.off_q + d + 1)));
+          if (r0 >= r1) continue;  // no row of this document in the tile
+          int64_t a, e;
+          doc_interval(mk, d, r1 - 1, kCausal, a, e);  // the union of its rows' intervals
+          if (a > e) continue;
+          bits_set_range(doc_bits(k), static_cast<int>(a / kBN), static_cast<int>(e / kBN));
+        }
+        if (!BLOCKS && threadIdx.x == 0) {
+          const int64_t f_lo = (lo_last[k] + kBN - 1) / kBN, f_hi = (hi_first[k] + 1) / kBN - 1;
+          if (f_lo <= f_hi) bits_set_range(full_bits(k), static_cast<int>(f_lo), static_cast<int>(f_hi));
+        }
+      }
+      if constexpr (BLOCKS) __syncthreads();  // the document sets filter the lists below
+    }
+    if constexpr (BLOCKS) {
+      const int64_t row0 = static_cast<int64_t>(b) * bl.b_stride + static_cast<int64_t>(h) * bl.h_stride;
+      // list l = 2 * k + f: query tile 2 * pair + k, f = 0 partial / 1 full (selects, not
+      // indexing, so that nothing here is forced into local memory)
+      auto count = [&](int k, int f) {
+        const int qt = 2 * pair + k;
+        const int32_t* num = f ? bl.num[1] : bl.num[0];
+        const int c = (qt < n_qtiles && num != nullptr) ? num[row0 * n_qtiles + qt] : 0;
+        return c < 0 ? 0 : (c > bl.max ? bl.max : c);
+      };
+      const int c00 = count(0, 0), c01 = count(0, 1), c10 = count(1, 0), c11 = count(1, 1);
+      for (int e = threadIdx.x; e < 4 * bl.max; e += kFwdThreads) {
+        const int l = e / bl.max, c = e - l * bl.max;
+        const int k = l >> 1, f = l & 1;
+        const int cl = k ? (f ? c11 : c10) : (f ? c01 : c00);
+        if (c >= cl) continue;
+        const int32_t* idx = f ? bl.idx[1] : bl.idx[0];
+        const int u = idx[(row0 * n_qtiles + 2 * pair + k) * bl.max + c];
+        if (u < 0 || u >= n_ktiles) continue;
+        bool full = f == 1;
+        if (!full) {
+          // a partial tile the mask_mod drops whole keeps nothing; one it keeps whole
+          // needs no per-element mask
+          if constexpr (kDoc) {
+            if (!bits_has(doc_bits(k), u)) continue;
+            full = tile_class_of(k ? lo_last[1] : lo_last[0], k ? hi_first[1] : hi_first[0], u * kBN, kBN,
+                                 Skv) == kTileFull;
+          } else {
+            if (u < sel(lo, k) || u >= sel(hi, k)) continue;
+            full = tile_class<MASK>(sel(q0, k), sel(q1, k), u * kBN, kBN, mk) == kTileFull;
+          }
+        }
+        const uint32_t bit = 1u << (u & 31);
+        if (full) atomicOr(full_bits(k) + (u >> 5), bit);
+        atomicOr(act_bits(k) + (u >> 5), bit);
+      }
+    }
+  }
+}
+
 template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     flex_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -289,96 +404,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   // ---------------------------------------------------------------- visit bitmaps
   // With a block mask or a document mask the key tiles a query tile visits are a set, not
-  // a range: full_k = tiles needing no element mask, act_k = every tile query tile k
-  // visits (complete at the setup barrier below).  Document masks build them from the
-  // documents; with a block mask as well, the document sets doc_k filter the lists.
+  // a range (build_visit_sets).
   constexpr bool kBits = BLOCKS || kDoc;
   uint32_t* blk = reinterpret_cast<uint32_t*>(sgen + L::kBlkOff);
   auto full_bits = [&](int k) { return blk + k * kBlkWords; };
   auto act_bits = [&](int k) { return blk + (2 + k) * kBlkWords; };
-  auto doc_bits = [&](int k) { return BLOCKS ? blk + (4 + k) * kBlkWords : blk + (2 + k) * kBlkWords; };
   int* doc_rows = reinterpret_cast<int*>(sgen + L::kDocOff);  // doc_floor of q0/q1-1 per tile
   if constexpr (kBits) {
-    for (int w = threadIdx.x; w < fwd_bitmaps(BLOCKS, kDoc) * kBlkWords; w += kFwdThreads) blk[w] = 0u;
-    if constexpr (kDoc) {
-      if (threadIdx.x < 4) {  // four independent binary searches, one per lane
-        const int k = threadIdx.x >> 1, qt = 2 * pair + k;
-        doc_rows[threadIdx.x] = qt < p.n_qtiles ? doc_floor(mk.off_q, mk.n_docs,
-                                                            (threadIdx.x & 1) ? sel(q1, k) - 1 : sel(q0, k))
-                                                : -1;
-      }
-    }
-    __syncthreads();
-    // Document rules: tile k's class bounds (the first row's last key, the last row's
-    // first key); FULL iff lo_last <= k0 and k1 - 1 <= hi_first.
-    int64_t lo_last[2] = {0, 0}, hi_first[2] = {-1, -1};
-    if constexpr (kDoc) {
-      constexpr bool kCausal = MASK == kMaskDocumentCausal;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        if (2 * pair + k >= p.n_qtiles) continue;
-        int64_t t;
-        doc_interval(mk, doc_rows[2 * k + 1], sel(q1, k) - 1, kCausal, lo_last[k], t);
-        doc_interval(mk, doc_rows[2 * k], sel(q0, k), kCausal, t, hi_first[k]);
-      }
-      // every document with rows in tile k: the key tiles those rows keep
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        if (2 * pair + k >= p.n_qtiles) continue;
-        const int d0 = max(doc_rows[2 * k], 0), d1 = min(doc_rows[2 * k + 1], mk.n_docs - 1);
-        for (int d = d0 + threadIdx.x; d <= d1; d += kFwdThreads) {
-          const int64_t r0 = max(static_cast<int64_t>(sel(q0, k)), static_cast<int64_t>(__ldg(mk.off_q + d)));
-          const int64_t r1 = min(static_cast<int64_t>(sel(q1, k)), static_cast<int64_t>(__ldg(mk.off_q + d + 1)));
-          if (r0 >= r1) continue;  // no row of this document in the tile
-          int64_t a, e;
-          doc_interval(mk, d, r1 - 1, kCausal, a, e);  // the union of its rows' intervals
-          if (a > e) continue;
-          bits_set_range(doc_bits(k), static_cast<int>(a / kBN), static_cast<int>(e / kBN));
-        }
-        if (!BLOCKS && threadIdx.x == 0) {
-          const int64_t f_lo = (lo_last[k] + kBN - 1) / kBN, f_hi = (hi_first[k] + 1) / kBN - 1;
-          if (f_lo <= f_hi) bits_set_range(full_bits(k), static_cast<int>(f_lo), static_cast<int>(f_hi));
-        }
-      }
-      if constexpr (BLOCKS) __syncthreads();  // the document sets filter the lists below
-    }
-    if constexpr (BLOCKS) {
-      const int64_t row0 = static_cast<int64_t>(b) * p.blk_b_stride + static_cast<int64_t>(h) * p.blk_h_stride;
-      // list l = 2 * k + f: query tile 2 * pair + k, f = 0 partial / 1 full (selects, not
-      // indexing, so that nothing here is forced into local memory)
-      auto count = [&](int k, int f) {
-        const int qt = 2 * pair + k;
-        const int32_t* num = f ? p.blk_num[1] : p.blk_num[0];
-        const int c = (qt < p.n_qtiles && num != nullptr) ? num[row0 * p.n_qtiles + qt] : 0;
-        return c < 0 ? 0 : (c > p.blk_max ? p.blk_max : c);
-      };
-      const int c00 = count(0, 0), c01 = count(0, 1), c10 = count(1, 0), c11 = count(1, 1);
-      for (int e = threadIdx.x; e < 4 * p.blk_max; e += kFwdThreads) {
-        const int l = e / p.blk_max, c = e - l * p.blk_max;
-        const int k = l >> 1, f = l & 1;
-        const int cl = k ? (f ? c11 : c10) : (f ? c01 : c00);
-        if (c >= cl) continue;
-        const int32_t* idx = f ? p.blk_idx[1] : p.blk_idx[0];
-        const int u = idx[(row0 * p.n_qtiles + 2 * pair + k) * p.blk_max + c];
-        if (u < 0 || u >= p.n_ktiles) continue;
-        bool full = f == 1;
-        if (!full) {
-          // a partial tile the mask_mod drops whole keeps nothing; one it keeps whole
-          // needs no per-element mask
-          if constexpr (kDoc) {
-            if (!bits_has(doc_bits(k), u)) continue;
-            full = tile_class_of(k ? lo_last[1] : lo_last[0], k ? hi_first[1] : hi_first[0], u * kBN, kBN,
-                                 p.Skv) == kTileFull;
-          } else {
-            if (u < sel(lo, k) || u >= sel(hi, k)) continue;
-            full = tile_class<MASK>(sel(q0, k), sel(q1, k), u * kBN, kBN, mk) == kTileFull;
-          }
-        }
-        const uint32_t bit = 1u << (u & 31);
-        if (full) atomicOr(full_bits(k) + (u >> 5), bit);
-        atomicOr(act_bits(k) + (u >> 5), bit);
-      }
-    }
+    const VisitLists bl{{p.blk_num[0], p.blk_num[1]}, {p.blk_idx[0], p.blk_idx[1]}, p.blk_max, p.blk_b_stride,
+                        p.blk_h_stride};
+    build_visit_sets<MASK, BLOCKS>(blk, doc_rows, bl, pair, b, h, q0, q1, lo, hi, mk, p.n_qtiles, p.n_ktiles, p.Skv);
   }
   // The walk over query tile k's key tiles (valid after the setup barrier); the CTA's
   // steps are the union of both walks: j = max of the two cursors.

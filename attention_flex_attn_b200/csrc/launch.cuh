@@ -21,10 +21,10 @@ struct Fp8Maps {
   CUtensorMap q, k, vt;
 };
 
-// V transpose into vt, then the 8-bit forward over (score_mod, mask_mod)
+// V transpose into vt, then the 8-bit forward over (score_mod, mask_mod, block mask)
 // (flex_fwd_fp8.cu).
-flex_status_t fp8_dispatch(int score, int mask, const uint8_t* v, uint8_t* vt, int64_t kv_rows, const Fp8Maps& m,
-                           const Fp8Params& p, int n_units, cudaStream_t s);
+flex_status_t fp8_dispatch(int score, int mask, bool blocks, const uint8_t* v, uint8_t* vt, int64_t kv_rows,
+                           const Fp8Maps& m, const Fp8Params& p, int n_units, cudaStream_t s);
 
 // Forward over every (dtype, score_mod, mask_mod) instantiation of one head dim and
 // block-mask mode.  Instantiated in flex_fwd_d{64,128}{,_blocks}.cu.

@@ -182,7 +182,7 @@ flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const voi
 
 /*
  * flex_attn_fwd_fp8_workspace_size -- bytes of device workspace flex_attn_fwd_fp8 needs
- * (a transposed copy of V, keys padded to a multiple of 128); 0 for D != 128.
+ * (a transposed copy of V, keys padded to a multiple of 128); 0 for D other than 64, 128.
  */
 size_t flex_attn_fwd_fp8_workspace_size(int B, int Hkv, int Skv, int D);
 
@@ -193,11 +193,10 @@ size_t flex_attn_fwd_fp8_workspace_size(int B, int Hkv, int Skv, int D);
  * descale_v * v8.  Computes O = softmax(mask_mod(score_mod(scale * q . k))) v with
  * fp32 accumulation; the probabilities enter the P.V product rounded to e4m3 (scaled
  * into the format's range and back, see the kernel header); O is written in bf16
- * [B, H, Sq, 128], LSE (natural log) in fp32 [B, H, Sq] (NULL allowed).
- *   D must be 128 (FLEX_ERR_UNSUPPORTED otherwise); scale and the descales finite, > 0.
- *   score_mod_id: NONE, ALIBI, ALIBI_SLOPES; mask_mod_id: NONE, CAUSAL, CAUSAL_FAST,
- *   SLIDING_WINDOW, KV_LE_Q_PLUS_OFFSET (the document rules and the tile map flag give
- *   FLEX_ERR_UNSUPPORTED).
+ * [B, H, Sq, D], LSE (natural log) in fp32 [B, H, Sq] (NULL allowed).
+ *   D must be 64 or 128 (FLEX_ERR_UNSUPPORTED otherwise); scale and the descales finite, > 0.
+ *   score_mod_id, mask_mod_id, mod_params: as for flex_attn_fwd (every mod, the captured
+ *   tensors, the debug tile map).
  *   workspace: at least flex_attn_fwd_fp8_workspace_size(B, Hkv, Skv, D) bytes,
  *   16-byte aligned; overwritten.
  */
@@ -206,6 +205,19 @@ flex_status_t flex_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, 
                                 float descale_q, float descale_k, float descale_v, int score_mod_id,
                                 int mask_mod_id, const flex_mod_params_t* mod_params, void* workspace,
                                 size_t workspace_bytes, flex_stream_t stream);
+
+/*
+ * flex_attn_fwd_fp8_block_sparse -- flex_attn_fwd_fp8 with a block mask: the key tiles each
+ * query tile visits come from block_mask (the rules and limits of
+ * flex_attn_fwd_block_sparse), the rest as flex_attn_fwd_fp8.
+ */
+flex_status_t flex_attn_fwd_fp8_block_sparse(const void* q8, const void* k8, const void* v8, void* o,
+                                             float* lse, int B, int H, int Hkv, int Sq, int Skv, int D,
+                                             float scale, float descale_q, float descale_k,
+                                             float descale_v, int score_mod_id, int mask_mod_id,
+                                             const flex_mod_params_t* mod_params,
+                                             const flex_block_mask_t* block_mask, void* workspace,
+                                             size_t workspace_bytes, flex_stream_t stream);
 
 /*
  * flex_attn_bwd_workspace_size -- bytes of device workspace flex_attn_bwd needs

@@ -195,16 +195,22 @@ def test_fp8_rejects_bad_args_on_host(lib):
         return lib.flex_attn_fwd_fp8(P(q), P(16), P(16), P(16), None, 1, 2, 1, 8, 8, D, scale, dq, dk, dv, score,
                                      mask, ctypes.byref(mp) if mp is not None else None, P(ws), wsb, None)
     assert f8(q=0) == 1
-    assert f8(D=64) == 2
+    assert f8(D=96) == 2
     assert f8(dq=0.0) == 1
     assert f8(dv=float("inf")) == 1
-    assert f8(mask=5) == 2                                   # document rules: not on the 8-bit path
-    assert f8(mp=fa.ModParams(0, 0, 1, 16, None, None, None, 0)) == 2   # tile map: not on the 8-bit path
+    assert f8(mask=5) == 1                                   # document rules without boundaries
+    assert f8(mp=fa.ModParams(0, 0, 1, None, None, None, None, 0)) == 1  # tile map flag without a buffer
+    bm = fa.BlockMaskC(32, 64, None, None, 1, 3, 1, 128, 128)           # batch must be 1 or B
+    assert lib.flex_attn_fwd_fp8_block_sparse(P(16), P(16), P(16), P(16), None, 1, 2, 1, 8, 8, 128, 0.1, 1.0, 1.0,
+                                              1.0, 0, 0, None, ctypes.byref(bm), P(64), 1 << 24, None) == 1
+    assert lib.flex_attn_fwd_fp8_block_sparse(P(16), P(16), P(16), P(16), None, 1, 2, 1, 8, 8, 128, 0.1, 1.0, 1.0,
+                                              1.0, 0, 0, None, None, P(64), 1 << 24, None) == 1
     assert f8(ws=0) == 4
     assert f8(wsb=100) == 4
     assert f8(q=8) == 3
     assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 128) == 2 * 4 * 128 * 384
-    assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 64) == 0
+    assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 64) == 2 * 4 * 64 * 384
+    assert fa.load_library().flex_attn_fwd_fp8_workspace_size(2, 4, 300, 96) == 0
 
 
 def _declared_arity():

@@ -29,8 +29,8 @@ def _fa():
     return fa
 
 
-def _inputs(B, H, Hkv, Sq, Skv, seed, spread=1.0, sigma=1.0, device="cpu"):
-    q, k, v = synth.qkv(B, H, Hkv, Sq, Skv, 128, seed=seed, sigma=sigma, device=device)
+def _inputs(B, H, Hkv, Sq, Skv, seed, spread=1.0, sigma=1.0, device="cpu", D=128):
+    q, k, v = synth.qkv(B, H, Hkv, Sq, Skv, D, seed=seed, sigma=sigma, device=device)
     return tuple((t.float() * spread).to(torch.float8_e4m3fn).cpu() for t in (q, k, v))
 
 
@@ -97,6 +97,31 @@ def test_ragged_gqa(mods, desc):
     _check(q8, k8, v8, o, lse, dq, dk, dv, scale, **mods)
 
 
+@pytest.mark.parametrize("mods", MODS[:5], ids=lambda m: "-".join(f"{k}" for k in m) or "no_mod")
+def test_ragged_gqa_d64(mods):
+    """Head dim 64: the tiles stay 128 bytes wide and TMA pads Q, K and V^T with zeros."""
+    fa = _fa()
+    B, H, Hkv, Sq, Skv = 2, 4, 2, 300, 700
+    q8, k8, v8 = _inputs(B, H, Hkv, Sq, Skv, seed=96, D=64)
+    scale = 0.125
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), descale_q=0.5, descale_k=2.0, descale_v=0.75, scale=scale,
+                        **mods)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    assert tuple(o.shape) == (B, H, Sq, 64)
+    _check(q8, k8, v8, o, lse, 0.5, 2.0, 0.75, scale, **mods)
+
+
+def test_d64_2048_sampled():
+    fa = _fa()
+    B, H, S = 2, 32, 2048
+    q8, k8, v8 = _inputs(B, H, 8, S, S, seed=104, device="cuda", D=64)
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), mask_mod="causal")
+    torch.cuda.synchronize()
+    rows = _sampled_rows(B, H, S, 2048, 105, [(0, 0, 0), (0, 0, 127), (0, 0, 128), (1, 31, 2047)])
+    _check(q8, k8, v8, o, lse, 1.0, 1.0, 1.0, 0.125, rows=rows, mask_mod="causal")
+
+
 def test_rows_without_keys():
     fa = _fa()
     q8, k8, v8 = _inputs(1, 2, 2, 250, 1024, seed=98)
@@ -155,3 +180,100 @@ def test_long_8192_sampled(mods):
              (0, 17, 1023), (0, 17, 1024), (0, 17, 1025), (1, 2, 4095)]
     rows = _sampled_rows(B, H, S, 2048, 103, fixed)
     _check(q8, k8, v8, o, lse, 1.0, 1.0, 1.0, scale, rows=rows, **mods)
+
+
+DOCS = np.array([[0, 90, 90, 250, 300], [0, 1, 200, 201, 300]], np.int32)
+
+
+@pytest.mark.parametrize("mask", ["document", "document_causal"])
+@pytest.mark.parametrize("D", [128, 64])
+def test_documents(mask, D):
+    """Packed documents (empty and one-token ones included) on the 8-bit path; keys past
+    the last boundary (Skv = 700 > 300) are in no document."""
+    fa = _fa()
+    B, H, Hkv, Sq, Skv = 2, 4, 2, 300, 700
+    q8, k8, v8 = _inputs(B, H, Hkv, Sq, Skv, seed=106, D=D)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), scale=scale, mask_mod=mask,
+                        doc_offsets=torch.from_numpy(DOCS).cuda(), score_mod="alibi")
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    _check(q8, k8, v8, o, lse, 1.0, 1.0, 1.0, scale, mask_mod=mask, doc_offsets=DOCS, score_mod="alibi")
+
+
+@pytest.mark.parametrize("mask,window,offset,docs", [("causal", 0, 0, None), ("sliding_window", 200, 0, None),
+                                                     ("kv_le_q_plus_offset", 0, -300, None),
+                                                     ("document_causal", 0, 0, DOCS[:1])])
+def test_tile_map_bit_exact(mask, window, offset, docs):
+    fa = _fa()
+    Sq, Skv = 640, 700
+    nq, nk = -(-Sq // 128), -(-Skv // 128)
+    q8, k8, v8 = _inputs(1, 1, 1, Sq, Skv, seed=107)
+    tm = torch.full((nq * nk,), 255, dtype=torch.uint8, device="cuda")
+    fa.fwd_fp8(q8.cuda(), k8.cuda(), v8.cuda(), mask_mod=mask, window=window, offset=offset, tile_map=tm,
+               doc_offsets=None if docs is None else torch.from_numpy(docs).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.tile_map(mask, Sq, Skv, window=window, offset=offset, doc_offsets=None if docs is None else docs[0])
+    np.testing.assert_array_equal(tm.cpu().numpy().reshape(nq, nk), ref)
+
+
+@pytest.mark.parametrize("mask,window,offset", [("causal", 0, 0), ("sliding_window", 300, 0),
+                                                ("kv_le_q_plus_offset", 0, -100)])
+def test_block_lists_from_tile_map_bitwise(mask, window, offset):
+    """Lists read off the analytic tile map visit the same tiles with the same classes in
+    the same order as the analytic 8-bit kernel: identical output bits."""
+    fa = _fa()
+    B, H, Hkv, S = 1, 4, 2, 1000
+    q8, k8, v8 = (t.cuda() for t in _inputs(B, H, Hkv, S, S, seed=108))
+    tm = oracle.tile_map(mask, S, S, window=window, offset=offset)
+    L = [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in oracle.block_mask_from_tile_map(tm, 1, 1)]
+    mods = dict(mask_mod=mask, window=window, offset=offset)
+    o1, l1 = fa.fwd_fp8(q8, k8, v8, **mods)
+    o2, l2 = fa.fwd_fp8_block_sparse(q8, k8, v8, *L, **mods)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("mods", [dict(), dict(mask_mod="causal", score_mod="alibi"),
+                                  dict(mask_mod="sliding_window", window=150)],
+                         ids=["no_mod", "causal-alibi", "window150"])
+def test_block_random_lists(mods):
+    """Random partial / full lists (duplicates, bad indices, over-long and negative counts)
+    against the oracle's block-sparse forward on the dequantized values, with the e4m3
+    bound of _check computed from P of the keep matrix the lists describe."""
+    from tests.helpers import random_block_lists
+    from tests.test_oracle_block_pins import _dense_keep
+    fa = _fa()
+    B, H, Hkv, Sq, Skv, D = 2, 4, 2, 300, 700, 128
+    nq, nk = -(-Sq // 128), -(-Skv // 128)
+    lists = random_block_lists(np.random.default_rng(109), B, H, nq, nk, max_blocks=nk + 2, p_full=0.35, p_part=0.35)
+    q8, k8, v8 = _inputs(B, H, Hkv, Sq, Skv, seed=110)
+    dq, dk, dv, scale = 0.5, 2.0, 0.75, 1.0 / math.sqrt(D)
+    L = [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in lists]
+    o, lse = fa.fwd_fp8_block_sparse(q8.cuda(), k8.cuda(), v8.cuda(), *L, descale_q=dq, descale_k=dk, descale_v=dv,
+                                     scale=scale, **mods)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    ro, rl = oracle.fwd_block_sparse(q8, k8, v8, *lists, scale=scale * dq * dk, **mods)
+    ro = ro * dv
+    # P of the keep matrix (torch float64) for the element-wise e4m3 bound
+    elem = oracle.mask_matrix(mods.get("mask_mod", "none"), Sq, Skv, mods.get("window", 0)).astype(bool)
+    keep = torch.from_numpy(_dense_keep(elem, *lists, B, H, Sq, Skv, 128, 128))
+    qq, kk = q8.double(), k8.double().repeat_interleave(H // Hkv, 1)
+    s = torch.einsum("bhid,bhjd->bhij", qq, kk) * scale * dq * dk
+    if mods.get("score_mod") == "alibi":
+        slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float64)
+        s = s + slopes[:, None, None] * (torch.arange(Skv)[None, :] - torch.arange(Sq)[:, None]).double()
+    s = s.masked_fill(~keep, float("-inf"))
+    live = keep.any(-1, keepdim=True)
+    P = (torch.softmax(s.masked_fill(~live, 0.0), -1) * live).numpy()
+    av = np.repeat(np.abs(v8.double().numpy()), H // Hkv, axis=1)
+    bound = dv * (2.0 ** -4 * np.einsum("bhij,bhjd->bhid", P, av)
+                  + 2.0 ** -16 * np.einsum("bhij,bhjd->bhid", (P > 0).astype(np.float64), av))
+    got = o.float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ro)
+    assert float((err / (1.05 * bound + 2.0 ** -8 * np.abs(ro) + 1e-4)).max()) <= 1.0
+    lg = lse.cpu().numpy().astype(np.float64)
+    dead = np.isneginf(rl)
+    assert np.array_equal(np.isneginf(lg), dead) and np.all(got[dead] == 0.0)
+    assert float(np.abs(lg[~dead] - rl[~dead]).max()) <= 1e-2
