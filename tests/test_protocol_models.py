@@ -228,6 +228,148 @@ def fwd_roles(sets, NS, issuers="two"):
     return roles, m.bars
 
 
+def fwd_persistent_roles(units, NS, wait_q_free=True):
+    """The persistent forward: one CTA runs the units (each a pair of key-tile sets) in
+    order with one MMA issuer.  The K/V ring and every barrier's phases run on across
+    units; the producer loads a unit's Q tiles once the issuer has committed the previous
+    unit's products (Q free).  The first P.V of a tile in a unit overwrites its O
+    accumulator; it needs no barrier of its own, since it waits for that tile's first P of
+    the unit, which its warpgroup writes only after its epilogue has read O of the
+    previous unit.  wait_q_free=False plants the mistake of loading Q without waiting."""
+    m = _Model()
+    bar_q, q_free = m.bar("q"), m.bar("q_free")
+    full = [m.bar(f"full{s}") for s in range(NS)]
+    empty = [m.bar(f"empty{s}") for s in range(NS)]
+    bar_s = [m.bar("s0"), m.bar("s1")]
+    bar_p = [[m.bar(f"p{k}{h}") for h in range(2)] for k in range(2)]
+    bar_o = [m.bar("o0"), m.bar("o1")]
+    drain = m.bar("drain")
+    work = [u for u in units if u[0] or u[1]]
+    steps_of = [sorted(set(u[0]) | set(u[1]), reverse=True) for u in work]
+
+    def rec(ui, t):
+        sets, steps = work[ui], steps_of[ui]
+        j, jn = steps[t], (steps[t + 1] if t + 1 < len(steps) else None)
+        r = {}
+        for k in range(2):
+            if j in sets[k]:
+                i = sets[k].index(j)
+                nxt = sets[k][i + 1] if i + 1 < len(sets[k]) else None
+                r[k] = "last" if nxt is None else ("pre" if nxt == jn else "later")
+        return r
+
+    def producer():
+        r = 0
+        for ui in range(len(work)):
+            if ui > 0 and wait_q_free:
+                yield ("wait", q_free, (ui - 1) & 1)
+            yield ("write", {("rec", NS): ("rec", ui, 0)})
+            yield ("expect", bar_q, TB)
+            yield ("tma", ("Q",), ("Q", ui), bar_q, TB)
+            for t, j in enumerate(steps_of[ui]):
+                for which in ("K", "V"):
+                    s = r % NS
+                    yield ("wait", empty[s], ((r // NS) & 1) ^ 1)
+                    if which == "V":
+                        yield ("write", {("rec", s): ("rec", ui, t + 1)})
+                    yield ("expect", full[s], TB)
+                    yield ("tma", ("slot", s), (which, ui, j), full[s], TB)
+                    r += 1
+        for e in range(max(0, r - NS), r):
+            yield ("wait", full[e % NS], (e // NS) & 1)
+
+    def S(ui, k, j, slot):
+        return ("mma", [(("Q",), ("Q", ui)), (("slot", slot), ("K", ui, j))],
+                {("S", k): ("S", ui, j), ("P", k, 0): ("Sx",), ("P", k, 1): ("Sx",)})
+
+    def PV(ui, k, j, half, slot, first):
+        reads = [(("P", k, half), ("P", ui, j, half)), (("slot", slot), ("V", ui, j))]
+        if not first:
+            reads.append((("O", k), ("O", ui)))
+        return ("mma", reads, {("O", k): ("O", ui)})
+
+    def issuer():
+        r = 0
+        np_, n_o = [0, 0], [0, 0]
+        for ui in range(len(work)):
+            yield ("wait", bar_q, ui & 1)
+            yield ("read", [(("rec", NS), ("rec", ui, 0))])
+            s_ready, started = [False, False], [False, False]
+            for t, j in enumerate(steps_of[ui]):
+                rK, rV = r, r + 1
+                r += 2
+                sK, sV = rK % NS, rV % NS
+                rc = rec(ui, t)
+                need = [k in rc and not s_ready[k] for k in range(2)]
+                if any(need):
+                    yield ("wait", full[sK], (rK // NS) & 1)
+                    for k in range(2):
+                        if need[k]:
+                            yield S(ui, k, j, sK)
+                            yield ("commit", bar_s[k])
+                yield ("commit", empty[sK])
+                yield ("wait", full[sV], (rV // NS) & 1)
+                yield ("read", [(("rec", sV), ("rec", ui, t + 1))])
+                next_k_ready = False
+                for k in range(2):
+                    if k not in rc:
+                        continue
+                    s_ready[k] = False
+                    for half in range(2):
+                        yield ("wait", bar_p[k][half], np_[k] & 1)
+                        yield PV(ui, k, j, half, sV, not started[k] and half == 0)
+                    started[k] = True
+                    np_[k] += 1
+                    if rc[k] == "pre":
+                        rK2 = rK + 2
+                        if not next_k_ready:
+                            yield ("wait", full[rK2 % NS], (rK2 // NS) & 1)
+                            next_k_ready = True
+                        yield S(ui, k, steps_of[ui][t + 1], rK2 % NS)
+                        yield ("commit", bar_s[k])
+                        s_ready[k] = True
+                    elif rc[k] == "last":
+                        yield ("commit", bar_o[k])
+                        n_o[k] += 1
+                yield ("commit", empty[sV])
+            yield ("commit", q_free)
+        yield ("commit", drain)
+        yield ("wait", drain, 0)
+
+    def softmax(k):
+        n, n_o = 0, 0
+        for ui in range(len(work)):
+            sets = work[ui][k]
+            for j in sets:
+                yield ("wait", bar_s[k], n & 1)
+                yield ("read", [(("S", k), ("S", ui, j))])
+                for half in range(2):
+                    yield ("write", {("P", k, half): ("P", ui, j, half)})
+                    yield ("arrive", bar_p[k][half])
+                n += 1
+            if sets:
+                yield ("wait", bar_o[k], n_o & 1)
+                yield ("read", [(("O", k), ("O", ui))])
+                n_o += 1
+
+    roles = {"producer": producer(), "I": issuer(), "sm0": softmax(0), "sm1": softmax(1)}
+    return roles, m.bars
+
+
+@pytest.mark.parametrize("NS", [5, 12])
+@pytest.mark.parametrize("kind", ["dense", "causal", "random"])
+def test_forward_persistent_protocol(NS, kind):
+    rng = random.Random(NS * 7 + len(kind))
+    cases = [[_sets(rng, rng.choice([1, 2, 3, 5]), kind) for _ in range(rng.randint(1, 5))] for _ in range(30)]
+    assert _schedules(lambda i: fwd_persistent_roles(cases[i], NS), len(cases)) == 0
+
+
+def test_forward_persistent_without_q_free_is_caught():
+    rng = random.Random(11)
+    cases = [[_sets(rng, rng.choice([1, 2, 3]), "dense") for _ in range(4)] for _ in range(40)]
+    assert _schedules(lambda i: fwd_persistent_roles(cases[i], 5, wait_q_free=False), len(cases)) > 0
+
+
 def _sets(rng, nk, kind):
     if kind == "dense":
         return [list(range(nk - 1, -1, -1))] * 2
