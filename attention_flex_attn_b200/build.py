@@ -17,11 +17,12 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libflexattn.so")
 OBJ_DIR = os.path.join(PKG, "_build")
-# Translation units: the forward and backward kernels per (head dim, block mask), the 8-bit
-# forward, decode, and the C ABI.
+# Translation units: the forward and backward kernels per (head dim, block mask), the
+# persistent forward per head dim, the 8-bit forward, decode, and the C ABI.
 # They compile in parallel and link into one shared library.
 SOURCES = [os.path.join(CSRC, f) for f in (
     "flex_fwd_d128.cu", "flex_fwd_d128_blocks.cu", "flex_fwd_d64.cu", "flex_fwd_d64_blocks.cu",
+    "flex_fwd_d128_persist.cu", "flex_fwd_d64_persist.cu",
     "flex_bwd_d128.cu", "flex_bwd_d64.cu", "flex_bwd_d128_blocks.cu", "flex_bwd_d64_blocks.cu", "flex_fwd_fp8.cu",
     "flex_decode_launch.cu", "flex_attn_api.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [

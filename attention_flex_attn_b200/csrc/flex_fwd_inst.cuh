@@ -1,7 +1,8 @@
 // flex_fwd_inst.cuh -- body of the forward instantiation units: sets the shared-memory
 // attribute once per kernel and device, and dispatches (dtype, score_mod, mask_mod)
 // onto the compile-time specialised kernels.  Included by flex_fwd_d*.cu only, each of
-// which instantiates fwd_dispatch for one (head dim, block mask) pair.
+// which instantiates fwd_dispatch for one (head dim, block mask) pair, or the persistent
+// launches for one head dim (FLEX_FWD_PERSISTENT_UNIT defined).
 #pragma once
 
 #include <atomic>
@@ -12,9 +13,20 @@
 namespace flexattn {
 namespace {
 
+// Masks whose work units carry uniform work (no mask, sliding window) can run on the
+// persistent kernel: one CTA per SM looping over the units, the K/V stream running on from
+// one unit to the next.  The host picks it (FwdParams::persist_grid > 0) when the units are
+// short; causal-like units grow with the query position, which the hardware block
+// scheduler balances better than a static assignment, and block and document masks keep
+// per-unit bitmaps.
+template <int MASK, bool BLOCKS>
+constexpr bool fwd_persistable() {
+  return !BLOCKS && (MASK == kMaskNone || MASK == kMaskSliding);
+}
+
 // Per-device "attribute already set" bits, one set per kernel instantiation (the tag
 // parameters make every instantiation own its static).
-template <int D, typename T, int SCORE, int MASK, bool BLOCKS, typename K>
+template <int D, typename T, int SCORE, int MASK, bool BLOCKS, bool PERSIST, typename K>
 bool ensure_smem_attr(K kernel, int bytes) {
   static std::atomic<uint64_t> done{0};
   int dev = 0;
@@ -26,12 +38,24 @@ bool ensure_smem_attr(K kernel, int bytes) {
   return true;
 }
 
+}  // namespace
+
+// The persistent kernels, instantiated in flex_fwd_d*_persist.cu.
+template <int D, typename T, int SCORE, int MASK>
+flex_status_t launch_fwd_persistent(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                    const FwdParams& p, cudaStream_t stream);
+
+namespace {
+
 template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
 flex_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                          int n_units, cudaStream_t stream) {
-  auto kern = flex_fwd_kernel<D, T, SCORE, MASK, BLOCKS>;
+  if constexpr (fwd_persistable<MASK, BLOCKS>()) {
+    if (p.persist_grid > 0) return launch_fwd_persistent<D, T, SCORE, MASK>(mq, mk, mv, p, stream);
+  }
+  auto kern = flex_fwd_kernel<D, T, SCORE, MASK, BLOCKS, false>;
   constexpr int kSmem = FwdSmem<D, BLOCKS, is_doc_mask(MASK)>::kAlloc;
-  if (!ensure_smem_attr<D, T, SCORE, MASK, BLOCKS>(kern, kSmem)) return FLEX_ERR_CUDA;
+  if (!ensure_smem_attr<D, T, SCORE, MASK, BLOCKS, false>(kern, kSmem)) return FLEX_ERR_CUDA;
   kern<<<n_units, kFwdThreads, kSmem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
 }
@@ -66,5 +90,37 @@ flex_status_t fwd_dispatch(flex_dtype_t dtype, int score, int mask, const CUtens
   if (dtype == FLEX_DTYPE_BF16) return dispatch_score<D, __nv_bfloat16, BLOCKS>(score, mask, mq, mk, mv, p, n_units, s);
   return dispatch_score<D, __half, BLOCKS>(score, mask, mq, mk, mv, p, n_units, s);
 }
+
+#ifdef FLEX_FWD_PERSISTENT_UNIT
+template <int D, typename T, int SCORE, int MASK>
+flex_status_t launch_fwd_persistent(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                    const FwdParams& p, cudaStream_t stream) {
+  static_assert(fwd_persistable<MASK, false>(), "no persistent kernel for this mask");
+  auto kern = flex_fwd_kernel<D, T, SCORE, MASK, false, true>;
+  constexpr int kSmem = FwdSmem<D, false, false>::kAlloc;
+  if (!ensure_smem_attr<D, T, SCORE, MASK, false, true>(kern, kSmem)) return FLEX_ERR_CUDA;
+  kern<<<p.persist_grid, kFwdThreads, kSmem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
+}
+
+// every (dtype, score_mod, mask) of head dim D that fwd_dispatch may send to the persistent kernel
+#define FLEX_FWD_PERSISTENT_INSTANCES(D)                                                                       \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskNone>(                              \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskSliding>(                           \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskNone>(                             \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskSliding>(                          \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskNone>(                       \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskSliding>(                    \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskNone>(                      \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskSliding>(                   \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);
+#endif
 
 }  // namespace flexattn

@@ -115,6 +115,8 @@ struct FwdParams {
   unsigned* status;    // device status word
   int H, Hkv, G, Sq, Skv;
   int n_qtiles, n_ktiles, n_pairs;
+  int n_units;         // B * H * n_pairs (the persistent kernel loops over them)
+  int persist_grid;    // CTAs of the persistent kernel: min(n_units, SMs)
   float scale_log2;    // scale * log2(e)
   const float* slopes; // alibi: captured per-head slopes [H], or nullptr for 2^(-8(h+1)/H)
   MaskArgs mask;       // document rules: boundaries of batch 0, advanced per batch below
@@ -142,8 +144,9 @@ struct FwdSmem {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  // barriers: q, full[NS], empty[NS], s_full[2], p_half[2][2], o_full[2], drain[2]; then tmem addr
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 4 + 2 + 2;
+  // barriers: q, full[NS], empty[NS], s_full[2], p_half[2][2], o_full[2], drain[2], q_free;
+  // then the tmem address
+  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 4 + 2 + 2 + 1;
   static constexpr int kTmemPtrOff = kBarOff + kNumBars * 8;
   // step records (kRec*): one per key/value slot, plus the first step's
   static constexpr int kRecOff = kTmemPtrOff + 16;
@@ -345,7 +348,14 @@ __device__ __forceinline__ void build_visit_sets(uint32_t* blk, int* doc_rows, c
   }
 }
 
-template <int D, typename T, int SCORE, int MASK, bool BLOCKS>
+// PERSIST: one CTA per SM loops over the units blockIdx.x, blockIdx.x + gridDim.x, ...
+// (analytic masks, one MMA issuer).  The K/V ring and every barrier's phases run on across
+// units, so the next unit's first key/value tiles load while the current one drains; the
+// producer reloads the Q tiles once the S products of the previous unit have completed
+// (q_free, committed by the issuer at the unit's last step, before its P.V products).  The first P.V of a tile in a unit, which overwrites its O accumulator, needs
+// no barrier of its own: it waits for that tile's first P of the unit, which the softmax
+// warpgroup writes only after its epilogue has read O of the previous unit.
+template <int D, typename T, int SCORE, int MASK, bool BLOCKS, bool PERSIST = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     flex_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -369,6 +379,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   auto bar_p = [&](int k, int half) { return sbase + L::kBarOff + 8u * (3 + 2 * NS + 2 * k + half); };
   auto bar_o = [&](int k) { return sbase + L::kBarOff + 8u * (7 + 2 * NS + k); };
   auto bar_drain = [&](int k) { return sbase + L::kBarOff + 8u * (9 + 2 * NS + k); };
+  const uint32_t bar_qfree = sbase + L::kBarOff + 8u * (11 + 2 * NS);
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(sgen + L::kTmemPtrOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + L::kTmemPtrOff + 4);
   uint32_t* rec_smem = reinterpret_cast<uint32_t*>(sgen + L::kRecOff);  // [NS] per V slot, [NS] first
@@ -377,30 +388,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ---------------------------------------------------------------- work unit
-  const int bh = blockIdx.x / p.n_pairs;
-  const int pair = p.n_pairs - 1 - (blockIdx.x % p.n_pairs);  // heavier (later) rows first
-  const int h = bh % p.H;
-  const int b = bh / p.H;
-  const int bkv = b * p.Hkv + h / p.G;
-
   // Per query tile k of the pair.  Read through sel() wherever k is not a compile-time
   // constant, so that no array is indexed at run time (that would put it in local memory).
+  constexpr bool kDoc = MASK == kMaskDocument || MASK == kMaskDocumentCausal;
+  static_assert(!PERSIST || (!BLOCKS && !kDoc), "the persistent kernel covers the analytic masks");
+  int bh, pair, h, b, bkv;
   int q0[2], q1[2], lo[2], hi[2];
   auto sel = [](const int (&a)[2], int k) { return k ? a[1] : a[0]; };
-  constexpr bool kDoc = MASK == kMaskDocument || MASK == kMaskDocumentCausal;
   MaskArgs mk = p.mask;
+  // unit -> (b, h, pair of query tiles), heavier (later) pairs first within a head
+  auto set_unit = [&](int unit) {
+    bh = unit / p.n_pairs;
+    pair = p.n_pairs - 1 - (unit % p.n_pairs);
+    h = bh % p.H;
+    b = bh / p.H;
+    bkv = b * p.Hkv + h / p.G;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int qt = 2 * pair + k;
+      q0[k] = qt * kBM;
+      q1[k] = min(q0[k] + kBM, p.Sq);
+      lo[k] = hi[k] = 0;
+      if (qt < p.n_qtiles && !kDoc) tile_range<MASK>(q0[k], q1[k], kBN, mk, lo[k], hi[k]);
+    }
+  };
+  set_unit(blockIdx.x);
   if constexpr (kDoc) {
     mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
     mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
   }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int qt = 2 * pair + k;
-    q0[k] = qt * kBM;
-    q1[k] = min(q0[k] + kBM, p.Sq);
-    lo[k] = hi[k] = 0;
-    if (qt < p.n_qtiles && !kDoc) tile_range<MASK>(q0[k], q1[k], kBN, mk, lo[k], hi[k]);
-  }
+  // the units of this CTA: blockIdx.x (+ gridDim.x ...) up to unit_end
+  const int unit_end = PERSIST ? p.n_units : static_cast<int>(blockIdx.x) + 1;
+  const int unit_step = PERSIST ? static_cast<int>(gridDim.x) : 1;
 
   // ---------------------------------------------------------------- visit bitmaps
   // With a block mask or a document mask the key tiles a query tile visits are a set, not
@@ -456,6 +475,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     mbar_init(bar_drain(0), 1);
     mbar_init(bar_drain(1), 1);
+    mbar_init(bar_qfree, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -482,11 +502,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (warp < kSoftmaxWarp0) {
     regs_dec<kAuxRegs>();
-    if (warp == kTmaWarp && lane == 0 && any_work) {
+    if (warp == kTmaWarp && lane == 0) {
       // ============================================================ TMA producer
-      int r = 0;
+      int r = 0;   // key/value loads issued (the ring position, across units)
+      int qn = 0;  // units whose Q tiles were loaded
       bool ok = true;
-      auto c0 = cursor(0), c1 = cursor(1);
       // record of the step at max(a0.cur, a1.cur) (copies: the caller's cursors stay put)
       auto make_rec = [](auto a0, auto a1) -> uint32_t {
         const int j = max(a0.cur, a1.cur);
@@ -500,33 +520,46 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (i1) rec |= a1.cur < 0 ? kRecLast1 : (a1.cur == jn ? kRecPre1 : 0u);
         return rec;
       };
-      // The first record is published with the Q barrier, which the issuer waits on first.
-      rec_smem[NS] = make_rec(c0, c1);
-      const int bytes_q = (act0 ? 1 : 0) * L::kTileBytes + (act1 ? 1 : 0) * L::kTileBytes;
-      mbar_arrive_expect_tx(bar_q, bytes_q);
-      for (int k = 0; k < 2; ++k) {
-        if (!(k == 0 ? act0 : act1)) continue;
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(q_smem(k) + c * L::kChunkBytes, &tmQ, bar_q, c * 64, sel(q0, k), bh);
-      }
-      for (int j = max(c0.cur, c1.cur); j >= 0 && ok; j = max(c0.cur, c1.cur)) {  // last to first
-        if (c0.cur == j) c0.advance();
-        if (c1.cur == j) c1.advance();
-        const uint32_t next_rec = make_rec(c0, c1);
-        for (int which = 0; which < 2 && ok; ++which, ++r) {
-          const int s = r % NS;
-          const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
-          if (!mbar_wait(bar_empty(s), ph ^ 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs) ||
-              *abort_flag) {
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          if (which == 1) rec_smem[s] = next_rec;  // released by the arrive below
-          mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
-          const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+      for (int unit = blockIdx.x; unit < unit_end && ok; unit += unit_step) {
+        if (PERSIST && unit != static_cast<int>(blockIdx.x)) set_unit(unit);
+        auto c0 = cursor(0), c1 = cursor(1);
+        const bool u0 = c0.cur >= 0, u1 = c1.cur >= 0;
+        if (!u0 && !u1) continue;  // no key for either tile: every role skips the unit
+        // the previous unit's products must be done with the Q tiles
+        if (qn > 0 && !mbar_wait(bar_qfree, static_cast<uint32_t>(qn - 1) & 1u, p.status, kStatusFwdTimeout,
+                                 kWaitTimeoutNs)) {
+          *abort_flag = 1;
+          break;
+        }
+        // The first record is published with the Q barrier, which the issuer waits on first.
+        rec_smem[NS] = make_rec(c0, c1);
+        const int bytes_q = (u0 ? 1 : 0) * L::kTileBytes + (u1 ? 1 : 0) * L::kTileBytes;
+        mbar_arrive_expect_tx(bar_q, bytes_q);
+        for (int k = 0; k < 2; ++k) {
+          if (!(k == 0 ? u0 : u1)) continue;
           for (int c = 0; c < kChunks; ++c)
-            tma_load_3d(kv_smem(s) + c * L::kChunkBytes, map, bar_full(s), c * 64, j * kBN, bkv);
+            tma_load_3d(q_smem(k) + c * L::kChunkBytes, &tmQ, bar_q, c * 64, sel(q0, k), bh);
+        }
+        ++qn;
+        for (int j = max(c0.cur, c1.cur); j >= 0 && ok; j = max(c0.cur, c1.cur)) {  // last to first
+          if (c0.cur == j) c0.advance();
+          if (c1.cur == j) c1.advance();
+          const uint32_t next_rec = make_rec(c0, c1);
+          for (int which = 0; which < 2 && ok; ++which, ++r) {
+            const int s = r % NS;
+            const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
+            if (!mbar_wait(bar_empty(s), ph ^ 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs) ||
+                *abort_flag) {
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            if (which == 1) rec_smem[s] = next_rec;  // released by the arrive below
+            mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
+            const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_3d(kv_smem(s) + c * L::kChunkBytes, map, bar_full(s), c * 64, j * kBN, bkv);
+          }
         }
       }
       // Every load issued must land before the CTA can exit.
@@ -534,11 +567,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int e = issued - NS < 0 ? 0 : issued - NS; e < issued; ++e)
         mbar_wait(bar_full(e % NS), static_cast<uint32_t>(e / NS) & 1u, p.status, kStatusFwdTimeout,
                   kWaitTimeoutNs);
-      mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
-    } else if (!two_issuers && warp == kMmaWarp && lane == 0 && any_work) {
+      if (qn > 0)
+        mbar_wait(bar_q, static_cast<uint32_t>(qn - 1) & 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+    } else if (!two_issuers && warp == kMmaWarp && lane == 0) {
       // ============================================================ MMA issuer (both tiles)
-      bool ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
-      tc_fence_after();
+      bool ok = true;
       int np[2] = {0, 0};
       // descriptor of chunk 0 / k-step 0; k-step kk adds ((kk/4)*chunk + (kk%4)*32) >> 4
       const uint64_t dq0 = smem_desc(q_smem(0), 16, 1024, kSwizzle128B);
@@ -595,44 +628,72 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         return true;
       };
-      uint32_t rec = rec_smem[NS];  // published with the Q barrier
-      for (int t = 0; !(rec & kRecEnd) && ok; ++t) {
-        const int rK = 2 * t, rV = rK + 1;
-        const int sK = rK % NS, sV = rV % NS;
-        const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
-        const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
-        if (need0 || need1) {
-          // K_j was not needed before: wait for it here (otherwise the previous step did)
-          if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+      int rb = 0;  // ring position of the unit's first key load
+      int qn = 0;  // units started (the Q barrier's phase)
+      for (int unit = blockIdx.x; unit < unit_end && ok; unit += unit_step) {
+        if (PERSIST && unit != static_cast<int>(blockIdx.x)) set_unit(unit);
+        // fin_k: query tile k has no key tile left in this unit
+        bool fin0 = cursor(0).cur < 0, fin1 = cursor(1).cur < 0;
+        if (fin0 && fin1) continue;  // no work in this unit
+        bool q_released = false;
+        if (!mbar_wait(bar_q, static_cast<uint32_t>(qn) & 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        ++qn;
+        tc_fence_after();
+        s_ready[0] = s_ready[1] = started[0] = started[1] = false;
+        uint32_t rec = rec_smem[NS];  // published with the Q barrier
+        int t = 0;
+        for (; !(rec & kRecEnd) && ok; ++t) {
+          const int rK = rb + 2 * t, rV = rK + 1;
+          const int sK = rK % NS, sV = rV % NS;
+          const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
+          const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
+          if (need0 || need1) {
+            // K_j was not needed before: wait for it here (otherwise the previous step did)
+            if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+                           kStatusFwdTimeout, kWaitTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (need0) {
+              issue_s(0, sK);
+              mma_commit(bar_s(0));
+            }
+            if (need1) {
+              issue_s(1, sK);
+              mma_commit(bar_s(1));
+            }
+          }
+          mma_commit(bar_empty(sK));
+          // The unit's last step: every S product of the unit has been issued, so Q is
+          // free once they complete; the next unit's Q loads during this step's P.V.
+          if (PERSIST && !q_released && (in0 ? (rec & kRecLast0) != 0 : fin0) &&
+              (in1 ? (rec & kRecLast1) != 0 : fin1)) {
+            mma_commit(bar_qfree);
+            q_released = true;
+          }
+          if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
                          kStatusFwdTimeout, kWaitTimeoutNs)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          if (need0) {
-            issue_s(0, sK);
-            mma_commit(bar_s(0));
-          }
-          if (need1) {
-            issue_s(1, sK);
-            mma_commit(bar_s(1));
-          }
+          const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
+          bool next_k_ready = false;
+          if (in0)
+            ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
+          if (ok && in1)
+            ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
+          if (!ok) break;
+          mma_commit(bar_empty(sV));
+          if (in0 && (rec & kRecLast0)) fin0 = true;
+          if (in1 && (rec & kRecLast1)) fin1 = true;
+          rec = next_rec;
         }
-        mma_commit(bar_empty(sK));
-        if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
-                       kStatusFwdTimeout, kWaitTimeoutNs)) {
-          ok = false;
-          break;
-        }
-        const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
-        bool next_k_ready = false;
-        if (in0)
-          ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
-        if (ok && in1)
-          ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
-        if (!ok) break;
-        mma_commit(bar_empty(sV));
-        rec = next_rec;
+        rb += 2 * t;
+        if (PERSIST && !q_released) mma_commit(bar_qfree);  // (only when the walk broke off)
       }
       if (!ok) *abort_flag = 1;
       // Drain: all MMAs this thread issued have completed before TMEM is released.
@@ -746,210 +807,227 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int k = (warp - kSoftmaxWarp0) >> 2;  // query tile of this warpgroup
     const int wq = warp & 3;          // TMEM lane quarter
     const int row = wq * 32 + lane;   // row inside the tile == TMEM lane
-    const int q0k = sel(q0, k), q1k = sel(q1, k);
-    const int qi = q0k + row;         // absolute query index
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + 128u * k;
     const uint32_t tO = tmem + lane_off + 256u + 128u * k;
-    const bool tile_valid = (2 * pair + k) < p.n_qtiles;
-    const bool write_map = p.tile_map != nullptr && bh == 0 && tile_valid && threadIdx.x % 128 == 0;
-    const int qt = 2 * pair + k;
-
-    const bool act_k = k == 0 ? act0 : act1;
-    if (write_map) {
-      for (int u = 0; u < p.n_ktiles; ++u)
-        if (!act_k || !has(k, u)) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + u] = kTileEmpty;
-    }
-
-    float m_used = -INFINITY;  // running max in log2 units (the reference of P and O)
-    float l_sum = 0.f;
-    const float sc = SCORE == kScoreAlibi ? 1.0f : p.scale_log2;
-    float slope2 = 0.f;
-    if (SCORE == kScoreAlibi)
-      slope2 = (p.slopes ? __ldg(p.slopes + h) : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
-               kLog2e;
-    // Document rules: this row's kept interval, looked up once (a binary search over the
-    // boundaries); the tile classes come from the visit bitmaps.
-    int64_t row_lo = 0, row_hi = -1;
-    if constexpr (kDoc) row_interval<MASK>(qi, mk, row_lo, row_hi);
-
     bool ok = true;
-    int n = 0;
-    // Key tiles from last to first: with alibi the bias grows with the key index, so the
-    // row maximum is met on the first tile and the lazy rescale of O almost never runs.
-    auto cur = cursor(k);
-    for (int j = cur.cur; j >= 0; j = cur.cur, ++n) {
-      // With a block mask the class comes from the walk (FULL listed or not).
-      const int cls_blk =
-          cur.cur_full ? (j * kBN + kBN > p.Skv ? kTileFullRagged : kTileFull) : kTilePartial;
-      cur.advance();
-      // Warp-uniform decision: the TMEM loads below are warp-collective.
-      const bool got = mbar_wait(bar_s(k), static_cast<uint32_t>(n) & 1u, p.status, kStatusFwdTimeout,
-                                 kWaitTimeoutNs) &&
-                       !*abort_flag;
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int k0 = j * kBN;
-      int cls;
-      if constexpr (kBits) cls = cls_blk;
-      else cls = tile_class<MASK>(q0k, q1k, k0, kBN, mk);
-      if (write_map)
-        p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] =
-            static_cast<uint8_t>(cls == kTileFullRagged ? kTilePartial : cls);
+    int n = 0;      // S tiles of this warpgroup so far (the S barrier's phase)
+    int o_par = 0;  // O completions waited for (the O barrier's phase)
+    for (int unit = blockIdx.x; unit < unit_end && ok; unit += unit_step) {
+      if (PERSIST && unit != static_cast<int>(blockIdx.x)) set_unit(unit);
+      const int q0k = sel(q0, k), q1k = sel(q1, k);
+      const int qi = q0k + row;         // absolute query index
+      const bool tile_valid = (2 * pair + k) < p.n_qtiles;
+      const bool write_map = p.tile_map != nullptr && bh == 0 && tile_valid && threadIdx.x % 128 == 0;
+      const int qt = 2 * pair + k;
 
-      uint32_t sr[kBN];
-      tmem_ld128(tS, sr);
-      float* s = reinterpret_cast<float*>(sr);
-      // Alibi: the bias slope2 * c of column c comes from four packed chains (columns
-      // 8i + 2r, 8i + 2r + 1), each stepped by 8 * slope2; the part common to the tile,
-      // slope2 * (k0 - qi), joins the running max instead of every element.  The _rn
-      // operations are never fused, so every instantiation rounds them alike.
-      const float base = SCORE == kScoreAlibi ? __fmul_rn(slope2, static_cast<float>(k0 - qi)) : 0.f;
-      if (SCORE == kScoreAlibi) {
-        const uint64_t scl2 = pack2(p.scale_log2, p.scale_log2);
-        const uint64_t astep = pack2(__fmul_rn(8.f, slope2), __fmul_rn(8.f, slope2));
-        uint64_t b0 = pack2(0.f, slope2), b1 = pack2(__fmul_rn(2.f, slope2), __fmul_rn(3.f, slope2));
-        uint64_t b2 = pack2(__fmul_rn(4.f, slope2), __fmul_rn(5.f, slope2));
-        uint64_t b3 = pack2(__fmul_rn(6.f, slope2), __fmul_rn(7.f, slope2));
-#pragma unroll
-        for (int c = 0; c < kBN; c += 8) {
-          unpack2(fma2(pack2(s[c], s[c + 1]), scl2, b0), s[c], s[c + 1]);
-          unpack2(fma2(pack2(s[c + 2], s[c + 3]), scl2, b1), s[c + 2], s[c + 3]);
-          unpack2(fma2(pack2(s[c + 4], s[c + 5]), scl2, b2), s[c + 4], s[c + 5]);
-          unpack2(fma2(pack2(s[c + 6], s[c + 7]), scl2, b3), s[c + 6], s[c + 7]);
-          b0 = add2(b0, astep);
-          b1 = add2(b1, astep);
-          b2 = add2(b2, astep);
-          b3 = add2(b3, astep);
-        }
+      const bool act_k = cursor(k).cur >= 0;
+      if (write_map) {
+        for (int u = 0; u < p.n_ktiles; ++u)
+          if (!act_k || !has(k, u)) p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + u] = kTileEmpty;
       }
-      if (cls != kTileFull) {
-        int c_lo, c_hi;
-        if (kBits && cls == kTileFullRagged)
-          col_interval<kMaskNone>(qi, k0, mk, c_lo, c_hi);
-        else
-          if constexpr (kDoc) col_interval_of(row_lo, row_hi, k0, c_lo, c_hi);
-          else col_interval<MASK>(qi, k0, mk, c_lo, c_hi);
-#pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if (c < c_lo || c > c_hi) s[c] = -INFINITY;
-      }
-      float mx0 = max3f(s[0], s[1], s[2]), mx1 = max3f(s[3], s[4], s[5]);
-      float mx2 = max3f(s[6], s[7], s[8]), mx3 = max3f(s[9], s[10], s[11]);
-#pragma unroll
-      for (int c = 12; c + 8 <= kBN - 4; c += 8) {
-        mx0 = max3f(mx0, s[c], s[c + 1]);
-        mx1 = max3f(mx1, s[c + 2], s[c + 3]);
-        mx2 = max3f(mx2, s[c + 4], s[c + 5]);
-        mx3 = max3f(mx3, s[c + 6], s[c + 7]);
-      }
-      mx0 = max3f(mx0, s[kBN - 4], s[kBN - 3]);
-      mx1 = max3f(mx1, s[kBN - 2], s[kBN - 1]);
-      const float mx = __fadd_rn(max3f(mx0, mx1, fmaxf(mx2, mx3)) * sc, base);
-      const bool need = mx > m_used + kRescaleThreshold;  // false while both are -inf
-      if (__any_sync(0xffffffffu, need)) {
-        float alpha = 1.0f;
-        if (need) {
-          alpha = ex2_approx(m_used - mx);  // 0 when m_used == -inf
-          m_used = mx;
-          l_sum *= alpha;
-        }
-        if (n > 0) {
-          const uint64_t a2 = pack2(alpha, alpha);
-#pragma unroll 1
-          for (int c = 0; c < D; c += 32) {
-            uint32_t r[32];
-            tmem_ld32(tO + c, r);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const uint64_t v = mul2(pack2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), a2);
-              r[e] = static_cast<uint32_t>(v);
-              r[e + 1] = static_cast<uint32_t>(v >> 32);
-            }
-            tmem_st32(tO + c, r);
-          }
-        }
-      }
-      const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-      const uint64_t sc2 = pack2(sc, sc);
-      const float nm = __fsub_rn(base, m_safe);
-      const uint64_t nm2 = pack2(nm, nm);
-      uint64_t acc2 = 0;  // two running partial sums (0.0f, 0.0f)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = 64 * half + 2 * i;
-          const uint64_t x2 = fma2(pack2(s[c], s[c + 1]), sc2, nm2);
-          uint64_t e2;
-          if (emu_pair(i)) {
-            e2 = exp2_poly2(x2);
-          } else {
-            float x0, x1;
-            unpack2(x2, x0, x1);
-            e2 = pack2(ex2_approx(x0), ex2_approx(x1));
-          }
-          acc2 = add2(acc2, e2);
-          float e0, e1;
-          unpack2(e2, e0, e1);
-          pk[i] = DtypeBits<T>::pack(e0, e1);
-        }
-        tmem_st32(tS + 32u * half, pk);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar_p(k, half));
-      }
-      float a0, a1;
-      unpack2(acc2, a0, a1);
-      l_sum += a0 + a1;
-    }
-    if (!ok) *abort_flag = 1;
 
-    // ---------------------------------------------------------------- epilogue
-    if (tile_valid) {
-      bool ran = ok && act_k;
-      if (ran) {
-        const bool got = mbar_wait(bar_o(k), 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+      float m_used = -INFINITY;  // running max in log2 units (the reference of P and O)
+      float l_sum = 0.f;
+      const float sc = SCORE == kScoreAlibi ? 1.0f : p.scale_log2;
+      float slope2 = 0.f;
+      if (SCORE == kScoreAlibi)
+        slope2 = (p.slopes ? __ldg(p.slopes + h) : exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.H))) *
+                 kLog2e;
+      // Document rules: this row's kept interval, looked up once (a binary search over the
+      // boundaries); the tile classes come from the visit bitmaps.
+      int64_t row_lo = 0, row_hi = -1;
+      if constexpr (kDoc) row_interval<MASK>(qi, mk, row_lo, row_hi);
+
+      int nu = 0;  // key tiles of this unit so far
+      // Key tiles from last to first: with alibi the bias grows with the key index, so the
+      // row maximum is met on the first tile and the lazy rescale of O almost never runs.
+      auto cur = cursor(k);
+      for (int j = cur.cur; j >= 0; j = cur.cur, ++n, ++nu) {
+        // With a block mask the class comes from the walk (FULL listed or not).
+        const int cls_blk =
+            cur.cur_full ? (j * kBN + kBN > p.Skv ? kTileFullRagged : kTileFull) : kTilePartial;
+        cur.advance();
+        // Warp-uniform decision: the TMEM loads below are warp-collective.
+        const bool got = mbar_wait(bar_s(k), static_cast<uint32_t>(n) & 1u, p.status, kStatusFwdTimeout,
+                                   kWaitTimeoutNs) &&
+                         !*abort_flag;
         if (!__all_sync(0xffffffffu, got)) {
-          *abort_flag = 1;
-          ran = false;
+          ok = false;
+          break;
         }
         tc_fence_after();
+        const int k0 = j * kBN;
+        int cls;
+        if constexpr (kBits) cls = cls_blk;
+        else cls = tile_class<MASK>(q0k, q1k, k0, kBN, mk);
+        if (write_map)
+          p.tile_map[static_cast<int64_t>(qt) * p.n_ktiles + j] =
+              static_cast<uint8_t>(cls == kTileFullRagged ? kTilePartial : cls);
+
+        uint32_t sr[kBN];
+        tmem_ld128(tS, sr);
+        float* s = reinterpret_cast<float*>(sr);
+        // Alibi: the bias slope2 * c of column c comes from four packed chains (columns
+        // 8i + 2r, 8i + 2r + 1), each stepped by 8 * slope2; the part common to the tile,
+        // slope2 * (k0 - qi), joins the running max instead of every element.  The _rn
+        // operations are never fused, so every instantiation rounds them alike.
+        const float base = SCORE == kScoreAlibi ? __fmul_rn(slope2, static_cast<float>(k0 - qi)) : 0.f;
+        if (SCORE == kScoreAlibi) {
+          const uint64_t scl2 = pack2(p.scale_log2, p.scale_log2);
+          const uint64_t astep = pack2(__fmul_rn(8.f, slope2), __fmul_rn(8.f, slope2));
+          uint64_t b0 = pack2(0.f, slope2), b1 = pack2(__fmul_rn(2.f, slope2), __fmul_rn(3.f, slope2));
+          uint64_t b2 = pack2(__fmul_rn(4.f, slope2), __fmul_rn(5.f, slope2));
+          uint64_t b3 = pack2(__fmul_rn(6.f, slope2), __fmul_rn(7.f, slope2));
+  #pragma unroll
+          for (int c = 0; c < kBN; c += 8) {
+            unpack2(fma2(pack2(s[c], s[c + 1]), scl2, b0), s[c], s[c + 1]);
+            unpack2(fma2(pack2(s[c + 2], s[c + 3]), scl2, b1), s[c + 2], s[c + 3]);
+            unpack2(fma2(pack2(s[c + 4], s[c + 5]), scl2, b2), s[c + 4], s[c + 5]);
+            unpack2(fma2(pack2(s[c + 6], s[c + 7]), scl2, b3), s[c + 6], s[c + 7]);
+            b0 = add2(b0, astep);
+            b1 = add2(b1, astep);
+            b2 = add2(b2, astep);
+            b3 = add2(b3, astep);
+          }
+        }
+        if (cls != kTileFull) {
+          int c_lo, c_hi;
+          if (kBits && cls == kTileFullRagged)
+            col_interval<kMaskNone>(qi, k0, mk, c_lo, c_hi);
+          else
+            if constexpr (kDoc) col_interval_of(row_lo, row_hi, k0, c_lo, c_hi);
+            else col_interval<MASK>(qi, k0, mk, c_lo, c_hi);
+  #pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c < c_lo || c > c_hi) s[c] = -INFINITY;
+        }
+        float mx0 = max3f(s[0], s[1], s[2]), mx1 = max3f(s[3], s[4], s[5]);
+        float mx2 = max3f(s[6], s[7], s[8]), mx3 = max3f(s[9], s[10], s[11]);
+  #pragma unroll
+        for (int c = 12; c + 8 <= kBN - 4; c += 8) {
+          mx0 = max3f(mx0, s[c], s[c + 1]);
+          mx1 = max3f(mx1, s[c + 2], s[c + 3]);
+          mx2 = max3f(mx2, s[c + 4], s[c + 5]);
+          mx3 = max3f(mx3, s[c + 6], s[c + 7]);
+        }
+        mx0 = max3f(mx0, s[kBN - 4], s[kBN - 3]);
+        mx1 = max3f(mx1, s[kBN - 2], s[kBN - 1]);
+        const float mx = __fadd_rn(max3f(mx0, mx1, fmaxf(mx2, mx3)) * sc, base);
+        const bool need = mx > m_used + kRescaleThreshold;  // false while both are -inf
+        if (__any_sync(0xffffffffu, need)) {
+          float alpha = 1.0f;
+          if (need) {
+            alpha = ex2_approx(m_used - mx);  // 0 when m_used == -inf
+            m_used = mx;
+            l_sum *= alpha;
+          }
+          if (nu > 0) {  // the unit's first tile finds O empty
+            const uint64_t a2 = pack2(alpha, alpha);
+  #pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+              uint32_t r[32];
+              tmem_ld32(tO + c, r);
+  #pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const uint64_t v = mul2(pack2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), a2);
+                r[e] = static_cast<uint32_t>(v);
+                r[e + 1] = static_cast<uint32_t>(v >> 32);
+              }
+              tmem_st32(tO + c, r);
+            }
+          }
+        }
+        const float m_safe = m_used == -INFINITY ? 0.f : m_used;
+        const uint64_t sc2 = pack2(sc, sc);
+        const float nm = __fsub_rn(base, m_safe);
+        const uint64_t nm2 = pack2(nm, nm);
+        uint64_t acc2 = 0;  // two running partial sums (0.0f, 0.0f)
+  #pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int c = 64 * half + 2 * i;
+            const uint64_t x2 = fma2(pack2(s[c], s[c + 1]), sc2, nm2);
+            uint64_t e2;
+            if (emu_pair(i)) {
+              e2 = exp2_poly2(x2);
+            } else {
+              float x0, x1;
+              unpack2(x2, x0, x1);
+              e2 = pack2(ex2_approx(x0), ex2_approx(x1));
+            }
+            acc2 = add2(acc2, e2);
+            float e0, e1;
+            unpack2(e2, e0, e1);
+            pk[i] = DtypeBits<T>::pack(e0, e1);
+          }
+          tmem_st32(tS + 32u * half, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar_p(k, half));
+        }
+        float a0, a1;
+        unpack2(acc2, a0, a1);
+        l_sum += a0 + a1;
       }
-      const bool row_ok = qi < p.Sq;
-      // A row has mass iff it ever saw a kept (finite) score.  The polynomial 2^x returns
-      // ~2^-125 rather than 0 for masked scores, so l_sum alone cannot tell.
-      const bool has_mass = ran && m_used != -INFINITY && l_sum > 0.f;
-      const float inv = has_mass ? 1.0f / l_sum : 0.f;
-      T* orow = reinterpret_cast<T*>(p.o) + (static_cast<int64_t>(bh) * p.Sq + qi) * D;
-#pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t r[32];
+      if (!ok) *abort_flag = 1;
+
+      // ---------------------------------------------------------------- epilogue
+      if (tile_valid) {
+        bool ran = ok && act_k;
         if (ran) {
-          tmem_ld32(tO + c, r);
+          const bool got = mbar_wait(bar_o(k), static_cast<uint32_t>(o_par) & 1u, p.status, kStatusFwdTimeout,
+                                     kWaitTimeoutNs);
+          ++o_par;
+          if (!__all_sync(0xffffffffu, got)) {
+            *abort_flag = 1;
+            ran = false;
+          }
+          tc_fence_after();
         }
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = has_mass ? __uint_as_float(r[2 * e]) * inv : 0.f;
-          const float bb = has_mass ? __uint_as_float(r[2 * e + 1]) * inv : 0.f;
-          w[e] = DtypeBits<T>::pack(a, bb);
+        // The output row's address is recomputed from the unit index behind an opaque copy,
+        // so that the compiler keeps neither it nor the head index live through the key
+        // tiles (in the persistent loop it cannot rebuild them from blockIdx).
+        const int ou = opaque_int(unit);
+        const int obh = ou / p.n_pairs;
+        const int oqi = (2 * (p.n_pairs - 1 - ou % p.n_pairs) + k) * kBM + row;
+        const bool row_ok = oqi < p.Sq;
+        // A row has mass iff it ever saw a kept (finite) score.  The polynomial 2^x returns
+        // ~2^-125 rather than 0 for masked scores, so l_sum alone cannot tell.
+        const bool has_mass = ran && m_used != -INFINITY && l_sum > 0.f;
+        const float inv = has_mass ? 1.0f / l_sum : 0.f;
+        T* orow = reinterpret_cast<T*>(p.o) + (static_cast<int64_t>(obh) * p.Sq + oqi) * D;
+  #pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          // defined on both paths: an undefined r would stay live around the unit loop
+          if (ran) {
+            tmem_ld32(tO + c, r);
+          } else {
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          uint32_t w[16];
+  #pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = has_mass ? __uint_as_float(r[2 * e]) * inv : 0.f;
+            const float bb = has_mass ? __uint_as_float(r[2 * e + 1]) * inv : 0.f;
+            w[e] = DtypeBits<T>::pack(a, bb);
+          }
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+  #pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
         }
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        if (row_ok && p.lse != nullptr) {
+          p.lse[static_cast<int64_t>(obh) * p.Sq + oqi] =
+              has_mass ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
         }
       }
-      if (row_ok && p.lse != nullptr) {
-        p.lse[static_cast<int64_t>(bh) * p.Sq + qi] =
-            has_mass ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
-      }
-    }
+    }  // unit
   }
 
   // ---------------------------------------------------------------- teardown

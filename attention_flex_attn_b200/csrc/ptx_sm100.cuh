@@ -293,6 +293,13 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return y;
 }
 
+// x, through a volatile move the compiler cannot look through or hoist: what is computed
+// from the result stays where it is written instead of being kept live from earlier.
+__device__ __forceinline__ int opaque_int(int x) {
+  asm volatile("mov.b32 %0, %0;" : "+r"(x));
+  return x;
+}
+
 // Packed pairs of fp32 (two lanes of one 64-bit register) for the f32x2 instructions.
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
   uint64_t r;

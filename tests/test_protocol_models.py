@@ -228,14 +228,17 @@ def fwd_roles(sets, NS, issuers="two"):
     return roles, m.bars
 
 
-def fwd_persistent_roles(units, NS, wait_q_free=True):
+def fwd_persistent_roles(units, NS, wait_q_free=True, q_free_at="last_step"):
     """The persistent forward: one CTA runs the units (each a pair of key-tile sets) in
     order with one MMA issuer.  The K/V ring and every barrier's phases run on across
-    units; the producer loads a unit's Q tiles once the issuer has committed the previous
-    unit's products (Q free).  The first P.V of a tile in a unit overwrites its O
-    accumulator; it needs no barrier of its own, since it waits for that tile's first P of
-    the unit, which its warpgroup writes only after its epilogue has read O of the
-    previous unit.  wait_q_free=False plants the mistake of loading Q without waiting."""
+    units; the producer loads a unit's Q tiles once the S products of the previous unit
+    have completed (Q free), which the issuer commits at the unit's last step, after that
+    step's S products and before its P.V products.  The first P.V of a tile in a unit
+    overwrites its O accumulator; it needs no barrier of its own, since it waits for that
+    tile's first P of the unit, which its warpgroup writes only after its epilogue has read
+    O of the previous unit.  Planted mistakes: wait_q_free=False (Q loaded without
+    waiting) and q_free_at="first_step" (Q released at the unit's first step, before the
+    S products of the later steps)."""
     m = _Model()
     bar_q, q_free = m.bar("q"), m.bar("q_free")
     full = [m.bar(f"full{s}") for s in range(NS)]
@@ -295,6 +298,8 @@ def fwd_persistent_roles(units, NS, wait_q_free=True):
             yield ("wait", bar_q, ui & 1)
             yield ("read", [(("rec", NS), ("rec", ui, 0))])
             s_ready, started = [False, False], [False, False]
+            fin = [not work[ui][0], not work[ui][1]]  # tile k has no key tile left
+            released = False
             for t, j in enumerate(steps_of[ui]):
                 rK, rV = r, r + 1
                 r += 2
@@ -308,6 +313,10 @@ def fwd_persistent_roles(units, NS, wait_q_free=True):
                             yield S(ui, k, j, sK)
                             yield ("commit", bar_s[k])
                 yield ("commit", empty[sK])
+                last_step = all(rc[k] == "last" if k in rc else fin[k] for k in range(2))
+                if not released and (last_step if q_free_at == "last_step" else t == 0):
+                    yield ("commit", q_free)
+                    released = True
                 yield ("wait", full[sV], (rV // NS) & 1)
                 yield ("read", [(("rec", sV), ("rec", ui, t + 1))])
                 next_k_ready = False
@@ -331,8 +340,9 @@ def fwd_persistent_roles(units, NS, wait_q_free=True):
                     elif rc[k] == "last":
                         yield ("commit", bar_o[k])
                         n_o[k] += 1
+                        fin[k] = True
                 yield ("commit", empty[sV])
-            yield ("commit", q_free)
+            assert released  # the last step always releases Q
         yield ("commit", drain)
         yield ("wait", drain, 0)
 
@@ -368,6 +378,12 @@ def test_forward_persistent_without_q_free_is_caught():
     rng = random.Random(11)
     cases = [[_sets(rng, rng.choice([1, 2, 3]), "dense") for _ in range(4)] for _ in range(40)]
     assert _schedules(lambda i: fwd_persistent_roles(cases[i], 5, wait_q_free=False), len(cases)) > 0
+
+
+def test_forward_persistent_q_released_early_is_caught():
+    rng = random.Random(12)
+    cases = [[_sets(rng, rng.choice([2, 3]), "dense") for _ in range(4)] for _ in range(40)]
+    assert _schedules(lambda i: fwd_persistent_roles(cases[i], 5, q_free_at="first_step"), len(cases)) > 0
 
 
 def _sets(rng, nk, kind):
