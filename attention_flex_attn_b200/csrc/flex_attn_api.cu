@@ -27,6 +27,7 @@ namespace {
 // Largest key-tile count per query tile that runs on the persistent forward kernel.
 constexpr int64_t kPersistMaxKeyTiles = 32;
 
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -157,6 +158,40 @@ void* symbol_ptr(Symbol which) {
 }
 
 void* decode_scratch_ptr() { return symbol_ptr(kSymScratch); }
+
+// Stream-ordered scratch of the forward's split units: a memory pool of the library's own
+// per device and context, which keeps its memory between calls (release threshold at the
+// maximum), so that steady-state calls neither map memory nor synchronise.
+cudaMemPool_t scratch_pool() {
+  constexpr int kMaxDevices = 64;
+  struct Entry {
+    unsigned long long ctx;
+    cudaMemPool_t pool;
+  };
+  static Entry cache[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  unsigned long long id = 0;
+  if (!current_context_id(&id)) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry& e = cache[dev];
+  if (e.pool && e.ctx == id) return e.pool;
+  cudaMemPoolProps props{};
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  cudaMemPool_t pool = nullptr;
+  if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+  uint64_t keep = UINT64_MAX;
+  if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+    cudaMemPoolDestroy(pool);
+    return nullptr;
+  }
+  e.ctx = id;
+  e.pool = pool;
+  return pool;
+}
 
 // Streaming multiprocessors of the current device (looked up once per device).
 int sm_count() {
@@ -360,10 +395,14 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   p.n_ktiles = (Skv + kBN - 1) / kBN;
   p.n_pairs = n_pairs;
   p.n_units = static_cast<int>(n_units);
+  p.n_full = p.n_items = static_cast<int>(n_units);
+  p.n_parts = 1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // Short units (few key tiles per query tile) run on the persistent kernel, where a
   // CTA's fill and drain would otherwise be a large share of its time.  On long units the
   // block scheduler's dynamic assignment wins (measured on B200, 128 rows per tile: 8 and
   // 3 key tiles 9 % and 7 % faster persistent, 32 at D = 64 2 % faster, 64 5 % slower).
+  void* split_ws = nullptr;
   if (!bm && (mask == kMaskNone || mask == kMaskSliding)) {
     int64_t span = p.n_ktiles;
     if (mask == kMaskSliding)
@@ -371,14 +410,45 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
     if (span <= kPersistMaxKeyTiles) {
       const int sms = sm_count();
       if (sms < 1) return FLEX_ERR_CUDA;
-      p.persist_grid = static_cast<int>(n_units < sms ? n_units : sms);
+      const int64_t grid = n_units < sms ? n_units : sms;
+      p.persist_grid = static_cast<int>(grid);
+      // The last round: R = n_units mod grid units would leave grid - R CTAs idle.  With
+      // R <= grid / 2 their key ranges split into parts (at most 4, at most one per key
+      // tile) that fill the round; the last part of each to finish merges them.  (B2 H32
+      // S2048: 512 units on 148 SMs take 4 rounds, as long as 592 units did.)  Not with
+      // the debug tile map, whose per-tile writes assume whole units.
+      const int64_t R = n_units % grid;
+      const int64_t parts = R > 0 ? std::min<int64_t>({kMaxParts, grid / R, span}) : 1;
+      if (parts >= 2 && !want_map) {
+        // counters: arrivals and parts ready, one each per (unit, tile, warp)
+        const size_t cnt_bytes = (2 * static_cast<size_t>(R) * 2 * 4 * sizeof(unsigned) + 255) / 256 * 256;
+        const size_t rows = static_cast<size_t>(R) * parts * 2 * kBM;
+        const size_t bytes = cnt_bytes + rows * sizeof(float2) + rows * D * sizeof(float);
+        cudaMemPool_t pool = scratch_pool();
+        if (pool && cudaMallocFromPoolAsync(&split_ws, bytes, pool, s) == cudaSuccess) {
+          if (cudaMemsetAsync(split_ws, 0, cnt_bytes, s) != cudaSuccess) {
+            cudaFreeAsync(split_ws, s);
+            return FLEX_ERR_CUDA;
+          }
+          char* base = static_cast<char*>(split_ws);
+          p.part_cnt = reinterpret_cast<unsigned*>(base);
+          p.part_ready_off = static_cast<int>(R * 2 * 4);
+          p.part_ml = reinterpret_cast<float2*>(base + cnt_bytes);
+          p.part_o = reinterpret_cast<float*>(base + cnt_bytes + rows * sizeof(float2));
+          p.n_full = static_cast<int>(n_units - R);
+          p.n_parts = static_cast<int>(parts);
+          p.n_items = static_cast<int>(n_units - R + R * parts);
+        } else {
+          split_ws = nullptr;  // no scratch: whole units only
+          cudaGetLastError();
+        }
+      }
     }
   }
   p.scale_log2 = scale * kLog2e;
   p.mask = mask_args(mask, mp, Skv);
   p.slopes = score_mod_id == FLEX_SCORE_ALIBI_SLOPES ? mp.alibi_slopes : nullptr;
   const int score = score_mod_id == FLEX_SCORE_NONE ? kScoreNone : kScoreAlibi;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int units = static_cast<int>(n_units);
   if (bm) {
     p.blk_num[0] = bm->kv_num_blocks;
@@ -391,8 +461,10 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
     return D == 128 ? fwd_dispatch<128, true>(dtype, score, mask, mq, mk, mv, p, units, s)
                     : fwd_dispatch<64, true>(dtype, score, mask, mq, mk, mv, p, units, s);
   }
-  return D == 128 ? fwd_dispatch<128, false>(dtype, score, mask, mq, mk, mv, p, units, s)
-                  : fwd_dispatch<64, false>(dtype, score, mask, mq, mk, mv, p, units, s);
+  const flex_status_t rc = D == 128 ? fwd_dispatch<128, false>(dtype, score, mask, mq, mk, mv, p, units, s)
+                                    : fwd_dispatch<64, false>(dtype, score, mask, mq, mk, mv, p, units, s);
+  if (split_ws && cudaFreeAsync(split_ws, s) != cudaSuccess && rc == FLEX_OK) return FLEX_ERR_CUDA;
+  return rc;
 }
 
 }  // namespace

@@ -96,6 +96,8 @@ constexpr int kMaxBlockKeyTiles = 2048;
 constexpr int kBlkWords = kMaxBlockKeyTiles / 32;
 // A FULL-listed key tile that runs past Skv: only the key-length rule masks it.
 constexpr int kTileFullRagged = 3;
+// Most parts the persistent kernel splits one unit's key ranges into (FwdParams::n_parts).
+constexpr int kMaxParts = 4;
 
 // Step record: what the MMA issuer does at one step of the CTA's walk over key tiles.
 // The TMA producer, which walks the same tiles ahead of time, writes the record of step
@@ -116,7 +118,17 @@ struct FwdParams {
   int H, Hkv, G, Sq, Skv;
   int n_qtiles, n_ktiles, n_pairs;
   int n_units;         // B * H * n_pairs (the persistent kernel loops over them)
-  int persist_grid;    // CTAs of the persistent kernel: min(n_units, SMs)
+  int persist_grid;    // CTAs of the persistent kernel (0: one CTA per unit)
+  // Persistent kernel: items [0, n_full) are whole units; items [n_full, n_items) split
+  // the last n_units - n_full units' key ranges into n_parts parts each.  The parts of a
+  // (unit, tile, warp) but the last to arrive leave their unnormalised O and (max, sum)
+  // per row in part_o / part_ml; the last merges them (counters in part_cnt).
+  int n_full, n_parts, n_items;
+  float* part_o;       // [split units][n_parts][2 tiles][D / 4][kBM rows] float4 (fp32 O)
+  float2* part_ml;     // [split units][n_parts][2 tiles][kBM rows] (max in log2 units, sum)
+  unsigned* part_cnt;  // arrivals, then (part_ready_off on) parts ready: [split units][2 tiles][4 warps],
+                       // zero at launch
+  int part_ready_off;
   float scale_log2;    // scale * log2(e)
   const float* slopes; // alibi: captured per-head slopes [H], or nullptr for 2^(-8(h+1)/H)
   MaskArgs mask;       // document rules: boundaries of batch 0, advanced per batch below
@@ -348,13 +360,15 @@ __device__ __forceinline__ void build_visit_sets(uint32_t* blk, int* doc_rows, c
   }
 }
 
-// PERSIST: one CTA per SM loops over the units blockIdx.x, blockIdx.x + gridDim.x, ...
-// (analytic masks, one MMA issuer).  The K/V ring and every barrier's phases run on across
-// units, so the next unit's first key/value tiles load while the current one drains; the
-// producer reloads the Q tiles once the S products of the previous unit have completed
-// (q_free, committed by the issuer at the unit's last step, before its P.V products).  The first P.V of a tile in a unit, which overwrites its O accumulator, needs
-// no barrier of its own: it waits for that tile's first P of the unit, which the softmax
-// warpgroup writes only after its epilogue has read O of the previous unit.
+// PERSIST: one CTA per SM loops over the items blockIdx.x, blockIdx.x + gridDim.x, ...
+// (analytic masks, one MMA issuer); an item is a unit or a part of one of the last units'
+// key ranges (FwdParams::n_full).  The K/V ring and every barrier's phases run on across
+// items, so the next item's first key/value tiles load while the current one drains; the
+// producer reloads the Q tiles once the S products of the previous item have completed
+// (q_free, committed by the issuer at the item's last step, before its P.V products).
+// The first P.V of a tile in an item, which overwrites its O accumulator, needs no barrier
+// of its own: it waits for that tile's first P of the item, which the softmax warpgroup
+// writes only after its epilogue has read O of the previous item.
 template <int D, typename T, int SCORE, int MASK, bool BLOCKS, bool PERSIST = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     flex_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -413,13 +427,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   };
   set_unit(blockIdx.x);
+  // item -> (unit, part): items from n_full on take part (item - n_full) % n_parts of
+  // unit n_full + (item - n_full) / n_parts, a contiguous share of each tile's key range
+  auto item_unit = [&](int item, int& part) {
+    part = -1;
+    if (!PERSIST || item < p.n_full) return item;
+    const int sidx = (item - p.n_full) / p.n_parts;
+    part = item - p.n_full - sidx * p.n_parts;
+    return p.n_full + sidx;
+  };
+  auto set_item = [&](int item) {
+    int part;
+    set_unit(item_unit(item, part));
+    if (part >= 0) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int n = hi[k] - lo[k];
+        if (n > 0) {
+          const int a = lo[k] + n * part / p.n_parts;
+          hi[k] = lo[k] + n * (part + 1) / p.n_parts;
+          lo[k] = a;
+        }
+      }
+    }
+  };
   if constexpr (kDoc) {
     mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
     mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
   }
-  // the units of this CTA: blockIdx.x (+ gridDim.x ...) up to unit_end
-  const int unit_end = PERSIST ? p.n_units : static_cast<int>(blockIdx.x) + 1;
-  const int unit_step = PERSIST ? static_cast<int>(gridDim.x) : 1;
+  // the items of this CTA: blockIdx.x (+ gridDim.x ...) up to item_end
+  const int item_end = PERSIST ? p.n_items : static_cast<int>(blockIdx.x) + 1;
+  const int item_step = PERSIST ? static_cast<int>(gridDim.x) : 1;
 
   // ---------------------------------------------------------------- visit bitmaps
   // With a block mask or a document mask the key tiles a query tile visits are a set, not
@@ -520,8 +558,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (i1) rec |= a1.cur < 0 ? kRecLast1 : (a1.cur == jn ? kRecPre1 : 0u);
         return rec;
       };
-      for (int unit = blockIdx.x; unit < unit_end && ok; unit += unit_step) {
-        if (PERSIST && unit != static_cast<int>(blockIdx.x)) set_unit(unit);
+      for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
+        if (PERSIST) set_item(item);
         auto c0 = cursor(0), c1 = cursor(1);
         const bool u0 = c0.cur >= 0, u1 = c1.cur >= 0;
         if (!u0 && !u1) continue;  // no key for either tile: every role skips the unit
@@ -630,8 +668,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       int rb = 0;  // ring position of the unit's first key load
       int qn = 0;  // units started (the Q barrier's phase)
-      for (int unit = blockIdx.x; unit < unit_end && ok; unit += unit_step) {
-        if (PERSIST && unit != static_cast<int>(blockIdx.x)) set_unit(unit);
+      for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
+        if (PERSIST) set_item(item);
         // fin_k: query tile k has no key tile left in this unit
         bool fin0 = cursor(0).cur < 0, fin1 = cursor(1).cur < 0;
         if (fin0 && fin1) continue;  // no work in this unit
@@ -813,8 +851,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bool ok = true;
     int n = 0;      // S tiles of this warpgroup so far (the S barrier's phase)
     int o_par = 0;  // O completions waited for (the O barrier's phase)
-    for (int unit = blockIdx.x; unit < unit_end && ok; unit += unit_step) {
-      if (PERSIST && unit != static_cast<int>(blockIdx.x)) set_unit(unit);
+    for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
+      if (PERSIST) set_item(item);
       const int q0k = sel(q0, k), q1k = sel(q1, k);
       const int qi = q0k + row;         // absolute query index
       const bool tile_valid = (2 * pair + k) < p.n_qtiles;
@@ -987,22 +1025,142 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           tc_fence_after();
         }
-        // The output row's address is recomputed from the unit index behind an opaque copy,
+        // The output row's address is recomputed from the item index behind an opaque copy,
         // so that the compiler keeps neither it nor the head index live through the key
         // tiles (in the persistent loop it cannot rebuild them from blockIdx).
-        const int ou = opaque_int(unit);
+        int opart;
+        const int ou = item_unit(opaque_int(item), opart);
         const int obh = ou / p.n_pairs;
         const int oqi = (2 * (p.n_pairs - 1 - ou % p.n_pairs) + k) * kBM + row;
         const bool row_ok = oqi < p.Sq;
         // A row has mass iff it ever saw a kept (finite) score.  The polynomial 2^x returns
         // ~2^-125 rather than 0 for masked scores, so l_sum alone cannot tell.
         const bool has_mass = ran && m_used != -INFINITY && l_sum > 0.f;
-        const float inv = has_mass ? 1.0f / l_sum : 0.f;
         T* orow = reinterpret_cast<T*>(p.o) + (static_cast<int64_t>(obh) * p.Sq + oqi) * D;
+        if (PERSIST && opart >= 0) {
+          // A part of a split unit.  Per warp (32 rows) the parts arrive on a counter; all
+          // but the last leave their rows' unnormalised O and (max, sum) in the workspace
+          // and count them ready; the last waits for those (their warps are past their
+          // key tiles, so the wait is their write time) and merges them with its own O,
+          // still in TMEM.  No warp waits for another of its own CTA.  A part's O is
+          // stored as [D / 4][kBM rows] float4s: the lanes of a warp, 32 consecutive rows,
+          // write and read 512 contiguous bytes per instruction.
+          const int64_t sidx = ou - p.n_full;
+          const int64_t slot0 = sidx * p.n_parts * 2 + k;  // (unit, part 0, tile k)
+          const int64_t cidx = (sidx * 2 + k) * 4 + wq;
+          unsigned* arrived = p.part_cnt + cidx;
+          unsigned* ready = p.part_cnt + p.part_ready_off + cidx;
+          unsigned done = 0;
+          if (lane == 0) done = atomicAdd(arrived, 1u);
+          done = __shfl_sync(0xffffffffu, done, 0);
+          const float m_own = has_mass ? m_used : -INFINITY;
+          const float l_own = has_mass ? l_sum : 0.f;
+          constexpr int64_t kPart4 = kBM * D / 4;  // float4s of one (part, tile) block
+          if (done != static_cast<unsigned>(p.n_parts - 1)) {
+            float4* dst = reinterpret_cast<float4*>(p.part_o) + (slot0 + 2 * opart) * kPart4 + row;
+  #pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+              uint32_t r[32];
+              if (ran) {
+                tmem_ld32(tO + c, r);
+              } else {
+  #pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = 0u;
+              }
+  #pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[(c / 4 + v) * kBM] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            }
+            p.part_ml[(slot0 + 2 * opart) * kBM + row] = make_float2(m_own, l_own);
+            __threadfence();  // this row's part is visible before the warp counts it ready
+            __syncwarp();
+            if (lane == 0) atomicAdd(ready, 1u);
+            continue;
+          }
+          bool got = true;
+          if (lane == 0)
+            got = wait_count_at_least(ready, static_cast<unsigned>(p.n_parts - 1), p.status, kStatusFwdTimeout,
+                                      kWaitTimeoutNs);
+          got = __shfl_sync(0xffffffffu, got, 0);  // (on a timeout the status says so; merged anyway)
+          __threadfence();
+          // merge: M = max of the maxima, L = sum of l_i 2^(m_i - M), O = sum of
+          // O_i 2^(m_i - M) / L (parts without mass weigh 0), summed in part order with
+          // this warp's own part in its place, so that the result does not depend on
+          // which part arrived last
+          float mi[kMaxParts], li[kMaxParts], wi[kMaxParts];
+          float M = -INFINITY;
+  #pragma unroll
+          for (int i = 0; i < kMaxParts; ++i) {
+            float2 ml = make_float2(-INFINITY, 0.f);
+            if (i == opart) ml = make_float2(m_own, l_own);
+            else if (i < p.n_parts) ml = __ldcg(p.part_ml + (slot0 + 2 * i) * kBM + row);
+            mi[i] = ml.x;
+            li[i] = ml.y;
+            M = fmaxf(M, ml.x);
+          }
+          float L = 0.f;
+  #pragma unroll
+          for (int i = 0; i < kMaxParts; ++i) {
+            wi[i] = mi[i] == -INFINITY ? 0.f : ex2_approx(mi[i] - M);
+            L = fmaf(li[i], wi[i], L);
+          }
+          const bool mass = got && M != -INFINITY && L > 0.f;
+          const float invL = mass ? 1.0f / L : 0.f;
+  #pragma unroll
+          for (int i = 0; i < kMaxParts; ++i) wi[i] *= invL;
+          const float4* src = reinterpret_cast<const float4*>(p.part_o) + slot0 * kPart4 + row;
+  #pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            uint32_t r[32];
+            if (ran) {
+              tmem_ld32(tO + c, r);
+            } else {
+  #pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = 0u;
+            }
+            float acc[32];
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+  #pragma unroll 1
+            for (int i = 0; i < p.n_parts; ++i) {
+              const float wpart = i == 0 ? wi[0] : i == 1 ? wi[1] : i == 2 ? wi[2] : wi[3];
+              float4 x[8];
+              if (i == opart) {
+  #pragma unroll
+                for (int v = 0; v < 8; ++v)
+                  x[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+              } else {
+  #pragma unroll
+                for (int v = 0; v < 8; ++v) x[v] = __ldcg(src + 2 * i * kPart4 + (c / 4 + v) * kBM);
+              }
+  #pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                acc[4 * v] = fmaf(wpart, x[v].x, acc[4 * v]);
+                acc[4 * v + 1] = fmaf(wpart, x[v].y, acc[4 * v + 1]);
+                acc[4 * v + 2] = fmaf(wpart, x[v].z, acc[4 * v + 2]);
+                acc[4 * v + 3] = fmaf(wpart, x[v].w, acc[4 * v + 3]);
+              }
+            }
+            if (row_ok) {
+              uint32_t w[16];
+  #pragma unroll
+              for (int e = 0; e < 16; ++e) w[e] = DtypeBits<T>::pack(acc[2 * e], acc[2 * e + 1]);
+              uint4* od = reinterpret_cast<uint4*>(orow + c);
+  #pragma unroll
+              for (int v = 0; v < 4; ++v) od[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+            }
+          }
+          if (row_ok && p.lse != nullptr)
+            p.lse[static_cast<int64_t>(obh) * p.Sq + oqi] = mass ? (M + lg2_approx(L)) * kLn2 : -INFINITY;
+          continue;
+        }
+        const float inv = has_mass ? 1.0f / l_sum : 0.f;
   #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           uint32_t r[32];
-          // defined on both paths: an undefined r would stay live around the unit loop
+          // defined on both paths: an undefined r would stay live around the item loop
           if (ran) {
             tmem_ld32(tO + c, r);
           } else {
@@ -1027,7 +1185,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               has_mass ? (m_used + lg2_approx(l_sum)) * kLn2 : -INFINITY;
         }
       }
-    }  // unit
+    }  // item
   }
 
   // ---------------------------------------------------------------- teardown

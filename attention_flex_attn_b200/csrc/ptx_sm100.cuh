@@ -69,6 +69,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
+// Bounded wait until the global counter *addr reaches `target` (acquire loads: what the
+// writers stored before their release of the counter is visible after).  Gives up after
+// timeout_ns of global time, ORs `code` into *status and returns false.
+__device__ __forceinline__ bool wait_count_at_least(const unsigned int* addr, unsigned int target,
+                                                    unsigned int* status, unsigned int code, uint64_t timeout_ns) {
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    if (v >= target) return true;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      atomicOr(status, code);
+      return false;
+    }
+    __nanosleep(32);
+  }
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -128,6 +128,39 @@ def test_long_8192(case):
     _run(q, k, v, 1.0 / math.sqrt(D), rows=rows, **mods)
 
 
+# ------------------------------------------------------------------ persistent kernel, split last round
+
+# Units (B*H*ceil(ceil(Sq/128)/2)) chosen so that on a 148-SM B200 the persistent kernel
+# splits the last round's units into 4, 3 or 2 parts (R = units mod 148 of them), with
+# windows that leave some parts empty, a ragged last query tile, a lone query tile in the
+# last pair, GQA, alibi and a key length unequal to the query length.  On another SM
+# count the split differs, and the oracle comparison holds all the same.
+SPLIT_CASES = [
+    (1, 38, 38, 1024, 1024, 128, dict()),                                        # R=4, 4 parts
+    (1, 49, 7, 1024, 1024, 128, dict(score_mod="alibi")),                        # R=48, 3 parts
+    (2, 32, 32, 2048, 2048, 128, dict()),                                        # R=68, 2 parts
+    (1, 38, 38, 1024, 1024, 64, dict(mask_mod="sliding_window", window=64)),      # empty parts
+    (1, 50, 10, 600, 600, 128, dict(mask_mod="sliding_window", window=200)),      # lone tile
+    (1, 40, 8, 1000, 1700, 64, dict(score_mod="alibi")),                         # ragged, Skv != Sq
+]
+
+
+@pytest.mark.parametrize("case", range(len(SPLIT_CASES)))
+def test_persistent_split_last_round(case):
+    B, H, Hkv, Sq, Skv, D, mods = SPLIT_CASES[case]
+    q, k, v = synth.qkv(B, H, Hkv, Sq, Skv, D, seed=synth.case_seed(6, case), device="cuda")
+    last = [(b, h, i) for b in range(B) for h in (0, H - 1) for i in (0, 127, 128, Sq - 129, Sq - 128, Sq - 1)]
+    rows = sample_rows(B, H, Sq, 2048, seed=60 + case, must=last)
+    _run(q, k, v, 1.0 / math.sqrt(D), rows=rows, **mods)
+    # the merge reads every part from memory in part order, whichever CTA merges: repeat
+    # calls agree bit for bit
+    fa = _fa()
+    o1, l1 = fa.fwd(q, k, v, **mods)
+    o2, l2 = fa.fwd(q, k, v, **mods)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 # ------------------------------------------------------------------ degenerate shapes
 
 @pytest.mark.parametrize("Sq,Skv", [(1, 1), (1, 300), (7, 1), (129, 129), (130, 5), (255, 513), (512, 128)])
