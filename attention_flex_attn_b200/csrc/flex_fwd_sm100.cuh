@@ -609,7 +609,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_wait(bar_q, static_cast<uint32_t>(qn - 1) & 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
     } else if (!two_issuers && warp == kMmaWarp && lane == 0) {
       // ============================================================ MMA issuer (both tiles)
+      // the first unit's Q (the persistent kernel waits for later units' in its item loop)
       bool ok = true;
+      if (any_work) {
+        ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+        tc_fence_after();
+      }
       int np[2] = {0, 0};
       // descriptor of chunk 0 / k-step 0; k-step kk adds ((kk/4)*chunk + (kk%4)*32) >> 4
       const uint64_t dq0 = smem_desc(q_smem(0), 16, 1024, kSwizzle128B);
@@ -666,72 +671,121 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         return true;
       };
-      int rb = 0;  // ring position of the unit's first key load
-      int qn = 0;  // units started (the Q barrier's phase)
-      for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
-        if (PERSIST) set_item(item);
-        // fin_k: query tile k has no key tile left in this unit
-        bool fin0 = cursor(0).cur < 0, fin1 = cursor(1).cur < 0;
-        if (fin0 && fin1) continue;  // no work in this unit
-        bool q_released = false;
-        if (!mbar_wait(bar_q, static_cast<uint32_t>(qn) & 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
-          ok = false;
-          break;
-        }
-        ++qn;
-        tc_fence_after();
-        s_ready[0] = s_ready[1] = started[0] = started[1] = false;
-        uint32_t rec = rec_smem[NS];  // published with the Q barrier
-        int t = 0;
-        for (; !(rec & kRecEnd) && ok; ++t) {
-          const int rK = rb + 2 * t, rV = rK + 1;
-          const int sK = rK % NS, sV = rV % NS;
-          const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
-          const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
-          if (need0 || need1) {
-            // K_j was not needed before: wait for it here (otherwise the previous step did)
-            if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+      if constexpr (!PERSIST) {
+        // One unit: a single pass over its steps.  (The item loop below, run for one
+        // unit, measured 13-18 % slower on B200 once a query tile visits more than 32
+        // key tiles; the persistent kernel runs only units of at most 32.)
+        if (any_work) {
+          uint32_t rec = rec_smem[NS];  // published with the Q barrier
+          for (int t = 0; !(rec & kRecEnd) && ok; ++t) {
+            const int rK = 2 * t, rV = rK + 1;
+            const int sK = rK % NS, sV = rV % NS;
+            const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
+            const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
+            if (need0 || need1) {
+              // K_j was not needed before: wait for it here (otherwise the previous step did)
+              if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+                             kStatusFwdTimeout, kWaitTimeoutNs)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              if (need0) {
+                issue_s(0, sK);
+                mma_commit(bar_s(0));
+              }
+              if (need1) {
+                issue_s(1, sK);
+                mma_commit(bar_s(1));
+              }
+            }
+            mma_commit(bar_empty(sK));
+            if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
                            kStatusFwdTimeout, kWaitTimeoutNs)) {
               ok = false;
               break;
             }
-            tc_fence_after();
-            if (need0) {
-              issue_s(0, sK);
-              mma_commit(bar_s(0));
-            }
-            if (need1) {
-              issue_s(1, sK);
-              mma_commit(bar_s(1));
-            }
+            const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
+            bool next_k_ready = false;
+            if (in0)
+              ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
+            if (ok && in1)
+              ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
+            if (!ok) break;
+            mma_commit(bar_empty(sV));
+            rec = next_rec;
           }
-          mma_commit(bar_empty(sK));
-          // The unit's last step: every S product of the unit has been issued, so Q is
-          // free once they complete; the next unit's Q loads during this step's P.V.
-          if (PERSIST && !q_released && (in0 ? (rec & kRecLast0) != 0 : fin0) &&
-              (in1 ? (rec & kRecLast1) != 0 : fin1)) {
-            mma_commit(bar_qfree);
-            q_released = true;
-          }
-          if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
-                         kStatusFwdTimeout, kWaitTimeoutNs)) {
-            ok = false;
-            break;
-          }
-          const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
-          bool next_k_ready = false;
-          if (in0)
-            ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
-          if (ok && in1)
-            ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
-          if (!ok) break;
-          mma_commit(bar_empty(sV));
-          if (in0 && (rec & kRecLast0)) fin0 = true;
-          if (in1 && (rec & kRecLast1)) fin1 = true;
-          rec = next_rec;
         }
-        rb += 2 * t;
-        if (PERSIST && !q_released) mma_commit(bar_qfree);  // (only when the walk broke off)
+      } else {
+        int rb = 0;  // ring position of the unit's first key load
+        int qn = 0;  // units started (the Q barrier's phase)
+        for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
+          if (PERSIST) set_item(item);
+          // fin_k: query tile k has no key tile left in this unit
+          bool fin0 = cursor(0).cur < 0, fin1 = cursor(1).cur < 0;
+          if (fin0 && fin1) continue;  // no work in this unit
+          bool q_released = false;
+          if (qn > 0 || !any_work) {  // (the first unit's Q, if it has work, was waited for above)
+            if (!mbar_wait(bar_q, static_cast<uint32_t>(qn) & 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          ++qn;
+          s_ready[0] = s_ready[1] = started[0] = started[1] = false;
+          uint32_t rec = rec_smem[NS];  // published with the Q barrier
+          int t = 0;
+          for (; !(rec & kRecEnd) && ok; ++t) {
+            const int rK = rb + 2 * t, rV = rK + 1;
+            const int sK = rK % NS, sV = rV % NS;
+            const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
+            const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
+            if (need0 || need1) {
+              // K_j was not needed before: wait for it here (otherwise the previous step did)
+              if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+                             kStatusFwdTimeout, kWaitTimeoutNs)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              if (need0) {
+                issue_s(0, sK);
+                mma_commit(bar_s(0));
+              }
+              if (need1) {
+                issue_s(1, sK);
+                mma_commit(bar_s(1));
+              }
+            }
+            mma_commit(bar_empty(sK));
+            // The unit's last step: every S product of the unit has been issued, so Q is
+            // free once they complete; the next unit's Q loads during this step's P.V.
+            if (PERSIST && !q_released && (in0 ? (rec & kRecLast0) != 0 : fin0) &&
+                (in1 ? (rec & kRecLast1) != 0 : fin1)) {
+              mma_commit(bar_qfree);
+              q_released = true;
+            }
+            if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
+                           kStatusFwdTimeout, kWaitTimeoutNs)) {
+              ok = false;
+              break;
+            }
+            const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
+            bool next_k_ready = false;
+            if (in0)
+              ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
+            if (ok && in1)
+              ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
+            if (!ok) break;
+            mma_commit(bar_empty(sV));
+            if (in0 && (rec & kRecLast0)) fin0 = true;
+            if (in1 && (rec & kRecLast1)) fin1 = true;
+            rec = next_rec;
+          }
+          rb += 2 * t;
+          if (PERSIST && !q_released) mma_commit(bar_qfree);  // (only when the walk broke off)
+        }
       }
       if (!ok) *abort_flag = 1;
       // Drain: all MMAs this thread issued have completed before TMEM is released.
