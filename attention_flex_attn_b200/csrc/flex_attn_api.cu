@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "flex_attn.h"
 #include "launch.cuh"
@@ -25,7 +26,7 @@ __device__ unsigned int g_status;
 namespace {
 
 // Largest key-tile count per query tile that runs on the persistent forward kernel.
-constexpr int64_t kPersistMaxKeyTiles = 32;
+constexpr int64_t kPersistMaxKeyTiles = 8;
 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -159,38 +160,57 @@ void* symbol_ptr(Symbol which) {
 
 void* decode_scratch_ptr() { return symbol_ptr(kSymScratch); }
 
-// Stream-ordered scratch of the forward's split units: a memory pool of the library's own
-// per device and context, which keeps its memory between calls (release threshold at the
-// maximum), so that steady-state calls neither map memory nor synchronise.
-cudaMemPool_t scratch_pool() {
-  constexpr int kMaxDevices = 64;
+// Workspace of the forward's split units, one per (context, stream) and kept for the
+// process's life: calls on one stream run in order and share it, calls on different
+// streams never do.  Sized for the most a launch can use (R * parts <= SMs split rows of
+// both tiles at D = 128); created zeroed on first use.  Each call takes the next tag for
+// the tagged counters, so they are never reset between calls.
+struct SplitWorkspace {
+  void* base;
+  unsigned tag;
+};
+
+bool split_workspace(cudaStream_t stream, int sms, SplitWorkspace* out, size_t* cnt_bytes_out,
+                     size_t* ml_bytes_out) {
   struct Entry {
     unsigned long long ctx;
-    cudaMemPool_t pool;
+    cudaStream_t stream;
+    void* base;
+    unsigned tag;
   };
-  static Entry cache[kMaxDevices] = {};
+  static std::vector<Entry> entries;
   static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   unsigned long long id = 0;
-  if (!current_context_id(&id)) return nullptr;
+  if (!current_context_id(&id)) return false;
+  const size_t rows = static_cast<size_t>(sms) * 2 * kBM;
+  const size_t cnt_bytes = (static_cast<size_t>(sms) * 2 * 4 * 2 * sizeof(unsigned long long) + 255) / 256 * 256;
+  const size_t ml_bytes = rows * sizeof(float2);
+  const size_t bytes = cnt_bytes + ml_bytes + rows * 128 * sizeof(float);
   std::lock_guard<std::mutex> lock(mu);
-  Entry& e = cache[dev];
-  if (e.pool && e.ctx == id) return e.pool;
-  cudaMemPoolProps props{};
-  props.allocType = cudaMemAllocationTypePinned;
-  props.location.type = cudaMemLocationTypeDevice;
-  props.location.id = dev;
-  cudaMemPool_t pool = nullptr;
-  if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
-  uint64_t keep = UINT64_MAX;
-  if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
-    cudaMemPoolDestroy(pool);
-    return nullptr;
+  for (Entry& e : entries) {
+    if (e.ctx == id && e.stream == stream) {
+      out->base = e.base;
+      out->tag = ++e.tag == 0 ? ++e.tag : e.tag;  // tag 0 is the zeroed state
+      *cnt_bytes_out = cnt_bytes;
+      *ml_bytes_out = ml_bytes;
+      return true;
+    }
   }
-  e.ctx = id;
-  e.pool = pool;
-  return pool;
+  void* base = nullptr;
+  if (cudaMalloc(&base, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (cudaMemsetAsync(base, 0, cnt_bytes, stream) != cudaSuccess) {  // ordered before the launch
+    cudaFree(base);
+    return false;
+  }
+  entries.push_back({id, stream, base, 1u});
+  out->base = base;
+  out->tag = 1u;
+  *cnt_bytes_out = cnt_bytes;
+  *ml_bytes_out = ml_bytes;
+  return true;
 }
 
 // Streaming multiprocessors of the current device (looked up once per device).
@@ -398,21 +418,21 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   p.n_full = p.n_items = static_cast<int>(n_units);
   p.n_parts = 1;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // Short units (few key tiles per query tile) run on the persistent kernel, where a
-  // CTA's fill and drain would otherwise be a large share of its time.  On long units the
-  // block scheduler's dynamic assignment wins (measured on B200, 128 rows per tile: 8 and
-  // 3 key tiles 9 % and 7 % faster persistent, 32 at D = 64 2 % faster, 64 5 % slower).
-  void* split_ws = nullptr;
+  // Units of uniform work (no mask or a sliding window, no block lists) run in rounds of
+  // one CTA per SM: on the persistent kernel when a query tile visits few key tiles (a
+  // CTA's fill and drain would otherwise be a large share of its time), else one CTA per
+  // unit, which the block scheduler places in waves.  (Measured on B200, 128-row tiles:
+  // 3 and 8 key tiles 8 % and 2 % faster persistent, 10 to 32 key tiles 4 to 11 % slower.)
   if (!bm && (mask == kMaskNone || mask == kMaskSliding)) {
     int64_t span = p.n_ktiles;
     if (mask == kMaskSliding)
       span = std::min<int64_t>(span, (static_cast<int64_t>(mp.window) + kBM - 1 + kBN - 1) / kBN + 1);
-    if (span <= kPersistMaxKeyTiles) {
-      const int sms = sm_count();
-      if (sms < 1) return FLEX_ERR_CUDA;
-      const int64_t grid = n_units < sms ? n_units : sms;
-      p.persist_grid = static_cast<int>(grid);
-      // The last round: R = n_units mod grid units would leave grid - R CTAs idle.  With
+    const int sms = sm_count();
+    if (sms < 1) return FLEX_ERR_CUDA;
+    const int64_t grid = n_units < sms ? n_units : sms;
+    if (span <= kPersistMaxKeyTiles) p.persist_grid = static_cast<int>(grid);
+    {
+      // The last round: R = n_units mod grid units would leave grid - R SMs idle.  With
       // R <= grid / 2 their key ranges split into parts (at most 4, at most one per key
       // tile) that fill the round; the last part of each to finish merges them.  (B2 H32
       // S2048: 512 units on 148 SMs take 4 rounds, as long as 592 units did.)  Not with
@@ -420,28 +440,18 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
       const int64_t R = n_units % grid;
       const int64_t parts = R > 0 ? std::min<int64_t>({kMaxParts, grid / R, span}) : 1;
       if (parts >= 2 && !want_map) {
-        // counters: arrivals and parts ready, one each per (unit, tile, warp)
-        const size_t cnt_bytes = (2 * static_cast<size_t>(R) * 2 * 4 * sizeof(unsigned) + 255) / 256 * 256;
-        const size_t rows = static_cast<size_t>(R) * parts * 2 * kBM;
-        const size_t bytes = cnt_bytes + rows * sizeof(float2) + rows * D * sizeof(float);
-        cudaMemPool_t pool = scratch_pool();
-        if (pool && cudaMallocFromPoolAsync(&split_ws, bytes, pool, s) == cudaSuccess) {
-          if (cudaMemsetAsync(split_ws, 0, cnt_bytes, s) != cudaSuccess) {
-            cudaFreeAsync(split_ws, s);
-            return FLEX_ERR_CUDA;
-          }
-          char* base = static_cast<char*>(split_ws);
-          p.part_cnt = reinterpret_cast<unsigned*>(base);
-          p.part_ready_off = static_cast<int>(R * 2 * 4);
+        SplitWorkspace ws{};
+        size_t cnt_bytes = 0, ml_bytes = 0;
+        if (split_workspace(s, sms, &ws, &cnt_bytes, &ml_bytes)) {
+          char* base = static_cast<char*>(ws.base);
+          p.part_cnt = reinterpret_cast<unsigned long long*>(base);
+          p.part_tag = ws.tag;
           p.part_ml = reinterpret_cast<float2*>(base + cnt_bytes);
-          p.part_o = reinterpret_cast<float*>(base + cnt_bytes + rows * sizeof(float2));
+          p.part_o = reinterpret_cast<float*>(base + cnt_bytes + ml_bytes);
           p.n_full = static_cast<int>(n_units - R);
           p.n_parts = static_cast<int>(parts);
           p.n_items = static_cast<int>(n_units - R + R * parts);
-        } else {
-          split_ws = nullptr;  // no scratch: whole units only
-          cudaGetLastError();
-        }
+        }  // else whole units only
       }
     }
   }
@@ -461,10 +471,8 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
     return D == 128 ? fwd_dispatch<128, true>(dtype, score, mask, mq, mk, mv, p, units, s)
                     : fwd_dispatch<64, true>(dtype, score, mask, mq, mk, mv, p, units, s);
   }
-  const flex_status_t rc = D == 128 ? fwd_dispatch<128, false>(dtype, score, mask, mq, mk, mv, p, units, s)
-                                    : fwd_dispatch<64, false>(dtype, score, mask, mq, mk, mv, p, units, s);
-  if (split_ws && cudaFreeAsync(split_ws, s) != cudaSuccess && rc == FLEX_OK) return FLEX_ERR_CUDA;
-  return rc;
+  return D == 128 ? fwd_dispatch<128, false>(dtype, score, mask, mq, mk, mv, p, units, s)
+                  : fwd_dispatch<64, false>(dtype, score, mask, mq, mk, mv, p, units, s);
 }
 
 }  // namespace

@@ -56,7 +56,7 @@ flex_status_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   auto kern = flex_fwd_kernel<D, T, SCORE, MASK, BLOCKS, false>;
   constexpr int kSmem = FwdSmem<D, BLOCKS, is_doc_mask(MASK)>::kAlloc;
   if (!ensure_smem_attr<D, T, SCORE, MASK, BLOCKS, false>(kern, kSmem)) return FLEX_ERR_CUDA;
-  kern<<<n_units, kFwdThreads, kSmem, stream>>>(mq, mk, mv, p);
+  kern<<<p.n_items, kFwdThreads, kSmem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FLEX_OK : FLEX_ERR_CUDA;
 }
 

@@ -122,13 +122,13 @@ struct FwdParams {
   // Persistent kernel: items [0, n_full) are whole units; items [n_full, n_items) split
   // the last n_units - n_full units' key ranges into n_parts parts each.  The parts of a
   // (unit, tile, warp) but the last to arrive leave their unnormalised O and (max, sum)
-  // per row in part_o / part_ml; the last merges them (counters in part_cnt).
+  // per row in part_o / part_ml; the last merges them.  The counters are tagged
+  // (tagged_add): every launch brings a new part_tag, so they are never zeroed.
   int n_full, n_parts, n_items;
   float* part_o;       // [split units][n_parts][2 tiles][D / 4][kBM rows] float4 (fp32 O)
   float2* part_ml;     // [split units][n_parts][2 tiles][kBM rows] (max in log2 units, sum)
-  unsigned* part_cnt;  // arrivals, then (part_ready_off on) parts ready: [split units][2 tiles][4 warps],
-                       // zero at launch
-  int part_ready_off;
+  unsigned long long* part_cnt;  // [split units][2 tiles][4 warps][arrived, ready]
+  unsigned part_tag;
   float scale_log2;    // scale * log2(e)
   const float* slopes; // alibi: captured per-head slopes [H], or nullptr for 2^(-8(h+1)/H)
   MaskArgs mask;       // document rules: boundaries of batch 0, advanced per batch below
@@ -426,12 +426,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (qt < p.n_qtiles && !kDoc) tile_range<MASK>(q0[k], q1[k], kBN, mk, lo[k], hi[k]);
     }
   };
-  set_unit(blockIdx.x);
   // item -> (unit, part): items from n_full on take part (item - n_full) % n_parts of
   // unit n_full + (item - n_full) / n_parts, a contiguous share of each tile's key range
+  // (the per-unit kernel runs item blockIdx.x, the persistent kernel a list of items)
   auto item_unit = [&](int item, int& part) {
     part = -1;
-    if (!PERSIST || item < p.n_full) return item;
+    if (item < p.n_full) return item;
     const int sidx = (item - p.n_full) / p.n_parts;
     part = item - p.n_full - sidx * p.n_parts;
     return p.n_full + sidx;
@@ -451,6 +451,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
   };
+  set_item(blockIdx.x);
   if constexpr (kDoc) {
     mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
     mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
@@ -1091,7 +1092,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ~2^-125 rather than 0 for masked scores, so l_sum alone cannot tell.
         const bool has_mass = ran && m_used != -INFINITY && l_sum > 0.f;
         T* orow = reinterpret_cast<T*>(p.o) + (static_cast<int64_t>(obh) * p.Sq + oqi) * D;
-        if (PERSIST && opart >= 0) {
+        if (opart >= 0) {
           // A part of a split unit.  Per warp (32 rows) the parts arrive on a counter; all
           // but the last leave their rows' unnormalised O and (max, sum) in the workspace
           // and count them ready; the last waits for those (their warps are past their
@@ -1101,11 +1102,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // write and read 512 contiguous bytes per instruction.
           const int64_t sidx = ou - p.n_full;
           const int64_t slot0 = sidx * p.n_parts * 2 + k;  // (unit, part 0, tile k)
-          const int64_t cidx = (sidx * 2 + k) * 4 + wq;
-          unsigned* arrived = p.part_cnt + cidx;
-          unsigned* ready = p.part_cnt + p.part_ready_off + cidx;
+          unsigned long long* arrived = p.part_cnt + ((sidx * 2 + k) * 4 + wq) * 2;
+          unsigned long long* ready = arrived + 1;
           unsigned done = 0;
-          if (lane == 0) done = atomicAdd(arrived, 1u);
+          if (lane == 0) done = tagged_add(arrived, p.part_tag);
           done = __shfl_sync(0xffffffffu, done, 0);
           const float m_own = has_mass ? m_used : -INFINITY;
           const float l_own = has_mass ? l_sum : 0.f;
@@ -1129,15 +1129,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             p.part_ml[(slot0 + 2 * opart) * kBM + row] = make_float2(m_own, l_own);
             __threadfence();  // this row's part is visible before the warp counts it ready
             __syncwarp();
-            if (lane == 0) atomicAdd(ready, 1u);
+            if (lane == 0) tagged_add(ready, p.part_tag);
             continue;
           }
           bool got = true;
           if (lane == 0)
-            got = wait_count_at_least(ready, static_cast<unsigned>(p.n_parts - 1), p.status, kStatusFwdTimeout,
-                                      kWaitTimeoutNs);
+            got = wait_tagged_at_least(ready, p.part_tag, static_cast<unsigned>(p.n_parts - 1), p.status,
+                                       kStatusFwdTimeout, kWaitTimeoutNs);
           got = __shfl_sync(0xffffffffu, got, 0);  // (on a timeout the status says so; merged anyway)
           __threadfence();
+          if (lane == 0) {  // every part is done with the counters: back to 0 under this tag (a
+            const unsigned long long zero = static_cast<unsigned long long>(p.part_tag) << 32;
+            *arrived = zero;  // replayed graph brings the same tag again)
+            *ready = zero;
+          }
           // merge: M = max of the maxima, L = sum of l_i 2^(m_i - M), O = sum of
           // O_i 2^(m_i - M) / L (parts without mass weigh 0), summed in part order with
           // this warp's own part in its place, so that the result does not depend on

@@ -69,16 +69,31 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
-// Bounded wait until the global counter *addr reaches `target` (acquire loads: what the
-// writers stored before their release of the counter is visible after).  Gives up after
-// timeout_ns of global time, ORs `code` into *status and returns false.
-__device__ __forceinline__ bool wait_count_at_least(const unsigned int* addr, unsigned int target,
-                                                    unsigned int* status, unsigned int code, uint64_t timeout_ns) {
+// Tagged counters: a 64-bit word (tag << 32) | count, where a count under another tag
+// reads as 0, so a caller that gives every launch a new tag never has to zero them.
+// Adds 1 to the count under `tag` and returns the count before.
+__device__ __forceinline__ unsigned int tagged_add(unsigned long long* c, unsigned int tag) {
+  unsigned long long seen = *reinterpret_cast<volatile unsigned long long*>(c), prev;
+  unsigned int cnt;
+  do {
+    prev = seen;
+    cnt = static_cast<unsigned int>(prev >> 32) == tag ? static_cast<unsigned int>(prev) : 0u;
+    seen = atomicCAS(c, prev, (static_cast<unsigned long long>(tag) << 32) | (cnt + 1u));
+  } while (seen != prev);
+  return cnt;
+}
+
+// Bounded wait until the tagged counter *c holds at least `target` under `tag` (acquire
+// loads: what the adders stored before their release of the counter is visible after).
+// Gives up after timeout_ns of global time, ORs `code` into *status and returns false.
+__device__ __forceinline__ bool wait_tagged_at_least(const unsigned long long* c, unsigned int tag,
+                                                     unsigned int target, unsigned int* status, unsigned int code,
+                                                     uint64_t timeout_ns) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
-    if (v >= target) return true;
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(c) : "memory");
+    if (static_cast<unsigned int>(v >> 32) == tag && static_cast<unsigned int>(v) >= target) return true;
     if (global_timer_ns() - t0 > timeout_ns) {
       atomicOr(status, code);
       return false;

@@ -161,6 +161,40 @@ def test_persistent_split_last_round(case):
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+def test_split_two_streams_and_graph_replay():
+    """Split launches on two streams at once each use their own workspace; a captured
+    graph, which replays the same counter tag, resets the counters after every merge.
+    Every result equals the eager single-stream result bit for bit."""
+    fa = _fa()
+    B, H, Hkv, Sq, Skv, D, mods = SPLIT_CASES[0]
+    q, k, v = synth.qkv(B, H, Hkv, Sq, Skv, D, seed=synth.case_seed(6, 0), device="cuda")
+    o_ref, l_ref = fa.fwd(q, k, v, **mods)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            outs.append(fa.fwd(q, k, v, **mods))
+        with torch.cuda.stream(s2):
+            outs.append(fa.fwd(q, k, v, **mods))
+    torch.cuda.synchronize()
+    for o, l in outs:
+        assert torch.equal(o, o_ref) and torch.equal(l, l_ref)
+    g_stream = torch.cuda.Stream()
+    with torch.cuda.stream(g_stream):
+        fa.fwd(q, k, v, **mods)  # creates this stream's workspace before the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=g_stream):
+        o_g, l_g = fa.fwd(q, k, v, **mods)
+    for _ in range(3):
+        o_g.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o_g, o_ref) and torch.equal(l_g, l_ref)
+    assert fa.device_status() == 0
+
+
 # ------------------------------------------------------------------ degenerate shapes
 
 @pytest.mark.parametrize("Sq,Skv", [(1, 1), (1, 300), (7, 1), (129, 129), (130, 5), (255, 513), (512, 128)])
