@@ -38,15 +38,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # dram read+write bytes per launch from ncu, keyed by the hash of the kernel sources
 # they were measured on (a changed kernel reports null until it is captured again)
 MEASURED_TRAFFIC = {
-    # flex_fwd_kernel<128,bf16,none,none>, B2 H32 S8192 D128: 402,710,784 B read +
-    # 113,622,272 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192.md)
-    "54190ee8878a9ab1": 516333056,
+    # flex_fwd_kernel<128,bf16,none,none> (one CTA per unit), B2 H32 S8192 D128:
+    # 402,723,328 B read + 114,665,984 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192.md)
+    "c9bf501cb9bd5bcb": 517389312,
 }
 MEASURED_DECODE_TRAFFIC = {
     # decode_split_kernel<128,f16,1,128>, B16 H32 Hkv32 cap8192, the bench's lengths and
-    # mask: 868,650,496 B read + 5,636,608 B written
+    # mask: 868,650,240 B read + 5,617,152 B written
     # (profiles/decode_split_kernel_f16_hkv32_bench.md)
-    "cfc6ae7c1e23a6be": 874287104,
+    "c56b25081c3bff63": 874267392,
 }
 # the forward kernel's sources: the roofline traffic below belongs to that kernel
 KERNEL_SOURCES = ["attention_flex_attn_b200/csrc/flex_fwd_sm100.cuh",
