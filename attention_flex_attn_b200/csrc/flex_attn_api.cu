@@ -26,7 +26,7 @@ __device__ unsigned int g_status;
 namespace {
 
 // Largest key-tile count per query tile that runs on the persistent forward kernel.
-constexpr int64_t kPersistMaxKeyTiles = 8;
+constexpr int64_t kPersistMaxKeyTiles = 32;
 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -421,8 +421,9 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   // Units of uniform work (no mask or a sliding window, no block lists) run in rounds of
   // one CTA per SM: on the persistent kernel when a query tile visits few key tiles (a
   // CTA's fill and drain would otherwise be a large share of its time), else one CTA per
-  // unit, which the block scheduler places in waves.  (Measured on B200, 128-row tiles:
-  // 3 and 8 key tiles 8 % and 2 % faster persistent, 10 to 32 key tiles 4 to 11 % slower.)
+  // unit, which the block scheduler places in waves.  (Measured on B200, 128-row tiles,
+  // persistent against per-unit: 3-4 key tiles +15 %, 8 +9 %, 10 +2 %, 16 +4 to +8 %,
+  // 32 at D = 64 +7 %, 32 at D = 128 -1 %, 48 and 64 -2 to -5 %, 128 equal.)
   if (!bm && (mask == kMaskNone || mask == kMaskSliding)) {
     int64_t span = p.n_ktiles;
     if (mask == kMaskSliding)

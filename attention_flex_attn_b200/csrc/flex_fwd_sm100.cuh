@@ -109,6 +109,7 @@ constexpr uint32_t kRecPre1 = 1u << 3;
 constexpr uint32_t kRecLast0 = 1u << 4;  // ... and this is its last key tile
 constexpr uint32_t kRecLast1 = 1u << 5;
 constexpr uint32_t kRecEnd = 1u << 6;    // no step: the walk is over
+constexpr uint32_t kRecNewItem = 1u << 7;  // persistent kernel: the first step of the next item
 
 struct FwdParams {
   void* o;
@@ -543,8 +544,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     regs_dec<kAuxRegs>();
     if (warp == kTmaWarp && lane == 0) {
       // ============================================================ TMA producer
-      int r = 0;   // key/value loads issued (the ring position, across units)
-      int qn = 0;  // units whose Q tiles were loaded
+      int r = 0;   // key/value loads issued (the ring position, across items)
+      int qn = 0;  // items whose Q tiles were loaded
       bool ok = true;
       // record of the step at max(a0.cur, a1.cur) (copies: the caller's cursors stay put)
       auto make_rec = [](auto a0, auto a1) -> uint32_t {
@@ -559,45 +560,100 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (i1) rec |= a1.cur < 0 ? kRecLast1 : (a1.cur == jn ? kRecPre1 : 0u);
         return rec;
       };
-      for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
-        if (PERSIST) set_item(item);
-        auto c0 = cursor(0), c1 = cursor(1);
-        const bool u0 = c0.cur >= 0, u1 = c1.cur >= 0;
-        if (!u0 && !u1) continue;  // no key for either tile: every role skips the unit
-        // the previous unit's products must be done with the Q tiles
-        if (qn > 0 && !mbar_wait(bar_qfree, static_cast<uint32_t>(qn - 1) & 1u, p.status, kStatusFwdTimeout,
-                                 kWaitTimeoutNs)) {
-          *abort_flag = 1;
-          break;
-        }
-        // The first record is published with the Q barrier, which the issuer waits on first.
-        rec_smem[NS] = make_rec(c0, c1);
-        const int bytes_q = (u0 ? 1 : 0) * L::kTileBytes + (u1 ? 1 : 0) * L::kTileBytes;
-        mbar_arrive_expect_tx(bar_q, bytes_q);
+      // Q of the current item (set_item state) on bar_q; u_k: query tile k has work
+      auto load_q = [&](bool u0, bool u1) {
+        mbar_arrive_expect_tx(bar_q, (u0 ? 1 : 0) * L::kTileBytes + (u1 ? 1 : 0) * L::kTileBytes);
         for (int k = 0; k < 2; ++k) {
           if (!(k == 0 ? u0 : u1)) continue;
           for (int c = 0; c < kChunks; ++c)
             tma_load_3d(q_smem(k) + c * L::kChunkBytes, &tmQ, bar_q, c * 64, sel(q0, k), bh);
         }
-        ++qn;
-        for (int j = max(c0.cur, c1.cur); j >= 0 && ok; j = max(c0.cur, c1.cur)) {  // last to first
-          if (c0.cur == j) c0.advance();
-          if (c1.cur == j) c1.advance();
-          const uint32_t next_rec = make_rec(c0, c1);
-          for (int which = 0; which < 2 && ok; ++which, ++r) {
-            const int s = r % NS;
-            const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
-            if (!mbar_wait(bar_empty(s), ph ^ 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs) ||
-                *abort_flag) {
+      };
+      if constexpr (PERSIST) {
+        // The items with work form one walk: at an item's last step the record carried
+        // with V is the next item's first one, flagged kRecNewItem; that item's Q loads
+        // once the issuer has released the previous Q (q_free).
+        auto next_work = [&](int it) {  // first item from `it` on with work (set_item state)
+          for (; it < item_end; it += item_step) {
+            set_item(it);
+            if (cursor(0).cur >= 0 || cursor(1).cur >= 0) break;
+          }
+          return it;
+        };
+        int item = next_work(static_cast<int>(blockIdx.x));
+        if (item < item_end) {
+          auto c0 = cursor(0), c1 = cursor(1);
+          rec_smem[NS] = make_rec(c0, c1);  // published with the Q barrier
+          load_q(c0.cur >= 0, c1.cur >= 0);
+          qn = 1;
+          while (ok) {
+            const int bkv_item = bkv;
+            int nxt = item_end;
+            for (int j = max(c0.cur, c1.cur); j >= 0 && ok; j = max(c0.cur, c1.cur)) {  // last to first
+              if (c0.cur == j) c0.advance();
+              if (c1.cur == j) c1.advance();
+              uint32_t next_rec = make_rec(c0, c1);
+              if (next_rec == kRecEnd) {  // the item's last step: chain the next item
+                nxt = next_work(item + item_step);
+                if (nxt < item_end) next_rec = make_rec(cursor(0), cursor(1)) | kRecNewItem;
+              }
+              for (int which = 0; which < 2 && ok; ++which, ++r) {
+                const int s = r % NS;
+                const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
+                if (!mbar_wait(bar_empty(s), ph ^ 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs) ||
+                    *abort_flag) {
+                  *abort_flag = 1;
+                  ok = false;
+                  break;
+                }
+                if (which == 1) rec_smem[s] = next_rec;  // released by the arrive below
+                mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
+                const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+                for (int c = 0; c < kChunks; ++c)
+                  tma_load_3d(kv_smem(s) + c * L::kChunkBytes, map, bar_full(s), c * 64, j * kBN, bkv_item);
+              }
+            }
+            if (!ok || nxt >= item_end) break;
+            item = nxt;  // set_item state is the next item's
+            c0 = cursor(0);
+            c1 = cursor(1);
+            // the previous item's S products must be done with the Q tiles
+            if (!mbar_wait(bar_qfree, static_cast<uint32_t>(qn - 1) & 1u, p.status, kStatusFwdTimeout,
+                           kWaitTimeoutNs)) {
               *abort_flag = 1;
-              ok = false;
               break;
             }
-            if (which == 1) rec_smem[s] = next_rec;  // released by the arrive below
-            mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
-            const CUtensorMap* map = which == 0 ? &tmK : &tmV;
-            for (int c = 0; c < kChunks; ++c)
-              tma_load_3d(kv_smem(s) + c * L::kChunkBytes, map, bar_full(s), c * 64, j * kBN, bkv);
+            load_q(c0.cur >= 0, c1.cur >= 0);
+            ++qn;
+          }
+        }
+      } else {
+        auto c0 = cursor(0), c1 = cursor(1);
+        const bool u0 = c0.cur >= 0, u1 = c1.cur >= 0;
+        if (u0 || u1) {
+          // The first record is published with the Q barrier, which the issuer waits on first.
+          rec_smem[NS] = make_rec(c0, c1);
+          load_q(u0, u1);
+          qn = 1;
+          for (int j = max(c0.cur, c1.cur); j >= 0 && ok; j = max(c0.cur, c1.cur)) {  // last to first
+            if (c0.cur == j) c0.advance();
+            if (c1.cur == j) c1.advance();
+            const uint32_t next_rec = make_rec(c0, c1);
+            for (int which = 0; which < 2 && ok; ++which, ++r) {
+              const int s = r % NS;
+              const uint32_t ph = static_cast<uint32_t>(r / NS) & 1u;
+              if (!mbar_wait(bar_empty(s), ph ^ 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs) ||
+                  *abort_flag) {
+                *abort_flag = 1;
+                ok = false;
+                break;
+              }
+              if (which == 1) rec_smem[s] = next_rec;  // released by the arrive below
+              mbar_arrive_expect_tx(bar_full(s), L::kTileBytes);
+              const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+              for (int c = 0; c < kChunks; ++c)
+                tma_load_3d(kv_smem(s) + c * L::kChunkBytes, map, bar_full(s), c * 64, j * kBN, bkv);
+            }
           }
         }
       }
@@ -672,120 +728,83 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         return true;
       };
-      if constexpr (!PERSIST) {
-        // One unit: a single pass over its steps.  (The item loop below, run for one
-        // unit, measured 13-18 % slower on B200 once a query tile visits more than 32
-        // key tiles; the persistent kernel runs only units of at most 32.)
-        if (any_work) {
-          uint32_t rec = rec_smem[NS];  // published with the Q barrier
-          for (int t = 0; !(rec & kRecEnd) && ok; ++t) {
-            const int rK = 2 * t, rV = rK + 1;
-            const int sK = rK % NS, sV = rV % NS;
-            const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
-            const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
-            if (need0 || need1) {
-              // K_j was not needed before: wait for it here (otherwise the previous step did)
-              if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
-                             kStatusFwdTimeout, kWaitTimeoutNs)) {
+      // One pass over the steps.  The persistent kernel's items chain their steps: the
+      // record of an item's last step is followed by the first record of the next item
+      // with work, flagged kRecNewItem, so the loop runs on across items.  (An item loop
+      // around the step loop measured 13-18 % slower on B200 in the per-unit kernel from
+      // 48 key tiles per query tile on, and 6-14 % per item in the persistent kernel.)
+      bool run = any_work;
+      if constexpr (PERSIST) {
+        if (!any_work) {  // the CTA's first item with work is a later one: bar_q's first phase
+          int it = blockIdx.x + item_step;
+          for (; it < item_end; it += item_step) {
+            set_item(it);
+            if (cursor(0).cur >= 0 || cursor(1).cur >= 0) break;
+          }
+          run = it < item_end;
+          if (run) {
+            ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
+            tc_fence_after();
+          }
+        }
+      }
+      if (run) {
+        uint32_t rec = rec_smem[NS];  // published with the Q barrier
+        [[maybe_unused]] int qn = 1;  // items started (the Q barrier's phase)
+        for (int t = 0; !(rec & kRecEnd) && ok; ++t) {
+          if constexpr (PERSIST) {
+            if (rec & kRecNewItem) {  // the next item's Q (loaded once q_free let it)
+              if (!mbar_wait(bar_q, static_cast<uint32_t>(qn) & 1u, p.status, kStatusFwdTimeout,
+                             kWaitTimeoutNs)) {
                 ok = false;
                 break;
               }
+              ++qn;
               tc_fence_after();
-              if (need0) {
-                issue_s(0, sK);
-                mma_commit(bar_s(0));
-              }
-              if (need1) {
-                issue_s(1, sK);
-                mma_commit(bar_s(1));
-              }
+              s_ready[0] = s_ready[1] = started[0] = started[1] = false;
             }
-            mma_commit(bar_empty(sK));
-            if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
-                           kStatusFwdTimeout, kWaitTimeoutNs)) {
-              ok = false;
-              break;
-            }
-            const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
-            bool next_k_ready = false;
-            if (in0)
-              ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
-            if (ok && in1)
-              ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
-            if (!ok) break;
-            mma_commit(bar_empty(sV));
-            rec = next_rec;
           }
-        }
-      } else {
-        int rb = 0;  // ring position of the unit's first key load
-        int qn = 0;  // units started (the Q barrier's phase)
-        for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
-          if (PERSIST) set_item(item);
-          // fin_k: query tile k has no key tile left in this unit
-          bool fin0 = cursor(0).cur < 0, fin1 = cursor(1).cur < 0;
-          if (fin0 && fin1) continue;  // no work in this unit
-          bool q_released = false;
-          if (qn > 0 || !any_work) {  // (the first unit's Q, if it has work, was waited for above)
-            if (!mbar_wait(bar_q, static_cast<uint32_t>(qn) & 1u, p.status, kStatusFwdTimeout, kWaitTimeoutNs)) {
+          const int rK = 2 * t, rV = rK + 1;
+          const int sK = rK % NS, sV = rV % NS;
+          const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
+          const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
+          if (need0 || need1) {
+            // K_j was not needed before: wait for it here (otherwise the previous step did)
+            if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
+                           kStatusFwdTimeout, kWaitTimeoutNs)) {
               ok = false;
               break;
             }
             tc_fence_after();
+            if (need0) {
+              issue_s(0, sK);
+              mma_commit(bar_s(0));
+            }
+            if (need1) {
+              issue_s(1, sK);
+              mma_commit(bar_s(1));
+            }
           }
-          ++qn;
-          s_ready[0] = s_ready[1] = started[0] = started[1] = false;
-          uint32_t rec = rec_smem[NS];  // published with the Q barrier
-          int t = 0;
-          for (; !(rec & kRecEnd) && ok; ++t) {
-            const int rK = rb + 2 * t, rV = rK + 1;
-            const int sK = rK % NS, sV = rV % NS;
-            const bool in0 = rec & kRecIn0, in1 = rec & kRecIn1;
-            const bool need0 = in0 && !s_ready[0], need1 = in1 && !s_ready[1];
-            if (need0 || need1) {
-              // K_j was not needed before: wait for it here (otherwise the previous step did)
-              if (!mbar_wait(bar_full(sK), static_cast<uint32_t>(rK / NS) & 1u, p.status,
-                             kStatusFwdTimeout, kWaitTimeoutNs)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              if (need0) {
-                issue_s(0, sK);
-                mma_commit(bar_s(0));
-              }
-              if (need1) {
-                issue_s(1, sK);
-                mma_commit(bar_s(1));
-              }
-            }
-            mma_commit(bar_empty(sK));
-            // The unit's last step: every S product of the unit has been issued, so Q is
-            // free once they complete; the next unit's Q loads during this step's P.V.
-            if (PERSIST && !q_released && (in0 ? (rec & kRecLast0) != 0 : fin0) &&
-                (in1 ? (rec & kRecLast1) != 0 : fin1)) {
-              mma_commit(bar_qfree);
-              q_released = true;
-            }
-            if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
-                           kStatusFwdTimeout, kWaitTimeoutNs)) {
-              ok = false;
-              break;
-            }
-            const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
-            bool next_k_ready = false;
-            if (in0)
-              ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
-            if (ok && in1)
-              ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
-            if (!ok) break;
-            mma_commit(bar_empty(sV));
-            if (in0 && (rec & kRecLast0)) fin0 = true;
-            if (in1 && (rec & kRecLast1)) fin1 = true;
-            rec = next_rec;
+          mma_commit(bar_empty(sK));
+          if (!mbar_wait(bar_full(sV), static_cast<uint32_t>(rV / NS) & 1u, p.status,
+                         kStatusFwdTimeout, kWaitTimeoutNs)) {
+            ok = false;
+            break;
           }
-          rb += 2 * t;
-          if (PERSIST && !q_released) mma_commit(bar_qfree);  // (only when the walk broke off)
+          const uint32_t next_rec = rec_smem[sV];  // the next step's record came with V
+          if constexpr (PERSIST) {
+            // the item's last step: every S product of the item has been issued, so Q is
+            // free once they complete; the next item's Q loads during this step's P.V
+            if (next_rec & (kRecNewItem | kRecEnd)) mma_commit(bar_qfree);
+          }
+          bool next_k_ready = false;
+          if (in0)
+            ok = tile_step(std::integral_constant<int, 0>{}, rec & kRecPre0, rec & kRecLast0, rK, sV, next_k_ready);
+          if (ok && in1)
+            ok = tile_step(std::integral_constant<int, 1>{}, rec & kRecPre1, rec & kRecLast1, rK, sV, next_k_ready);
+          if (!ok) break;
+          mma_commit(bar_empty(sV));
+          rec = next_rec;
         }
       }
       if (!ok) *abort_flag = 1;

@@ -231,14 +231,16 @@ def fwd_roles(sets, NS, issuers="two"):
 def fwd_persistent_roles(units, NS, wait_q_free=True, q_free_at="last_step"):
     """The persistent forward: one CTA runs the units (each a pair of key-tile sets) in
     order with one MMA issuer.  The K/V ring and every barrier's phases run on across
-    units; the producer loads a unit's Q tiles once the S products of the previous unit
-    have completed (Q free), which the issuer commits at the unit's last step, after that
-    step's S products and before its P.V products.  The first P.V of a tile in a unit
-    overwrites its O accumulator; it needs no barrier of its own, since it waits for that
-    tile's first P of the unit, which its warpgroup writes only after its epilogue has read
-    O of the previous unit.  Planted mistakes: wait_q_free=False (Q loaded without
-    waiting) and q_free_at="first_step" (Q released at the unit's first step, before the
-    S products of the later steps)."""
+    units, and so does the issuer's step loop: the record carried with V of a unit's last
+    step is the next unit's first record (flagged as a new unit), at which the issuer
+    waits for the next phase of the Q barrier.  The producer loads a unit's Q tiles once
+    the S products of the previous unit have completed (Q free), which the issuer commits
+    at the unit's last step, after reading the chained record and before that step's P.V
+    products.  The first P.V of a tile in a unit overwrites its O accumulator; it needs
+    no barrier of its own, since it waits for that tile's first P of the unit, which its
+    warpgroup writes only after its epilogue has read O of the previous unit.  Planted
+    mistakes: wait_q_free=False (Q loaded without waiting) and q_free_at="first_step" (Q
+    released at the unit's first step, before the S products of the later steps)."""
     m = _Model()
     bar_q, q_free = m.bar("q"), m.bar("q_free")
     full = [m.bar(f"full{s}") for s in range(NS)]
@@ -261,12 +263,18 @@ def fwd_persistent_roles(units, NS, wait_q_free=True, q_free_at="last_step"):
                 r[k] = "last" if nxt is None else ("pre" if nxt == jn else "later")
         return r
 
+    def after(ui, t):  # the record carried with V of step t of unit ui
+        if t + 1 < len(steps_of[ui]):
+            return ("rec", ui, t + 1)
+        return ("rec", ui + 1, 0) if ui + 1 < len(work) else ("end",)
+
     def producer():
         r = 0
         for ui in range(len(work)):
-            if ui > 0 and wait_q_free:
+            if ui == 0:
+                yield ("write", {("rec", NS): ("rec", 0, 0)})  # later units' come chained
+            elif wait_q_free:
                 yield ("wait", q_free, (ui - 1) & 1)
-            yield ("write", {("rec", NS): ("rec", ui, 0)})
             yield ("expect", bar_q, TB)
             yield ("tma", ("Q",), ("Q", ui), bar_q, TB)
             for t, j in enumerate(steps_of[ui]):
@@ -274,7 +282,7 @@ def fwd_persistent_roles(units, NS, wait_q_free=True, q_free_at="last_step"):
                     s = r % NS
                     yield ("wait", empty[s], ((r // NS) & 1) ^ 1)
                     if which == "V":
-                        yield ("write", {("rec", s): ("rec", ui, t + 1)})
+                        yield ("write", {("rec", s): after(ui, t)})
                     yield ("expect", full[s], TB)
                     yield ("tma", ("slot", s), (which, ui, j), full[s], TB)
                     r += 1
@@ -295,8 +303,9 @@ def fwd_persistent_roles(units, NS, wait_q_free=True, q_free_at="last_step"):
         r = 0
         np_, n_o = [0, 0], [0, 0]
         for ui in range(len(work)):
-            yield ("wait", bar_q, ui & 1)
-            yield ("read", [(("rec", NS), ("rec", ui, 0))])
+            yield ("wait", bar_q, ui & 1)  # unit 0: before the loop; later: at the chained record
+            if ui == 0:
+                yield ("read", [(("rec", NS), ("rec", 0, 0))])
             s_ready, started = [False, False], [False, False]
             fin = [not work[ui][0], not work[ui][1]]  # tile k has no key tile left
             released = False
@@ -313,12 +322,17 @@ def fwd_persistent_roles(units, NS, wait_q_free=True, q_free_at="last_step"):
                             yield S(ui, k, j, sK)
                             yield ("commit", bar_s[k])
                 yield ("commit", empty[sK])
-                last_step = all(rc[k] == "last" if k in rc else fin[k] for k in range(2))
-                if not released and (last_step if q_free_at == "last_step" else t == 0):
+                if q_free_at == "first_step" and t == 0 and not released:
                     yield ("commit", q_free)
                     released = True
                 yield ("wait", full[sV], (rV // NS) & 1)
-                yield ("read", [(("rec", sV), ("rec", ui, t + 1))])
+                yield ("read", [(("rec", sV), after(ui, t))])
+                # the chained record says this is the unit's last step
+                last_step = t + 1 == len(steps_of[ui])
+                assert last_step == all(rc[k] == "last" if k in rc else fin[k] for k in range(2))
+                if last_step and not released:
+                    yield ("commit", q_free)
+                    released = True
                 next_k_ready = False
                 for k in range(2):
                     if k not in rc:
