@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # they were measured on (a changed kernel reports null until it is captured again)
 MEASURED_TRAFFIC = {
     # flex_fwd_kernel<128,bf16,none,none> (one CTA per unit), B2 H32 S8192 D128:
-    # 402,723,328 B read + 114,665,984 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192.md)
-    "c9bf501cb9bd5bcb": 517389312,
+    # 402,722,816 B read + 114,174,720 B written (profiles/flex_fwd_kernel_bf16_nomod_S8192.md)
+    "35374352ecfe85fe": 516897536,
 }
 MEASURED_DECODE_TRAFFIC = {
     # decode_split_kernel<128,f16,1,128>, B16 H32 Hkv32 cap8192, the bench's lengths and
@@ -487,10 +487,39 @@ def per_case(fa, q, k, v, scale, o, lse, args):
         out[name]["tflops_dense_equiv"] = dense / t / 1e12
         if name.startswith("sliding"):
             out[name]["tflops_useful"] = useful_window / t / 1e12
+    out.update(mha2048_cases(fa))
     out.update(block_cases(fa, q, k, v, scale, o, lse))
     out.update(captured_cases(fa, q, k, v, scale, o, lse))
     out.update(bwd_cases(fa, q, k, v, scale))
     out.update(fp8_cases(fa, q, k, v, scale))
+    return out
+
+
+def mha2048_cases(fa):
+    """The MHA configuration at S=2048 (B2 H32 D128 bf16, N(0, 1) inputs, scale 1/sqrt(128)):
+    no_mod, alibi, sliding window 256 (causal), causal via mask_mod, causal=True.  These
+    inputs (96 MiB) fit in L2, so iterations run L2-warm; the kernel is tensor-bound."""
+    import torch
+    import synth
+    dev = torch.device("cuda")
+    B, H, S, D = 2, 32, 2048, 128
+    q, k, v = synth.qkv(B, H, H, S, S, D, seed=synth.case_seed(1, 0), device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    dense = fwd_flops(B, H, S, S, D)
+    W = 256
+    useful_window = 4.0 * D * B * H * (W * (W + 1) // 2 + (S - W) * W)
+    cases = {"s2048_no_mod": dict(), "s2048_alibi": dict(score_mod="alibi"),
+             "s2048_sliding_window_256": dict(mask_mod="sliding_window", window=W),
+             "s2048_causal_via_mask": dict(mask_mod="causal"), "s2048_causal_fast": dict(mask_mod="causal_fast")}
+    out = {}
+    for name, mods in cases.items():
+        st = _time_stats(lambda: fa.fwd(q, k, v, out=o, lse_out=lse, **mods))
+        if "sliding" in name:
+            out[name] = _case_row(st, useful_window, "tflops_useful")
+        else:
+            out[name] = _case_row(st, dense * (0.5 if "causal" in name else 1.0))
+        out[name]["l2"] = "warm"
     return out
 
 
