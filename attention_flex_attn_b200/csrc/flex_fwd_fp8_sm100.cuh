@@ -51,6 +51,7 @@ struct Fp8Params {
   unsigned* status;
   int H, Hkv, G, Sq, Skv, Skv_pad, D;
   int n_qtiles, n_ktiles, n_pairs;
+  int bh_total, head_group;  // B * H; units run in groups of head_group heads (unit_coords_of)
   float scale_log2;   // scale * descale_q * descale_k * log2(e)
   float descale_v;
   const float* slopes;
@@ -163,8 +164,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   auto p_smem = [&](int k) { return sbase + static_cast<uint32_t>(L::kPOff + k * L::kTileBytes); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / p.n_pairs;
-  const int pair = p.n_pairs - 1 - (blockIdx.x % p.n_pairs);
+  int bh, pair;
+  unit_coords_of(static_cast<int>(blockIdx.x), p.n_pairs, p.head_group, p.bh_total, bh, pair);
   const int h = bh % p.H, b = bh / p.H;
   const int bkv = b * p.Hkv + h / p.G;
   int q0[2], q1[2], lo[2], hi[2];

@@ -111,6 +111,9 @@ constexpr uint32_t kRecLast1 = 1u << 5;
 constexpr uint32_t kRecEnd = 1u << 6;    // no step: the walk is over
 constexpr uint32_t kRecNewItem = 1u << 7;  // persistent kernel: the first step of the next item
 
+struct FwdParams;
+__device__ __forceinline__ void unit_coords(const FwdParams& p, int unit, int& bh, int& pair);
+
 struct FwdParams {
   void* o;
   float* lse;
@@ -119,6 +122,8 @@ struct FwdParams {
   int H, Hkv, G, Sq, Skv;
   int n_qtiles, n_ktiles, n_pairs;
   int n_units;         // B * H * n_pairs (the persistent kernel loops over them)
+  int bh_total;        // B * H
+  int head_group;      // units run in groups of head_group heads (unit_coords)
   int persist_grid;    // CTAs of the persistent kernel (0: one CTA per unit)
   // Persistent kernel: items [0, n_full) are whole units; items [n_full, n_items) split
   // the last n_units - n_full units' key ranges into n_parts parts each.  The parts of a
@@ -141,6 +146,25 @@ struct FwdParams {
   int blk_max;
   int blk_b_stride, blk_h_stride;
 };
+
+// unit -> (b * H + h, pair of query tiles).  Heads run in groups of head_group; within a
+// group the pairs run from the last to the first (under causal masks the heaviest first),
+// each pair over all the group's heads, so that the block scheduler's last wave holds the
+// lightest units while the group's K/V stay in L2.  head_group = 1: head by head.
+__device__ __forceinline__ void unit_coords_of(int unit, int n_pairs, int head_group, int bh_total, int& bh,
+                                               int& pair) {
+  const int per_group = head_group * n_pairs;
+  const int gi = unit / per_group;
+  const int base = gi * head_group;
+  const int gh = min(head_group, bh_total - base);  // heads in this group
+  const int r = unit - gi * per_group;
+  pair = n_pairs - 1 - r / gh;
+  bh = base + r % gh;
+}
+__device__ __forceinline__ void unit_coords(const FwdParams& p, int unit, int& bh, int& pair) {
+  unit_coords_of(unit, p.n_pairs, p.head_group, p.bh_total, bh, pair);
+}
+
 
 // Block-mask / document bitmaps: full0, full1, act0, act1, and with both a block mask
 // and a document mask the document sets doc0, doc1 (kBlkWords words each).
@@ -411,10 +435,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   int q0[2], q1[2], lo[2], hi[2];
   auto sel = [](const int (&a)[2], int k) { return k ? a[1] : a[0]; };
   MaskArgs mk = p.mask;
-  // unit -> (b, h, pair of query tiles), heavier (later) pairs first within a head
+  // unit -> (b, h, pair of query tiles), later (heavier) pairs first (unit_coords)
   auto set_unit = [&](int unit) {
-    bh = unit / p.n_pairs;
-    pair = p.n_pairs - 1 - (unit % p.n_pairs);
+    unit_coords(p, unit, bh, pair);
     h = bh % p.H;
     b = bh / p.H;
     bkv = b * p.Hkv + h / p.G;
@@ -1104,8 +1127,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // tiles (in the persistent loop it cannot rebuild them from blockIdx).
         int opart;
         const int ou = item_unit(opaque_int(item), opart);
-        const int obh = ou / p.n_pairs;
-        const int oqi = (2 * (p.n_pairs - 1 - ou % p.n_pairs) + k) * kBM + row;
+        int obh, opair;
+        unit_coords(p, ou, obh, opair);
+        const int oqi = (2 * opair + k) * kBM + row;
         const bool row_ok = oqi < p.Sq;
         // A row has mass iff it ever saw a kept (finite) score.  The polynomial 2^x returns
         // ~2^-125 rather than 0 for masked scores, so l_sum alone cannot tell.
