@@ -702,6 +702,17 @@ flex_status_t bwd_common(const void* q, const void* k, const void* v, const void
   p.D = D;
   p.n_qtiles = n_qtiles;
   p.n_ktiles = n_ktiles;
+  p.q_group = 0;
+  p.kv_group = 1;
+  if (!bm && (mask == kMaskCausal || mask == kMaskOffset)) {
+    // heaviest tiles first over groups of heads whose shared operands stay in L2: the dQ
+    // kernel reads K/V of its kv head, the dK/dV kernel Q and dO of the kv head's G heads
+    // (measured on B200, causal B2 H32 S8192: see the design notes)
+    p.q_group = head_group_for(mask, static_cast<int64_t>(B) * H, H / Hkv, Skv, D, 2);
+    const int64_t qdo_bytes = static_cast<int64_t>(H / Hkv) * Sq * D * 2 * 2;
+    p.kv_group = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(B) * Hkv,
+                                                    std::max<int64_t>(1, (int64_t{32} << 20) / qdo_bytes)));
+  }
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.slopes = score_mod_id == FLEX_SCORE_ALIBI_SLOPES ? mp.alibi_slopes : nullptr;

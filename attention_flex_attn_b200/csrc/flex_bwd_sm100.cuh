@@ -62,6 +62,12 @@ struct BwdParams {
   unsigned* status;
   int B, H, Hkv, G, Sq, Skv, D, Sq_pad;
   int n_qtiles, n_ktiles;
+  // CTA order (unit_coords_of): the dQ kernel runs head by head with its query tiles in
+  // order (q_group 0), or under causal-like masks the last (heaviest) query tiles first
+  // over groups of q_group query heads; the dK/dV kernel runs its key tiles in order over
+  // groups of kv_group kv heads (1: head by head; under causal masks the first key tiles
+  // see the most queries)
+  int q_group, kv_group;
   float scale;
   float scale_log2;       // scale * log2(e)
   const float* slopes;    // alibi slope tensor [H] or nullptr
@@ -297,8 +303,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto v_smem = [&](int s) { return sbase + static_cast<uint32_t>(L::kKVOff + (KS + s) * L::kTileBytes); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % p.n_qtiles;
-  const int bh = blockIdx.x / p.n_qtiles;
+  int qt, bh;
+  if (p.q_group > 0) {
+    unit_coords_of(static_cast<int>(blockIdx.x), p.n_qtiles, p.q_group, p.B * p.H, bh, qt);
+  } else {
+    qt = blockIdx.x % p.n_qtiles;
+    bh = blockIdx.x / p.n_qtiles;
+  }
   const int h = bh % p.H, b = bh / p.H;
   const int bkv = b * p.Hkv + h / p.G;
   const int q0 = qt * kBM, q1 = min(q0 + kBM, p.Sq);
@@ -657,8 +668,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto stat_slot = [&](int s) { return slot_base(s) + 2 * L::kTileBytes; };  // byte offset from sbase
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x % p.n_ktiles;
-  const int bkv = blockIdx.x / p.n_ktiles;
+  int kt, bkv;
+  unit_coords_of(static_cast<int>(blockIdx.x), p.n_ktiles, p.kv_group, p.B * p.Hkv, bkv, kt);
+  kt = p.n_ktiles - 1 - kt;  // ascending: under causal masks the first key tiles see the most queries
   const int hk = bkv % p.Hkv, b = bkv / p.Hkv;
   const int k0 = kt * kBN;
   MaskArgs mk = p.mask;
