@@ -27,6 +27,8 @@ namespace {
 
 // Largest key-tile count per query tile that runs on the persistent forward kernel.
 constexpr int64_t kPersistMaxKeyTiles = 32;
+// Largest K + V footprint (bytes) with which causal-like masks run persistent.
+constexpr int64_t kPersistRisingMaxKvBytes = int64_t{80} << 20;
 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -439,15 +441,24 @@ flex_status_t fwd_common(const void* q, const void* k, const void* v, void* o, f
   // unit, which the block scheduler places in waves.  (Measured on B200, 128-row tiles,
   // persistent against per-unit: 3-4 key tiles +15 %, 8 +9 %, 10 +2 %, 16 +4 to +8 %,
   // 32 at D = 64 +7 %, 32 at D = 128 -1 %, 48 and 64 -2 to -5 %, 128 equal.)
-  if (!bm && (mask == kMaskNone || mask == kMaskSliding)) {
+  const bool uniform = mask == kMaskNone || mask == kMaskSliding;
+  const bool rising = mask == kMaskCausal || mask == kMaskOffset;
+  if (!bm && (uniform || rising)) {
     int64_t span = p.n_ktiles;
     if (mask == kMaskSliding)
       span = std::min<int64_t>(span, (static_cast<int64_t>(mp.window) + kBM - 1 + kBN - 1) / kBN + 1);
     const int sms = sm_count();
     if (sms < 1) return FLEX_ERR_CUDA;
     const int64_t grid = n_units < sms ? n_units : sms;
-    if (span <= kPersistMaxKeyTiles) p.persist_grid = static_cast<int>(grid);
-    {
+    // Causal-like units run persistent only while every head's K and V fit in L2 at once:
+    // then all units form one list, heaviest first, which the kernel's snake order over
+    // the CTAs spreads evenly.
+    const int64_t kv_bytes = static_cast<int64_t>(B) * Hkv * Skv * D * 2 * 2;
+    if (span <= kPersistMaxKeyTiles && (uniform || kv_bytes <= kPersistRisingMaxKvBytes)) {
+      p.persist_grid = static_cast<int>(grid);
+      if (rising) p.head_group = static_cast<int>(bh);
+    }
+    if (uniform) {
       // The last round: R = n_units mod grid units would leave grid - R SMs idle.  With
       // R <= grid / 2 their key ranges split into parts (at most 4, at most one per key
       // tile) that fill the round; the last part of each to finish merges them.  (B2 H32

@@ -13,15 +13,14 @@
 namespace flexattn {
 namespace {
 
-// Masks whose work units carry uniform work (no mask, sliding window) can run on the
-// persistent kernel: one CTA per SM looping over the units, the K/V stream running on from
-// one unit to the next.  The host picks it (FwdParams::persist_grid > 0) when the units are
-// short; causal-like units grow with the query position, which the hardware block
-// scheduler balances better than a static assignment, and block and document masks keep
-// per-unit bitmaps.
+// The analytic masks without documents can run on the persistent kernel: one CTA per SM
+// walking its units back to back, the K/V stream running on from one unit to the next.
+// The host picks it (FwdParams::persist_grid > 0) when the units are short, and for
+// causal-like masks only while all K/V fit in L2 (their units, sorted heaviest first,
+// spread over the CTAs in snake order).  Block and document masks keep per-unit bitmaps.
 template <int MASK, bool BLOCKS>
 constexpr bool fwd_persistable() {
-  return !BLOCKS && (MASK == kMaskNone || MASK == kMaskSliding);
+  return !BLOCKS && (MASK == kMaskNone || MASK == kMaskSliding || MASK == kMaskCausal || MASK == kMaskOffset);
 }
 
 // Per-device "attribute already set" bits, one set per kernel instantiation (the tag
@@ -104,22 +103,38 @@ flex_status_t launch_fwd_persistent(const CUtensorMap& mq, const CUtensorMap& mk
 }
 
 // every (dtype, score_mod, mask) of head dim D that fwd_dispatch may send to the persistent kernel
-#define FLEX_FWD_PERSISTENT_INSTANCES(D)                                                                       \
-  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskNone>(                              \
-      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
-  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskSliding>(                           \
-      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
-  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskNone>(                             \
-      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
-  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskSliding>(                          \
-      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
-  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskNone>(                       \
-      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
-  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskSliding>(                    \
-      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
-  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskNone>(                      \
-      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);             \
-  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskSliding>(                   \
+#define FLEX_FWD_PERSISTENT_INSTANCES(D) \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskNone>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskSliding>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskCausal>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreNone, kMaskOffset>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskNone>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskSliding>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskCausal>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __half, kScoreAlibi, kMaskOffset>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskNone>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskSliding>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskCausal>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreNone, kMaskOffset>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskNone>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskSliding>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskCausal>( \
+      const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t); \
+  template flex_status_t launch_fwd_persistent<D, __nv_bfloat16, kScoreAlibi, kMaskOffset>( \
       const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, const FwdParams&, cudaStream_t);
 #endif
 

@@ -480,9 +480,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mk.off_q += static_cast<int64_t>(b) * (mk.n_docs + 1);
     mk.off_kv += static_cast<int64_t>(b) * (mk.n_docs + 1);
   }
-  // the items of this CTA: blockIdx.x (+ gridDim.x ...) up to item_end
+  // The items of this CTA: one per round of gridDim.x items, in snake order (odd rounds
+  // reversed), so that an item list sorted heaviest first spreads evenly over the CTAs;
+  // items from item_end on do not exist.  The per-unit kernel has one round: blockIdx.x.
   const int item_end = PERSIST ? p.n_items : static_cast<int>(blockIdx.x) + 1;
   const int item_step = PERSIST ? static_cast<int>(gridDim.x) : 1;
+  const int n_rounds = PERSIST ? (p.n_items + item_step - 1) / item_step : 1;
+  auto round_item = [&](int rr) {
+    const int c = (PERSIST && (rr & 1)) ? item_step - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x);
+    return rr * item_step + c;
+  };
 
   // ---------------------------------------------------------------- visit bitmaps
   // With a block mask or a document mask the key tiles a query tile visits are a set, not
@@ -596,14 +603,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // The items with work form one walk: at an item's last step the record carried
         // with V is the next item's first one, flagged kRecNewItem; that item's Q loads
         // once the issuer has released the previous Q (q_free).
-        auto next_work = [&](int it) {  // first item from `it` on with work (set_item state)
-          for (; it < item_end; it += item_step) {
+        int rr = -1;  // round of the current item
+        auto next_work = [&]() {  // the next round's item with work (set_item state), or item_end
+          while (++rr < n_rounds) {
+            const int it = round_item(rr);
+            if (it >= item_end) continue;
             set_item(it);
-            if (cursor(0).cur >= 0 || cursor(1).cur >= 0) break;
+            if (cursor(0).cur >= 0 || cursor(1).cur >= 0) return it;
           }
-          return it;
+          return item_end;
         };
-        int item = next_work(static_cast<int>(blockIdx.x));
+        int item = next_work();
         if (item < item_end) {
           auto c0 = cursor(0), c1 = cursor(1);
           rec_smem[NS] = make_rec(c0, c1);  // published with the Q barrier
@@ -617,7 +627,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (c1.cur == j) c1.advance();
               uint32_t next_rec = make_rec(c0, c1);
               if (next_rec == kRecEnd) {  // the item's last step: chain the next item
-                nxt = next_work(item + item_step);
+                nxt = next_work();
                 if (nxt < item_end) next_rec = make_rec(cursor(0), cursor(1)) | kRecNewItem;
               }
               for (int which = 0; which < 2 && ok; ++which, ++r) {
@@ -759,12 +769,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool run = any_work;
       if constexpr (PERSIST) {
         if (!any_work) {  // the CTA's first item with work is a later one: bar_q's first phase
-          int it = blockIdx.x + item_step;
-          for (; it < item_end; it += item_step) {
+          run = false;
+          for (int rr = 1; rr < n_rounds && !run; ++rr) {
+            const int it = round_item(rr);
+            if (it >= item_end) continue;
             set_item(it);
-            if (cursor(0).cur >= 0 || cursor(1).cur >= 0) break;
+            run = cursor(0).cur >= 0 || cursor(1).cur >= 0;
           }
-          run = it < item_end;
           if (run) {
             ok = mbar_wait(bar_q, 0, p.status, kStatusFwdTimeout, kWaitTimeoutNs);
             tc_fence_after();
@@ -948,7 +959,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bool ok = true;
     int n = 0;      // S tiles of this warpgroup so far (the S barrier's phase)
     int o_par = 0;  // O completions waited for (the O barrier's phase)
-    for (int item = blockIdx.x; item < item_end && ok; item += item_step) {
+    for (int rr = 0; rr < n_rounds && ok; ++rr) {
+      const int item = round_item(rr);
+      if (item >= item_end) continue;
       if (PERSIST) set_item(item);
       const int q0k = sel(q0, k), q1k = sel(q1, k);
       const int qi = q0k + row;         // absolute query index
