@@ -27,7 +27,8 @@ MASK_MODS = {"none": 0, "causal": 1, "sliding_window": 2, "kv_le_q_plus_offset":
 FLAG_TILE_MAP = 1
 
 # The symbols include/flex_attn.h declares.
-EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_fwd_fp8_workspace_size", "flex_attn_fwd_fp8",
+EXPORTED = ["flex_attn_fwd", "flex_attn_fwd_block_sparse", "flex_attn_fwd_host_workspace_size", "flex_attn_fwd_host",
+            "flex_attn_fwd_fp8_workspace_size", "flex_attn_fwd_fp8",
             "flex_attn_fwd_fp8_block_sparse",
             "flex_attn_bwd_workspace_size", "flex_attn_bwd",
             "flex_attn_bwd_block_sparse_workspace_size", "flex_attn_bwd_block_sparse",
@@ -78,6 +79,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.flex_attn_fwd_block_sparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams),
                                                ctypes.POINTER(BlockMaskC), I, P]
     lib.flex_attn_fwd_block_sparse.restype = I
+    lib.flex_attn_fwd_host_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.flex_attn_fwd_host_workspace_size.restype = SZ
+    lib.flex_attn_fwd_host.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, ctypes.POINTER(ModParams), I, P,
+                                       SZ, P]
+    lib.flex_attn_fwd_host.restype = I
     lib.flex_attn_fwd_fp8_workspace_size.argtypes = [I, I, I, I]
     lib.flex_attn_fwd_fp8_workspace_size.restype = SZ
     lib.flex_attn_fwd_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, F, F, F, I, I, ctypes.POINTER(ModParams),
@@ -367,6 +373,53 @@ def _fp8(bm, q8, k8, v8, descale_q, descale_k, descale_v, scale, score_mod, mask
         _check(lib.flex_attn_fwd_fp8(*args, *tail), "flex_attn_fwd_fp8")
     else:
         _check(lib.flex_attn_fwd_fp8_block_sparse(*args, ctypes.byref(bm), *tail), "flex_attn_fwd_fp8_block_sparse")
+    return o, lse
+
+
+def fwd_host_workspace_size(B, H, Hkv, Sq, Skv, D) -> int:
+    return int(load_library().flex_attn_fwd_host_workspace_size(B, H, Hkv, Sq, Skv, D))
+
+
+def fwd_host(q, k, v, scale=None, score_mod="none", mask_mod="none", window=0, offset=0, return_lse=True,
+             out=None, lse_out=None, alibi_slopes=None, doc_offsets=None, doc_offsets_kv=None, status=None,
+             workspace=None, device=None):
+    """The forward on HOST tensors (flex_attn_fwd_host): q [B,H,Sq,D], k/v [B,Hkv,Skv,D] CPU
+    tensors (pinned memory lets the copies overlap the kernels), results in host tensors
+    (``out`` / ``lse_out``, allocated pinned when not given).  The library copies chunks of
+    kv heads to ``device`` (default: the current CUDA device) and back while it computes
+    the previous ones.  Captured tensors and ``status`` are CUDA tensors as in fwd;
+    ``workspace``: optional device buffer of fwd_host_workspace_size bytes.  Returns
+    (O, LSE) once the results are in host memory (the call synchronises its stream)."""
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or not t.is_contiguous():
+            raise FlexAttnError(f"{n} must be a contiguous CPU tensor")
+    B, H, Hkv, Sq, Skv, D = _check_fwd_shapes(q, k, v, out, lse_out if return_lse else None)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = out if out is not None else torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    lse = None
+    if return_lse:
+        lse = lse_out if lse_out is not None else torch.empty((B, H, Sq), dtype=torch.float32).pin_memory()
+    for t, n in ((o, "out"), (lse, "lse_out")):
+        if t is not None and not t.is_contiguous():
+            raise FlexAttnError(f"{n} must be contiguous")
+    need = fwd_host_workspace_size(B, H, Hkv, Sq, Skv, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    elif (not workspace.is_cuda or workspace.device != dev or not workspace.is_contiguous()
+          or workspace.numel() * workspace.element_size() < need):
+        raise FlexAttnError(f"workspace must be a contiguous CUDA tensor of at least {need} bytes on {dev}")
+    mp, score = _mod_params(B, H, score_mod, mask_mod, window, offset, None, alibi_slopes, doc_offsets,
+                            doc_offsets_kv, _status_word(status, dev))
+    with torch.cuda.device(dev):
+        stream = _stream(dev)
+        rc = lib.flex_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Skv, D,
+                                    float(scale), score, MASK_MODS[mask_mod], ctypes.byref(mp), DTYPES[q.dtype],
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), stream)
+        _check(rc, "flex_attn_fwd_host")
+        torch.cuda.current_stream(dev).synchronize()
     return o, lse
 
 

@@ -526,6 +526,185 @@ flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const voi
                     block_mask, dtype, stream);
 }
 
+}  // extern "C"
+
+namespace flexattn {
+namespace {
+
+// ---------------------------------------------------------------- forward from host buffers
+
+// The built-in alibi slopes of the query heads, computed as the kernels compute them (so a
+// chunk that starts at head h0 reads slopes[h0 ..] and gets the same bits).
+__global__ void alibi_slope_table_kernel(float* out, int H) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h < H) out[h] = exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(H));
+}
+
+// flex_attn_fwd_host splits the work into chunks of hc kv heads (and their G query heads)
+// of one batch, about kHostChunks in all, and keeps kHostBuffers chunks on the device.
+constexpr int kHostChunks = 16;
+constexpr int kHostBuffers = 3;
+
+struct HostPlan {
+  int per_batch, hc, n, nb;
+  size_t q_bytes, kv_bytes, lse_bytes, buf_bytes, slope_off, total;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+HostPlan host_plan(int B, int H, int Hkv, int Sq, int Skv, int D) {
+  HostPlan pl{};
+  const int G = H / Hkv;
+  const int want = std::max(1, std::min(Hkv, (kHostChunks + B - 1) / B));
+  pl.hc = (Hkv + want - 1) / want;
+  pl.per_batch = (Hkv + pl.hc - 1) / pl.hc;
+  pl.n = B * pl.per_batch;
+  pl.nb = std::min(kHostBuffers, pl.n);
+  pl.q_bytes = align256(static_cast<size_t>(pl.hc) * G * Sq * D * 2);
+  pl.kv_bytes = align256(static_cast<size_t>(pl.hc) * Skv * D * 2);
+  pl.lse_bytes = align256(static_cast<size_t>(pl.hc) * G * Sq * sizeof(float));
+  pl.buf_bytes = 2 * pl.q_bytes + 2 * pl.kv_bytes + pl.lse_bytes;  // Q, K, V, O, LSE
+  pl.slope_off = static_cast<size_t>(pl.nb) * pl.buf_bytes;
+  pl.total = pl.slope_off + align256(static_cast<size_t>(H) * sizeof(float));
+  return pl;
+}
+
+// The copy streams and events of the host pipeline, one set per context, created on first
+// use and kept for the process's life.  A call holds the set's mutex while it enqueues, so
+// every wait on an event is enqueued after that call's record of it.
+struct HostPipe {
+  unsigned long long ctx;
+  cudaStream_t in, out;
+  cudaEvent_t start, end, ev_in[kHostBuffers], ev_comp[kHostBuffers], ev_out[kHostBuffers];
+  std::mutex mu;
+};
+
+HostPipe* host_pipe() {
+  static std::vector<HostPipe*> pipes;
+  static std::mutex mu;
+  unsigned long long id = 0;
+  if (!current_context_id(&id)) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  for (HostPipe* hp : pipes)
+    if (hp->ctx == id) return hp;
+  HostPipe* hp = new HostPipe();
+  hp->ctx = id;
+  bool ok = cudaStreamCreateWithFlags(&hp->in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&hp->out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp->start, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp->end, cudaEventDisableTiming) == cudaSuccess;
+  for (int i = 0; ok && i < kHostBuffers; ++i)
+    ok = cudaEventCreateWithFlags(&hp->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&hp->ev_comp[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&hp->ev_out[i], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    return nullptr;  // (the partly created set is leaked: this only happens when CUDA fails)
+  }
+  pipes.push_back(hp);
+  return hp;
+}
+
+}  // namespace
+}  // namespace flexattn
+
+extern "C" {
+
+size_t flex_attn_fwd_host_workspace_size(int B, int H, int Hkv, int Sq, int Skv, int D) {
+  if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0 || (D != 64 && D != 128)) return 0;
+  return flexattn::host_plan(B, H, Hkv, Sq, Skv, D).total;
+}
+
+flex_status_t flex_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                 int Hkv, int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
+                                 const flex_mod_params_t* mod_params, flex_dtype_t dtype, void* workspace,
+                                 size_t workspace_bytes, flex_stream_t stream) {
+  using namespace flexattn;
+  if (!q || !k || !v || !o) return FLEX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || H % Hkv != 0) return FLEX_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FLEX_ERR_UNSUPPORTED;
+  if (dtype != FLEX_DTYPE_BF16 && dtype != FLEX_DTYPE_F16) return FLEX_ERR_UNSUPPORTED;
+  if (score_mod_id != FLEX_SCORE_NONE && score_mod_id != FLEX_SCORE_ALIBI && score_mod_id != FLEX_SCORE_ALIBI_SLOPES)
+    return FLEX_ERR_INVALID_ARG;
+  const flex_mod_params_t zero{};
+  const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
+  if (mp.flags & FLEX_FLAG_TILE_MAP) return FLEX_ERR_INVALID_ARG;  // the debug map covers whole calls only
+  const int mask = mask_kind(mask_mod_id);
+  if (mask < 0) return FLEX_ERR_INVALID_ARG;
+  if (const flex_status_t ds = check_documents(mask, mp); ds != FLEX_OK) return ds;
+  const HostPlan pl = host_plan(B, H, Hkv, Sq, Skv, D);
+  if (!workspace || workspace_bytes < pl.total) return FLEX_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FLEX_ERR_MISALIGNED;
+  HostPipe* hp = host_pipe();
+  if (!hp) return FLEX_ERR_CUDA;
+  const int G = H / Hkv;
+  const size_t es = 2;  // bytes per element
+  char* ws = static_cast<char*>(workspace);
+  float* slopes = reinterpret_cast<float*>(ws + pl.slope_off);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(hp->mu);
+  flex_status_t rc = FLEX_OK;
+  auto cuda_ok = [&rc](cudaError_t e) {
+    if (e != cudaSuccess && rc == FLEX_OK) rc = FLEX_ERR_CUDA;
+    return e == cudaSuccess;
+  };
+  // the copy streams start after the work already on the caller's stream
+  cuda_ok(cudaEventRecord(hp->start, cs));
+  cuda_ok(cudaStreamWaitEvent(hp->in, hp->start, 0));
+  cuda_ok(cudaStreamWaitEvent(hp->out, hp->start, 0));
+  const float* table = mp.alibi_slopes;
+  if (score_mod_id == FLEX_SCORE_ALIBI) {
+    alibi_slope_table_kernel<<<(H + 127) / 128, 128, 0, cs>>>(slopes, H);
+    cuda_ok(cudaGetLastError());
+    table = slopes;
+  }
+  for (int c = 0; c < pl.n && rc == FLEX_OK; ++c) {
+    const int b = c / pl.per_batch, hk0 = (c % pl.per_batch) * pl.hc;
+    const int nk = std::min(Hkv, hk0 + pl.hc) - hk0, nh = nk * G, h0 = hk0 * G;
+    const int buf = c % pl.nb;
+    char* base = ws + static_cast<size_t>(buf) * pl.buf_bytes;
+    char* dq = base;
+    char* dk = dq + pl.q_bytes;
+    char* dv = dk + pl.kv_bytes;
+    char* dout = dv + pl.kv_bytes;
+    float* dlse = reinterpret_cast<float*>(dout + pl.q_bytes);
+    const size_t q_off = (static_cast<size_t>(b) * H + h0) * Sq * D * es, q_len = static_cast<size_t>(nh) * Sq * D * es;
+    const size_t kv_off = (static_cast<size_t>(b) * Hkv + hk0) * Skv * D * es,
+                 kv_len = static_cast<size_t>(nk) * Skv * D * es;
+    const size_t l_off = (static_cast<size_t>(b) * H + h0) * Sq, l_len = static_cast<size_t>(nh) * Sq * sizeof(float);
+    // in: this buffer's inputs were read by the forward of chunk c - nb
+    if (c >= pl.nb) cuda_ok(cudaStreamWaitEvent(hp->in, hp->ev_comp[buf], 0));
+    cuda_ok(cudaMemcpyAsync(dq, static_cast<const char*>(q) + q_off, q_len, cudaMemcpyHostToDevice, hp->in));
+    cuda_ok(cudaMemcpyAsync(dk, static_cast<const char*>(k) + kv_off, kv_len, cudaMemcpyHostToDevice, hp->in));
+    cuda_ok(cudaMemcpyAsync(dv, static_cast<const char*>(v) + kv_off, kv_len, cudaMemcpyHostToDevice, hp->in));
+    cuda_ok(cudaEventRecord(hp->ev_in[buf], hp->in));
+    // compute, on the caller's stream: after the inputs, and after chunk c - nb's outputs left
+    cuda_ok(cudaStreamWaitEvent(cs, hp->ev_in[buf], 0));
+    if (c >= pl.nb) cuda_ok(cudaStreamWaitEvent(cs, hp->ev_out[buf], 0));
+    if (rc != FLEX_OK) break;
+    flex_mod_params_t cp = mp;
+    if (score_mod_id != FLEX_SCORE_NONE) cp.alibi_slopes = table + h0;
+    if (cp.doc_offsets_q) cp.doc_offsets_q += static_cast<size_t>(b) * (mp.n_docs + 1);
+    if (cp.doc_offsets_kv) cp.doc_offsets_kv += static_cast<size_t>(b) * (mp.n_docs + 1);
+    rc = fwd_common(dq, dk, dv, dout, lse ? dlse : nullptr, 1, nh, nk, Sq, Skv, D, scale,
+                    score_mod_id == FLEX_SCORE_NONE ? FLEX_SCORE_NONE : FLEX_SCORE_ALIBI_SLOPES, mask_mod_id, &cp,
+                    nullptr, dtype, stream);
+    cuda_ok(cudaEventRecord(hp->ev_comp[buf], cs));
+    // out: O and LSE of this chunk
+    cuda_ok(cudaStreamWaitEvent(hp->out, hp->ev_comp[buf], 0));
+    cuda_ok(cudaMemcpyAsync(static_cast<char*>(o) + q_off, dout, q_len, cudaMemcpyDeviceToHost, hp->out));
+    if (lse) cuda_ok(cudaMemcpyAsync(lse + l_off, dlse, l_len, cudaMemcpyDeviceToHost, hp->out));
+    cuda_ok(cudaEventRecord(hp->ev_out[buf], hp->out));
+  }
+  // the caller's stream reaches its next work only after every copy (also after an error)
+  const bool joined = cudaEventRecord(hp->end, hp->out) == cudaSuccess &&
+                      cudaStreamWaitEvent(cs, hp->end, 0) == cudaSuccess &&
+                      cudaEventRecord(hp->start, hp->in) == cudaSuccess &&
+                      cudaStreamWaitEvent(cs, hp->start, 0) == cudaSuccess;
+  if (!joined && rc == FLEX_OK) rc = FLEX_ERR_CUDA;
+  return rc;
+}
+
 size_t flex_attn_fwd_fp8_workspace_size(int B, int Hkv, int Skv, int D) {
   if (B < 1 || Hkv < 1 || Skv < 1 || (D != 64 && D != 128)) return 0;
   const size_t skv_pad = (static_cast<size_t>(Skv) + 127) / 128 * 128;

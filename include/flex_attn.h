@@ -181,6 +181,40 @@ flex_status_t flex_attn_fwd_block_sparse(const void* q, const void* k, const voi
                                          flex_stream_t stream);
 
 /*
+ * flex_attn_fwd_host_workspace_size -- bytes of device workspace flex_attn_fwd_host needs:
+ * three chunk buffers (Q, K, V, O, LSE of one chunk of kv heads) and a table of H slopes;
+ * 0 for invalid sizes.
+ */
+size_t flex_attn_fwd_host_workspace_size(int B, int H, int Hkv, int Sq, int Skv, int D);
+
+/*
+ * flex_attn_fwd_host -- flex_attn_fwd on HOST buffers (the forward of FlyDSL PR 931,
+ * Summary, with the operands of torch-mlir PR 4366, Description, living in host memory):
+ * q, k, v are read from and o, lse written to host memory in the layouts of flex_attn_fwd.
+ * The work is split into chunks of kv heads of one batch (about 16 in all); chunk c's
+ * copy to the device, the forward on chunk c - 1 and the copy of chunk c - 2's O and LSE
+ * back run at the same time (copies on two streams of the library's own, the forward on
+ * `stream`), so the call takes about as long as its host-to-device copies.  The results
+ * equal flex_attn_fwd's on the same values up to the summation order of key-range parts
+ * (the split of a last round of units depends on the number of units per launch).
+ *   q, k, v, o, lse: host pointers (lse may be NULL).  Page-locked (pinned) memory lets the
+ *   copies run asynchronously and overlap; pageable memory works but serialises them.
+ *   The host buffers must stay valid and untouched until `stream` has passed this call.
+ *   score_mod_id, mask_mod_id, mod_params: as flex_attn_fwd; captured tensors
+ *   (alibi_slopes, doc_offsets_*) are DEVICE pointers as there; FLEX_FLAG_TILE_MAP is
+ *   rejected (FLEX_ERR_INVALID_ARG).
+ *   workspace: device memory, at least flex_attn_fwd_host_workspace_size(...) bytes,
+ *   16-byte aligned; in use until `stream` has passed this call.
+ * Asynchronous on `stream`: work queued on it before the call runs first, and work queued
+ * after it starts only once every copy has finished.  Calls from several host threads are
+ * serialised while they enqueue (they share the library's copy streams).
+ */
+flex_status_t flex_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                 int Hkv, int Sq, int Skv, int D, float scale, int score_mod_id, int mask_mod_id,
+                                 const flex_mod_params_t* mod_params, flex_dtype_t dtype, void* workspace,
+                                 size_t workspace_bytes, flex_stream_t stream);
+
+/*
  * flex_attn_fwd_fp8_workspace_size -- bytes of device workspace flex_attn_fwd_fp8 needs
  * (a transposed copy of V, keys padded to a multiple of 128); 0 for D other than 64, 128.
  */

@@ -190,6 +190,28 @@ def test_bwd_rejects_bad_args_on_host(lib):
     assert fa.bwd_workspace_size(2, 4, 300) == 2 * 2 * 4 * 384 * 4
 
 
+def test_fwd_host_rejects_bad_args_on_host(lib):
+    def fh(q=16, ws=64, wsb=1 << 30, D=128, H=2, Hkv=1, score=0, mask=0, mp=None):
+        return lib.flex_attn_fwd_host(P(q), P(16), P(16), P(16), None, 1, H, Hkv, 8, 8, D, 0.1, score, mask,
+                                      ctypes.byref(mp) if mp is not None else None, 0, P(ws), wsb, None)
+    assert fh(q=0) == 1
+    assert fh(H=3, Hkv=2) == 1
+    assert fh(D=96) == 2
+    assert fh(mask=9) == 1
+    assert fh(score=7) == 1
+    tile_map = fa.ModParams(0, 0, fa.FLAG_TILE_MAP, 16, None, None, None, 0, None)
+    assert fh(mp=tile_map) == 1
+    assert fh(ws=0) == 4
+    assert fh(wsb=16) == 4
+    assert fh(ws=24) == 3
+    # three chunk buffers (Q, K, V, O of hc kv heads, 256-byte aligned, and their LSE) and
+    # the slope table: B=2 H=32 Hkv=32 S=8192 D=128 -> 16 chunks of 4 kv heads
+    q_bytes = 4 * 8192 * 128 * 2
+    lse_bytes = 4 * 8192 * 4
+    assert fa.fwd_host_workspace_size(2, 32, 32, 8192, 8192, 128) == 3 * (4 * q_bytes + lse_bytes) + 256
+    assert fa.fwd_host_workspace_size(2, 3, 2, 8, 8, 128) == 0
+
+
 def test_fp8_rejects_bad_args_on_host(lib):
     def f8(q=16, ws=64, wsb=1 << 24, D=128, scale=0.1, dq=1.0, dk=1.0, dv=1.0, score=0, mask=0, mp=None):
         return lib.flex_attn_fwd_fp8(P(q), P(16), P(16), P(16), None, 1, 2, 1, 8, 8, D, scale, dq, dk, dv, score,
