@@ -159,3 +159,35 @@ def test_decode_matches_forward_single_row():
     torch.cuda.synchronize()
     assert (o1.float() - o2.float()).abs().max().item() < 2e-2
     assert (l1 - l2).abs().max().item() < 1e-2
+
+
+def test_decode_grouped_graph_replay():
+    """A CUDA graph of a grouped-query decode (the persistent kernel and the combine):
+    each replay, with new lengths written into the captured kv_len tensor, equals an
+    eager call, because the chunk list is built on the device from kv_len."""
+    fa = _fa()
+    B, H, Hkv, cap, D = 4, 16, 4, 2048, 128
+    q, kc, vc, _, mask = _inputs(B, H, Hkv, cap, D, seed=3800, lens=[1] * B, mask_p=0.1)
+    d = torch.device("cuda")
+    q, kc, vc, mask = q.to(d), kc.to(d), vc.to(d), mask.to(d)
+    kv_len = torch.full((B,), cap, dtype=torch.int32, device=d)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, 1), dtype=torch.float32, device=d)
+    ws = torch.empty(fa.decode_workspace_size(B, H, Hkv, cap, D), dtype=torch.uint8, device=d)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fa.decode(q, kc, vc, kv_len, SCALE, mask=mask, out=out, lse_out=lse, workspace=ws)  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fa.decode(q, kc, vc, kv_len, SCALE, mask=mask, out=out, lse_out=lse, workspace=ws)
+    for lens in ([cap, 1, 700, 1500], [0, 2048, 64, 65], [1000, 1000, 1000, 1000]):
+        kv_len.copy_(torch.tensor(lens, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        ref_o, ref_l = fa.decode(q, kc, vc, kv_len, SCALE, mask=mask)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref_o) and torch.equal(lse, ref_l), lens
+    assert fa.device_status() == 0
