@@ -540,13 +540,15 @@ __global__ void alibi_slope_table_kernel(float* out, int H) {
   if (h < H) out[h] = exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(H));
 }
 
-// flex_attn_fwd_host splits the work into chunks of hc kv heads (and their G query heads)
-// of one batch, about kHostChunks in all, and keeps kHostBuffers chunks on the device.
+// flex_attn_fwd_host splits the work into about kHostChunks chunks and keeps kHostBuffers of
+// them on the device: with fewer batches than that, ranges of hc kv heads (and their G
+// query heads) of one batch; otherwise runs of bc whole batches (contiguous in every
+// tensor, so a run is one forward call over bc batches).
 constexpr int kHostChunks = 16;
 constexpr int kHostBuffers = 3;
 
 struct HostPlan {
-  int per_batch, hc, n, nb;
+  int per_batch, hc, bc, n, nb;  // chunks per batch, kv heads per chunk, batches per chunk
   size_t q_bytes, kv_bytes, lse_bytes, buf_bytes, slope_off, total;
 };
 
@@ -555,14 +557,23 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 HostPlan host_plan(int B, int H, int Hkv, int Sq, int Skv, int D) {
   HostPlan pl{};
   const int G = H / Hkv;
-  const int want = std::max(1, std::min(Hkv, (kHostChunks + B - 1) / B));
-  pl.hc = (Hkv + want - 1) / want;
-  pl.per_batch = (Hkv + pl.hc - 1) / pl.hc;
-  pl.n = B * pl.per_batch;
+  if (B >= kHostChunks) {  // runs of whole batches
+    pl.bc = (B + kHostChunks - 1) / kHostChunks;
+    pl.hc = Hkv;
+    pl.per_batch = 1;
+    pl.n = (B + pl.bc - 1) / pl.bc;
+  } else {  // kv-head ranges of one batch
+    const int want = std::max(1, std::min(Hkv, (kHostChunks + B - 1) / B));
+    pl.bc = 1;
+    pl.hc = (Hkv + want - 1) / want;
+    pl.per_batch = (Hkv + pl.hc - 1) / pl.hc;
+    pl.n = B * pl.per_batch;
+  }
   pl.nb = std::min(kHostBuffers, pl.n);
-  pl.q_bytes = align256(static_cast<size_t>(pl.hc) * G * Sq * D * 2);
-  pl.kv_bytes = align256(static_cast<size_t>(pl.hc) * Skv * D * 2);
-  pl.lse_bytes = align256(static_cast<size_t>(pl.hc) * G * Sq * sizeof(float));
+  const size_t heads = static_cast<size_t>(pl.bc) * pl.hc;  // kv heads of one chunk
+  pl.q_bytes = align256(heads * G * Sq * D * 2);
+  pl.kv_bytes = align256(heads * Skv * D * 2);
+  pl.lse_bytes = align256(heads * G * Sq * sizeof(float));
   pl.buf_bytes = 2 * pl.q_bytes + 2 * pl.kv_bytes + pl.lse_bytes;  // Q, K, V, O, LSE
   pl.slope_off = static_cast<size_t>(pl.nb) * pl.buf_bytes;
   pl.total = pl.slope_off + align256(static_cast<size_t>(H) * sizeof(float));
@@ -659,7 +670,9 @@ flex_status_t flex_attn_fwd_host(const void* q, const void* k, const void* v, vo
     table = slopes;
   }
   for (int c = 0; c < pl.n && rc == FLEX_OK; ++c) {
-    const int b = c / pl.per_batch, hk0 = (c % pl.per_batch) * pl.hc;
+    // batches [b, b + nbat) and, of each, kv heads [hk0, hk0 + nk) (all of them when nbat > 1)
+    const int b = (c / pl.per_batch) * pl.bc, nbat = std::min(B, b + pl.bc) - b;
+    const int hk0 = (c % pl.per_batch) * pl.hc;
     const int nk = std::min(Hkv, hk0 + pl.hc) - hk0, nh = nk * G, h0 = hk0 * G;
     const int buf = c % pl.nb;
     char* base = ws + static_cast<size_t>(buf) * pl.buf_bytes;
@@ -668,10 +681,12 @@ flex_status_t flex_attn_fwd_host(const void* q, const void* k, const void* v, vo
     char* dv = dk + pl.kv_bytes;
     char* dout = dv + pl.kv_bytes;
     float* dlse = reinterpret_cast<float*>(dout + pl.q_bytes);
-    const size_t q_off = (static_cast<size_t>(b) * H + h0) * Sq * D * es, q_len = static_cast<size_t>(nh) * Sq * D * es;
+    const size_t q_off = (static_cast<size_t>(b) * H + h0) * Sq * D * es,
+                 q_len = static_cast<size_t>(nbat) * nh * Sq * D * es;
     const size_t kv_off = (static_cast<size_t>(b) * Hkv + hk0) * Skv * D * es,
-                 kv_len = static_cast<size_t>(nk) * Skv * D * es;
-    const size_t l_off = (static_cast<size_t>(b) * H + h0) * Sq, l_len = static_cast<size_t>(nh) * Sq * sizeof(float);
+                 kv_len = static_cast<size_t>(nbat) * nk * Skv * D * es;
+    const size_t l_off = (static_cast<size_t>(b) * H + h0) * Sq,
+                 l_len = static_cast<size_t>(nbat) * nh * Sq * sizeof(float);
     // in: this buffer's inputs were read by the forward of chunk c - nb
     if (c >= pl.nb) cuda_ok(cudaStreamWaitEvent(hp->in, hp->ev_comp[buf], 0));
     cuda_ok(cudaMemcpyAsync(dq, static_cast<const char*>(q) + q_off, q_len, cudaMemcpyHostToDevice, hp->in));
@@ -686,7 +701,7 @@ flex_status_t flex_attn_fwd_host(const void* q, const void* k, const void* v, vo
     if (score_mod_id != FLEX_SCORE_NONE) cp.alibi_slopes = table + h0;
     if (cp.doc_offsets_q) cp.doc_offsets_q += static_cast<size_t>(b) * (mp.n_docs + 1);
     if (cp.doc_offsets_kv) cp.doc_offsets_kv += static_cast<size_t>(b) * (mp.n_docs + 1);
-    rc = fwd_common(dq, dk, dv, dout, lse ? dlse : nullptr, 1, nh, nk, Sq, Skv, D, scale,
+    rc = fwd_common(dq, dk, dv, dout, lse ? dlse : nullptr, nbat, nh, nk, Sq, Skv, D, scale,
                     score_mod_id == FLEX_SCORE_NONE ? FLEX_SCORE_NONE : FLEX_SCORE_ALIBI_SLOPES, mask_mod_id, &cp,
                     nullptr, dtype, stream);
     cuda_ok(cudaEventRecord(hp->ev_comp[buf], cs));

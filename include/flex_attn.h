@@ -191,7 +191,8 @@ size_t flex_attn_fwd_host_workspace_size(int B, int H, int Hkv, int Sq, int Skv,
  * flex_attn_fwd_host -- flex_attn_fwd on HOST buffers (the forward of FlyDSL PR 931,
  * Summary, with the operands of torch-mlir PR 4366, Description, living in host memory):
  * q, k, v are read from and o, lse written to host memory in the layouts of flex_attn_fwd.
- * The work is split into chunks of kv heads of one batch (about 16 in all); chunk c's
+ * The work is split into about 16 chunks (ranges of kv heads of one batch, or, with 16 or
+ * more batches, runs of whole batches); chunk c's
  * copy to the device, the forward on chunk c - 1 and the copy of chunk c - 2's O and LSE
  * back run at the same time (copies on two streams of the library's own, the forward on
  * `stream`), so the call takes about as long as its host-to-device copies.  The results

@@ -210,6 +210,10 @@ def test_fwd_host_rejects_bad_args_on_host(lib):
     lse_bytes = 4 * 8192 * 4
     assert fa.fwd_host_workspace_size(2, 32, 32, 8192, 8192, 128) == 3 * (4 * q_bytes + lse_bytes) + 256
     assert fa.fwd_host_workspace_size(2, 3, 2, 8, 8, 128) == 0
+    # 16 or more batches: runs of whole batches, B=32 H=4 Hkv=2 S=100 D=64 -> runs of 2
+    # batches (4 kv heads, 8 query heads) per chunk
+    buf = 2 * (8 * 100 * 64 * 2) + 2 * (4 * 100 * 64 * 2) + 3328
+    assert fa.fwd_host_workspace_size(32, 4, 2, 100, 100, 64) == 3 * buf + 256
 
 
 def test_fp8_rejects_bad_args_on_host(lib):

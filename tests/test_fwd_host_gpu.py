@@ -99,3 +99,24 @@ def test_without_lse_and_into_given_buffers():
     assert (o.float() - od.cpu().float()).abs().max().item() <= 4e-3
     o2, _ = fa.fwd_host(hq, hk, hv, mask_mod="causal", return_lse=False, workspace=ws)  # workspace reused
     assert torch.equal(o2, o)
+
+
+def test_many_batches_run_in_batch_chunks():
+    """B = 40 (at least 16 batches: chunks are runs of whole batches), GQA 4/2, ragged
+    Sq = Skv = 200, D = 64 f16, causal documents with per-batch boundaries and the built-in
+    alibi: against the oracle (all rows) and the device forward."""
+    fa = _fa()
+    B, H, Hkv, S, D = 40, 4, 2, 200, 64
+    q, k, v = synth.qkv(B, H, Hkv, S, S, D, seed=123, dtype="f16")
+    rng = np.random.default_rng(124)
+    offs = np.array([[0, *sorted(rng.integers(1, S, size=2).tolist()), S] for _ in range(B)], np.int32)
+    mods = dict(mask_mod="document_causal", doc_offsets=offs, score_mod="alibi")
+    m = dict(mods, doc_offsets=torch.as_tensor(offs).cuda())
+    hq, hk, hv = _pinned(q, k, v)
+    o, lse = fa.fwd_host(hq, hk, hv, **m)
+    od, ld = fa.fwd(q.cuda(), k.cuda(), v.cuda(), **m)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    assert (o.float() - od.cpu().float()).abs().max().item() <= 4e-3
+    ro, rl = oracle.fwd(q, k, v, scale=1.0 / math.sqrt(D), **mods)
+    compare(o, lse, ro, rl, "fwd_host batch runs")
