@@ -640,9 +640,19 @@ flex_status_t flex_attn_fwd_host(const void* q, const void* k, const void* v, vo
   const flex_mod_params_t zero{};
   const flex_mod_params_t& mp = mod_params ? *mod_params : zero;
   if (mp.flags & FLEX_FLAG_TILE_MAP) return FLEX_ERR_INVALID_ARG;  // the debug map covers whole calls only
+  // the checks each chunk's forward makes again, here before any copy is queued
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FLEX_ERR_INVALID_ARG;
   const int mask = mask_kind(mask_mod_id);
   if (mask < 0) return FLEX_ERR_INVALID_ARG;
+  if (mask == kMaskSliding && mp.window < 1) return FLEX_ERR_INVALID_ARG;
+  if (score_mod_id == FLEX_SCORE_ALIBI_SLOPES) {
+    if (!mp.alibi_slopes) return FLEX_ERR_INVALID_ARG;
+    if (!aligned4(mp.alibi_slopes)) return FLEX_ERR_MISALIGNED;
+  }
   if (const flex_status_t ds = check_documents(mask, mp); ds != FLEX_OK) return ds;
+  if ((mask == kMaskDocument || mask == kMaskDocumentCausal) && (Skv + kBN - 1) / kBN > kMaxBlockKeyTiles)
+    return FLEX_ERR_UNSUPPORTED;
+  if (mp.status_out && !aligned4(mp.status_out)) return FLEX_ERR_MISALIGNED;
   const HostPlan pl = host_plan(B, H, Hkv, Sq, Skv, D);
   if (!workspace || workspace_bytes < pl.total) return FLEX_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FLEX_ERR_MISALIGNED;

@@ -204,6 +204,11 @@ def test_fwd_host_rejects_bad_args_on_host(lib):
     assert fh(ws=0) == 4
     assert fh(wsb=16) == 4
     assert fh(ws=24) == 3
+    assert lib.flex_attn_fwd_host(P(16), P(16), P(16), P(16), None, 1, 2, 1, 8, 8, 128, -1.0, 0, 0, None, 0, P(64),
+                                  1 << 30, None) == 1                       # scale <= 0
+    assert fh(score=2) == 1                                                # slope table missing
+    window0 = fa.ModParams(0, 0, 0, None, None, None, None, 0, None)
+    assert fh(mask=2, mp=window0) == 1                                     # sliding window of 0
     # three chunk buffers (Q, K, V, O of hc kv heads, 256-byte aligned, and their LSE) and
     # the slope table: B=2 H=32 Hkv=32 S=8192 D=128 -> 16 chunks of 4 kv heads
     q_bytes = 4 * 8192 * 128 * 2
