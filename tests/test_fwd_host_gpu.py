@@ -120,3 +120,16 @@ def test_many_batches_run_in_batch_chunks():
     assert (o.float() - od.cpu().float()).abs().max().item() <= 4e-3
     ro, rl = oracle.fwd(q, k, v, scale=1.0 / math.sqrt(D), **mods)
     compare(o, lse, ro, rl, "fwd_host batch runs")
+
+
+def test_pageable_host_memory():
+    """Pageable (not pinned) host tensors: the copies serialise but the results are those
+    of the pinned case, bit for bit."""
+    fa = _fa()
+    B, H, Hkv, S, D = 1, 8, 2, 700, 128
+    q, k, v = synth.qkv(B, H, Hkv, S, S, D, seed=125)
+    op, lp = fa.fwd_host(*_pinned(q, k, v), mask_mod="sliding_window", window=300)
+    oq, lq = fa.fwd_host(q.contiguous(), k.contiguous(), v.contiguous(), mask_mod="sliding_window", window=300,
+                         out=torch.empty(q.shape, dtype=q.dtype), lse_out=torch.empty((B, H, S)))
+    assert not oq.is_pinned()
+    assert torch.equal(op, oq) and torch.equal(lp, lq)
